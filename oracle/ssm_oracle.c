@@ -1,0 +1,196 @@
+/*
+ * ssm_oracle.c -- plain fp64 CPU oracle of the selective-SSM mixer core.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline leg may load this library. The product path never
+ * calls it, and it shares no code, header or constant with the CUDA sources.
+ *
+ * Everything here is written straight from the definitions, with plain loops,
+ * in double precision, no blocking, no fusion and no reordering:
+ *
+ *   conv:     xc_t[c] = silu(bias[c] + sum_k w[c,k] * win_t[c,k]), where the
+ *             window holds the K-1 previous inputs of the same sequence (the
+ *             carried conv state, or zeros, before the sequence's first token)
+ *             followed by x_t; the newest input pairs with w[c,K-1].
+ *             Source: tp_builder.py (TensorRT-Model-Connect, Mamba family),
+ *             _add_mamba_tp_layer, conv-state shift and depthwise conv step;
+ *             "Scaling State-Space Models on Multiple GPUs with Tensor
+ *             Parallelism", Fig. 1 (channel-separable 1D convolution).
+ *   delta:    D_t[c] = softplus(dt_t[c] + dt_bias[c])   (same builder, dt step,
+ *             written there as log(exp(v) + 1)).
+ *   scan:     dA = exp(D_t[c] A[c,n]); h_t[c,n] = dA h_{t-1}[c,n] + D_t[c] u_t[c] B_t[n];
+ *             y_t[c] = (sum_n C_t[n] h_t[c,n] + Dskip[c] u_t[c]) * silu(z_t[c])
+ *             (same builder: discretisation, state update, readout, D skip,
+ *             gate; Fig. 1: state update over the sequence, then gating).
+ *   packing:  every sequence of a packed batch starts from its own initial
+ *             state; nothing flows across a cu_seqlens boundary ("PackMamba:
+ *             Efficient Processing of Variable-Length Sequences in Mamba
+ *             training", abstract).
+ *   decode:   one token per row updates the cached conv and SSM state in place
+ *             (tp_builder.py: present_conv / present_ssm outputs; "Scaling
+ *             State-Space Models...", abstract: SSM cache across prefill and
+ *             decode).
+ *
+ * Channels are independent, so the outer (sequence, channel) loops may run on
+ * several OpenMP threads; each (sequence, channel) is computed by one thread in
+ * token order, so results do not depend on the thread count.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stddef.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_MAX_N 256
+#define ORACLE_MAX_K 64
+
+static double silu(double v) { return v / (1.0 + exp(-v)); }
+
+/* softplus(v) = log(1 + exp(v)), evaluated without overflow. */
+static double softplus(double v) { return (v > 0.0 ? v : 0.0) + log1p(exp(-fabs(v))); }
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* Value of the conv window for sequence s, channel c at sequence position p
+ * (p < 0 reaches into the carried state: position -1 is the newest state
+ * entry, stored at index K-2). */
+static double window_value(const double *x, const double *state_in, int64_t D, int K,
+                           int64_t start, int64_t s, int64_t c, int64_t p)
+{
+    if (p >= 0) return x[(start + p) * D + c];
+    if (state_in == NULL) return 0.0;
+    return state_in[(s * D + c) * (K - 1) + (K - 1) + p];
+}
+
+/*
+ * x, xc: (tok, D). w: (D, K). bias: (D) or NULL. cu: S+1 offsets.
+ * state_in, state_out: (S, D, K-1) or NULL; they must not alias.
+ */
+void oracle_causal_conv1d(const double *x, double *xc, const double *w, const double *bias,
+                          int64_t tok, int64_t D, int K, const int64_t *cu, int64_t S,
+                          const double *state_in, double *state_out, int apply_silu)
+{
+    (void)tok;
+#pragma omp parallel for collapse(2) schedule(dynamic, 16)
+    for (int64_t s = 0; s < S; ++s) {
+        for (int64_t c = 0; c < D; ++c) {
+            const int64_t start = cu[s];
+            const int64_t len = cu[s + 1] - cu[s];
+            for (int64_t t = 0; t < len; ++t) {
+                double acc = bias ? bias[c] : 0.0;
+                for (int k = 0; k < K; ++k) {
+                    const int64_t p = t - (K - 1) + k;
+                    acc += w[c * K + k] * window_value(x, state_in, D, K, start, s, c, p);
+                }
+                xc[(start + t) * D + c] = apply_silu ? silu(acc) : acc;
+            }
+            if (state_out) {
+                for (int j = 0; j < K - 1; ++j) {
+                    const int64_t p = len - (K - 1) + j;
+                    state_out[(s * D + c) * (K - 1) + j] =
+                        window_value(x, state_in, D, K, start, s, c, p);
+                }
+            }
+        }
+    }
+}
+
+/*
+ * u, delta, z, y: (tok, D). A: (D, N). B, C: (tok, N). Dskip, dt_bias: (D) or
+ * NULL. h0, h_final: (S, D, N) or NULL (they may be the same array: each
+ * (sequence, channel) reads its h0 before writing its h_final). z == NULL
+ * means no gate. Tokens of empty sequences do not exist, so nothing is written
+ * for them; their h_final is h0 (or zeros).
+ */
+void oracle_selective_scan(const double *u, const double *delta, const double *A,
+                           const double *B, const double *C, const double *Dskip,
+                           const double *z, const double *dt_bias, int delta_softplus,
+                           const double *h0, const int64_t *cu, int64_t S, int64_t tok,
+                           int64_t D, int N, double *y, double *h_final)
+{
+    (void)tok;
+    if (N > ORACLE_MAX_N) return;
+#pragma omp parallel for collapse(2) schedule(dynamic, 16)
+    for (int64_t s = 0; s < S; ++s) {
+        for (int64_t c = 0; c < D; ++c) {
+            double h[ORACLE_MAX_N];
+            for (int n = 0; n < N; ++n) h[n] = h0 ? h0[(s * D + c) * N + n] : 0.0;
+            for (int64_t t = cu[s]; t < cu[s + 1]; ++t) {
+                double d = delta[t * D + c] + (dt_bias ? dt_bias[c] : 0.0);
+                if (delta_softplus) d = softplus(d);
+                const double ut = u[t * D + c];
+                double acc = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    const double dA = exp(d * A[c * N + n]);
+                    h[n] = dA * h[n] + d * ut * B[t * N + n];
+                    acc += C[t * N + n] * h[n];
+                }
+                double yt = acc + (Dskip ? Dskip[c] : 0.0) * ut;
+                if (z) yt *= silu(z[t * D + c]);
+                y[t * D + c] = yt;
+            }
+            if (h_final)
+                for (int n = 0; n < N; ++n) h_final[(s * D + c) * N + n] = h[n];
+        }
+    }
+}
+
+/*
+ * One decode token per row b. Slot s = idx[b] (or b when idx is NULL); rows
+ * with s < 0 are skipped and their y row is left untouched. conv_state:
+ * (n_slots, D, K-1), ssm_state: (n_slots, D, N); both are updated in place.
+ * x, dt, z, y: (Bt, D); B, C: (Bt, N).
+ */
+void oracle_state_update(double *conv_state, double *ssm_state, const double *x,
+                         const double *dt, const double *B, const double *C, const double *z,
+                         const double *conv_w, const double *conv_b, const double *A,
+                         const double *Dskip, const double *dt_bias, int delta_softplus,
+                         const int64_t *idx, int64_t n_slots, double *y, int64_t Bt,
+                         int64_t D, int N, int K)
+{
+    if (N > ORACLE_MAX_N || K > ORACLE_MAX_K) return;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < Bt; ++b) {
+        for (int64_t c = 0; c < D; ++c) {
+            const int64_t s = idx ? idx[b] : b;
+            if (s < 0 || s >= n_slots) continue;
+            double win[ORACLE_MAX_K];
+            for (int j = 0; j < K - 1; ++j) win[j] = conv_state[(s * D + c) * (K - 1) + j];
+            win[K - 1] = x[b * D + c];
+            double acc = conv_b ? conv_b[c] : 0.0;
+            for (int k = 0; k < K; ++k) acc += conv_w[c * K + k] * win[k];
+            const double xcv = silu(acc);
+            for (int j = 0; j < K - 1; ++j) conv_state[(s * D + c) * (K - 1) + j] = win[j + 1];
+
+            double d = dt[b * D + c] + (dt_bias ? dt_bias[c] : 0.0);
+            if (delta_softplus) d = softplus(d);
+            double *h = ssm_state + (s * D + c) * N;
+            double sum = 0.0;
+            for (int n = 0; n < N; ++n) {
+                const double dA = exp(d * A[c * N + n]);
+                h[n] = dA * h[n] + d * xcv * B[b * N + n];
+                sum += C[b * N + n] * h[n];
+            }
+            double yt = sum + (Dskip ? Dskip[c] : 0.0) * xcv;
+            if (z) yt *= silu(z[b * D + c]);
+            y[b * D + c] = yt;
+        }
+    }
+}
