@@ -1,0 +1,200 @@
+/*
+ * ssm_causal.h -- C ABI of the B200 (sm_100a) selective-SSM mixer core.
+ *
+ * Three operations, each one asynchronous call on a caller-given stream:
+ *
+ *   ssm_causal_conv1d           causal depthwise conv1d + bias + SiLU over packed
+ *                               sequences, with carried conv state in and out
+ *   ssm_selective_scan_fwd      selective scan (dA = exp(delta*A),
+ *                               h_t = dA*h_{t-1} + delta*u_t*B_t,
+ *                               y_t = (C_t.h_t + Dskip*u_t) * silu(z_t)) over packed
+ *                               sequences, with optional h0 and final-state output
+ *   ssm_selective_state_update  one decode token per row: conv-state shift, conv,
+ *                               softplus, state update in place, readout and gate
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *   never allocates, frees or retains memory, and never synchronises the host.
+ * - Layouts are row-major and token-major with channels contiguous:
+ *   activations (tok, D); B and C (tok, N), one group shared by all channels;
+ *   A (D, N); conv weight (D, K); Dskip, dt_bias, conv bias (D);
+ *   SSM state (S, D, N) fp32; conv state (S, D, K-1), oldest entry first.
+ * - Packed variable-length sequences are described by cu_seqlens, S+1 int32
+ *   offsets on the device: sequence s owns tokens [cu[s], cu[s+1]). It must be
+ *   non-decreasing with cu[0] = 0 and cu[S] = tok (ssm_check_cu_seqlens checks
+ *   a host copy). Nothing flows across a boundary: each sequence starts from
+ *   its own initial state. Kernels clamp every offset into [0, tok], so a bad
+ *   array gives wrong values but never an out-of-bounds access. Sequences may
+ *   be empty. cu_seqlens == NULL means a dense batch of S rows of tok/S tokens.
+ * - Floating-point work is fp32 throughout (fp32 state, fp32 accumulation);
+ *   bf16 tensors are converted on load and rounded to nearest even on store.
+ * - Results are deterministic: no atomics take part in the arithmetic.
+ * - Every call returns SSM_OK (0) or a negative status and then launches
+ *   nothing; ssm_last_error() gives a message for the calling thread.
+ *
+ * Sources (titles of the pages this follows):
+ * - tp_builder.py (TensorRT-Model-Connect, Mamba family), _add_mamba_tp_layer:
+ *   the per-token mixer math (conv-state shift, depthwise conv, softplus of dt,
+ *   discretisation dA = exp(delta*A) and dB = delta*B, state update, C readout,
+ *   D skip, silu(z) gate) and the present_conv / present_ssm state outputs.
+ * - "Scaling State-Space Models on Multiple GPUs with Tensor Parallelism"
+ *   (Dutt, Shah, Masarani, Gandhi): Fig. 1 (mixer dataflow) and the abstract
+ *   (SSM state cache carried across prefill and decode).
+ * - "PackMamba: Efficient Processing of Variable-Length Sequences in Mamba
+ *   training", abstract: packed sequences with no information passed between
+ *   sequences.
+ */
+#ifndef SSM_CAUSAL_H
+#define SSM_CAUSAL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *ssm_stream_t;
+
+typedef enum { SSM_F32 = 0, SSM_BF16 = 1 } ssm_dtype;
+
+enum {
+    SSM_OK = 0,
+    SSM_ERR_INVALID_ARGUMENT = -1, /* null required pointer, bad size, unsupported N or K */
+    SSM_ERR_UNSUPPORTED_DTYPE = -2,
+    SSM_ERR_MISALIGNED = -3,       /* a pointer is not aligned to its element size */
+    SSM_ERR_BAD_SEQLENS = -4,      /* cu_seqlens rejected (host check) */
+    SSM_ERR_WORKSPACE = -5,        /* workspace given but too small */
+    SSM_ERR_CUDA = -6              /* a CUDA launch or runtime call failed */
+};
+
+/* Message describing the last failing call on this host thread ("" if none). */
+const char *ssm_last_error(void);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int ssm_version(void);
+
+/* Number of kernels this library has launched in this process (all calls,
+ * all threads). Lets a caller count launches inside a timed region. */
+unsigned long long ssm_launch_count(void);
+
+/*
+ * Tuning knob for ssm_selective_scan_fwd: states of one channel handled per
+ * lane (4, 8 or 16; 16 / value lanes then share a channel), or 0 to let the
+ * library choose from the number of (sequence, channel) pairs. Process-wide;
+ * not thread-safe against concurrent scan calls. Returns SSM_OK or
+ * SSM_ERR_INVALID_ARGUMENT.
+ */
+int ssm_set_scan_states_per_lane(int states_per_lane);
+
+/*
+ * Checks a HOST copy of cu_seqlens (S+1 entries): cu[0] == 0, non-decreasing,
+ * cu[S] == tok. Returns SSM_OK or SSM_ERR_BAD_SEQLENS. Touches no device.
+ */
+int ssm_check_cu_seqlens(const int32_t *cu_seqlens_host, int64_t S, int64_t tok);
+
+/*
+ * Causal depthwise conv1d (+ bias, + SiLU) over packed sequences.
+ * Follows tp_builder.py, _add_mamba_tp_layer (conv-state shift and conv step):
+ *   xc[t,c] = act(bias[c] + sum_{k<K} w[c,k] * win_t[c,k])
+ * where win_t holds the K-1 inputs of the same sequence before t (the carried
+ * conv state, or zeros, before the sequence's first token) and then x[t,c];
+ * the newest input pairs with w[c,K-1]. act is SiLU when apply_silu != 0.
+ *
+ *   x              (tok, D) of x_dtype; read only
+ *   xc             (tok, D) of x_dtype; written; must not overlap x
+ *   weight         (D, K) fp32;  bias: (D) fp32 or NULL (= 0)
+ *   tok, D         tokens in the call (>= 0) and channels (>= 1)
+ *   K              conv width, 2..4
+ *   cu_seqlens, S  see the conventions above (S >= 1)
+ *   conv_state_in  (S, D, K-1) of state_dtype or NULL (= zeros)
+ *   conv_state_out (S, D, K-1) of state_dtype or NULL (= not written): the last
+ *                  K-1 entries of [conv_state_in || x_seq] per sequence, so a
+ *                  sequence shorter than K-1 keeps part of its carried state.
+ *                  May be the same buffer as conv_state_in.
+ * Launches 1 kernel, or 2 when conv_state_out is given.
+ */
+int ssm_causal_conv1d(const void *x, void *xc, const float *weight, const float *bias,
+                      int64_t tok, int64_t D, int K, const int32_t *cu_seqlens, int64_t S,
+                      const void *conv_state_in, void *conv_state_out, int apply_silu,
+                      ssm_dtype x_dtype, ssm_dtype state_dtype, ssm_stream_t stream);
+
+/*
+ * Bytes of optional scratch for ssm_selective_scan_fwd with S packed
+ * sequences (a longest-first schedule of the sequences). Passing a NULL
+ * workspace is always allowed: sequences are then scheduled in index order.
+ */
+size_t ssm_scan_workspace_size(int64_t tok, int64_t D, int N, int64_t S);
+
+/*
+ * Selective scan over packed sequences.
+ * Follows tp_builder.py, _add_mamba_tp_layer (dt softplus, dA = exp(delta*A),
+ * dBx = delta*B*u, h = dA*h + dBx, y = C.h + D*u, times silu(z)), run over each
+ * sequence in order as Fig. 1 of "Scaling State-Space Models on Multiple GPUs
+ * with Tensor Parallelism" describes, resetting at every cu_seqlens boundary
+ * ("PackMamba", abstract).
+ *
+ *   u              (tok, D) act_dtype: the conv output xc
+ *   delta          (tok, D) act_dtype: raw dt (delta_softplus != 0) or delta
+ *   A              (D, N) fp32 (negative reals for a decaying state)
+ *   B, C           (tok, N) act_dtype
+ *   Dskip          (D) fp32 or NULL (= 0)
+ *   z              (tok, D) act_dtype or NULL (= no gate)
+ *   dt_bias        (D) fp32 or NULL (= 0), added before the softplus
+ *   delta_softplus 1: delta = softplus(dt + dt_bias); 0: delta = dt + dt_bias
+ *   h0             (S, D, N) fp32 or NULL (= zeros)
+ *   cu_seqlens, S  see the conventions above
+ *   y              (tok, D) act_dtype, written; tokens outside every sequence
+ *                  are left untouched
+ *   h_final        (S, D, N) fp32 or NULL; may be the same buffer as h0
+ *   tok, D, N      N must be 16
+ *   workspace      NULL or >= ssm_scan_workspace_size() bytes of device
+ *                  scratch, 256-byte aligned; its contents are overwritten
+ * y must not overlap u, delta, z, B or C.
+ */
+int ssm_selective_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                           const void *C, const float *Dskip, const void *z,
+                           const float *dt_bias, int delta_softplus, const float *h0,
+                           const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
+                           int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
+                           size_t workspace_bytes, ssm_stream_t stream);
+
+/*
+ * One decode token per row, updating the cached states in place.
+ * Follows the whole of tp_builder.py, _add_mamba_tp_layer for one token (its
+ * conv_state / ssm_state inputs and present_conv / present_ssm outputs) and
+ * the SSM cache of "Scaling State-Space Models...", abstract and Fig. 2 (1).
+ * For row b with slot s = state_indices[b] (or b when state_indices is NULL):
+ *   win = [conv_state[s] || x[b]]; xc = silu(conv_b + sum_k conv_w[:,k]*win[k]);
+ *   conv_state[s] = last K-1 of win; delta = softplus(dt[b] + dt_bias) (flag);
+ *   ssm_state[s] = exp(delta*A)*ssm_state[s] + delta*xc*B[b];
+ *   y[b] = (C[b].ssm_state[s] + Dskip*xc) * silu(z[b]).
+ *
+ *   conv_state     (n_slots, D, K-1) of conv_state_dtype, updated in place
+ *   ssm_state      (n_slots, D, N) fp32, updated in place
+ *   x, dt, z       (Bt, D) act_dtype (z may be NULL = no gate)
+ *   B, C           (Bt, N) act_dtype
+ *   conv_w (D, K), conv_b (D) or NULL, A (D, N), Dskip (D) or NULL,
+ *   dt_bias (D) or NULL: fp32
+ *   state_indices  (Bt) int32 or NULL (= identity, needs n_slots >= Bt). A row
+ *                  with index -1 (any negative) is skipped and its y row is
+ *                  left untouched; an index >= n_slots is skipped as well.
+ *                  Two rows naming the same slot race (undefined result).
+ *   y              (Bt, D) act_dtype
+ *   N must be 16; K in 2..4.
+ */
+int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x,
+                               const void *dt, const void *B, const void *C, const void *z,
+                               const float *conv_w, const float *conv_b, const float *A,
+                               const float *Dskip, const float *dt_bias, int delta_softplus,
+                               const int32_t *state_indices, int64_t n_slots, void *y,
+                               int64_t Bt, int64_t D, int N, int K, ssm_dtype act_dtype,
+                               ssm_dtype conv_state_dtype, ssm_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSM_CAUSAL_H */

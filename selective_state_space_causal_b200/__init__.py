@@ -1,0 +1,22 @@
+"""B200-native (sm_100a) selective-SSM mixer core.
+
+The computation lives in ``libssm_causal.so`` (hand-written CUDA behind the C
+ABI declared in ``include/ssm_causal.h``); this package is its thin Python
+binding. Importing it loads the library and fails loudly if it is missing.
+"""
+
+from ._lib import (  # noqa: F401
+    SSM_BF16,
+    SSM_F32,
+    SsmError,
+    lib,
+    ssm_causal_conv1d,
+    ssm_check_cu_seqlens,
+    ssm_last_error,
+    ssm_launch_count,
+    ssm_scan_workspace_size,
+    ssm_selective_scan_fwd,
+    ssm_selective_state_update,
+    ssm_set_scan_states_per_lane,
+    ssm_version,
+)

@@ -1,0 +1,161 @@
+"""ctypes binding of libssm_causal.so (argument marshalling only).
+
+Each function here has the name of the C entry point it calls and does
+nothing but turn tensors into pointers, dtypes into enums and the current
+torch stream into a stream handle; every step of the computation runs in the
+library's CUDA kernels. There is no fallback: if the library is missing the
+import fails, and a failing call raises SsmError with the library's message.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(HERE, "libssm_causal.so")
+
+SSM_F32, SSM_BF16 = 0, 1
+STATUS = {0: "SSM_OK", -1: "SSM_ERR_INVALID_ARGUMENT", -2: "SSM_ERR_UNSUPPORTED_DTYPE",
+          -3: "SSM_ERR_MISALIGNED", -4: "SSM_ERR_BAD_SEQLENS", -5: "SSM_ERR_WORKSPACE",
+          -6: "SSM_ERR_CUDA"}
+
+# (name, restype, argtypes) of every symbol include/ssm_causal.h declares
+_vp, _i64, _int, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = [
+    ("ssm_last_error", ctypes.c_char_p, []),
+    ("ssm_version", _int, []),
+    ("ssm_launch_count", ctypes.c_ulonglong, []),
+    ("ssm_set_scan_states_per_lane", _int, [_int]),
+    ("ssm_check_cu_seqlens", _int, [_vp, _i64, _i64]),
+    ("ssm_causal_conv1d", _int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _i64, _vp, _vp, _int,
+                                 _int, _int, _vp]),
+    ("ssm_scan_workspace_size", _sz, [_i64, _i64, _int, _i64]),
+    ("ssm_selective_scan_fwd", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64,
+                                      _vp, _vp, _i64, _i64, _int, _int, _vp, _sz, _vp]),
+    ("ssm_selective_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                          _vp, _int, _vp, _i64, _vp, _i64, _i64, _int, _int, _int,
+                                          _int, _vp]),
+]
+
+
+class SsmError(RuntimeError):
+    def __init__(self, code: int, message: str):
+        super().__init__(f"{STATUS.get(code, code)}: {message}")
+        self.code = code
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIBRARY):
+        raise ImportError(
+            f"{LIBRARY} is missing: build it with `python -m selective_state_space_causal_b200.build`"
+        )
+    lib = ctypes.CDLL(LIBRARY)
+    for name, res, args in SIGNATURES:
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(code: int) -> None:
+    if code != 0:
+        raise SsmError(code, lib.ssm_last_error().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dtype(t) -> int:
+    import torch
+
+    if t.dtype == torch.bfloat16:
+        return SSM_BF16
+    if t.dtype == torch.float32:
+        return SSM_F32
+    raise SsmError(-2, f"unsupported tensor dtype {t.dtype}")
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream if isinstance(stream, int) else stream.cuda_stream
+    import torch
+
+    return torch.cuda.current_stream().cuda_stream
+
+
+def ssm_last_error() -> str:
+    return lib.ssm_last_error().decode()
+
+
+def ssm_version() -> int:
+    return lib.ssm_version()
+
+
+def ssm_launch_count() -> int:
+    return int(lib.ssm_launch_count())
+
+
+def ssm_set_scan_states_per_lane(n: int) -> None:
+    _check(lib.ssm_set_scan_states_per_lane(int(n)))
+
+
+def ssm_check_cu_seqlens(cu_seqlens_host, tok: int) -> None:
+    """Check a host (CPU, int32, contiguous) copy of cu_seqlens."""
+    S = cu_seqlens_host.numel() - 1
+    _check(lib.ssm_check_cu_seqlens(_ptr(cu_seqlens_host), S, int(tok)))
+
+
+def ssm_scan_workspace_size(tok: int, D: int, N: int, S: int) -> int:
+    return int(lib.ssm_scan_workspace_size(tok, D, N, S))
+
+
+def ssm_causal_conv1d(x, xc, weight, bias=None, cu_seqlens=None, S=None, conv_state_in=None,
+                      conv_state_out=None, apply_silu=True, stream=None):
+    """x, xc: (tok, D); weight (D, K) fp32; states (S, D, K-1)."""
+    tok, D = x.shape
+    K = weight.shape[1]
+    if S is None:
+        S = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
+    st = conv_state_in if conv_state_in is not None else conv_state_out
+    sdt = _dtype(st) if st is not None else _dtype(x)
+    _check(lib.ssm_causal_conv1d(_ptr(x), _ptr(xc), _ptr(weight), _ptr(bias), tok, D, K,
+                                 _ptr(cu_seqlens), S, _ptr(conv_state_in), _ptr(conv_state_out),
+                                 int(bool(apply_silu)), _dtype(x), sdt, _stream(stream)))
+
+
+def ssm_selective_scan_fwd(u, delta, A, B, C, y, Dskip=None, z=None, dt_bias=None,
+                           delta_softplus=True, h0=None, h_final=None, cu_seqlens=None, S=None,
+                           workspace=None, stream=None):
+    """u, delta, z, y: (tok, D); A (D, N); B, C (tok, N); h0 / h_final (S, D, N) fp32."""
+    tok, D = u.shape
+    N = A.shape[1]
+    if S is None:
+        S = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ssm_selective_scan_fwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C),
+                                      _ptr(Dskip), _ptr(z), _ptr(dt_bias), int(bool(delta_softplus)),
+                                      _ptr(h0), _ptr(cu_seqlens), S, _ptr(y), _ptr(h_final), tok, D,
+                                      N, _dtype(u), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def ssm_selective_state_update(conv_state, ssm_state, x, dt, B, C, y, conv_w, A, z=None,
+                               conv_b=None, Dskip=None, dt_bias=None, delta_softplus=True,
+                               state_indices=None, stream=None):
+    """conv_state (slots, D, K-1); ssm_state (slots, D, N) fp32; x, dt, z, y (Bt, D)."""
+    Bt, D = x.shape
+    N = A.shape[1]
+    K = conv_w.shape[1]
+    _check(lib.ssm_selective_state_update(
+        _ptr(conv_state), _ptr(ssm_state), _ptr(x), _ptr(dt), _ptr(B), _ptr(C), _ptr(z),
+        _ptr(conv_w), _ptr(conv_b), _ptr(A), _ptr(Dskip), _ptr(dt_bias), int(bool(delta_softplus)),
+        _ptr(state_indices), ssm_state.shape[0], _ptr(y), Bt, D, N, K, _dtype(x),
+        _dtype(conv_state), _stream(stream)))

@@ -1,0 +1,232 @@
+// api.cu -- the extern "C" boundary: argument validation, dispatch, errors.
+//
+// Every entry point validates its arguments on the host before touching the
+// device (the tensor-parallel builder this library follows rejects bad shapes
+// up front as well: tp_builder.py, _validate_mamba_tp), then launches its
+// kernels asynchronously on the caller's stream. Failures return a negative
+// status and leave a message in a thread-local buffer.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "../../include/ssm_causal.h"
+#include "internal.h"
+
+namespace ssm {
+void set_scan_npt(int npt);
+size_t scan_order_bytes(int64_t S);
+}  // namespace ssm
+
+namespace {
+
+thread_local std::string g_error;
+std::atomic<unsigned long long> g_launches{0};
+
+int fail(int code, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_error = buf;
+    return code;
+}
+
+int ok()
+{
+    g_error.clear();
+    return SSM_OK;
+}
+
+size_t esize(ssm_dtype t) { return t == SSM_BF16 ? 2 : 4; }
+
+bool valid_dtype(ssm_dtype t) { return t == SSM_F32 || t == SSM_BF16; }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+ssm::DType dt(ssm_dtype t) { return t == SSM_BF16 ? ssm::DType::BF16 : ssm::DType::F32; }
+
+int finish(cudaError_t e, int launched, const char *what)
+{
+    g_launches.fetch_add((unsigned long long)launched, std::memory_order_relaxed);
+    if (e != cudaSuccess)
+        return fail(SSM_ERR_CUDA, "%s: CUDA error %d (%s)", what, (int)e, cudaGetErrorString(e));
+    return ok();
+}
+
+// Common checks of the packed-sequence description.
+int check_seqs(const char *fn, const int32_t *cu, int64_t S, int64_t tok)
+{
+    if (S < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: S must be >= 1 (got %lld)", fn, (long long)S);
+    if (S > 65535)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: at most 65535 sequences per call (got %lld)", fn,
+                    (long long)S);
+    if (tok < 0 || tok > (int64_t)INT32_MAX)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: tok out of range (%lld)", fn, (long long)tok);
+    if (!cu && tok % S != 0)
+        return fail(SSM_ERR_INVALID_ARGUMENT,
+                    "%s: without cu_seqlens, tok (%lld) must be a multiple of S (%lld)", fn,
+                    (long long)tok, (long long)S);
+    if (cu && !aligned(cu, 4)) return fail(SSM_ERR_MISALIGNED, "%s: cu_seqlens misaligned", fn);
+    return SSM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ssm_last_error(void) { return g_error.c_str(); }
+
+int ssm_version(void) { return 100; }
+
+unsigned long long ssm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int ssm_set_scan_states_per_lane(int npt)
+{
+    if (npt != 0 && npt != 4 && npt != 8 && npt != 16)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "ssm_set_scan_states_per_lane: use 0, 4, 8 or 16");
+    ssm::set_scan_npt(npt);
+    return ok();
+}
+
+int ssm_check_cu_seqlens(const int32_t *cu, int64_t S, int64_t tok)
+{
+    if (!cu) return fail(SSM_ERR_INVALID_ARGUMENT, "ssm_check_cu_seqlens: null pointer");
+    if (S < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "ssm_check_cu_seqlens: S must be >= 1");
+    if (cu[0] != 0) return fail(SSM_ERR_BAD_SEQLENS, "cu_seqlens[0] = %d, expected 0", cu[0]);
+    for (int64_t i = 0; i < S; ++i)
+        if (cu[i + 1] < cu[i])
+            return fail(SSM_ERR_BAD_SEQLENS, "cu_seqlens decreases at %lld (%d -> %d)",
+                        (long long)i, cu[i], cu[i + 1]);
+    if ((int64_t)cu[S] != tok)
+        return fail(SSM_ERR_BAD_SEQLENS, "cu_seqlens[S] = %d, expected tok = %lld", cu[S],
+                    (long long)tok);
+    return ok();
+}
+
+int ssm_causal_conv1d(const void *x, void *xc, const float *weight, const float *bias,
+                      int64_t tok, int64_t D, int K, const int32_t *cu_seqlens, int64_t S,
+                      const void *conv_state_in, void *conv_state_out, int apply_silu,
+                      ssm_dtype x_dtype, ssm_dtype state_dtype, ssm_stream_t stream)
+{
+    const char *fn = "ssm_causal_conv1d";
+    if (!valid_dtype(x_dtype) || !valid_dtype(state_dtype))
+        return fail(SSM_ERR_UNSUPPORTED_DTYPE, "%s: unknown dtype", fn);
+    if (D < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: D must be >= 1", fn);
+    if (K < 2 || K > 4) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: K must be 2..4 (got %d)", fn, K);
+    if (int r = check_seqs(fn, cu_seqlens, S, tok)) return r;
+    if (!weight) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: weight is NULL", fn);
+    if (tok > 0 && (!x || !xc)) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: x or xc is NULL", fn);
+    if (conv_state_out && S * D > 0 && !x && tok > 0)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: x is NULL", fn);
+    const size_t es = esize(x_dtype), ss = esize(state_dtype);
+    if (!aligned(x, es) || !aligned(xc, es) || !aligned(weight, 4) || !aligned(bias, 4) ||
+        !aligned(conv_state_in, ss) || !aligned(conv_state_out, ss))
+        return fail(SSM_ERR_MISALIGNED, "%s: a pointer is not aligned to its element size", fn);
+    if (x && xc && tok > 0) {
+        const char *a = static_cast<const char *>(x), *b = static_cast<const char *>(xc);
+        const size_t bytes = (size_t)tok * D * es;
+        if (a < b + bytes && b < a + bytes)
+            return fail(SSM_ERR_INVALID_ARGUMENT, "%s: xc overlaps x", fn);
+    }
+    ssm::ConvArgs a{x, xc, weight, bias, tok, D, K, cu_seqlens, S, conv_state_in,
+                    conv_state_out, apply_silu, dt(x_dtype), dt(state_dtype),
+                    aligned(x, 16) && aligned(xc, 16)};
+    int launched = 0;
+    cudaError_t e = ssm::launch_conv1d(a, reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
+size_t ssm_scan_workspace_size(int64_t tok, int64_t D, int N, int64_t S)
+{
+    (void)tok; (void)D; (void)N;
+    return S > 1 ? ssm::scan_order_bytes(S) : 0;
+}
+
+int ssm_selective_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                           const void *C, const float *Dskip, const void *z,
+                           const float *dt_bias, int delta_softplus, const float *h0,
+                           const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
+                           int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
+                           size_t workspace_bytes, ssm_stream_t stream)
+{
+    const char *fn = "ssm_selective_scan_fwd";
+    if (!valid_dtype(act_dtype)) return fail(SSM_ERR_UNSUPPORTED_DTYPE, "%s: unknown dtype", fn);
+    if (N != 16) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: N must be 16 (got %d)", fn, N);
+    if (D < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: D must be >= 1", fn);
+    if (int r = check_seqs(fn, cu_seqlens, S, tok)) return r;
+    if (!A) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: A is NULL", fn);
+    if (tok > 0 && (!u || !delta || !B || !C || !y))
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: u, delta, B, C and y are required", fn);
+    const size_t es = esize(act_dtype);
+    if (!aligned(u, es) || !aligned(delta, es) || !aligned(z, es) || !aligned(y, es) ||
+        !aligned(A, 4) || !aligned(Dskip, 4) || !aligned(dt_bias, 4) || !aligned(h0, 4) ||
+        !aligned(h_final, 4))
+        return fail(SSM_ERR_MISALIGNED, "%s: a pointer is not aligned to its element size", fn);
+    if (!aligned(B, 16) || !aligned(C, 16))
+        return fail(SSM_ERR_MISALIGNED, "%s: B and C must be 16-byte aligned", fn);
+    const size_t need = ssm_scan_workspace_size(tok, D, N, S);
+    if (workspace && workspace_bytes < need)
+        return fail(SSM_ERR_WORKSPACE, "%s: workspace has %zu bytes, needs %zu", fn,
+                    workspace_bytes, need);
+    if (workspace && !aligned(workspace, 256))
+        return fail(SSM_ERR_MISALIGNED, "%s: workspace must be 256-byte aligned", fn);
+    if (y && tok > 0) {
+        const size_t bytes = (size_t)tok * D * es;
+        const void *ins[3] = {u, delta, z};
+        for (const void *in : ins) {
+            if (!in) continue;
+            const char *a = static_cast<const char *>(in), *b = static_cast<const char *>(y);
+            if (a < b + bytes && b < a + bytes)
+                return fail(SSM_ERR_INVALID_ARGUMENT, "%s: y overlaps an input", fn);
+        }
+    }
+    const bool vec = aligned(u, 16) && aligned(delta, 16) && aligned(y, 16) &&
+                     (!z || aligned(z, 16));
+    ssm::ScanArgs a{u, delta, A, B, C, Dskip, z, dt_bias, delta_softplus, h0, cu_seqlens, S,
+                    y, h_final, tok, D, N, dt(act_dtype),
+                    workspace ? static_cast<int32_t *>(workspace) : nullptr, vec};
+    int launched = 0;
+    cudaError_t e = ssm::launch_scan(a, reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
+int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x,
+                               const void *dt_, const void *B, const void *C, const void *z,
+                               const float *conv_w, const float *conv_b, const float *A,
+                               const float *Dskip, const float *dt_bias, int delta_softplus,
+                               const int32_t *state_indices, int64_t n_slots, void *y,
+                               int64_t Bt, int64_t D, int N, int K, ssm_dtype act_dtype,
+                               ssm_dtype conv_state_dtype, ssm_stream_t stream)
+{
+    const char *fn = "ssm_selective_state_update";
+    if (!valid_dtype(act_dtype) || !valid_dtype(conv_state_dtype))
+        return fail(SSM_ERR_UNSUPPORTED_DTYPE, "%s: unknown dtype", fn);
+    if (N != 16) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: N must be 16 (got %d)", fn, N);
+    if (K < 2 || K > 4) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: K must be 2..4 (got %d)", fn, K);
+    if (D < 1 || Bt < 0 || Bt > 65535 || n_slots < 0)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: bad sizes (D=%lld, Bt=%lld, n_slots=%lld)", fn,
+                    (long long)D, (long long)Bt, (long long)n_slots);
+    if (!state_indices && n_slots < Bt)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: identity slots need n_slots >= Bt", fn);
+    if (Bt > 0 && (!conv_state || !ssm_state || !x || !dt_ || !B || !C || !conv_w || !A || !y))
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: a required pointer is NULL", fn);
+    const size_t es = esize(act_dtype);
+    if (!aligned(x, es) || !aligned(dt_, es) || !aligned(B, es) || !aligned(C, es) ||
+        !aligned(z, es) || !aligned(y, es) || !aligned(conv_state, esize(conv_state_dtype)) ||
+        !aligned(conv_w, 4) || !aligned(conv_b, 4) || !aligned(A, 4) || !aligned(Dskip, 4) ||
+        !aligned(dt_bias, 4) || !aligned(state_indices, 4))
+        return fail(SSM_ERR_MISALIGNED, "%s: a pointer is not aligned to its element size", fn);
+    if (!aligned(ssm_state, 16))
+        return fail(SSM_ERR_MISALIGNED, "%s: ssm_state must be 16-byte aligned", fn);
+    ssm::DecodeArgs a{conv_state, ssm_state, x, dt_, B, C, z, conv_w, conv_b, A, Dskip, dt_bias,
+                      delta_softplus, state_indices, n_slots, y, Bt, D, N, K, dt(act_dtype),
+                      dt(conv_state_dtype)};
+    int launched = 0;
+    cudaError_t e = ssm::launch_decode(a, reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
+}  // extern "C"

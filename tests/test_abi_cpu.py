@@ -1,0 +1,136 @@
+"""The C-ABI library on the host: it loads without a GPU, exports every symbol
+the header declares, and rejects bad arguments before touching any device."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import selective_state_space_causal_b200 as ssm
+from selective_state_space_causal_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssm_causal.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^[A-Za-z_][\w\s\*]*?\b(ssm_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_three_operations():
+    names = declared_functions()
+    for op in ("ssm_causal_conv1d", "ssm_selective_scan_fwd", "ssm_selective_state_update"):
+        assert op in names
+
+
+def test_library_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIBRARY], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (\w+)$", out, flags=re.M))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(_lib.lib, name)
+
+
+def test_binding_covers_every_declared_symbol():
+    bound = {name for name, _, _ in _lib.SIGNATURES}
+    assert bound == set(declared_functions())
+
+
+# --- argument validation (fake device addresses; nothing reaches a device) ---
+L = _lib.lib
+A16 = 0x10000  # 16-byte aligned fake address
+
+
+def _err():
+    return ssm.ssm_last_error()
+
+
+def conv(**kw):
+    args = dict(x=A16, xc=A16 + 0x100000, w=A16, b=None, tok=64, D=32, K=4, cu=None, S=1,
+                si=None, so=None, silu=1, xdt=1, sdt=1)
+    args.update(kw)
+    return L.ssm_causal_conv1d(args["x"], args["xc"], args["w"], args["b"], args["tok"],
+                               args["D"], args["K"], args["cu"], args["S"], args["si"],
+                               args["so"], args["silu"], args["xdt"], args["sdt"], None)
+
+
+def scan(**kw):
+    a = dict(u=A16, dt=A16 + 0x200000, A=A16, B=A16, C=A16, Dsk=None, z=None, dtb=None, sp=1,
+             h0=None, cu=None, S=1, y=A16 + 0x400000, hf=None, tok=64, D=32, N=16, adt=1,
+             ws=None, wsb=0)
+    a.update(kw)
+    return L.ssm_selective_scan_fwd(a["u"], a["dt"], a["A"], a["B"], a["C"], a["Dsk"], a["z"],
+                                    a["dtb"], a["sp"], a["h0"], a["cu"], a["S"], a["y"], a["hf"],
+                                    a["tok"], a["D"], a["N"], a["adt"], a["ws"], a["wsb"], None)
+
+
+def decode(**kw):
+    a = dict(cs=A16, ss=A16, x=A16, dt=A16, B=A16, C=A16, z=None, w=A16, b=None, A=A16, Dsk=None,
+             dtb=None, sp=1, idx=None, slots=8, y=A16, Bt=8, D=32, N=16, K=4, adt=1, cdt=1)
+    a.update(kw)
+    return L.ssm_selective_state_update(a["cs"], a["ss"], a["x"], a["dt"], a["B"], a["C"],
+                                        a["z"], a["w"], a["b"], a["A"], a["Dsk"], a["dtb"],
+                                        a["sp"], a["idx"], a["slots"], a["y"], a["Bt"], a["D"],
+                                        a["N"], a["K"], a["adt"], a["cdt"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(K=5), -1), (dict(K=1), -1), (dict(S=0), -1), (dict(tok=63, S=2), -1),
+    (dict(D=0), -1), (dict(x=None), -1), (dict(w=None), -1), (dict(xc=A16 + 1), -3),
+    (dict(xdt=7), -2), (dict(xc=A16 + 64), -1), (dict(S=70000, tok=70000), -1),
+    (dict(cu=A16 + 2), -3),
+])
+def test_conv_rejects(kw, code):
+    assert conv(**kw) == code
+    assert _err()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=8), -1), (dict(N=32), -1), (dict(u=None), -1), (dict(A=None), -1),
+    (dict(B=A16 + 8), -3), (dict(u=A16 + 1), -3), (dict(adt=3), -2),
+    (dict(y=A16 + 0x200000), -1), (dict(S=3, tok=64), -1),
+    (dict(cu=A16, S=4, ws=A16, wsb=8), -5), (dict(cu=A16, S=4, ws=A16 + 16, wsb=4096), -3),
+])
+def test_scan_rejects(kw, code):
+    assert scan(**kw) == code
+    assert _err()
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=4), -1), (dict(K=6), -1), (dict(slots=4), -1), (dict(ss=A16 + 4), -3),
+    (dict(x=None), -1), (dict(cdt=5), -2), (dict(Bt=70000, slots=70000), -1),
+])
+def test_decode_rejects(kw, code):
+    assert decode(**kw) == code
+    assert _err()
+
+
+def test_workspace_size():
+    assert ssm.ssm_scan_workspace_size(100, 64, 16, 1) == 0
+    n = ssm.ssm_scan_workspace_size(65536, 5120, 16, 34)
+    assert n >= 34 * 4 and n % 256 == 0
+
+
+def test_check_cu_seqlens_host():
+    import torch
+
+    good = torch.tensor([0, 3, 3, 10], dtype=torch.int32)
+    ssm.ssm_check_cu_seqlens(good, 10)
+    for bad, tok in (([1, 3, 10], 10), ([0, 5, 3, 10], 10), ([0, 3, 9], 10)):
+        with pytest.raises(ssm.SsmError) as ei:
+            ssm.ssm_check_cu_seqlens(torch.tensor(bad, dtype=torch.int32), tok)
+        assert ei.value.code == -4
+
+
+def test_tuning_knob():
+    for n in (0, 4, 8, 16):
+        ssm.ssm_set_scan_states_per_lane(n)
+    with pytest.raises(ssm.SsmError):
+        ssm.ssm_set_scan_states_per_lane(3)
+    ssm.ssm_set_scan_states_per_lane(0)

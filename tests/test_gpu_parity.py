@@ -1,0 +1,239 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Sizes span several channel tiles and token chunks with ragged tails; packed
+cases include empty sequences and sequences shorter than the conv window.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import selective_state_space_causal_b200 as ssm
+from selective_state_space_causal_b200 import synth
+from gpu_helpers import (TOL_BF16, TOL_F32, act_dtype, assert_close, cu_tensor, dev, host,
+                         run_conv, run_scan)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _auto_variant():
+    ssm.ssm_set_scan_states_per_lane(0)
+    yield
+    ssm.ssm_set_scan_states_per_lane(0)
+
+
+def _layer_inputs(seed, tok, D, bf16, K=4, random_bias=True, random_A=True):
+    prm = synth.make_params(seed, D, K=K, random_bias=random_bias, random_A=random_A,
+                            random_D=True)
+    act = synth.make_activations(seed, tok, D, bf16=bf16)
+    return prm, act
+
+
+# ---------------------------------------------------------------------------
+# conv
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bf16", [False, True])
+@pytest.mark.parametrize("K", [2, 3, 4])
+@pytest.mark.parametrize("D", [40, 30])  # vector path / scalar path
+def test_conv_packed_with_state(orc, bf16, K, D):
+    lens = [70, 0, 1, 2, 3, 33, 5, 64]
+    tok = sum(lens)
+    prm, act = _layer_inputs(1, tok, D, bf16, K=K)
+    st = synth.make_states(2, len(lens), D, K=K, bf16=bf16)["conv_state"]
+    cu_d, cu_h = cu_tensor(lens)
+    dt_ = act_dtype(bf16)
+    x = dev(act["x"], dt_)
+    xc, so = run_conv(x, dev(prm.conv_w), dev(prm.conv_b), cu=cu_d, state_in=dev(st, dt_),
+                      want_state=True)
+    ref, ref_st = orc.causal_conv1d(act["x"], prm.conv_w, prm.conv_b, cu_seqlens=cu_h,
+                                    state_in=st, want_state=True)
+    tol = TOL_BF16 if bf16 else TOL_F32
+    assert_close(host(xc), ref, bf16, tol, "xc")
+    assert np.array_equal(host(so), ref_st), "conv state out must be exact"
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_conv_dense_no_state_and_inplace_state(orc, bf16):
+    B, L, D = 3, 100, 64
+    tok = B * L
+    prm, act = _layer_inputs(3, tok, D, bf16)
+    dt_ = act_dtype(bf16)
+    x = dev(act["x"], dt_)
+    xc, so = run_conv(x, dev(prm.conv_w), dev(prm.conv_b), S=B, want_state=True)
+    ref, ref_st = orc.causal_conv1d(act["x"], prm.conv_w, prm.conv_b, S=B, want_state=True)
+    assert_close(host(xc), ref, bf16, TOL_BF16 if bf16 else TOL_F32, "xc")
+    assert np.array_equal(host(so), ref_st)
+    # in place: state_out is the same buffer as state_in
+    st = synth.make_states(4, B, D, bf16=bf16)["conv_state"]
+    st_d = dev(st, dt_)
+    xc2, _ = run_conv(x, dev(prm.conv_w), dev(prm.conv_b), S=B, state_in=st_d, want_state=True,
+                      state_inplace=True)
+    ref2, ref_st2 = orc.causal_conv1d(act["x"], prm.conv_w, prm.conv_b, S=B, state_in=st,
+                                      want_state=True)
+    assert_close(host(xc2), ref2, bf16, TOL_BF16 if bf16 else TOL_F32, "xc in-place state")
+    assert np.array_equal(host(st_d), ref_st2)
+
+
+def test_conv_no_silu(orc):
+    prm, act = _layer_inputs(5, 90, 48, True)
+    x = dev(act["x"], torch.bfloat16)
+    xc, _ = run_conv(x, dev(prm.conv_w), dev(prm.conv_b), apply_silu=False)
+    ref = orc.causal_conv1d(act["x"], prm.conv_w, prm.conv_b, apply_silu=False)
+    assert_close(host(xc), ref, True, TOL_BF16, "xc (no silu)")
+
+
+# ---------------------------------------------------------------------------
+# scan
+# ---------------------------------------------------------------------------
+
+def _scan_case(orc, seed, lens, D, bf16, npt=0, with_z=True, with_h0=True, softplus=True,
+               workspace=False, inplace=False):
+    ssm.ssm_set_scan_states_per_lane(npt)
+    tok = sum(lens)
+    prm, act = _layer_inputs(seed, tok, D, bf16)
+    S = len(lens)
+    h0 = synth.make_states(seed + 1, S, D, bf16=bf16, scale=0.3)["h0"] if with_h0 else None
+    # u: any bf16-exact values; reuse x through silu-free draws
+    u = act["x"]
+    dt_raw = act["dt"] if softplus else np.abs(act["dt"]) * 0.2 + 1e-3
+    if bf16 and not softplus:
+        dt_raw = synth.round_bf16(dt_raw)
+    cu_d, cu_h = cu_tensor(lens)
+    dt_ = act_dtype(bf16)
+    h0_d = dev(h0)
+    y, hf = run_scan(dev(u, dt_), dev(dt_raw, dt_), dev(prm.A), dev(act["B"], dt_),
+                     dev(act["C"], dt_), Dskip=dev(prm.Dskip),
+                     z=dev(act["z"], dt_) if with_z else None,
+                     dt_bias=dev(prm.dt_bias) if softplus else None, delta_softplus=softplus,
+                     h0=h0_d, cu=cu_d, inplace_state=inplace and with_h0, workspace=workspace,
+                     y_fill=-7.0)
+    ry, rh = orc.selective_scan(u, dt_raw, prm.A, act["B"], act["C"], Dskip=prm.Dskip,
+                                z=act["z"] if with_z else None,
+                                dt_bias=prm.dt_bias if softplus else None,
+                                delta_softplus=softplus, h0=h0, cu_seqlens=cu_h, want_state=True)
+    tol = TOL_BF16 if bf16 else TOL_F32
+    assert_close(host(y), ry, bf16, tol, "y")
+    assert_close(host(hf), rh, False, tol, "h_final")
+    return host(y), host(hf)
+
+
+@pytest.mark.parametrize("npt", [4, 8, 16])
+@pytest.mark.parametrize("bf16", [False, True])
+def test_scan_variants_packed(orc, npt, bf16):
+    _scan_case(orc, 10, [130, 0, 1, 7, 64, 65, 200], 200, bf16, npt=npt)
+
+
+@pytest.mark.parametrize("npt", [4, 8, 16])
+def test_scan_scalar_path(orc, npt):
+    _scan_case(orc, 11, [50, 77], 30, True, npt=npt)
+
+
+def test_scan_options(orc):
+    _scan_case(orc, 12, [90, 40], 72, True, with_z=False, with_h0=False)
+    _scan_case(orc, 13, [90, 40], 72, False, softplus=False)
+    _scan_case(orc, 14, [90, 40], 72, True, inplace=True)
+
+
+def test_scan_workspace_schedule_is_bit_identical(orc):
+    lens = [33, 400, 0, 129, 7, 260]
+    y1, h1 = _scan_case(orc, 15, lens, 96, True, workspace=False)
+    y2, h2 = _scan_case(orc, 15, lens, 96, True, workspace=True)
+    assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
+
+
+def test_scan_tokens_outside_sequences_untouched():
+    D, N = 64, 16
+    tok = 50
+    cu = torch.tensor([0, 10, 30], dtype=torch.int32, device="cuda")  # last 20 tokens unowned
+    u = torch.randn(tok, D, device="cuda").bfloat16()
+    A = -torch.rand(D, N, device="cuda") - 0.5
+    Bm = torch.randn(tok, N, device="cuda").bfloat16()
+    y = torch.full((tok, D), 3.0, device="cuda").bfloat16()
+    ssm.ssm_selective_scan_fwd(u, u, A, Bm, Bm, y, cu_seqlens=cu, S=2)
+    torch.cuda.synchronize()
+    assert torch.all(y[30:] == 3.0)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_layer_arithmetic_fp32_bound_at_scale(orc, bf16):
+    """Mamba-130M layer shape at reduced length: conv then scan.
+
+    With fp32 activations the whole path must meet 1e-4 * rms(y); with bf16
+    activations the bf16 bound applies (each call checked on its own inputs).
+    """
+    B, L, D = 2, 1024, 1536
+    tok = B * L
+    prm = synth.make_params(0, D)
+    act = synth.make_activations(0, tok, D, bf16=bf16)
+    dt_ = act_dtype(bf16)
+    x = dev(act["x"], dt_)
+    xc, cs = run_conv(x, dev(prm.conv_w), dev(prm.conv_b), S=B, want_state=True)
+    ref_xc = orc.causal_conv1d(act["x"], prm.conv_w, prm.conv_b, S=B)
+    tol = TOL_BF16 if bf16 else TOL_F32
+    assert_close(host(xc), ref_xc, bf16, tol, "xc")
+    xc_h = host(xc)
+    y, hf = run_scan(xc, dev(act["dt"], dt_), dev(prm.A), dev(act["B"], dt_), dev(act["C"], dt_),
+                     Dskip=dev(prm.Dskip), z=dev(act["z"], dt_), dt_bias=dev(prm.dt_bias), S=B)
+    ry, rh = orc.selective_scan(xc_h, act["dt"], prm.A, act["B"], act["C"], Dskip=prm.Dskip,
+                                z=act["z"], dt_bias=prm.dt_bias, S=B, want_state=True)
+    assert_close(host(y), ry, bf16, tol, "y")
+    assert_close(host(hf), rh, False, tol, "h_final")
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bf16", [False, True])
+@pytest.mark.parametrize("K", [2, 4])
+def test_decode_state_indices(orc, bf16, K):
+    n_slots, Bt, D, N = 11, 6, 200, 16
+    prm, act = _layer_inputs(20, Bt, D, bf16, K=K)
+    st = synth.make_states(21, n_slots, D, K=K, bf16=bf16, scale=0.3)
+    idx = np.array([7, -1, 0, 3, 10, 4], dtype=np.int32)
+    dt_ = act_dtype(bf16)
+    cs_d = dev(st["conv_state"], dt_)
+    ss_d = dev(st["h0"])
+    y = torch.full((Bt, D), 9.0, device="cuda", dtype=dt_)
+    ssm.ssm_selective_state_update(cs_d, ss_d, dev(act["x"], dt_), dev(act["dt"], dt_),
+                                   dev(act["B"], dt_), dev(act["C"], dt_), y, dev(prm.conv_w),
+                                   dev(prm.A), z=dev(act["z"], dt_), conv_b=dev(prm.conv_b),
+                                   Dskip=dev(prm.Dskip), dt_bias=dev(prm.dt_bias),
+                                   state_indices=torch.from_numpy(idx).cuda())
+    ry, rcs, rss = orc.state_update(st["conv_state"], st["h0"], act["x"], act["dt"], act["B"],
+                                    act["C"], act["z"], prm.conv_w, prm.conv_b, prm.A, prm.Dskip,
+                                    prm.dt_bias, state_indices=idx,
+                                    y_init=np.full((Bt, D), 9.0))
+    tol = TOL_BF16 if bf16 else TOL_F32
+    live = idx >= 0
+    assert_close(host(y)[live], ry[live], bf16, tol, "y")
+    assert np.all(host(y)[~live] == 9.0), "skipped rows must keep their y"
+    used = sorted(int(i) for i in idx if i >= 0)
+    unused = [s for s in range(n_slots) if s not in used]
+    gcs, gss = host(cs_d), host(ss_d)
+    assert np.array_equal(gcs[unused], np.asarray(st["conv_state"], np.float64)[unused])
+    assert np.array_equal(gss[unused], np.asarray(st["h0"], np.float64)[unused])
+    assert np.array_equal(gcs[used], rcs[used]), "conv state shift must be exact"
+    assert_close(gss[used], rss[used], False, tol, "ssm state")
+
+
+def test_decode_identity_slots(orc):
+    Bt, D = 5, 136
+    prm, act = _layer_inputs(22, Bt, D, True)
+    st = synth.make_states(23, Bt, D, bf16=True, scale=0.3)
+    cs_d = dev(st["conv_state"], torch.bfloat16)
+    ss_d = dev(st["h0"])
+    y = torch.empty((Bt, D), device="cuda", dtype=torch.bfloat16)
+    ssm.ssm_selective_state_update(cs_d, ss_d, dev(act["x"], torch.bfloat16),
+                                   dev(act["dt"], torch.bfloat16), dev(act["B"], torch.bfloat16),
+                                   dev(act["C"], torch.bfloat16), y, dev(prm.conv_w), dev(prm.A),
+                                   z=None, conv_b=dev(prm.conv_b), Dskip=dev(prm.Dskip),
+                                   dt_bias=dev(prm.dt_bias))
+    ry, rcs, rss = orc.state_update(st["conv_state"], st["h0"], act["x"], act["dt"], act["B"],
+                                    act["C"], None, prm.conv_w, prm.conv_b, prm.A, prm.Dskip,
+                                    prm.dt_bias)
+    assert_close(host(y), ry, True, TOL_BF16, "y")
+    assert np.array_equal(host(cs_d), rcs)
+    assert_close(host(ss_d), rss, False, TOL_BF16, "ssm state")
