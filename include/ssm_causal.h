@@ -81,13 +81,26 @@ int ssm_version(void);
 unsigned long long ssm_launch_count(void);
 
 /*
- * Tuning knob for ssm_selective_scan_fwd: states of one channel handled per
- * lane (4, 8 or 16; 16 / value lanes then share a channel), or 0 to let the
- * library choose from the number of (sequence, channel) pairs. Process-wide;
- * not thread-safe against concurrent scan calls. Returns SSM_OK or
- * SSM_ERR_INVALID_ARGUMENT.
+ * Tuning knob for ssm_selective_scan_fwd's kernel variant: states of one
+ * channel per lane (2, 4, 8 or 16; 16 / value lanes then share a channel) and
+ * the schedule (1: next chunk prefetched into registers; 2: tiles staged by
+ * TMA; 3: TMA staging with each chunk split in time over four warps, which
+ * combine their segments through a carry step; only 2 or 4 states per lane).
+ * 0 lets the library choose. Applies to the 16-byte vector path; the scalar
+ * path always uses 4 states per lane and register prefetch. Process-wide; not thread-safe against concurrent scan calls.
+ * Returns SSM_OK or SSM_ERR_INVALID_ARGUMENT. Results differ between variants
+ * only in the order of the readout sum.
  */
-int ssm_set_scan_states_per_lane(int states_per_lane);
+int ssm_set_scan_variant(int states_per_lane, int schedule);
+
+/*
+ * Device-side status of the scan kernels on the current device: 0 while every
+ * bounded wait for a TMA tile completed, 1 once a wait gave up (the results of
+ * that call are then unspecified; the kernel still terminates). Synchronises
+ * the device. clear != 0 resets the flag. Returns SSM_ERR_CUDA if the query
+ * itself fails.
+ */
+int ssm_scan_device_status(int clear);
 
 /*
  * Checks a HOST copy of cu_seqlens (S+1 entries): cu[0] == 0, non-decreasing,

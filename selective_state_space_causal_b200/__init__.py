@@ -14,9 +14,10 @@ from ._lib import (  # noqa: F401
     ssm_check_cu_seqlens,
     ssm_last_error,
     ssm_launch_count,
+    ssm_scan_device_status,
     ssm_scan_workspace_size,
     ssm_selective_scan_fwd,
     ssm_selective_state_update,
-    ssm_set_scan_states_per_lane,
+    ssm_set_scan_variant,
     ssm_version,
 )

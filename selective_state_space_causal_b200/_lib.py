@@ -26,7 +26,8 @@ SIGNATURES = [
     ("ssm_last_error", ctypes.c_char_p, []),
     ("ssm_version", _int, []),
     ("ssm_launch_count", ctypes.c_ulonglong, []),
-    ("ssm_set_scan_states_per_lane", _int, [_int]),
+    ("ssm_set_scan_variant", _int, [_int, _int]),
+    ("ssm_scan_device_status", _int, [_int]),
     ("ssm_check_cu_seqlens", _int, [_vp, _i64, _i64]),
     ("ssm_causal_conv1d", _int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _i64, _vp, _vp, _int,
                                  _int, _int, _vp]),
@@ -48,7 +49,7 @@ class SsmError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIBRARY):
         raise ImportError(
-            f"{LIBRARY} is missing: build it with `python -m selective_state_space_causal_b200.build`"
+            f"{LIBRARY} is missing: build it with `python selective_state_space_causal_b200/build.py`"
         )
     lib = ctypes.CDLL(LIBRARY)
     for name, res, args in SIGNATURES:
@@ -104,8 +105,15 @@ def ssm_launch_count() -> int:
     return int(lib.ssm_launch_count())
 
 
-def ssm_set_scan_states_per_lane(n: int) -> None:
-    _check(lib.ssm_set_scan_states_per_lane(int(n)))
+def ssm_set_scan_variant(states_per_lane: int, schedule: int = 0) -> None:
+    _check(lib.ssm_set_scan_variant(int(states_per_lane), int(schedule)))
+
+
+def ssm_scan_device_status(clear: bool = False) -> int:
+    code = lib.ssm_scan_device_status(int(bool(clear)))
+    if code < 0:
+        _check(code)
+    return code
 
 
 def ssm_check_cu_seqlens(cu_seqlens_host, tok: int) -> None:

@@ -1,7 +1,8 @@
 """Build the CUDA library (sm_100a) in-tree: libssm_causal.so next to this file.
 
-Run ``python -m selective_state_space_causal_b200.build`` (or call
-``build_library()``). nvcc cross-compiles for sm_100a without a GPU.
+Run ``python selective_state_space_causal_b200/build.py`` (by path: importing
+the package needs the built library) or call ``build_library()``. nvcc
+cross-compiles for sm_100a without a GPU.
 """
 
 from __future__ import annotations

@@ -14,8 +14,9 @@
 #include "internal.h"
 
 namespace ssm {
-void set_scan_npt(int npt);
+void set_scan_variant(int npt, int sched);
 size_t scan_order_bytes(int64_t S);
+int read_scan_status(bool clear);
 }  // namespace ssm
 
 namespace {
@@ -83,12 +84,23 @@ int ssm_version(void) { return 100; }
 
 unsigned long long ssm_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
-int ssm_set_scan_states_per_lane(int npt)
+int ssm_set_scan_variant(int npt, int sched)
 {
-    if (npt != 0 && npt != 4 && npt != 8 && npt != 16)
-        return fail(SSM_ERR_INVALID_ARGUMENT, "ssm_set_scan_states_per_lane: use 0, 4, 8 or 16");
-    ssm::set_scan_npt(npt);
+    const bool npt_ok = npt == 0 || npt == 2 || npt == 4 || npt == 8 || npt == 16;
+    const bool sched_ok = sched >= 0 && sched <= 3;
+    if (!npt_ok || !sched_ok)
+        return fail(SSM_ERR_INVALID_ARGUMENT,
+                    "ssm_set_scan_variant: states per lane 0, 2, 4, 8 or 16; schedule 0..3");
+    ssm::set_scan_variant(npt, sched);
     return ok();
+}
+
+int ssm_scan_device_status(int clear)
+{
+    const int v = ssm::read_scan_status(clear != 0);
+    if (v < 0) return fail(SSM_ERR_CUDA, "ssm_scan_device_status: CUDA query failed");
+    g_error.clear();
+    return v;
 }
 
 int ssm_check_cu_seqlens(const int32_t *cu, int64_t S, int64_t tok)

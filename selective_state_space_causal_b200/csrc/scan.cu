@@ -10,33 +10,42 @@
 //   y     = (sum_n C_t[n] h[n] + Dskip[c] * u) * silu(z)
 //
 // Design. The scan is bound by the special-function unit: every (token,
-// channel) needs N = 16 exponentials against only ~8 bytes of DRAM traffic in
-// bf16. The kernel therefore spends as few issue slots as possible on anything
-// but the 16 dA exponentials and their 4 FMA-pipe companions:
+// channel) needs N = 16 exponentials against ~8 bytes of DRAM traffic in bf16,
+// so the kernel spends as few issue slots and as little latency as it can on
+// anything but the 16 dA exponentials:
 //
-// * A CTA owns one sequence and CH channels. A channel's N = 16 states are split
-//   over TPC = 16 / NPT adjacent lanes (NPT states each) so that small batches
-//   still fill 148 SMs; h stays in fp32 registers for the whole sequence.
-// * The sequence is walked in chunks of TCH tokens. Each chunk's per-(token,
-//   channel) work (softplus, delta*u, silu(z), bf16 unpacking) is done ONCE in a
-//   cooperative pre-pass into shared memory, from 16-byte loads that were issued
-//   one chunk ahead into registers (software prefetch), so the DRAM latency of
-//   chunk k+1 hides behind the recurrence of chunk k.
-// * In the recurrence each lane reads delta and delta*u (broadcast within the
-//   channel) and 4-wide B/C vectors from shared memory, runs NPT exps + FMAs per
-//   token, and the TPC partial readouts are combined with a transposed butterfly
-//   over shuffles: after log2(TPC) steps lane `sub` holds the full sum of token
-//   `sub` of the group, which it gates and writes back in place.
+// * A CTA owns one sequence and CH channels. A channel's 16 states are split
+//   over TPC = 16 / NPT adjacent lanes (NPT states each); h stays in fp32
+//   registers, two states per packed fp32x2 register, for the whole sequence.
+// * The sequence is walked in chunks of TCH tokens. The chunk's tiles of u, dt,
+//   z (TCH x CH) and B, C (TCH x 16) are brought into shared memory by TMA
+//   (cp.async.bulk.tensor, completion on an mbarrier) one chunk ahead, so no
+//   registers are held by loads in flight. Where TMA cannot be used (rows not
+//   16-byte aligned) a variant prefetches the next chunk into registers.
+// * Each chunk's per-(token, channel) work (softplus, delta*u, silu(z), bf16
+//   unpacking) is done once, in a cooperative pre-pass into shared memory.
+// * The recurrence runs on packed fp32x2 FMUL/FFMA (sm_100a), one MUFU ex2 per
+//   state and token, and the TPC partial readouts are combined with a
+//   transposed butterfly over shuffles: after log2(TPC) steps lane `sub` holds
+//   the full sum of token `sub` of the group, which it gates and writes back.
 // * Tokens past a sequence's end are padded with delta = 0 (dA = 1, no input),
 //   which leaves h unchanged, so the inner loop needs no tail branch.
 // * Packed sequences are scheduled longest-first when scratch is supplied.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace ssm {
+
+// Set by a kernel whose bounded wait on a TMA completion gave up.
+__device__ int g_scan_status = 0;
+
 namespace {
 
 constexpr int kN = 16;
+constexpr unsigned kSpinLimit = 1u << 21;
 
 struct Params {
     const void *u, *delta, *B, *C, *z;
@@ -49,26 +58,260 @@ struct Params {
     int delta_softplus;
 };
 
-template <typename T, int NPT_, int CH_, int TCH_, int VEC_>
+constexpr size_t align128(size_t v) { return (v + 127) / 128 * 128; }
+
+template <typename T, int NPT_, int BATCH_, int CH_, int TCH_, int VEC_>
 struct Cfg {
-    static constexpr int NPT = NPT_, CH = CH_, TCH = TCH_, VEC = VEC_;
+    static constexpr int NPT = NPT_, BATCH = BATCH_, CH = CH_, TCH = TCH_, VEC = VEC_;
     static constexpr int TPC = kN / NPT;                  // lanes per channel
     static constexpr int THREADS = CH * TPC;
     static constexpr int CV = CH / VEC;                   // channel vectors per row
     static constexpr int ITEMS = TCH * CV;                // (token, vector) items per chunk
     static constexpr int IPT = ITEMS / THREADS;           // items per thread
-    static constexpr int SROW = CH + 4;                   // padded smem row, floats
-    static constexpr int BCVEC = 16 / sizeof(T);          // B/C elements per 16-byte load
-    static constexpr int BCN = TCH * kN / BCVEC;          // 16-byte B (or C) loads per chunk
+    static constexpr int ROW2 = CH + 2 * (CH / 16);       // padded smem row, in float2
+    static constexpr int BCVEC = 16 / sizeof(T);          // B/C elements per 16 bytes
+    static constexpr int BCN = TCH * kN / BCVEC;          // 16-byte B (or C) pieces per chunk
     static constexpr int BPT = (BCN + THREADS - 1) / THREADS;
-    static constexpr size_t SMEM = sizeof(float) * (4 * TCH * SROW + 2 * TCH * kN);
+    // shared memory: derived arrays, then (TMA kernel only) the raw tiles
+    static constexpr size_t OFF_DX = 0;
+    static constexpr size_t OFF_UG = align128(OFF_DX + sizeof(float2) * TCH * ROW2);
+    static constexpr size_t OFF_B = align128(OFF_UG + sizeof(float2) * TCH * ROW2);
+    static constexpr size_t OFF_C = align128(OFF_B + sizeof(float) * TCH * kN);
+    static constexpr size_t SMEM = align128(OFF_C + sizeof(float) * TCH * kN);
+    static constexpr size_t RAW_ACT = sizeof(T) * TCH * CH;   // one u / dt / z tile
+    static constexpr size_t RAW_BC = sizeof(T) * TCH * kN;    // one B / C tile
+    static constexpr size_t OFF_RU = SMEM;
+    static constexpr size_t OFF_RDT = OFF_RU + align128(RAW_ACT);
+    static constexpr size_t OFF_RZ = OFF_RDT + align128(RAW_ACT);
+    static constexpr size_t OFF_RB = OFF_RZ + align128(RAW_ACT);
+    static constexpr size_t OFF_RC = OFF_RB + align128(RAW_BC);
+    static constexpr size_t OFF_BAR = OFF_RC + align128(RAW_BC);
+    static constexpr size_t SMEM_TMA = OFF_BAR + 128;
+    static_assert(CH % 16 == 0, "channel tile is a multiple of 16");
+    static_assert(NPT % 2 == 0, "states come in packed pairs");
     static_assert(ITEMS % THREADS == 0, "items must divide evenly");
     static_assert(THREADS % CV == 0, "each thread keeps one channel vector");
     static_assert(TCH % TPC == 0, "chunk must hold whole token groups");
     static_assert(THREADS <= 1024 && (THREADS % 32) == 0, "block size");
+    static_assert(RAW_ACT % 128 == 0 && RAW_BC % 128 == 0, "TMA tiles stay 128-byte aligned");
 };
 
-// Raw prefetch register of one (token, vector) item: 16 bytes, or one element.
+// Column of channel c in a padded float2 row: 16 B of padding after every 16
+// channels keeps both the 16-byte pre-pass stores and the per-token reads free
+// of bank conflicts.
+__device__ __forceinline__ int col2(int c) { return c + 2 * (c >> 4); }
+
+// Store VEC consecutive float2 values (16-byte aligned when VEC is even).
+template <int VEC>
+__device__ __forceinline__ void st_pairs(float2 *dst, const float (&a)[VEC], const float (&b)[VEC])
+{
+    if constexpr (VEC % 2 == 0) {
+#pragma unroll
+        for (int e = 0; e < VEC; e += 2)
+            *reinterpret_cast<float4 *>(dst + e) = make_float4(a[e], b[e], a[e + 1], b[e + 1]);
+    } else {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) dst[e] = make_float2(a[e], b[e]);
+    }
+}
+
+// Derived per-(token, channel) values of one pre-pass item.
+template <int VEC>
+__device__ __forceinline__ void prepass_item(float2 *dx_row, float2 *ug_row, bool live,
+                                             const float (&fdt)[VEC], const float (&fu)[VEC],
+                                             const float (&fz)[VEC], bool has_z,
+                                             const float (&dtb)[VEC], int softplus)
+{
+    float vd[VEC], vdx[VEC], vu[VEC], vg[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        float d = fdt[e] + dtb[e];
+        if (softplus) d = softplus_f(d);
+        vd[e] = live ? d : 0.f;
+        vdx[e] = live ? d * fu[e] : 0.f;
+        vu[e] = live ? fu[e] : 0.f;
+        vg[e] = live ? (has_z ? silu_f(fz[e]) : 1.f) : 0.f;
+    }
+    st_pairs<VEC>(dx_row, vd, vdx);
+    st_pairs<VEC>(ug_row, vu, vg);
+}
+
+// Recurrence over one staged chunk for one lane: NPT states of channel `mycol`
+// (padded column), tokens [0, ntr) of the chunk in groups of TPC.
+template <class K>
+__device__ __forceinline__ void recur_chunk(const float2 *__restrict__ sDX, float2 *sUG,
+                                            const float *__restrict__ sB,
+                                            const float *__restrict__ sC, int ntr, int mycol,
+                                            int sub, const f32x2 (&A2p)[K::NPT / 2],
+                                            f32x2 (&hp)[K::NPT / 2], float dsk)
+{
+    constexpr int NPT = K::NPT, TPC = K::TPC, ROW2 = K::ROW2, NP = K::NPT / 2;
+    for (int tt = 0; tt < ntr; tt += TPC) {
+        float yp[TPC];
+        if constexpr (K::BATCH) {
+            // all exponentials of the group first, then the dependent FMAs
+            f32x2 dA[TPC][NP], bx[TPC][NP], cc[TPC][NP];
+#pragma unroll
+            for (int q = 0; q < TPC; ++q) {
+                const int tq = tt + q;
+                const float2 v = sDX[tq * ROW2 + mycol];
+                const f32x2 dd = pk2(v.x, v.x), xx = pk2(v.y, v.y);
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    const float2 b2 = *reinterpret_cast<const float2 *>(sB + tq * kN + sub * NPT + 2 * j);
+                    const float2 c2 = *reinterpret_cast<const float2 *>(sC + tq * kN + sub * NPT + 2 * j);
+                    float a0, a1;
+                    upk2(mul2(dd, A2p[j]), a0, a1);
+                    dA[q][j] = pk2(ex2_approx(a0), ex2_approx(a1));
+                    bx[q][j] = mul2(xx, pk2(b2.x, b2.y));
+                    cc[q][j] = pk2(c2.x, c2.y);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < TPC; ++q) {
+                f32x2 acc = 0ull;
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    hp[j] = fma2(dA[q][j], hp[j], bx[q][j]);
+                    acc = fma2(cc[q][j], hp[j], acc);
+                }
+                float s0, s1;
+                upk2(acc, s0, s1);
+                yp[q] = s0 + s1;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < TPC; ++q) {
+                const int tq = tt + q;
+                const float2 v = sDX[tq * ROW2 + mycol];
+                const f32x2 dd = pk2(v.x, v.x), xx = pk2(v.y, v.y);
+                f32x2 acc = 0ull;
+#pragma unroll
+                for (int j = 0; j < NP; ++j) {
+                    const float2 b2 = *reinterpret_cast<const float2 *>(sB + tq * kN + sub * NPT + 2 * j);
+                    const float2 c2 = *reinterpret_cast<const float2 *>(sC + tq * kN + sub * NPT + 2 * j);
+                    float a0, a1;
+                    upk2(mul2(dd, A2p[j]), a0, a1);
+                    const f32x2 dA = pk2(ex2_approx(a0), ex2_approx(a1));
+                    hp[j] = fma2(dA, hp[j], mul2(xx, pk2(b2.x, b2.y)));
+                    acc = fma2(pk2(c2.x, c2.y), hp[j], acc);
+                }
+                float s0, s1;
+                upk2(acc, s0, s1);
+                yp[q] = s0 + s1;
+            }
+        }
+        // transposed butterfly: lane `sub` ends with the full sum of token tt+sub
+#pragma unroll
+        for (int w = TPC / 2; w >= 1; w >>= 1) {
+            const bool upper = (sub & w) != 0;
+#pragma unroll
+            for (int i = 0; i < w; ++i) {
+                const float send = upper ? yp[i] : yp[i + w];
+                const float keep = upper ? yp[i + w] : yp[i];
+                yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+            }
+        }
+        float2 *q2 = sUG + (tt + sub) * ROW2 + mycol;
+        const float2 ug = *q2;
+        q2->x = (yp[0] + dsk * ug.x) * ug.y;
+    }
+}
+
+// Writes y for this thread's pre-pass items of the chunk (y sits in sUG.x).
+template <class K, typename T>
+__device__ __forceinline__ void store_y(T *Y, const float2 *sUG, int tid, int nt, bool vvalid,
+                                        int vcol, int64_t t0, int64_t D, int64_t cg)
+{
+    constexpr int VEC = K::VEC;
+#pragma unroll
+    for (int i = 0; i < K::IPT; ++i) {
+        const int tl = (tid + i * K::THREADS) / K::CV;
+        if (tl < nt && vvalid) {
+            float out[VEC];
+            const float2 *src = sUG + tl * K::ROW2 + vcol;
+            if constexpr (VEC % 2 == 0) {
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    const float4 v = *reinterpret_cast<const float4 *>(src + e);
+                    out[e] = v.x;
+                    out[e + 1] = v.z;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) out[e] = src[e].x;
+            }
+            store_vec<T, VEC>(Y + (t0 + tl) * D + cg, out);
+        }
+    }
+}
+
+// Per-CTA setup shared by both kernels.
+struct Lane {
+    int64_t seq, start, end, cbase, c0, cg;
+    int sub, mycol, cvl, vcol;
+    bool cvalid, vvalid;
+};
+
+template <class K>
+__device__ __forceinline__ Lane lane_setup(const Params &p)
+{
+    Lane l;
+    const int tid = threadIdx.x;
+    l.sub = tid % K::TPC;
+    const int cl = tid / K::TPC;
+    l.cbase = (int64_t)blockIdx.x * K::CH;
+    l.c0 = l.cbase + cl;
+    l.cvalid = l.c0 < p.D;
+    int64_t seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    l.seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
+    if (p.cu) {
+        l.start = clamp_off(p.cu[l.seq], p.tok);
+        l.end = max(clamp_off(p.cu[l.seq + 1], p.tok), l.start);
+    } else {
+        l.start = l.seq * p.L;
+        l.end = l.start + p.L;
+    }
+    l.mycol = col2(cl);
+    l.cvl = tid % K::CV;
+    l.cg = l.cbase + (int64_t)l.cvl * K::VEC;
+    l.vvalid = l.cg < p.D;  // D % VEC == 0 on the vector paths
+    l.vcol = col2(l.cvl * K::VEC);
+    return l;
+}
+
+template <class K>
+__device__ __forceinline__ void load_state(const Params &p, const Lane &l, f32x2 (&A2p)[K::NPT / 2],
+                                           f32x2 (&hp)[K::NPT / 2])
+{
+#pragma unroll
+    for (int j = 0; j < K::NPT; j += 2) {
+        const int64_t ai = l.c0 * kN + l.sub * K::NPT + j;
+        const int64_t hi = (l.seq * p.D + l.c0) * kN + l.sub * K::NPT + j;
+        A2p[j / 2] = l.cvalid ? pk2(__ldg(p.A + ai) * kLog2e, __ldg(p.A + ai + 1) * kLog2e) : 0ull;
+        hp[j / 2] = (l.cvalid && p.h0) ? pk2(p.h0[hi], p.h0[hi + 1]) : 0ull;
+    }
+}
+
+template <class K>
+__device__ __forceinline__ void save_state(const Params &p, const Lane &l,
+                                           const f32x2 (&hp)[K::NPT / 2])
+{
+    if (p.h_final && l.cvalid) {
+#pragma unroll
+        for (int j = 0; j < K::NPT; j += 2) {
+            float lo, hi;
+            upk2(hp[j / 2], lo, hi);
+            const int64_t o = (l.seq * p.D + l.c0) * kN + l.sub * K::NPT + j;
+            p.h_final[o] = lo;
+            p.h_final[o + 1] = hi;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Variant 1: next chunk prefetched into registers (any alignment).
+// ---------------------------------------------------------------------------
 template <typename T, int VEC> struct Raw { using type = uint4; };
 template <typename T> struct Raw<T, 1> { using type = T; };
 
@@ -90,68 +333,37 @@ template <class K, typename T>
 __global__ void __launch_bounds__(K::THREADS)
 scan_kernel(const Params p)
 {
-    constexpr int NPT = K::NPT, CH = K::CH, TCH = K::TCH, VEC = K::VEC, TPC = K::TPC;
-    constexpr int THREADS = K::THREADS, CV = K::CV, IPT = K::IPT, SROW = K::SROW;
+    constexpr int VEC = K::VEC, IPT = K::IPT, THREADS = K::THREADS, CV = K::CV, TCH = K::TCH;
     using RawT = typename Raw<T, VEC>::type;
-
-    extern __shared__ __align__(16) float smem[];
-    float *sD = smem;                 // delta                [TCH][SROW]
-    float *sDX = sD + TCH * SROW;     // delta * u            [TCH][SROW]
-    float *sU = sDX + TCH * SROW;     // u, then y in place   [TCH][SROW]
-    float *sG = sU + TCH * SROW;      // silu(z) (or 1)       [TCH][SROW]
-    float *sB = sG + TCH * SROW;      // B                    [TCH][16]
-    float *sC = sB + TCH * kN;        // C                    [TCH][16]
+    extern __shared__ __align__(128) unsigned char smem[];
+    float2 *sDX = reinterpret_cast<float2 *>(smem + K::OFF_DX);
+    float2 *sUG = reinterpret_cast<float2 *>(smem + K::OFF_UG);
+    float *sB = reinterpret_cast<float *>(smem + K::OFF_B);
+    float *sC = reinterpret_cast<float *>(smem + K::OFF_C);
 
     const int tid = threadIdx.x;
-    const int chl = tid / TPC, sub = tid % TPC;
-    const int64_t cbase = (int64_t)blockIdx.x * CH;
-    const int64_t c = cbase + chl;
-    const bool cvalid = c < p.D;
-    int64_t seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
-    seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
-    int64_t start, end;
-    if (p.cu) {
-        start = clamp_off(p.cu[seq], p.tok);
-        end = max(clamp_off(p.cu[seq + 1], p.tok), start);
-    } else {
-        start = seq * p.L;
-        end = start + p.L;
-    }
-
+    const Lane l = lane_setup<K>(p);
     const T *U = static_cast<const T *>(p.u);
     const T *DT = static_cast<const T *>(p.delta);
     const T *Z = static_cast<const T *>(p.z);
     const T *Bp = static_cast<const T *>(p.B);
     const T *Cp = static_cast<const T *>(p.C);
-    T *Y = static_cast<T *>(p.y);
 
-    // per-lane constants: A * log2(e), the state, Dskip
-    float A2[NPT], h[NPT];
-#pragma unroll
-    for (int j = 0; j < NPT; ++j) {
-        A2[j] = cvalid ? __ldg(p.A + c * kN + sub * NPT + j) * kLog2e : 0.f;
-        h[j] = (cvalid && p.h0) ? p.h0[(seq * p.D + c) * kN + sub * NPT + j] : 0.f;
-    }
-    const float dsk = (cvalid && p.Dskip) ? __ldg(p.Dskip + c) : 0.f;
-
-    // this thread's channel vector in the pre-pass is fixed (THREADS % CV == 0)
-    const int cvl = tid % CV;
-    const int64_t cg = cbase + (int64_t)cvl * VEC;
-    const bool vvalid = cg < p.D;  // D % VEC == 0 on the vector path
+    f32x2 A2p[K::NPT / 2], hp[K::NPT / 2];
+    load_state<K>(p, l, A2p, hp);
+    const float dsk = (l.cvalid && p.Dskip) ? __ldg(p.Dskip + l.c0) : 0.f;
     float dtb[VEC];
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) dtb[i] = (vvalid && p.dt_bias) ? __ldg(p.dt_bias + cg + i) : 0.f;
+    for (int i = 0; i < VEC; ++i) dtb[i] = (l.vvalid && p.dt_bias) ? __ldg(p.dt_bias + l.cg + i) : 0.f;
 
     RawT rdt[IPT], ru[IPT], rz[IPT];
     uint4 rb[K::BPT], rc[K::BPT];
-
     auto prefetch = [&](int64_t t0) {
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
-            const int tl = (tid + i * THREADS) / CV;
-            const int64_t row = t0 + tl;
-            if (row < end && vvalid) {
-                const int64_t off = row * p.D + cg;
+            const int64_t row = t0 + (tid + i * THREADS) / CV;
+            if (row < l.end && l.vvalid) {
+                const int64_t off = row * p.D + l.cg;
                 rdt[i] = ld_raw<T, VEC>(DT + off);
                 ru[i] = ld_raw<T, VEC>(U + off);
                 if (Z) rz[i] = ld_raw<T, VEC>(Z + off);
@@ -161,7 +373,7 @@ scan_kernel(const Params p)
         for (int i = 0; i < K::BPT; ++i) {
             const int q = tid + i * THREADS;
             const int64_t row = t0 + (q * K::BCVEC) / kN;
-            if (q < K::BCN && row < end) {
+            if (q < K::BCN && row < l.end) {
                 const int64_t off = t0 * kN + (int64_t)q * K::BCVEC;
                 rb[i] = ldg16(Bp + off);
                 rc[i] = ldg16(Cp + off);
@@ -169,42 +381,21 @@ scan_kernel(const Params p)
         }
     };
 
-    if (start < end) prefetch(start);
-
-    for (int64_t t0 = start; t0 < end; t0 += TCH) {
-        const int nt = (int)min((int64_t)TCH, end - t0);
-
-        // ---- pre-pass: per-(token, channel) scalars into shared memory ----
+    if (l.start < l.end) prefetch(l.start);
+    for (int64_t t0 = l.start; t0 < l.end; t0 += TCH) {
+        const int nt = (int)min((int64_t)TCH, l.end - t0);
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
             const int tl = (tid + i * THREADS) / CV;
-            float vd[VEC], vdx[VEC], vu[VEC], vg[VEC];
-            if (tl < nt && vvalid) {
-                float fdt[VEC], fu[VEC], fz[VEC];
+            float fdt[VEC], fu[VEC], fz[VEC];
+            const bool live = tl < nt && l.vvalid;
+            if (live) {
                 unpack<T, VEC>(rdt[i], fdt);
                 unpack<T, VEC>(ru[i], fu);
                 if (Z) unpack<T, VEC>(rz[i], fz);
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) {
-                    float d = fdt[e] + dtb[e];
-                    if (p.delta_softplus) d = softplus_f(d);
-                    vd[e] = d;
-                    vdx[e] = d * fu[e];
-                    vu[e] = fu[e];
-                    vg[e] = Z ? silu_f(fz[e]) : 1.f;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) vd[e] = vdx[e] = vu[e] = vg[e] = 0.f;
             }
-            const int so = tl * SROW + cvl * VEC;
-#pragma unroll
-            for (int e = 0; e < VEC; ++e) {
-                sD[so + e] = vd[e];
-                sDX[so + e] = vdx[e];
-                sU[so + e] = vu[e];
-                sG[so + e] = vg[e];
-            }
+            prepass_item<VEC>(sDX + tl * K::ROW2 + l.vcol, sUG + tl * K::ROW2 + l.vcol, live, fdt,
+                              fu, fz, Z != nullptr, dtb, p.delta_softplus);
         }
 #pragma unroll
         for (int i = 0; i < K::BPT; ++i) {
@@ -223,36 +414,374 @@ scan_kernel(const Params p)
             }
         }
         __syncthreads();
+        if (t0 + TCH < l.end) prefetch(t0 + TCH);
+        const int ntr = ((nt + K::TPC - 1) / K::TPC) * K::TPC;
+        recur_chunk<K>(sDX, sUG, sB, sC, ntr, l.mycol, l.sub, A2p, hp, dsk);
+        __syncthreads();
+        store_y<K, T>(static_cast<T *>(p.y), sUG, tid, nt, l.vvalid, l.vcol, t0, p.D, l.cg);
+        // The next pre-pass rewrites only slots this thread just read (sUG) or
+        // slots no thread reads after the barrier above, so no barrier here.
+    }
+    save_state<K>(p, l, hp);
+}
 
-        if (t0 + TCH < end) prefetch(t0 + TCH);
+// ---------------------------------------------------------------------------
+// Variant 2: tiles brought in by TMA one chunk ahead (16-byte aligned rows).
+// ---------------------------------------------------------------------------
+struct Maps {
+    CUtensorMap u, dt, z, b, c;
+};
 
-        // ---- recurrence over the chunk ----
-        const int ntr = ((nt + TPC - 1) / TPC) * TPC;
-        for (int tt = 0; tt < ntr; tt += TPC) {
+__device__ __forceinline__ uint32_t saddr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void tma_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];"
+        :: "r"(saddr(dst)), "l"(map), "r"(x), "r"(y), "r"(saddr(bar)) : "memory");
+}
+
+// Waits for phase `parity` of the barrier with a bounded number of
+// non-blocking polls (about 0.2 s in all; a tile normally lands within a few
+// microseconds). On timeout it records the failure in g_scan_status and marks
+// `failed`, after which this thread no longer waits at all, so the kernel
+// always terminates.
+__device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &failed)
+{
+    if (failed) return;
+    for (unsigned i = 0; i < kSpinLimit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done) : "r"(saddr(bar)), "r"(parity) : "memory");
+        if (done) return;
+        if (i >= 32) __nanosleep(64);
+    }
+    failed = true;
+    atomicOr(&g_scan_status, 1);
+}
+
+template <class K, typename T>
+__global__ void __launch_bounds__(K::THREADS)
+scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
+{
+    constexpr int VEC = K::VEC, IPT = K::IPT, THREADS = K::THREADS, CV = K::CV, TCH = K::TCH;
+    constexpr int CH = K::CH;
+    extern __shared__ __align__(128) unsigned char smem[];
+    float2 *sDX = reinterpret_cast<float2 *>(smem + K::OFF_DX);
+    float2 *sUG = reinterpret_cast<float2 *>(smem + K::OFF_UG);
+    float *sB = reinterpret_cast<float *>(smem + K::OFF_B);
+    float *sC = reinterpret_cast<float *>(smem + K::OFF_C);
+    T *rU = reinterpret_cast<T *>(smem + K::OFF_RU);
+    T *rDT = reinterpret_cast<T *>(smem + K::OFF_RDT);
+    T *rZ = reinterpret_cast<T *>(smem + K::OFF_RZ);
+    T *rB = reinterpret_cast<T *>(smem + K::OFF_RB);
+    T *rC = reinterpret_cast<T *>(smem + K::OFF_RC);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+
+    const int tid = threadIdx.x;
+    const Lane l = lane_setup<K>(p);
+    const uint32_t tx_bytes = (uint32_t)((has_z ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
+
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(saddr(bar)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    auto issue = [&](int64_t t0) {
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                     :: "r"(saddr(bar)), "r"(tx_bytes) : "memory");
+        const int x = (int)l.cbase, y = (int)t0;
+        tma_2d(rU, &m.u, bar, x, y);
+        tma_2d(rDT, &m.dt, bar, x, y);
+        if (has_z) tma_2d(rZ, &m.z, bar, x, y);
+        tma_2d(rB, &m.b, bar, 0, y);
+        tma_2d(rC, &m.c, bar, 0, y);
+    };
+    if (tid == 0 && l.start < l.end) issue(l.start);
+
+    f32x2 A2p[K::NPT / 2], hp[K::NPT / 2];
+    load_state<K>(p, l, A2p, hp);
+    const float dsk = (l.cvalid && p.Dskip) ? __ldg(p.Dskip + l.c0) : 0.f;
+    float dtb[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) dtb[i] = (l.vvalid && p.dt_bias) ? __ldg(p.dt_bias + l.cg + i) : 0.f;
+
+    uint32_t parity = 0;
+    bool failed = false;
+    for (int64_t t0 = l.start; t0 < l.end; t0 += TCH) {
+        const int nt = (int)min((int64_t)TCH, l.end - t0);
+        mbar_wait(bar, parity, failed);
+        parity ^= 1u;
+#pragma unroll
+        for (int i = 0; i < IPT; ++i) {
+            const int tl = (tid + i * THREADS) / CV;
+            const int ro = tl * CH + l.cvl * VEC;
+            float fdt[VEC], fu[VEC], fz[VEC];
+            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rDT + ro), fdt);
+            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rU + ro), fu);
+            if (has_z) unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rZ + ro), fz);
+            prepass_item<VEC>(sDX + tl * K::ROW2 + l.vcol, sUG + tl * K::ROW2 + l.vcol,
+                              tl < nt && l.vvalid, fdt, fu, fz, has_z != 0, dtb,
+                              p.delta_softplus);
+        }
+#pragma unroll
+        for (int i = 0; i < K::BPT; ++i) {
+            const int q = tid + i * THREADS;
+            if (q < K::BCN) {
+                const int e0 = q * K::BCVEC;
+                const bool live = e0 / kN < nt;
+                float fb[K::BCVEC], fc[K::BCVEC];
+                unpack16<T, K::BCVEC>(*reinterpret_cast<const uint4 *>(rB + e0), fb);
+                unpack16<T, K::BCVEC>(*reinterpret_cast<const uint4 *>(rC + e0), fc);
+#pragma unroll
+                for (int e = 0; e < K::BCVEC; ++e) {
+                    sB[e0 + e] = live ? fb[e] : 0.f;
+                    sC[e0 + e] = live ? fc[e] : 0.f;
+                }
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && t0 + TCH < l.end) {
+            // the raw tiles were read through the generic proxy; order those
+            // reads before the next asynchronous-proxy writes into them
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(t0 + TCH);
+        }
+        const int ntr = ((nt + K::TPC - 1) / K::TPC) * K::TPC;
+        recur_chunk<K>(sDX, sUG, sB, sC, ntr, l.mycol, l.sub, A2p, hp, dsk);
+        __syncthreads();
+        store_y<K, T>(static_cast<T *>(p.y), sUG, tid, nt, l.vvalid, l.vcol, t0, p.D, l.cg);
+    }
+    save_state<K>(p, l, hp);
+}
+
+// ---------------------------------------------------------------------------
+// Variant 3: time-split chunks (TMA staging). A chunk of SEG x TS tokens is
+// cut into SEG segments handled by different warps, which multiplies the
+// warps available to sequences x channels pairs that are too few to fill the
+// GPU. Each segment first runs its tokens from a zero state, keeping dA and
+// delta*u*B in registers and forming its decay product P = prod dA and local
+// state hl; the segments' (P, hl) pairs meet in shared memory, every warp
+// folds those of the segments before its own onto the chunk's incoming state
+// (h_in = P * h_in + hl), and then replays its tokens from the true state
+// with the register-resident dA, so every exponential is computed once.
+// ---------------------------------------------------------------------------
+template <typename T, int NPT_, int SEG_, int TS_, int CH_>
+struct TsCfg {
+    static constexpr int NPT = NPT_, SEG = SEG_, TS = TS_, CH = CH_;
+    static constexpr int TPC = kN / NPT, NP = NPT / 2;
+    static constexpr int TCH = SEG * TS;                  // tokens per chunk
+    static constexpr int LANES = CH * TPC;                // threads per segment
+    static constexpr int THREADS = SEG * LANES;
+    static constexpr int PV = 2;                          // channels per pre-pass item
+    static constexpr int ITEMS = TCH * CH / PV;
+    static constexpr int IPT = (ITEMS + THREADS - 1) / THREADS;
+    static constexpr int ROW2 = CH + 2 * (CH / 16);
+    static constexpr int BCE = TCH * kN;                  // B (or C) elements per chunk
+    static constexpr size_t OFF_DX = 0;
+    static constexpr size_t OFF_UG = align128(OFF_DX + sizeof(float2) * TCH * ROW2);
+    static constexpr size_t OFF_B = align128(OFF_UG + sizeof(float2) * TCH * ROW2);
+    static constexpr size_t OFF_C = align128(OFF_B + sizeof(float) * BCE);
+    static constexpr size_t OFF_XF = align128(OFF_C + sizeof(float) * BCE);
+    static constexpr size_t RAW_ACT = sizeof(T) * TCH * CH;
+    static constexpr size_t RAW_BC = sizeof(T) * BCE;
+    static constexpr size_t OFF_RU = align128(OFF_XF + sizeof(float) * THREADS * 2 * NPT);
+    static constexpr size_t OFF_RDT = OFF_RU + align128(RAW_ACT);
+    static constexpr size_t OFF_RZ = OFF_RDT + align128(RAW_ACT);
+    static constexpr size_t OFF_RB = OFF_RZ + align128(RAW_ACT);
+    static constexpr size_t OFF_RC = OFF_RB + align128(RAW_BC);
+    static constexpr size_t OFF_BAR = OFF_RC + align128(RAW_BC);
+    static constexpr size_t SMEM = OFF_BAR + 128;
+    static_assert(NPT == 2 || NPT == 4, "two or four states per lane");
+    static_assert(TS % TPC == 0, "segments hold whole token groups");
+    static_assert((CH * sizeof(T)) % 16 == 0, "TMA rows are whole 16-byte units");
+    static_assert(THREADS % 32 == 0 && THREADS <= 1024, "block size");
+};
+
+template <class K, typename T>
+__global__ void __launch_bounds__(K::THREADS)
+scan_ts_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
+{
+    constexpr int NPT = K::NPT, NP = K::NP, TPC = K::TPC, SEG = K::SEG, TS = K::TS;
+    constexpr int CH = K::CH, TCH = K::TCH, LANES = K::LANES, THREADS = K::THREADS;
+    constexpr int ROW2 = K::ROW2, PV = K::PV;
+    extern __shared__ __align__(128) unsigned char smem[];
+    float2 *sDX = reinterpret_cast<float2 *>(smem + K::OFF_DX);
+    float2 *sUG = reinterpret_cast<float2 *>(smem + K::OFF_UG);
+    float *sB = reinterpret_cast<float *>(smem + K::OFF_B);
+    float *sC = reinterpret_cast<float *>(smem + K::OFF_C);
+    float *sXF = reinterpret_cast<float *>(smem + K::OFF_XF);
+    T *rU = reinterpret_cast<T *>(smem + K::OFF_RU);
+    T *rDT = reinterpret_cast<T *>(smem + K::OFF_RDT);
+    T *rZ = reinterpret_cast<T *>(smem + K::OFF_RZ);
+    T *rB = reinterpret_cast<T *>(smem + K::OFF_RB);
+    T *rC = reinterpret_cast<T *>(smem + K::OFF_RC);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+
+    const int tid = threadIdx.x;
+    const int seg = tid / LANES, r = tid % LANES;
+    const int cl = r / TPC, sub = r % TPC;
+    const int64_t cbase = (int64_t)blockIdx.x * CH;
+    const int64_t c0 = cbase + cl;
+    const bool cvalid = c0 < p.D;
+    int64_t seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
+    int64_t start, end;
+    if (p.cu) {
+        start = clamp_off(p.cu[seq], p.tok);
+        end = max(clamp_off(p.cu[seq + 1], p.tok), start);
+    } else {
+        start = seq * p.L;
+        end = start + p.L;
+    }
+    const int mycol = col2(cl);
+    const uint32_t tx_bytes = (uint32_t)((has_z ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
+
+    if (tid == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(saddr(bar)) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    auto issue = [&](int64_t t0) {
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                     :: "r"(saddr(bar)), "r"(tx_bytes) : "memory");
+        const int x = (int)cbase, y = (int)t0;
+        tma_2d(rU, &m.u, bar, x, y);
+        tma_2d(rDT, &m.dt, bar, x, y);
+        if (has_z) tma_2d(rZ, &m.z, bar, x, y);
+        tma_2d(rB, &m.b, bar, 0, y);
+        tma_2d(rC, &m.c, bar, 0, y);
+    };
+    if (tid == 0 && start < end) issue(start);
+
+    // A * log2(e) and the chunk's incoming state (identical in every segment)
+    f32x2 A2p[NP], hp[NP];
+#pragma unroll
+    for (int j = 0; j < NPT; j += 2) {
+        const int64_t ai = c0 * kN + sub * NPT + j;
+        const int64_t hi = (seq * p.D + c0) * kN + sub * NPT + j;
+        A2p[j / 2] = cvalid ? pk2(__ldg(p.A + ai) * kLog2e, __ldg(p.A + ai + 1) * kLog2e) : 0ull;
+        hp[j / 2] = (cvalid && p.h0) ? pk2(p.h0[hi], p.h0[hi + 1]) : 0ull;
+    }
+    const float dsk = (cvalid && p.Dskip) ? __ldg(p.Dskip + c0) : 0.f;
+
+    uint32_t parity = 0;
+    bool failed = false;
+    for (int64_t t0 = start; t0 < end; t0 += TCH) {
+        const int nt = (int)min((int64_t)TCH, end - t0);
+        mbar_wait(bar, parity, failed);
+        parity ^= 1u;
+
+        // ---- pre-pass: items of PV channels of one token ----
+#pragma unroll
+        for (int i = 0; i < K::IPT; ++i) {
+            const int it = tid + i * THREADS;
+            if (it < K::ITEMS) {
+                const int tl = it / (CH / PV), pc = (it % (CH / PV)) * PV;
+                const int64_t cg = cbase + pc;
+                const bool live = tl < nt && cg < p.D;
+                float fdt[PV], fu[PV], fz[PV], dtb[PV];
+#pragma unroll
+                for (int e = 0; e < PV; ++e) {
+                    fdt[e] = to_f32(rDT[tl * CH + pc + e]);
+                    fu[e] = to_f32(rU[tl * CH + pc + e]);
+                    fz[e] = has_z ? to_f32(rZ[tl * CH + pc + e]) : 0.f;
+                    dtb[e] = (live && p.dt_bias) ? __ldg(p.dt_bias + cg + e) : 0.f;
+                }
+                prepass_item<PV>(sDX + tl * ROW2 + col2(pc), sUG + tl * ROW2 + col2(pc), live, fdt,
+                                 fu, fz, has_z != 0, dtb, p.delta_softplus);
+            }
+        }
+        for (int e = tid; e < K::BCE; e += THREADS) {
+            const bool live = e / kN < nt;
+            sB[e] = live ? to_f32(rB[e]) : 0.f;
+            sC[e] = live ? to_f32(rC[e]) : 0.f;
+        }
+        __syncthreads();
+        if (tid == 0 && t0 + TCH < end) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(t0 + TCH);
+        }
+
+        // ---- phase 1: this segment from a zero state ----
+        f32x2 dA[TS][NP], bx[TS][NP], hl[NP], P[NP];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            hl[j] = 0ull;
+            P[j] = pk2(1.f, 1.f);
+        }
+#pragma unroll
+        for (int t = 0; t < TS; ++t) {
+            const int tq = seg * TS + t;
+            const float2 v = sDX[tq * ROW2 + mycol];
+            const f32x2 dd = pk2(v.x, v.x), xx = pk2(v.y, v.y);
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const float2 b2 = *reinterpret_cast<const float2 *>(sB + tq * kN + sub * NPT + 2 * j);
+                float a0, a1;
+                upk2(mul2(dd, A2p[j]), a0, a1);
+                dA[t][j] = pk2(ex2_approx(a0), ex2_approx(a1));
+                bx[t][j] = mul2(xx, pk2(b2.x, b2.y));
+                hl[j] = fma2(dA[t][j], hl[j], bx[t][j]);
+                P[j] = mul2(P[j], dA[t][j]);
+            }
+        }
+        float *xf = sXF + (size_t)tid * 2 * NPT;
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            float a, b;
+            upk2(P[j], a, b);
+            xf[2 * j] = a;
+            xf[2 * j + 1] = b;
+            upk2(hl[j], a, b);
+            xf[NPT + 2 * j] = a;
+            xf[NPT + 2 * j + 1] = b;
+        }
+        __syncthreads();
+
+        // ---- phase 2: carry across the segments ----
+        f32x2 hs[NP];
+#pragma unroll
+        for (int j = 0; j < NP; ++j) hs[j] = hp[j];
+#pragma unroll
+        for (int v = 0; v < SEG; ++v) {
+            if (v == seg) {
+#pragma unroll
+                for (int j = 0; j < NP; ++j) hs[j] = hp[j];
+            }
+            const float *src = sXF + (size_t)(v * LANES + r) * 2 * NPT;
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+                const f32x2 Pv = pk2(src[2 * j], src[2 * j + 1]);
+                const f32x2 hv = pk2(src[NPT + 2 * j], src[NPT + 2 * j + 1]);
+                hp[j] = fma2(Pv, hp[j], hv);  // after the loop: the chunk's outgoing state
+            }
+        }
+
+        // ---- phase 3: replay the segment from its true incoming state ----
+#pragma unroll
+        for (int t = 0; t < TS; t += TPC) {
             float yp[TPC];
 #pragma unroll
             for (int q = 0; q < TPC; ++q) {
-                const int tq = tt + q;
-                const float d = sD[tq * SROW + chl];
-                const float dx = sDX[tq * SROW + chl];
-                float bv[NPT], cv[NPT];
+                const int tq = seg * TS + t + q;
+                f32x2 acc = 0ull;
 #pragma unroll
-                for (int j = 0; j < NPT; j += 4) {
-                    const float4 b4 = *reinterpret_cast<const float4 *>(sB + tq * kN + sub * NPT + j);
-                    const float4 c4 = *reinterpret_cast<const float4 *>(sC + tq * kN + sub * NPT + j);
-                    bv[j] = b4.x; bv[j + 1] = b4.y; bv[j + 2] = b4.z; bv[j + 3] = b4.w;
-                    cv[j] = c4.x; cv[j + 1] = c4.y; cv[j + 2] = c4.z; cv[j + 3] = c4.w;
+                for (int j = 0; j < NP; ++j) {
+                    const float2 c2 = *reinterpret_cast<const float2 *>(sC + tq * kN + sub * NPT + 2 * j);
+                    hs[j] = fma2(dA[t + q][j], hs[j], bx[t + q][j]);
+                    acc = fma2(pk2(c2.x, c2.y), hs[j], acc);
                 }
-                float acc = 0.f;
-#pragma unroll
-                for (int j = 0; j < NPT; ++j) {
-                    const float dA = ex2_approx(d * A2[j]);
-                    h[j] = fmaf(dA, h[j], dx * bv[j]);
-                    acc = fmaf(cv[j], h[j], acc);
-                }
-                yp[q] = acc;
+                float s0, s1;
+                upk2(acc, s0, s1);
+                yp[q] = s0 + s1;
             }
-            // transposed butterfly: lane `sub` ends with the full sum of token tt+sub
 #pragma unroll
             for (int w = TPC / 2; w >= 1; w >>= 1) {
                 const bool upper = (sub & w) != 0;
@@ -263,31 +792,39 @@ scan_kernel(const Params p)
                     yp[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
                 }
             }
-            const int tq = tt + sub;
-            const float uval = sU[tq * SROW + chl];
-            sU[tq * SROW + chl] = (yp[0] + dsk * uval) * sG[tq * SROW + chl];
+            float2 *q2 = sUG + (seg * TS + t + sub) * ROW2 + mycol;
+            const float2 ug = *q2;
+            q2->x = (yp[0] + dsk * ug.x) * ug.y;
         }
         __syncthreads();
 
-        // ---- write y (same (token, vector) items as the pre-pass) ----
+        // ---- write y ----
+        T *Y = static_cast<T *>(p.y);
 #pragma unroll
-        for (int i = 0; i < IPT; ++i) {
-            const int tl = (tid + i * THREADS) / CV;
-            if (tl < nt && vvalid) {
-                float out[VEC];
-                const int so = tl * SROW + cvl * VEC;
+        for (int i = 0; i < K::IPT; ++i) {
+            const int it = tid + i * THREADS;
+            if (it < K::ITEMS) {
+                const int tl = it / (CH / PV), pc = (it % (CH / PV)) * PV;
+                const int64_t cg = cbase + pc;
+                if (tl < nt && cg < p.D) {
+                    float out[PV];
 #pragma unroll
-                for (int e = 0; e < VEC; ++e) out[e] = sU[so + e];
-                store_vec<T, VEC>(Y + (t0 + tl) * p.D + cg, out);
+                    for (int e = 0; e < PV; ++e) out[e] = sUG[tl * ROW2 + col2(pc) + e].x;
+                    store_vec<T, PV>(Y + (t0 + tl) * p.D + cg, out);
+                }
             }
         }
-        // The next pre-pass rewrites only slots this thread just read (sU) or
-        // slots no thread reads after the barrier above, so no barrier here.
+        // the next pre-pass rewrites sUG only at this thread's own items
     }
-
-    if (cvalid && p.h_final) {
+    if (p.h_final && cvalid && seg == 0) {
 #pragma unroll
-        for (int j = 0; j < NPT; ++j) p.h_final[(seq * p.D + c) * kN + sub * NPT + j] = h[j];
+        for (int j = 0; j < NPT; j += 2) {
+            float lo, hi;
+            upk2(hp[j / 2], lo, hi);
+            const int64_t o = (seq * p.D + c0) * kN + sub * NPT + j;
+            p.h_final[o] = lo;
+            p.h_final[o + 1] = hi;
+        }
     }
 }
 
@@ -334,51 +871,165 @@ order_kernel(const int32_t *__restrict__ cu, int64_t S, int64_t tok, int32_t *__
         order[i] = (int32_t)(0xFFFFFFFFu - (unsigned)(keys[i] & 0xFFFFFFFFull));
 }
 
-template <class K, typename T>
-cudaError_t run(const Params &p, cudaStream_t stream, int *launches)
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 {
-    const unsigned gx = (unsigned)((p.D + K::CH - 1) / K::CH);
-    const unsigned gy = (unsigned)p.S;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess || q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }();
+    return fn;
+}
+
+// 2-D tile map over a row-major (rows, inner) tensor; out-of-range reads fill 0.
+bool encode(CUtensorMap *map, const void *base, bool bf16, uint64_t inner, uint64_t rows,
+            uint32_t box_inner, uint32_t box_rows)
+{
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    const uint64_t es = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * es};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <class K, typename T>
+cudaError_t run(const Params &p, bool tma, cudaStream_t stream, int *launches)
+{
+    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
+    if constexpr (K::VEC * sizeof(T) == 16) {
+    if (tma && p.tok > 0) {
+        Maps m;
+        const bool bf = sizeof(T) == 2;
+        bool ok = encode(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
+                  encode(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+                  encode(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+                  encode(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+        if (ok) {
+            if (p.z) ok = encode(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+            else m.z = m.u;  // never loaded
+        }
+        if (ok) {
+            cudaError_t e = cudaFuncSetAttribute(scan_tma_kernel<K, T>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)K::SMEM_TMA);
+            if (e != cudaSuccess) return e;
+            scan_tma_kernel<K, T><<<grid, K::THREADS, K::SMEM_TMA, stream>>>(p, m, p.z ? 1 : 0);
+            ++*launches;
+            return cudaGetLastError();
+        }
+        // no tensor-map encoder: fall through to the register-prefetch variant
+    }
+    } else {
+        (void)tma;
+    }
     cudaError_t e = cudaFuncSetAttribute(scan_kernel<K, T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)K::SMEM);
     if (e != cudaSuccess) return e;
-    scan_kernel<K, T><<<dim3(gx, gy), K::THREADS, K::SMEM, stream>>>(p);
+    scan_kernel<K, T><<<grid, K::THREADS, K::SMEM, stream>>>(p);
     ++*launches;
     return cudaGetLastError();
 }
 
-// Variants: NPT states per lane, CH channels per CTA, TCH tokens per chunk.
-template <typename T, int VEC>
-cudaError_t dispatch(const Params &p, int npt, cudaStream_t s, int *n)
+template <class K, typename T>
+cudaError_t run_ts(const Params &p, cudaStream_t stream, int *launches)
 {
-    switch (npt) {
-    case 16: return run<Cfg<T, 16, 128, 32, VEC>, T>(p, s, n);
-    case 8: return run<Cfg<T, 8, 64, 64, VEC>, T>(p, s, n);
-    default: return run<Cfg<T, 4, 32, 64, VEC>, T>(p, s, n);
+    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
+    Maps m;
+    const bool bf = sizeof(T) == 2;
+    bool ok = p.tok > 0 && encode(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+              encode(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+    if (ok) {
+        if (p.z) ok = encode(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+        else m.z = m.u;  // never loaded
+    }
+    if (!ok) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(scan_ts_kernel<K, T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)K::SMEM);
+    if (e != cudaSuccess) return e;
+    scan_ts_kernel<K, T><<<grid, K::THREADS, K::SMEM, stream>>>(p, m, p.z ? 1 : 0);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+int g_forced_npt = 0, g_forced_sched = 0;
+
+// Variants: NPT states per lane; schedule 1: register prefetch, 2: TMA
+// staging, 3: TMA staging with time-split chunks; CH channels per CTA, TCH
+// tokens per chunk.
+template <typename T, int VEC>
+cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n)
+{
+    if constexpr (VEC == 1) {
+        (void)npt; (void)sched;
+        return run<Cfg<T, 4, 0, 32, 64, 1>, T>(p, false, s, n);
+    } else {
+        // TMA variants use shorter chunks: their raw tiles add shared memory,
+        // and without prefetch registers the CTA count per SM is set by it
+        if (sched == 3 && p.tok > 0) {
+            cudaError_t e = npt == 2 ? run_ts<TsCfg<T, 2, 4, 8, 8>, T>(p, s, n)
+                                     : run_ts<TsCfg<T, 4, 4, 8, 8>, T>(p, s, n);
+            if (e != cudaErrorNotSupported) return e;
+        }
+        if (sched >= 2) {
+            if (npt == 16) return run<Cfg<T, 16, 0, 128, 16, VEC>, T>(p, true, s, n);
+            if (npt == 8) return run<Cfg<T, 8, 0, 64, 32, VEC>, T>(p, true, s, n);
+            if (npt == 2) return run<Cfg<T, 2, 0, 16, 64, VEC>, T>(p, true, s, n);
+            return run<Cfg<T, 4, 0, 32, 32, VEC>, T>(p, true, s, n);
+        }
+        if (npt == 16) return run<Cfg<T, 16, 0, 128, 32, VEC>, T>(p, false, s, n);
+        if (npt == 8) return run<Cfg<T, 8, 0, 64, 64, VEC>, T>(p, false, s, n);
+        if (npt == 2) return run<Cfg<T, 2, 0, 16, 64, VEC>, T>(p, false, s, n);
+        return run<Cfg<T, 4, 0, 32, 64, VEC>, T>(p, false, s, n);
     }
 }
 
-int g_forced_npt = 0;
-
-// States per lane: as many as keep at least ~4 warps per SM sub-partition
-// busy (148 SMs x 4 SMSPs); fewer states per lane split a channel over more
-// lanes when there are few (sequence, channel) pairs.
-int pick_npt(int64_t S, int64_t D)
+// Measured on B200: with few (sequence, channel) pairs, splitting a channel's
+// states over more lanes wins (more warps); with many, fewer lanes per channel
+// win (fewer instructions per exponential). TMA staging throughout.
+void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
 {
-    if (g_forced_npt) return g_forced_npt;
     const int64_t pairs = S * D;
-    const int64_t want_warps = 148 * 4 * 4;
-    if (pairs / 32 >= want_warps) return 16;
-    if (pairs * 2 / 32 >= want_warps) return 8;
-    return 4;
+    const int npt_auto = pairs < (1 << 15) ? 2 : (pairs < (1 << 17) ? 4 : 8);
+    *npt = g_forced_npt ? g_forced_npt : npt_auto;
+    *sched = g_forced_sched ? g_forced_sched : 2;
 }
 
 }  // namespace
 
-void set_scan_npt(int npt) { g_forced_npt = (npt == 4 || npt == 8 || npt == 16) ? npt : 0; }
+void set_scan_variant(int npt, int sched)
+{
+    g_forced_npt = (npt == 2 || npt == 4 || npt == 8 || npt == 16) ? npt : 0;
+    g_forced_sched = (sched >= 1 && sched <= 3) ? sched : 0;
+}
 
 size_t scan_order_bytes(int64_t S) { return (size_t)((S * 4 + 255) / 256) * 256; }
+
+int read_scan_status(bool clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_scan_status, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_scan_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+    }
+    return v;
+}
 
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t stream, int *launches)
 {
@@ -395,13 +1046,14 @@ cudaError_t launch_scan(const ScanArgs &a, cudaStream_t stream, int *launches)
         if (e != cudaSuccess) return e;
         p.order = a.order;
     }
-    const int npt = pick_npt(a.S, a.D);
+    int npt, sched;
+    pick_variant(a.S, a.D, &npt, &sched);
     if (a.dtype == DType::BF16) {
-        if (a.vec && a.D % 8 == 0) return dispatch<__nv_bfloat16, 8>(p, npt, stream, launches);
-        return dispatch<__nv_bfloat16, 1>(p, npt, stream, launches);
+        if (a.vec && a.D % 8 == 0) return dispatch<__nv_bfloat16, 8>(p, npt, sched, stream, launches);
+        return dispatch<__nv_bfloat16, 1>(p, npt, sched, stream, launches);
     }
-    if (a.vec && a.D % 4 == 0) return dispatch<float, 4>(p, npt, stream, launches);
-    return dispatch<float, 1>(p, npt, stream, launches);
+    if (a.vec && a.D % 4 == 0) return dispatch<float, 4>(p, npt, sched, stream, launches);
+    return dispatch<float, 1>(p, npt, sched, stream, launches);
 }
 
 }  // namespace ssm

@@ -129,8 +129,9 @@ def test_check_cu_seqlens_host():
 
 
 def test_tuning_knob():
-    for n in (0, 4, 8, 16):
-        ssm.ssm_set_scan_states_per_lane(n)
-    with pytest.raises(ssm.SsmError):
-        ssm.ssm_set_scan_states_per_lane(3)
-    ssm.ssm_set_scan_states_per_lane(0)
+    for n, c in ((0, 0), (2, 1), (4, 1), (4, 2), (4, 3), (8, 2), (16, 1), (16, 2)):
+        ssm.ssm_set_scan_variant(n, c)
+    for n, c in ((3, 1), (16, 4), (4, -1)):
+        with pytest.raises(ssm.SsmError):
+            ssm.ssm_set_scan_variant(n, c)
+    ssm.ssm_set_scan_variant(0, 0)

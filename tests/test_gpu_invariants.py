@@ -27,9 +27,9 @@ BF = torch.bfloat16
 @pytest.fixture(autouse=True)
 def _fixed_variant():
     # the packed and per-sequence runs must use the same kernel variant
-    ssm.ssm_set_scan_states_per_lane(4)
+    ssm.ssm_set_scan_variant(4, 2)
     yield
-    ssm.ssm_set_scan_states_per_lane(0)
+    ssm.ssm_set_scan_variant(0, 0)
 
 
 def _params(seed, D):
@@ -50,9 +50,9 @@ def _acts(seed, tok, D):
     return {k: dev(v, BF) for k, v in a.items()}
 
 
-@pytest.mark.parametrize("npt", [4, 16])
-def test_pack_equals_separate(npt):
-    ssm.ssm_set_scan_states_per_lane(npt)
+@pytest.mark.parametrize("variant", [(4, 1), (4, 2), (4, 3), (2, 3), (8, 2), (16, 2)])
+def test_pack_equals_separate(variant):
+    ssm.ssm_set_scan_variant(*variant)
     lens = [100, 0, 3, 1, 257, 64]
     D = 96
     p = _params(1, D)
@@ -143,3 +143,22 @@ def test_prefill_then_decode_bf16_against_oracle_chain(orc, k):
         assert_close(host(y), ry, True, TOL_BF16, f"decode y at step {t - L0}")
     assert np.array_equal(host(c), rc)
     assert_close(host(h), rh, False, TOL_BF16, "state after the decode steps")
+
+
+@pytest.mark.parametrize("variant", [(4, 3), (2, 3)])
+def test_chunked_prefill_time_split_variant(variant):
+    """The time-split kernel combines segments through their decay products, so
+    a call boundary moves the segment boundaries: equal to the fp32 bound."""
+    ssm.ssm_set_scan_variant(*variant)
+    L, D = 700, 64
+    p = _params(9, D)
+    a = {k: dev(v) for k, v in synth.make_activations(10, L, D, bf16=True).items()}
+    y, hf, cs = _prefill(p, a["x"], a["dt"], a["z"], a["B"], a["C"], S=1)
+    for L1 in (1, 31, 33, 64, 333):
+        s1, s2 = slice(0, L1), slice(L1, L)
+        y1, h1, c1 = _prefill(p, a["x"][s1], a["dt"][s1], a["z"][s1], a["B"][s1], a["C"][s1], S=1)
+        y2, h2, c2 = _prefill(p, a["x"][s2], a["dt"][s2], a["z"][s2], a["B"][s2], a["C"][s2], S=1,
+                              conv_state=c1, h0=h1)
+        assert_close(host(torch.cat([y1, y2])), host(y), False, TOL_F32, f"y split at {L1}")
+        assert_close(host(h2), host(hf), False, TOL_F32, f"h split at {L1}")
+        assert torch.equal(c2, cs), L1

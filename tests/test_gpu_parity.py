@@ -18,9 +18,9 @@ pytestmark = pytest.mark.gpu
 
 @pytest.fixture(autouse=True)
 def _auto_variant():
-    ssm.ssm_set_scan_states_per_lane(0)
+    ssm.ssm_set_scan_variant(0, 0)
     yield
-    ssm.ssm_set_scan_states_per_lane(0)
+    ssm.ssm_set_scan_variant(0, 0)
 
 
 def _layer_inputs(seed, tok, D, bf16, K=4, random_bias=True, random_A=True):
@@ -88,9 +88,12 @@ def test_conv_no_silu(orc):
 # scan
 # ---------------------------------------------------------------------------
 
-def _scan_case(orc, seed, lens, D, bf16, npt=0, with_z=True, with_h0=True, softplus=True,
-               workspace=False, inplace=False):
-    ssm.ssm_set_scan_states_per_lane(npt)
+VARIANTS = [(2, 1), (2, 2), (2, 3), (4, 1), (4, 2), (4, 3), (8, 1), (8, 2), (16, 1), (16, 2)]
+
+
+def _scan_case(orc, seed, lens, D, bf16, variant=(0, 0), with_z=True, with_h0=True,
+               softplus=True, workspace=False, inplace=False):
+    ssm.ssm_set_scan_variant(*variant)
     tok = sum(lens)
     prm, act = _layer_inputs(seed, tok, D, bf16)
     S = len(lens)
@@ -119,15 +122,15 @@ def _scan_case(orc, seed, lens, D, bf16, npt=0, with_z=True, with_h0=True, softp
     return host(y), host(hf)
 
 
-@pytest.mark.parametrize("npt", [4, 8, 16])
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("bf16", [False, True])
-def test_scan_variants_packed(orc, npt, bf16):
-    _scan_case(orc, 10, [130, 0, 1, 7, 64, 65, 200], 200, bf16, npt=npt)
+def test_scan_variants_packed(orc, variant, bf16):
+    _scan_case(orc, 10, [130, 0, 1, 7, 64, 65, 200], 200, bf16, variant=variant)
 
 
-@pytest.mark.parametrize("npt", [4, 8, 16])
-def test_scan_scalar_path(orc, npt):
-    _scan_case(orc, 11, [50, 77], 30, True, npt=npt)
+@pytest.mark.parametrize("variant", VARIANTS)
+def test_scan_scalar_path(orc, variant):
+    _scan_case(orc, 11, [50, 77], 30, True, variant=variant)
 
 
 def test_scan_options(orc):
@@ -141,6 +144,11 @@ def test_scan_workspace_schedule_is_bit_identical(orc):
     y1, h1 = _scan_case(orc, 15, lens, 96, True, workspace=False)
     y2, h2 = _scan_case(orc, 15, lens, 96, True, workspace=True)
     assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
+
+
+def test_scan_device_status_clean():
+    """No bounded TMA wait gave up during the tests so far."""
+    assert ssm.ssm_scan_device_status(clear=True) == 0
 
 
 def test_scan_tokens_outside_sequences_untouched():
