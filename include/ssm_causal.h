@@ -206,6 +206,34 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
                                int64_t Bt, int64_t D, int N, int K, ssm_dtype act_dtype,
                                ssm_dtype conv_state_dtype, ssm_stream_t stream);
 
+/*
+ * ssm_selective_scan_fwd without a workspace, for callers that cannot
+ * allocate device memory when they call it: an inference engine that reserves
+ * all of its device memory at start-up and forbids allocation afterwards, or a
+ * plugin whose host framework owns the device allocator and hands it no
+ * scratch. Not part of the method the pages describe (the paper has no
+ * counterpart); it is a packaging of the same scan.
+ *
+ * Arguments, results and errors are those of ssm_selective_scan_fwd. The
+ * longest-first schedule of packed sequences lives in a fixed 16 KB array
+ * inside the library instead of a workspace, so a call may name at most 4096
+ * packed sequences; larger S with cu_seqlens is rejected with
+ * SSM_ERR_INVALID_ARGUMENT before anything is launched. The library allocates
+ * nothing for this call: every GPU that loads the library holds the array
+ * until the process exits. The first call on a device looks the array's
+ * address up (with that device current) and caches it; make that first call
+ * before any stream capture. All calls on a device share the one array and
+ * each overwrites it completely before reading it, so nothing needs clearing,
+ * but two such calls that run at the same time on one GPU (different streams
+ * without ordering between them) race on it and give unspecified results.
+ */
+int ssm_selective_scan_fwd_noalloc(const void *u, const void *delta, const float *A,
+                                   const void *B, const void *C, const float *Dskip,
+                                   const void *z, const float *dt_bias, int delta_softplus,
+                                   const float *h0, const int32_t *cu_seqlens, int64_t S,
+                                   void *y, float *h_final, int64_t tok, int64_t D, int N,
+                                   ssm_dtype act_dtype, ssm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

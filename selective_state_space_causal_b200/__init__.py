@@ -17,6 +17,7 @@ from ._lib import (  # noqa: F401
     ssm_scan_device_status,
     ssm_scan_workspace_size,
     ssm_selective_scan_fwd,
+    ssm_selective_scan_fwd_noalloc,
     ssm_selective_state_update,
     ssm_set_scan_variant,
     ssm_version,

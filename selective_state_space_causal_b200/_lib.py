@@ -34,6 +34,8 @@ SIGNATURES = [
     ("ssm_scan_workspace_size", _sz, [_i64, _i64, _int, _i64]),
     ("ssm_selective_scan_fwd", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64,
                                       _vp, _vp, _i64, _i64, _int, _int, _vp, _sz, _vp]),
+    ("ssm_selective_scan_fwd_noalloc", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
+                                              _vp, _i64, _vp, _vp, _i64, _i64, _int, _int, _vp]),
     ("ssm_selective_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _int, _vp, _i64, _vp, _i64, _i64, _int, _int, _int,
                                           _int, _vp]),
@@ -153,6 +155,25 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, y, Dskip=None, z=None, dt_bias=Non
                                       _ptr(Dskip), _ptr(z), _ptr(dt_bias), int(bool(delta_softplus)),
                                       _ptr(h0), _ptr(cu_seqlens), S, _ptr(y), _ptr(h_final), tok, D,
                                       N, _dtype(u), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def ssm_selective_scan_fwd_noalloc(u, delta, A, B, C, y, Dskip=None, z=None, dt_bias=None,
+                                   delta_softplus=True, h0=None, h_final=None, cu_seqlens=None,
+                                   S=None, stream=None):
+    """ssm_selective_scan_fwd with the library's fixed scratch instead of a workspace.
+
+    For callers that cannot allocate device memory at call time (an engine
+    that reserved all device memory at start-up, or a plugin whose framework
+    owns the allocator). At most 4096 packed sequences per call; concurrent
+    calls on one GPU share the scratch and race."""
+    tok, D = u.shape
+    N = A.shape[1]
+    if S is None:
+        S = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
+    _check(lib.ssm_selective_scan_fwd_noalloc(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(cu_seqlens), S, _ptr(y), _ptr(h_final), tok, D,
+        N, _dtype(u), _stream(stream)))
 
 
 def ssm_selective_state_update(conv_state, ssm_state, x, dt, B, C, y, conv_w, A, z=None,

@@ -17,6 +17,8 @@ namespace ssm {
 void set_scan_variant(int npt, int sched);
 size_t scan_order_bytes(int64_t S);
 int read_scan_status(bool clear);
+cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
+int64_t noalloc_max_sequences();
 }  // namespace ssm
 
 namespace {
@@ -239,6 +241,33 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
     int launched = 0;
     cudaError_t e = ssm::launch_decode(a, reinterpret_cast<cudaStream_t>(stream), &launched);
     return finish(e, launched, fn);
+}
+
+// For callers that cannot allocate device memory: the same scan, with its
+// schedule scratch in a fixed device array owned by the library instead of a
+// caller-allocated workspace. It forwards to ssm_selective_scan_fwd.
+int ssm_selective_scan_fwd_noalloc(const void *u, const void *delta, const float *A,
+                                   const void *B, const void *C, const float *Dskip,
+                                   const void *z, const float *dt_bias, int delta_softplus,
+                                   const float *h0, const int32_t *cu_seqlens, int64_t S,
+                                   void *y, float *h_final, int64_t tok, int64_t D, int N,
+                                   ssm_dtype act_dtype, ssm_stream_t stream)
+{
+    const char *fn = "ssm_selective_scan_fwd_noalloc";
+    if (cu_seqlens && S > ssm::noalloc_max_sequences())
+        return fail(SSM_ERR_INVALID_ARGUMENT,
+                    "%s: at most %lld packed sequences per call (got %lld); the fixed scratch "
+                    "holds one schedule entry per sequence",
+                    fn, (long long)ssm::noalloc_max_sequences(), (long long)S);
+    void *scratch = nullptr;
+    size_t bytes = 0;
+    cudaError_t e = ssm::noalloc_scratch(&scratch, &bytes);
+    if (e != cudaSuccess)
+        return fail(SSM_ERR_CUDA, "%s: looking up the fixed scratch failed: %s", fn,
+                    cudaGetErrorString(e));
+    return ssm_selective_scan_fwd(u, delta, A, B, C, Dskip, z, dt_bias, delta_softplus, h0,
+                                  cu_seqlens, S, y, h_final, tok, D, N, act_dtype, scratch, bytes,
+                                  stream);
 }
 
 }  // extern "C"

@@ -34,6 +34,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -1055,5 +1057,46 @@ cudaError_t launch_scan(const ScanArgs &a, cudaStream_t stream, int *launches)
     if (a.vec && a.D % 4 == 0) return dispatch<float, 4>(p, npt, sched, stream, launches);
     return dispatch<float, 1>(p, npt, sched, stream, launches);
 }
+
+}  // namespace ssm
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for callers that cannot allocate device memory.
+//
+// The longest-first schedule of ssm_selective_scan_fwd normally lives in a
+// caller-allocated workspace. ssm_selective_scan_fwd_noalloc uses this
+// file-scope array instead: every GPU that loads the library holds its 16 KB
+// until the process exits, and every call on a device shares it.
+// ---------------------------------------------------------------------------
+namespace ssm {
+
+constexpr int64_t kNoallocMaxSeqs = 4096;
+static __device__ __align__(256) int32_t g_noalloc_order[kNoallocMaxSeqs];
+
+// Device address of g_noalloc_order on the current device. The first request
+// on a device looks it up (with that device current) and caches it; later
+// requests reuse the cached value.
+cudaError_t noalloc_scratch(void **ptr, size_t *bytes)
+{
+    constexpr int kMaxDevices = 64;
+    static void *cached[kMaxDevices] = {};
+    static std::mutex lock;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> guard(lock);
+    if (!cached[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_order);
+        if (e != cudaSuccess) return e;
+        cached[dev] = p;
+    }
+    *ptr = cached[dev];
+    *bytes = sizeof(g_noalloc_order);
+    return cudaSuccess;
+}
+
+int64_t noalloc_max_sequences() { return kNoallocMaxSeqs; }
 
 }  // namespace ssm
