@@ -266,7 +266,7 @@ def bench_headline(args, world, peaks, rank_dev):
     achieved = st.scan_exps() / (scan_ms * 1e-3) / 1e9
     sha = source_sha("scan.cu", "common.cuh")
     traffic = recorded_traffic("scan_kernel", sha)
-    roofline = {"kernel": "scan_kernel", "bound": "alu", "unit": "Gexp/s",
+    roofline = {"kernel": "scan_kernel (scan_tma_kernel)", "bound": "alu", "unit": "Gexp/s",
                 "achieved": round(achieved, 1), "peak": round(mufu, 1),
                 "frac": round(achieved / mufu, 4), "traffic": traffic,
                 "kernel_ms": round(scan_ms, 5),
