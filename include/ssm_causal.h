@@ -94,13 +94,13 @@ unsigned long long ssm_launch_count(void);
 int ssm_set_scan_variant(int states_per_lane, int schedule);
 
 /*
- * Device-side status of the scan kernels on the current device: 0 while every
- * bounded wait for a TMA tile completed, 1 once a wait gave up (the results of
- * that call are then unspecified; the kernel still terminates). Synchronises
- * the device. clear != 0 resets the flag. Returns SSM_ERR_CUDA if the query
- * itself fails.
+ * Device-side status of the library's kernels on the current device: 0 while
+ * every bounded wait for a TMA tile completed; bit 0 set once a scan kernel's
+ * wait gave up, bit 1 once a conv kernel's did (the results of that call are
+ * then unspecified; the kernel still terminates). Synchronises the device.
+ * clear != 0 resets the flags. Returns SSM_ERR_CUDA if the query itself fails.
  */
-int ssm_scan_device_status(int clear);
+int ssm_device_status(int clear);
 
 /*
  * Checks a HOST copy of cu_seqlens (S+1 entries): cu[0] == 0, non-decreasing,
@@ -196,7 +196,8 @@ int ssm_selective_scan_fwd(const void *u, const void *delta, const float *A, con
  *                  left untouched; an index >= n_slots is skipped as well.
  *                  Two rows naming the same slot race (undefined result).
  *   y              (Bt, D) act_dtype
- *   N must be 16; K in 2..4.
+ *   N must be 16; K in 2..4. ssm_state, A, B, C and (for K = 4) conv_w must be
+ *   16-byte aligned, else SSM_ERR_MISALIGNED.
  */
 int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x,
                                const void *dt, const void *B, const void *C, const void *z,

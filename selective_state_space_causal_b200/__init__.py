@@ -14,7 +14,7 @@ from ._lib import (  # noqa: F401
     ssm_check_cu_seqlens,
     ssm_last_error,
     ssm_launch_count,
-    ssm_scan_device_status,
+    ssm_device_status,
     ssm_scan_workspace_size,
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_noalloc,

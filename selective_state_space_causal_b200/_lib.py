@@ -27,7 +27,7 @@ SIGNATURES = [
     ("ssm_version", _int, []),
     ("ssm_launch_count", ctypes.c_ulonglong, []),
     ("ssm_set_scan_variant", _int, [_int, _int]),
-    ("ssm_scan_device_status", _int, [_int]),
+    ("ssm_device_status", _int, [_int]),
     ("ssm_check_cu_seqlens", _int, [_vp, _i64, _i64]),
     ("ssm_causal_conv1d", _int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _i64, _vp, _vp, _int,
                                  _int, _int, _vp]),
@@ -111,8 +111,8 @@ def ssm_set_scan_variant(states_per_lane: int, schedule: int = 0) -> None:
     _check(lib.ssm_set_scan_variant(int(states_per_lane), int(schedule)))
 
 
-def ssm_scan_device_status(clear: bool = False) -> int:
-    code = lib.ssm_scan_device_status(int(bool(clear)))
+def ssm_device_status(clear: bool = False) -> int:
+    code = lib.ssm_device_status(int(bool(clear)))
     if code < 0:
         _check(code)
     return code

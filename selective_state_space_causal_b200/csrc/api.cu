@@ -17,6 +17,7 @@ namespace ssm {
 void set_scan_variant(int npt, int sched);
 size_t scan_order_bytes(int64_t S);
 int read_scan_status(bool clear);
+int read_conv_status(bool clear);
 cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
 int64_t noalloc_max_sequences();
 }  // namespace ssm
@@ -97,12 +98,13 @@ int ssm_set_scan_variant(int npt, int sched)
     return ok();
 }
 
-int ssm_scan_device_status(int clear)
+int ssm_device_status(int clear)
 {
-    const int v = ssm::read_scan_status(clear != 0);
-    if (v < 0) return fail(SSM_ERR_CUDA, "ssm_scan_device_status: CUDA query failed");
+    const int a = ssm::read_scan_status(clear != 0);
+    const int b = ssm::read_conv_status(clear != 0);
+    if (a < 0 || b < 0) return fail(SSM_ERR_CUDA, "ssm_device_status: CUDA query failed");
     g_error.clear();
-    return v;
+    return (a ? 1 : 0) | (b ? 2 : 0);
 }
 
 int ssm_check_cu_seqlens(const int32_t *cu, int64_t S, int64_t tok)
@@ -233,8 +235,10 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
         !aligned(conv_w, 4) || !aligned(conv_b, 4) || !aligned(A, 4) || !aligned(Dskip, 4) ||
         !aligned(dt_bias, 4) || !aligned(state_indices, 4))
         return fail(SSM_ERR_MISALIGNED, "%s: a pointer is not aligned to its element size", fn);
-    if (!aligned(ssm_state, 16))
-        return fail(SSM_ERR_MISALIGNED, "%s: ssm_state must be 16-byte aligned", fn);
+    if (!aligned(ssm_state, 16) || !aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16) ||
+        (K == 4 && !aligned(conv_w, 16)))
+        return fail(SSM_ERR_MISALIGNED,
+                    "%s: ssm_state, A, B, C (and conv_w when K = 4) must be 16-byte aligned", fn);
     ssm::DecodeArgs a{conv_state, ssm_state, x, dt_, B, C, z, conv_w, conv_b, A, Dskip, dt_bias,
                       delta_softplus, state_indices, n_slots, y, Bt, D, N, K, dt(act_dtype),
                       dt(conv_state_dtype)};

@@ -14,14 +14,21 @@
 // inputs in registers, so every input is read from DRAM once; the K-1 halo rows
 // at a strip's start are re-read from L2. Consecutive threads own consecutive
 // channel vectors, so each token row is read and written fully coalesced.
+// A strip that lies inside one sequence issues all of its loads before any
+// arithmetic, which keeps enough bytes in flight to run at HBM speed.
 #include "common.cuh"
 #include "internal.h"
+#include "tma.cuh"
 
 namespace ssm {
+
+// Set by a conv kernel whose bounded wait on its TMA tile gave up.
+__device__ int g_conv_status = 0;
+
 namespace {
 
-constexpr int kStrip = 32;
-constexpr int kThreads = 256;
+constexpr int kStrip = 16;
+constexpr int kThreads = 128;
 
 struct Seqs {
     const int32_t *cu;  // nullptr: dense rows of L tokens
@@ -46,6 +53,20 @@ struct Seqs {
         return lo;
     }
 };
+
+template <typename T, int VEC, int K>
+__device__ __forceinline__ void conv_out(const float (&wk)[K][VEC], const float (&bv)[VEC],
+                                         const float (&win)[K][VEC], int apply_silu,
+                                         float (&out)[VEC])
+{
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+        float acc = bv[i];
+#pragma unroll
+        for (int k = 0; k < K; ++k) acc = fmaf(wk[k][i], win[k][i], acc);
+        out[i] = apply_silu ? silu_f(acc) : acc;
+    }
+}
 
 template <typename T, typename TS, int VEC, int K>
 __global__ void __launch_bounds__(kThreads)
@@ -73,8 +94,36 @@ conv1d_kernel(const T *__restrict__ x, T *__restrict__ xc, const float *__restri
     int64_t s_start = sq.off(s);
     int64_t s_end = max(sq.off(s + 1), s_start);
 
+    if constexpr (VEC * sizeof(T) == 16) {
+        // Fast path: the strip and its K-1 halo rows lie inside one sequence.
+        // All loads are issued before any use, so each thread keeps
+        // (kStrip + K - 1) x 16 bytes in flight.
+        if (t0 - (K - 1) >= s_start && t0 + kStrip <= s_end) {
+            uint4 raw[kStrip + K - 1];
+#pragma unroll
+            for (int r = 0; r < kStrip + K - 1; ++r)
+                raw[r] = ldg16(x + (t0 - (K - 1) + r) * D + c0);
+            float win[K][VEC];
+#pragma unroll
+            for (int k = 0; k < K - 1; ++k) unpack16<T, VEC>(raw[k], win[k]);
+#pragma unroll
+            for (int t = 0; t < kStrip; ++t) {
+                unpack16<T, VEC>(raw[t + K - 1], win[K - 1]);
+                float out[VEC];
+                conv_out<T, VEC, K>(wk, bv, win, apply_silu, out);
+                store_vec<T, VEC>(xc + (t0 + t) * D + c0, out);
+#pragma unroll
+                for (int k = 0; k < K - 1; ++k)
+#pragma unroll
+                    for (int i = 0; i < VEC; ++i) win[k][i] = win[k + 1][i];
+            }
+            return;
+        }
+    }
+
+    // General path: sequence starts inside the strip or its halo.
     // win[j] is the input K-1-j positions before the current token.
-    float win[K - 1][VEC];
+    float win[K][VEC];
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) {
         const int64_t pos = t0 - (K - 1) + j;
@@ -104,23 +153,120 @@ conv1d_kernel(const T *__restrict__ x, T *__restrict__ xc, const float *__restri
                 for (int i = 0; i < VEC; ++i)
                     win[j][i] = state_in ? to_f32(state_in[(s * D + c0 + i) * (K - 1) + j]) : 0.f;
         }
-        float xv[VEC], out[VEC];
-        load_vec<T, VEC>(x + t * D + c0, xv);
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) {
-            float acc = bv[i];
-#pragma unroll
-            for (int k = 0; k < K - 1; ++k) acc = fmaf(wk[k][i], win[k][i], acc);
-            acc = fmaf(wk[K - 1][i], xv[i], acc);
-            out[i] = apply_silu ? silu_f(acc) : acc;
-        }
+        load_vec<T, VEC>(x + t * D + c0, win[K - 1]);
+        float out[VEC];
+        conv_out<T, VEC, K>(wk, bv, win, apply_silu, out);
         store_vec<T, VEC>(xc + t * D + c0, out);
 #pragma unroll
-        for (int j = 0; j < K - 2; ++j)
+        for (int j = 0; j < K - 1; ++j)
 #pragma unroll
             for (int i = 0; i < VEC; ++i) win[j][i] = win[j + 1][i];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// TMA-tiled variant (16-byte aligned rows). A CTA owns kTileT tokens x one
+// 128-byte row of channels: one TMA box of kTileT + K - 1 rows (the K - 1 halo
+// rows may start before token 0 or run past the last token; those read zeros)
+// lands in shared memory, then each thread slides the K-tap window over its
+// kTileG tokens of one 16-byte channel vector and writes 16-byte outputs.
+// Many small CTAs per SM overlap one CTA's load with another's arithmetic.
+// ---------------------------------------------------------------------------
+constexpr int kTileT = 128;      // tokens per CTA
+constexpr int kTileG = 8;        // tokens per thread
+constexpr int kTileThreads = 128;
+
+template <typename T, typename TS, int K>
+__global__ void __launch_bounds__(kTileThreads)
+conv1d_tma_kernel(const __grid_constant__ CUtensorMap xmap, T *__restrict__ xc,
+                  const float *__restrict__ w, const float *__restrict__ bias, Seqs sq, int64_t D,
+                  const TS *__restrict__ state_in, int apply_silu)
+{
+    constexpr int VEC = 16 / sizeof(T);        // channels per 16-byte vector
+    constexpr int CW = 128 / sizeof(T);        // channels per tile row (128 bytes)
+    constexpr int NV = CW / VEC;               // vectors per row
+    constexpr int ROWS = kTileT + K - 1;
+    static_assert(NV * (kTileT / kTileG) == kTileThreads, "one thread per (vector, token group)");
+    __shared__ __align__(128) T tile[ROWS * CW];
+    __shared__ __align__(8) uint64_t bar;
+
+    const int tid = threadIdx.x;
+    const int64_t t0 = (int64_t)blockIdx.x * kTileT;
+    const int64_t cbase = (int64_t)blockIdx.y * CW;
+    if (tid == 0) mbar_init(&bar);
+    __syncthreads();
+    if (tid == 0) {
+        mbar_expect_tx(&bar, (uint32_t)(ROWS * CW * sizeof(T)));
+        tma_2d(tile, &xmap, &bar, (int)cbase, (int)(t0 - (K - 1)));
+    }
+
+    const int v = tid % NV, g = tid / NV;
+    const int64_t c0 = cbase + (int64_t)v * VEC;
+    const int64_t ta = t0 + (int64_t)g * kTileG;
+    const bool active = c0 < D && ta < sq.tok;
+    float wk[K][VEC], bv[VEC];
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) win[K - 2][i] = xv[i];
+    for (int i = 0; i < VEC; ++i) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) wk[k][i] = active ? __ldg(w + (c0 + i) * K + k) : 0.f;
+        bv[i] = (active && bias) ? __ldg(bias + c0 + i) : 0.f;
+    }
+    // every thread waits, so no thread leaves while the copy is in flight
+    bool failed = false;
+    mbar_wait(&bar, 0, failed, &g_conv_status, 1);
+    if (!active) return;
+
+    const int64_t tb = min(ta + (int64_t)kTileG, sq.tok);
+    int64_t s = sq.find(ta);
+    int64_t s_start = sq.off(s);
+    int64_t s_end = max(sq.off(s + 1), s_start);
+    // tile row of token position pos
+    auto row = [&](int64_t pos) { return (int)(pos - (t0 - (K - 1))); };
+
+    if (ta - (K - 1) >= s_start && ta + kTileG <= s_end) {
+        float win[K][VEC];
+#pragma unroll
+        for (int k = 0; k < K - 1; ++k)
+            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(tile + row(ta - (K - 1) + k) * CW + v * VEC), win[k]);
+#pragma unroll
+        for (int t = 0; t < kTileG; ++t) {
+            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(tile + row(ta + t) * CW + v * VEC), win[K - 1]);
+            float out[VEC];
+            conv_out<T, VEC, K>(wk, bv, win, apply_silu, out);
+            store_vec<T, VEC>(xc + (ta + t) * D + c0, out);
+#pragma unroll
+            for (int k = 0; k < K - 1; ++k)
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) win[k][i] = win[k + 1][i];
+        }
+        return;
+    }
+
+    // tokens near a sequence boundary: rebuild the window for every token
+    for (int64_t t = ta; t < tb; ++t) {
+        while (t >= s_end && s < sq.S - 1) {
+            ++s;
+            s_start = s_end;
+            s_end = max(sq.off(s + 1), s_start);
+        }
+        if (t >= s_end) break;  // token outside every sequence
+        float win[K][VEC];
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            const int64_t pos = t - (K - 1) + k;
+            if (pos >= s_start) {
+                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(tile + row(pos) * CW + v * VEC), win[k]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i)
+                    win[k][i] = state_in
+                        ? to_f32(state_in[(s * D + c0 + i) * (K - 1) + (K - 1) + (pos - s_start)])
+                        : 0.f;
+            }
+        }
+        float out[VEC];
+        conv_out<T, VEC, K>(wk, bv, win, apply_silu, out);
+        store_vec<T, VEC>(xc + t * D + c0, out);
     }
 }
 
@@ -160,7 +306,14 @@ cudaError_t run(const ConvArgs &a, cudaStream_t stream, int *launches)
         const int64_t nvec = vec ? a.D / V : a.D;
         const int64_t threads = nvec * ((a.tok + kStrip - 1) / kStrip);
         const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
-        if (vec)
+        CUtensorMap map;
+        if (vec && encode_2d(&map, a.x, sizeof(T) == 2, a.D, a.tok, 128 / sizeof(T),
+                             kTileT + K - 1)) {
+            const dim3 grid((unsigned)((a.tok + kTileT - 1) / kTileT),
+                            (unsigned)((a.D * sizeof(T) + 127) / 128));
+            conv1d_tma_kernel<T, TS, K><<<grid, kTileThreads, 0, stream>>>(
+                map, static_cast<T *>(a.xc), a.w, a.bias, sq, a.D, st_in, a.apply_silu);
+        } else if (vec)
             conv1d_kernel<T, TS, V, K><<<blocks, kThreads, 0, stream>>>(
                 x, static_cast<T *>(a.xc), a.w, a.bias, sq, a.D, st_in, a.apply_silu);
         else
@@ -200,6 +353,17 @@ cudaError_t launch_conv1d(const ConvArgs &a, cudaStream_t stream, int *launches)
     if (xb) return by_k<__nv_bfloat16, float>(a, stream, launches);
     if (sb) return by_k<float, __nv_bfloat16>(a, stream, launches);
     return by_k<float, float>(a, stream, launches);
+}
+
+int read_conv_status(bool clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_conv_status, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_conv_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+    }
+    return v;
 }
 
 }  // namespace ssm

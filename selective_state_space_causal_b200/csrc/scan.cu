@@ -31,13 +31,11 @@
 // * Tokens past a sequence's end are padded with delta = 0 (dA = 1, no input),
 //   which leaves h unchanged, so the inner loop needs no tail branch.
 // * Packed sequences are scheduled longest-first when scratch is supplied.
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
+#include "tma.cuh"
 
 namespace ssm {
 
@@ -47,7 +45,6 @@ __device__ int g_scan_status = 0;
 namespace {
 
 constexpr int kN = 16;
-constexpr unsigned kSpinLimit = 1u << 21;
 
 struct Params {
     const void *u, *delta, *B, *C, *z;
@@ -434,40 +431,6 @@ struct Maps {
     CUtensorMap u, dt, z, b, c;
 };
 
-__device__ __forceinline__ uint32_t saddr(const void *p)
-{
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void tma_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x, int y)
-{
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%2, %3}], [%4];"
-        :: "r"(saddr(dst)), "l"(map), "r"(x), "r"(y), "r"(saddr(bar)) : "memory");
-}
-
-// Waits for phase `parity` of the barrier with a bounded number of
-// non-blocking polls (about 0.2 s in all; a tile normally lands within a few
-// microseconds). On timeout it records the failure in g_scan_status and marks
-// `failed`, after which this thread no longer waits at all, so the kernel
-// always terminates.
-__device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &failed)
-{
-    if (failed) return;
-    for (unsigned i = 0; i < kSpinLimit; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-            " selp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(done) : "r"(saddr(bar)), "r"(parity) : "memory");
-        if (done) return;
-        if (i >= 32) __nanosleep(64);
-    }
-    failed = true;
-    atomicOr(&g_scan_status, 1);
-}
-
 template <class K, typename T>
 __global__ void __launch_bounds__(K::THREADS)
 scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
@@ -490,14 +453,10 @@ scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
     const Lane l = lane_setup<K>(p);
     const uint32_t tx_bytes = (uint32_t)((has_z ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
 
-    if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(saddr(bar)) : "memory");
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+    if (tid == 0) mbar_init(bar);
     __syncthreads();
     auto issue = [&](int64_t t0) {
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                     :: "r"(saddr(bar)), "r"(tx_bytes) : "memory");
+        mbar_expect_tx(bar, tx_bytes);
         const int x = (int)l.cbase, y = (int)t0;
         tma_2d(rU, &m.u, bar, x, y);
         tma_2d(rDT, &m.dt, bar, x, y);
@@ -518,7 +477,7 @@ scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
     bool failed = false;
     for (int64_t t0 = l.start; t0 < l.end; t0 += TCH) {
         const int nt = (int)min((int64_t)TCH, l.end - t0);
-        mbar_wait(bar, parity, failed);
+        mbar_wait(bar, parity, failed, &g_scan_status, 1);
         parity ^= 1u;
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
@@ -552,7 +511,7 @@ scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
         if (tid == 0 && t0 + TCH < l.end) {
             // the raw tiles were read through the generic proxy; order those
             // reads before the next asynchronous-proxy writes into them
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            fence_proxy_async();
             issue(t0 + TCH);
         }
         const int ntr = ((nt + K::TPC - 1) / K::TPC) * K::TPC;
@@ -645,14 +604,10 @@ scan_ts_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
     const int mycol = col2(cl);
     const uint32_t tx_bytes = (uint32_t)((has_z ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
 
-    if (tid == 0) {
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(saddr(bar)) : "memory");
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+    if (tid == 0) mbar_init(bar);
     __syncthreads();
     auto issue = [&](int64_t t0) {
-        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                     :: "r"(saddr(bar)), "r"(tx_bytes) : "memory");
+        mbar_expect_tx(bar, tx_bytes);
         const int x = (int)cbase, y = (int)t0;
         tma_2d(rU, &m.u, bar, x, y);
         tma_2d(rDT, &m.dt, bar, x, y);
@@ -677,7 +632,7 @@ scan_ts_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
     bool failed = false;
     for (int64_t t0 = start; t0 < end; t0 += TCH) {
         const int nt = (int)min((int64_t)TCH, end - t0);
-        mbar_wait(bar, parity, failed);
+        mbar_wait(bar, parity, failed, &g_scan_status, 1);
         parity ^= 1u;
 
         // ---- pre-pass: items of PV channels of one token ----
@@ -707,7 +662,7 @@ scan_ts_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
         }
         __syncthreads();
         if (tid == 0 && t0 + TCH < end) {
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            fence_proxy_async();
             issue(t0 + TCH);
         }
 
@@ -876,36 +831,6 @@ order_kernel(const int32_t *__restrict__ cu, int64_t S, int64_t tok, int32_t *__
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
-                cudaSuccess || q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }();
-    return fn;
-}
-
-// 2-D tile map over a row-major (rows, inner) tensor; out-of-range reads fill 0.
-bool encode(CUtensorMap *map, const void *base, bool bf16, uint64_t inner, uint64_t rows,
-            uint32_t box_inner, uint32_t box_rows)
-{
-    auto fn = tensor_map_encoder();
-    if (!fn) return false;
-    const uint64_t es = bf16 ? 2 : 4;
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner * es};
-    cuuint32_t box[2] = {box_inner, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <class K, typename T>
 cudaError_t run(const Params &p, bool tma, cudaStream_t stream, int *launches)
 {
@@ -914,12 +839,12 @@ cudaError_t run(const Params &p, bool tma, cudaStream_t stream, int *launches)
     if (tma && p.tok > 0) {
         Maps m;
         const bool bf = sizeof(T) == 2;
-        bool ok = encode(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
-                  encode(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
-                  encode(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
-                  encode(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+        bool ok = encode_2d(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
+                  encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+                  encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+                  encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
         if (ok) {
-            if (p.z) ok = encode(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+            if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
             else m.z = m.u;  // never loaded
         }
         if (ok) {
@@ -951,12 +876,12 @@ cudaError_t run_ts(const Params &p, cudaStream_t stream, int *launches)
     const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
     Maps m;
     const bool bf = sizeof(T) == 2;
-    bool ok = p.tok > 0 && encode(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
-              encode(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
-              encode(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
-              encode(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+    bool ok = p.tok > 0 && encode_2d(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+              encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
     if (ok) {
-        if (p.z) ok = encode(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+        if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
         else m.z = m.u;  // never loaded
     }
     if (!ok) return cudaErrorNotSupported;

@@ -1,0 +1,107 @@
+// tma.cuh -- TMA tile loads, mbarrier waits and tensor-map encoding (sm_100a).
+//
+// Loads are plain per-CTA tile copies (cp.async.bulk.tensor, no multicast) of
+// this GPU's own memory into the calling CTA's shared memory; completion is
+// tracked by an mbarrier with an expected transaction byte count.
+#pragma once
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssm {
+
+// Non-blocking polls before a wait gives up (about 0.2 s with the back-off;
+// a tile normally lands within microseconds).
+constexpr unsigned kTmaSpinLimit = 1u << 21;
+
+__device__ __forceinline__ uint32_t saddr(const void *p)
+{
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" :: "r"(saddr(bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(saddr(bar)), "r"(bytes) : "memory");
+}
+
+// 2-D tile load: box at (x = inner coordinate, y = row) into dst.
+__device__ __forceinline__ void tma_2d(void *dst, const CUtensorMap *map, uint64_t *bar, int x,
+                                       int y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3}], [%4];"
+        :: "r"(saddr(dst)), "l"(map), "r"(x), "r"(y), "r"(saddr(bar)) : "memory");
+}
+
+// Order earlier generic-proxy reads of shared memory before later TMA writes.
+__device__ __forceinline__ void fence_proxy_async()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Waits for phase `parity` of the barrier with a bounded number of
+// non-blocking polls. On timeout it sets bit `code` of *status and marks
+// `failed`, after which this thread no longer waits at all, so a kernel
+// always terminates.
+__device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &failed,
+                                          int *status, int code)
+{
+    if (failed) return;
+    for (unsigned i = 0; i < kTmaSpinLimit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done) : "r"(saddr(bar)), "r"(parity) : "memory");
+        if (done) return;
+        if (i >= 32) __nanosleep(64);
+    }
+    failed = true;
+    atomicOr(status, code);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess || q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }();
+    return fn;
+}
+
+// 2-D tile map over a row-major (rows, inner) tensor of bf16 or fp32;
+// out-of-range reads fill zeros. Returns false if the map cannot be encoded.
+inline bool encode_2d(CUtensorMap *map, const void *base, bool bf16, uint64_t inner, uint64_t rows,
+                      uint32_t box_inner, uint32_t box_rows)
+{
+    auto fn = tensor_map_encoder();
+    if (!fn) return false;
+    const uint64_t es = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * es};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+              const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace ssm

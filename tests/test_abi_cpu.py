@@ -104,6 +104,7 @@ def test_scan_rejects(kw, code):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(N=4), -1), (dict(K=6), -1), (dict(slots=4), -1), (dict(ss=A16 + 4), -3),
+    (dict(A=A16 + 4), -3), (dict(B=A16 + 8), -3), (dict(w=A16 + 4), -3),
     (dict(x=None), -1), (dict(cdt=5), -2), (dict(Bt=70000, slots=70000), -1),
 ])
 def test_decode_rejects(kw, code):

@@ -148,7 +148,7 @@ def test_scan_workspace_schedule_is_bit_identical(orc):
 
 def test_scan_device_status_clean():
     """No bounded TMA wait gave up during the tests so far."""
-    assert ssm.ssm_scan_device_status(clear=True) == 0
+    assert ssm.ssm_device_status(clear=True) == 0
 
 
 def test_scan_tokens_outside_sequences_untouched():

@@ -66,4 +66,4 @@ def test_noalloc_matches_workspace_entry_point_twice():
         torch.cuda.synchronize()
         assert_close(host(y), host(y_ref), True, TOL_BF16, "y")
         assert_close(host(h), host(h_ref), False, TOL_BF16, "h_final")
-    assert ssm.ssm_scan_device_status(clear=True) == 0
+    assert ssm.ssm_device_status(clear=True) == 0
