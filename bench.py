@@ -172,18 +172,26 @@ def _barrier_sync(world):
 
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
 
 
 def _max_over_ranks(x: float, world: int) -> float:
+    """Slowest rank's value (timings are taken per rank on the device)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Units all ranks processed per second, in G/s, over the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3) / 1e9
 
 
 class HeadlineStep:
@@ -260,7 +268,7 @@ def bench_headline(args, world, peaks, rank_dev):
     ms = start.elapsed_time(stop) / K
     scan_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
     ms_max = _max_over_ranks(ms, world)
-    value = st.units() * world / (ms_max * 1e-3) / 1e9
+    value = whole_job_rate(st.units(), world, ms_max)
 
     mufu = mufu_peak_gexp(peaks["sm_max_mhz"])
     achieved = st.scan_exps() / (scan_ms * 1e-3) / 1e9
@@ -308,7 +316,7 @@ def bench_headline(args, world, peaks, rank_dev):
     stop.record()
     _barrier_sync(world)
     ems = _max_over_ranks(start.elapsed_time(stop) / Ke, world)
-    res["e2e"] = {"value": st.units() * world / (ems * 1e-3) / 1e9, "unit": UNIT,
+    res["e2e"] = {"value": whole_job_rate(st.units(), world, ems), "unit": UNIT,
                   "ms_per_step": ems, "h2d_bytes_per_step": int(h2d),
                   "d2h_bytes_per_step": int(d2h)}
     del st
