@@ -111,10 +111,93 @@ __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
     return d;
 }
 
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b)
+{
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for two values on the FMA pipe instead of the special-function unit.
+// x is clamped to [-126, 126] and split as n + f with n = round(x) (adding and
+// subtracting 1.5 * 2^23 rounds to an integer held in the low mantissa bits)
+// and f in [-0.5, 0.5]; 2^f comes from a degree-5 polynomial whose
+// coefficients were fitted here for minimal relative error on [-0.5, 0.5]
+// (2.3e-7 when evaluated in fp32), and 2^n is added into the exponent bits:
+// the float bits of x + 1.5 * 2^23 are 0x4B400000 + n, and shifting them left
+// by 23 leaves exactly n << 23 (mod 2^32).
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float &r0, float &r1)
+{
+    x0 = fminf(fmaxf(x0, -126.0f), 126.0f);
+    x1 = fminf(fmaxf(x1, -126.0f), 126.0f);
+    const f32x2 X = pk2(x0, x1);
+    const f32x2 T = add2(X, pk2(12582912.0f, 12582912.0f));
+    const f32x2 N = add2(T, pk2(-12582912.0f, -12582912.0f));  // exact
+    const f32x2 F = fma2(N, pk2(-1.0f, -1.0f), X);                // x - n, exact
+    f32x2 P = fma2(pk2(0.00132764782756567f, 0.00132764782756567f), F,
+                   pk2(0.009675521403551102f, 0.009675521403551102f));
+    P = fma2(P, F, pk2(0.05550713092088699f, 0.05550713092088699f));
+    P = fma2(P, F, pk2(0.24022120237350464f, 0.24022120237350464f));
+    P = fma2(P, F, pk2(0.6931469440460205f, 0.6931469440460205f));
+    P = fma2(P, F, pk2(1.0000001192092896f, 1.0000001192092896f));
+    float p0, p1, t0, t1;
+    upk2(P, p0, p1);
+    upk2(T, t0, t1);
+    r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// softplus of two values as softplus_fast, with exp on the FMA pipe.
+__device__ __forceinline__ void softplus2(float v0, float v1, float &d0, float &d1)
+{
+    float e0, e1;
+    exp2_fma2(-fabsf(v0) * kLog2e, -fabsf(v1) * kLog2e, e0, e1);
+    const f32x2 S = pk2(__fdividef(e0, 2.0f + e0), __fdividef(e1, 2.0f + e1));
+    const f32x2 X = mul2(S, S);
+    f32x2 P = fma2(pk2(0.28178291674498446f, 0.28178291674498446f), X,
+                   pk2(0.27960550702657632f, 0.27960550702657632f));
+    P = fma2(P, X, pk2(0.40024919874690540f, 0.40024919874690540f));
+    P = fma2(P, X, pk2(0.66666314227845440f, 0.66666314227845440f));
+    P = fma2(P, X, pk2(2.0000000079702546f, 2.0000000079702546f));
+    float l0, l1;
+    upk2(mul2(S, P), l0, l1);
+    d0 = fmaxf(v0, 0.0f) + l0;
+    d1 = fmaxf(v1, 0.0f) + l1;
+}
+
+// silu of two values, exp on the FMA pipe: z / (1 + 2^(-z log2 e)).
+__device__ __forceinline__ void silu2(float z0, float z1, float &g0, float &g1)
+{
+    float e0, e1;
+    exp2_fma2(-z0 * kLog2e, -z1 * kLog2e, e0, e1);
+    g0 = __fdividef(z0, 1.0f + e0);
+    g1 = __fdividef(z1, 1.0f + e1);
+}
+
 // silu(v) = v * sigmoid(v); exp(-v) overflowing to +inf gives -0 for v << 0.
 __device__ __forceinline__ float silu_f(float v)
 {
     return __fdividef(v, 1.0f + __expf(-v));
+}
+
+// softplus(v) = max(v, 0) + log1p(e) with e = exp(-|v|) in (0, 1], and
+// log1p(e) = 2 atanh(s), s = e / (2 + e) in (0, 1/3]. 2 atanh(s) / s is a
+// polynomial in s^2; the degree-4 coefficients below were fitted here for
+// minimal relative error on [0, 1/9] (max 4e-9, below fp32 resolution). Two
+// special-function ops (2^x and 1/x) and ten FMA-pipe ops; relative error of
+// the result ~5e-7.
+__device__ __forceinline__ float softplus_fast(float v)
+{
+    float e;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-fabsf(v) * kLog2e));
+    const float s = __fdividef(e, 2.0f + e);
+    const float x = s * s;
+    float p = 0.28178291674498446f;
+    p = fmaf(p, x, 0.27960550702657632f);
+    p = fmaf(p, x, 0.40024919874690540f);
+    p = fmaf(p, x, 0.66666314227845440f);
+    p = fmaf(p, x, 2.0000000079702546f);
+    return fmaxf(v, 0.0f) + s * p;
 }
 
 // softplus(v) = log(1 + e^v), taken as v itself above 20 where the two agree
