@@ -431,95 +431,267 @@ struct Maps {
     CUtensorMap u, dt, z, b, c;
 };
 
+// Shapes of the TMA-staged kernel. Per (token, channel) shared memory holds
+// (delta, delta, delta*u, delta*u) as one float4, so a lane gets both packed
+// operands of its recurrence from one 16-byte load, and TPC partial readouts.
+// The raw u, dt, z, B, C tiles are double-buffered: chunk k+1 lands while
+// chunk k is computed, and chunk k's u and z stay readable for its output.
+template <typename T, int NPT_, int CH_, int TCH_>
+struct TmaCfg {
+    static constexpr int NPT = NPT_, CH = CH_, TCH = TCH_;
+    static constexpr int TPC = kN / NPT, NP = NPT / 2;
+    static constexpr int THREADS = CH * TPC;
+    static constexpr int VEC = 16 / sizeof(T);
+    static constexpr int CV = CH / VEC;
+    static constexpr int ITEMS = TCH * CV;
+    static constexpr int IPT = (ITEMS + THREADS - 1) / THREADS;
+    static constexpr int ROWP = CH + CH / 8;               // float4 per row of sDD
+    static constexpr int ROWY = CH * TPC + (CH / 8) * 4;   // floats per row of sYP
+    static constexpr int BCN = TCH * kN / VEC;             // 16-byte B (or C) pieces
+    static constexpr size_t RAW_ACT = sizeof(T) * TCH * CH;
+    static constexpr size_t RAW_BC = sizeof(T) * TCH * kN;
+    static constexpr size_t STAGE = 3 * align128(RAW_ACT) + 2 * align128(RAW_BC);
+    static constexpr size_t OFF_DD = 0;
+    static constexpr size_t OFF_YP = align128(OFF_DD + 16 * (size_t)TCH * ROWP);
+    static constexpr size_t OFF_B = align128(OFF_YP + 4 * (size_t)TCH * ROWY);
+    static constexpr size_t OFF_C = align128(OFF_B + 4 * (size_t)TCH * kN);
+    static constexpr size_t OFF_RAW = align128(OFF_C + 4 * (size_t)TCH * kN);
+    static constexpr size_t OFF_BAR = OFF_RAW + 2 * STAGE;
+    static constexpr size_t SMEM = OFF_BAR + 128;
+    static_assert(NPT % 2 == 0 && CH % 8 == 0, "shape");
+    static_assert(VEC == 8 || VEC == 4, "16-byte vectors");
+    static_assert(THREADS % CV == 0, "each thread keeps one channel vector");
+    static_assert(THREADS <= 1024 && THREADS % 32 == 0, "block size");
+};
+
+// float4 column of channel c in a padded sDD row (16 B after every 8 channels).
+__device__ __forceinline__ int col4(int c) { return c + (c >> 3); }
+// float offset of (channel c, lane sub) in a padded sYP row.
+template <int TPC>
+__device__ __forceinline__ int coly(int c, int sub) { return c * TPC + sub + 4 * (c >> 3); }
+
 template <class K, typename T>
 __global__ void __launch_bounds__(K::THREADS)
 scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
 {
-    constexpr int VEC = K::VEC, IPT = K::IPT, THREADS = K::THREADS, CV = K::CV, TCH = K::TCH;
-    constexpr int CH = K::CH;
+    constexpr int NPT = K::NPT, NP = K::NP, TPC = K::TPC, CH = K::CH, TCH = K::TCH;
+    constexpr int VEC = K::VEC, CV = K::CV, IPT = K::IPT, THREADS = K::THREADS;
+    constexpr int ROWP = K::ROWP, ROWY = K::ROWY;
     extern __shared__ __align__(128) unsigned char smem[];
-    float2 *sDX = reinterpret_cast<float2 *>(smem + K::OFF_DX);
-    float2 *sUG = reinterpret_cast<float2 *>(smem + K::OFF_UG);
+    float4 *sDD = reinterpret_cast<float4 *>(smem + K::OFF_DD);
+    float *sYP = reinterpret_cast<float *>(smem + K::OFF_YP);
     float *sB = reinterpret_cast<float *>(smem + K::OFF_B);
     float *sC = reinterpret_cast<float *>(smem + K::OFF_C);
-    T *rU = reinterpret_cast<T *>(smem + K::OFF_RU);
-    T *rDT = reinterpret_cast<T *>(smem + K::OFF_RDT);
-    T *rZ = reinterpret_cast<T *>(smem + K::OFF_RZ);
-    T *rB = reinterpret_cast<T *>(smem + K::OFF_RB);
-    T *rC = reinterpret_cast<T *>(smem + K::OFF_RC);
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+    auto raw = [&](int stage, int which) -> T * {
+        size_t off = K::OFF_RAW + (size_t)stage * K::STAGE;
+        off += which < 3 ? (size_t)which * align128(K::RAW_ACT)
+                         : 3 * align128(K::RAW_ACT) + (size_t)(which - 3) * align128(K::RAW_BC);
+        return reinterpret_cast<T *>(smem + off);
+    };  // which: 0 u, 1 dt, 2 z, 3 B, 4 C
 
     const int tid = threadIdx.x;
-    const Lane l = lane_setup<K>(p);
+    const int cl = tid / TPC, sub = tid % TPC;
+    const int64_t cbase = (int64_t)blockIdx.x * CH;
+    const int64_t c0 = cbase + cl;
+    const bool cvalid = c0 < p.D;
+    int64_t seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
+    int64_t start, end;
+    if (p.cu) {
+        start = clamp_off(p.cu[seq], p.tok);
+        end = max(clamp_off(p.cu[seq + 1], p.tok), start);
+    } else {
+        start = seq * p.L;
+        end = start + p.L;
+    }
     const uint32_t tx_bytes = (uint32_t)((has_z ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
 
-    if (tid == 0) mbar_init(bar);
+    if (tid == 0) {
+        mbar_init(&bar[0]);
+        mbar_init(&bar[1]);
+    }
     __syncthreads();
-    auto issue = [&](int64_t t0) {
-        mbar_expect_tx(bar, tx_bytes);
-        const int x = (int)l.cbase, y = (int)t0;
-        tma_2d(rU, &m.u, bar, x, y);
-        tma_2d(rDT, &m.dt, bar, x, y);
-        if (has_z) tma_2d(rZ, &m.z, bar, x, y);
-        tma_2d(rB, &m.b, bar, 0, y);
-        tma_2d(rC, &m.c, bar, 0, y);
+    auto issue = [&](int64_t t0, int stage) {
+        mbar_expect_tx(&bar[stage], tx_bytes);
+        const int x = (int)cbase, y = (int)t0;
+        tma_2d(raw(stage, 0), &m.u, &bar[stage], x, y);
+        tma_2d(raw(stage, 1), &m.dt, &bar[stage], x, y);
+        if (has_z) tma_2d(raw(stage, 2), &m.z, &bar[stage], x, y);
+        tma_2d(raw(stage, 3), &m.b, &bar[stage], 0, y);
+        tma_2d(raw(stage, 4), &m.c, &bar[stage], 0, y);
     };
-    if (tid == 0 && l.start < l.end) issue(l.start);
+    if (tid == 0 && start < end) issue(start, 0);
 
-    f32x2 A2p[K::NPT / 2], hp[K::NPT / 2];
-    load_state<K>(p, l, A2p, hp);
-    const float dsk = (l.cvalid && p.Dskip) ? __ldg(p.Dskip + l.c0) : 0.f;
-    float dtb[VEC];
+    // recurrence lane: A * log2(e) and the state, two states per register
+    f32x2 A2p[NP], hp[NP];
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) dtb[i] = (l.vvalid && p.dt_bias) ? __ldg(p.dt_bias + l.cg + i) : 0.f;
+    for (int j = 0; j < NPT; j += 2) {
+        const int64_t ai = c0 * kN + sub * NPT + j;
+        const int64_t hi = (seq * p.D + c0) * kN + sub * NPT + j;
+        A2p[j / 2] = cvalid ? pk2(__ldg(p.A + ai) * kLog2e, __ldg(p.A + ai + 1) * kLog2e) : 0ull;
+        hp[j / 2] = (cvalid && p.h0) ? pk2(p.h0[hi], p.h0[hi + 1]) : 0ull;
+    }
+    const int mycol = col4(cl);
+    const int myy = coly<TPC>(cl, sub);
 
-    uint32_t parity = 0;
+    // pre-pass / output lane: one 16-byte channel vector
+    const int cvl = tid % CV;
+    const int64_t cg = cbase + (int64_t)cvl * VEC;
+    const bool vvalid = cg < p.D;
+    float dtb[VEC], dsk[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+        dtb[i] = (vvalid && p.dt_bias) ? __ldg(p.dt_bias + cg + i) : 0.f;
+        dsk[i] = (vvalid && p.Dskip) ? __ldg(p.Dskip + cg + i) : 0.f;
+    }
+    const int vcol = col4(cvl * VEC);
+    const int vy = coly<TPC>(cvl * VEC, 0);
+
     bool failed = false;
-    for (int64_t t0 = l.start; t0 < l.end; t0 += TCH) {
-        const int nt = (int)min((int64_t)TCH, l.end - t0);
-        mbar_wait(bar, parity, failed, &g_scan_status, 1);
-        parity ^= 1u;
+    int k = 0;
+    for (int64_t t0 = start; t0 < end; t0 += TCH, ++k) {
+        const int stage = k & 1;
+        const int nt = (int)min((int64_t)TCH, end - t0);
+        mbar_wait(&bar[stage], (uint32_t)((k >> 1) & 1), failed, &g_scan_status, 1);
+
+        // ---- pre-pass: (delta, delta, delta*u, delta*u) per (token, channel) ----
+        const T *rU = raw(stage, 0), *rDT = raw(stage, 1);
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
+            if (tid + i * THREADS >= K::ITEMS) break;
             const int tl = (tid + i * THREADS) / CV;
-            const int ro = tl * CH + l.cvl * VEC;
-            float fdt[VEC], fu[VEC], fz[VEC];
-            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rDT + ro), fdt);
-            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rU + ro), fu);
-            if (has_z) unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rZ + ro), fz);
-            prepass_item<VEC>(sDX + tl * K::ROW2 + l.vcol, sUG + tl * K::ROW2 + l.vcol,
-                              tl < nt && l.vvalid, fdt, fu, fz, has_z != 0, dtb,
-                              p.delta_softplus);
+            const bool live = tl < nt && vvalid;
+            float fdt[VEC], fu[VEC];
+            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rDT + tl * CH + cvl * VEC), fdt);
+            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rU + tl * CH + cvl * VEC), fu);
+            float4 *dst = sDD + tl * ROWP + vcol;
+#pragma unroll
+            for (int e = 0; e < VEC; e += 2) {
+                float d0 = fdt[e] + dtb[e], d1 = fdt[e + 1] + dtb[e + 1];
+                if (p.delta_softplus) softplus2(d0, d1, d0, d1);
+                d0 = live ? d0 : 0.f;
+                d1 = live ? d1 : 0.f;
+                float x0, x1;
+                upk2(mul2(pk2(d0, d1), pk2(fu[e], fu[e + 1])), x0, x1);
+                dst[e] = make_float4(d0, d0, x0, x0);
+                dst[e + 1] = make_float4(d1, d1, x1, x1);
+            }
         }
-#pragma unroll
-        for (int i = 0; i < K::BPT; ++i) {
-            const int q = tid + i * THREADS;
-            if (q < K::BCN) {
-                const int e0 = q * K::BCVEC;
+        {
+            const T *rB = raw(stage, 3), *rC = raw(stage, 4);
+            for (int q = tid; q < K::BCN; q += THREADS) {
+                const int e0 = q * VEC;
                 const bool live = e0 / kN < nt;
-                float fb[K::BCVEC], fc[K::BCVEC];
-                unpack16<T, K::BCVEC>(*reinterpret_cast<const uint4 *>(rB + e0), fb);
-                unpack16<T, K::BCVEC>(*reinterpret_cast<const uint4 *>(rC + e0), fc);
+                float fb[VEC], fc[VEC];
+                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rB + e0), fb);
+                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rC + e0), fc);
 #pragma unroll
-                for (int e = 0; e < K::BCVEC; ++e) {
-                    sB[e0 + e] = live ? fb[e] : 0.f;
-                    sC[e0 + e] = live ? fc[e] : 0.f;
+                for (int e = 0; e < VEC; e += 4) {
+                    *reinterpret_cast<float4 *>(sB + e0 + e) = live
+                        ? make_float4(fb[e], fb[e + 1], fb[e + 2], fb[e + 3])
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4 *>(sC + e0 + e) = live
+                        ? make_float4(fc[e], fc[e + 1], fc[e + 2], fc[e + 3])
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
             }
         }
         __syncthreads();
-        if (tid == 0 && t0 + TCH < l.end) {
-            // the raw tiles were read through the generic proxy; order those
-            // reads before the next asynchronous-proxy writes into them
+        if (tid == 0 && t0 + TCH < end) {
+            // the other stage was last read by the previous chunk's output pass,
+            // which every thread finished before the barrier above
             fence_proxy_async();
-            issue(t0 + TCH);
+            issue(t0 + TCH, stage ^ 1);
         }
-        const int ntr = ((nt + K::TPC - 1) / K::TPC) * K::TPC;
-        recur_chunk<K>(sDX, sUG, sB, sC, ntr, l.mycol, l.sub, A2p, hp, dsk);
+
+        // ---- recurrence: packed fp32x2, one ex2 per state and token ----
+#pragma unroll 4
+        for (int tq = 0; tq < nt; ++tq) {
+            const float4 v = sDD[tq * ROWP + mycol];
+            const f32x2 dd = pk2(v.x, v.y), xx = pk2(v.z, v.w);
+            f32x2 acc = 0ull;
+#pragma unroll
+            for (int j = 0; j + 1 < NP; j += 2) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(sB + tq * kN + sub * NPT + 2 * j);
+                const float4 c4 = *reinterpret_cast<const float4 *>(sC + tq * kN + sub * NPT + 2 * j);
+                float a0, a1, a2, a3;
+                upk2(mul2(dd, A2p[j]), a0, a1);
+                upk2(mul2(dd, A2p[j + 1]), a2, a3);
+                const f32x2 dA0 = pk2(ex2_approx(a0), ex2_approx(a1));
+                const f32x2 dA1 = pk2(ex2_approx(a2), ex2_approx(a3));
+                hp[j] = fma2(dA0, hp[j], mul2(xx, pk2(b4.x, b4.y)));
+                hp[j + 1] = fma2(dA1, hp[j + 1], mul2(xx, pk2(b4.z, b4.w)));
+                acc = fma2(pk2(c4.x, c4.y), hp[j], acc);
+                acc = fma2(pk2(c4.z, c4.w), hp[j + 1], acc);
+            }
+            if constexpr (NP % 2 == 1) {  // NPT == 2: one pair
+                const float2 b2 = *reinterpret_cast<const float2 *>(sB + tq * kN + sub * NPT);
+                const float2 c2 = *reinterpret_cast<const float2 *>(sC + tq * kN + sub * NPT);
+                float a0, a1;
+                upk2(mul2(dd, A2p[NP - 1]), a0, a1);
+                const f32x2 dA = pk2(ex2_approx(a0), ex2_approx(a1));
+                hp[NP - 1] = fma2(dA, hp[NP - 1], mul2(xx, pk2(b2.x, b2.y)));
+                acc = fma2(pk2(c2.x, c2.y), hp[NP - 1], acc);
+            }
+            float s0, s1;
+            upk2(acc, s0, s1);
+            sYP[tq * ROWY + myy] = s0 + s1;
+        }
         __syncthreads();
-        store_y<K, T>(static_cast<T *>(p.y), sUG, tid, nt, l.vvalid, l.vcol, t0, p.D, l.cg);
+
+        // ---- output: sum the partial readouts, skip, gate, store y ----
+        const T *rU2 = raw(stage, 0), *rZ = raw(stage, 2);
+        T *Y = static_cast<T *>(p.y);
+#pragma unroll
+        for (int i = 0; i < IPT; ++i) {
+            if (tid + i * THREADS >= K::ITEMS) break;
+            const int tl = (tid + i * THREADS) / CV;
+            if (tl < nt && vvalid) {
+                float fu[VEC], fz[VEC], out[VEC];
+                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rU2 + tl * CH + cvl * VEC), fu);
+                if (has_z) unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rZ + tl * CH + cvl * VEC), fz);
+                const float *yp = sYP + tl * ROWY + vy;
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) {
+                    float sum = 0.f;
+                    if constexpr (TPC >= 4) {
+#pragma unroll
+                        for (int q = 0; q < TPC; q += 4) {
+                            const float4 v4 = *reinterpret_cast<const float4 *>(yp + e * TPC + q);
+                            sum += (v4.x + v4.y) + (v4.z + v4.w);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < TPC; ++q) sum += yp[e * TPC + q];
+                    }
+                    out[e] = fmaf(dsk[e], fu[e], sum);
+                }
+                if (has_z) {
+#pragma unroll
+                    for (int e = 0; e < VEC; e += 2) {
+                        float g0, g1;
+                        silu2(fz[e], fz[e + 1], g0, g1);
+                        out[e] *= g0;
+                        out[e + 1] *= g1;
+                    }
+                }
+                store_vec<T, VEC>(Y + (t0 + tl) * p.D + cg, out);
+            }
+        }
+        // next chunk's pre-pass and recurrence rewrite sDD, sB, sC, sYP only
+        // after its first barrier, which follows every thread's output pass
     }
-    save_state<K>(p, l, hp);
+    if (p.h_final && cvalid) {
+#pragma unroll
+        for (int j = 0; j < NPT; j += 2) {
+            float lo, hi;
+            upk2(hp[j / 2], lo, hi);
+            const int64_t o = (seq * p.D + c0) * kN + sub * NPT + j;
+            p.h_final[o] = lo;
+            p.h_final[o + 1] = hi;
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -832,40 +1004,38 @@ order_kernel(const int32_t *__restrict__ cu, int64_t S, int64_t tok, int32_t *__
 // host side
 // ---------------------------------------------------------------------------
 template <class K, typename T>
-cudaError_t run(const Params &p, bool tma, cudaStream_t stream, int *launches)
+cudaError_t run(const Params &p, cudaStream_t stream, int *launches)
 {
     const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
-    if constexpr (K::VEC * sizeof(T) == 16) {
-    if (tma && p.tok > 0) {
-        Maps m;
-        const bool bf = sizeof(T) == 2;
-        bool ok = encode_2d(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
-                  encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
-                  encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
-                  encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
-        if (ok) {
-            if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
-            else m.z = m.u;  // never loaded
-        }
-        if (ok) {
-            cudaError_t e = cudaFuncSetAttribute(scan_tma_kernel<K, T>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)K::SMEM_TMA);
-            if (e != cudaSuccess) return e;
-            scan_tma_kernel<K, T><<<grid, K::THREADS, K::SMEM_TMA, stream>>>(p, m, p.z ? 1 : 0);
-            ++*launches;
-            return cudaGetLastError();
-        }
-        // no tensor-map encoder: fall through to the register-prefetch variant
-    }
-    } else {
-        (void)tma;
-    }
     cudaError_t e = cudaFuncSetAttribute(scan_kernel<K, T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)K::SMEM);
     if (e != cudaSuccess) return e;
     scan_kernel<K, T><<<grid, K::THREADS, K::SMEM, stream>>>(p);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+template <class K, typename T>
+cudaError_t run_tma(const Params &p, cudaStream_t stream, int *launches)
+{
+    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
+    Maps m;
+    const bool bf = sizeof(T) == 2;
+    bool ok = p.tok > 0 && encode_2d(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+              encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+    if (ok) {
+        if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+        else m.z = m.u;  // never loaded
+    }
+    if (!ok) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(scan_tma_kernel<K, T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)K::SMEM);
+    if (e != cudaSuccess) return e;
+    scan_tma_kernel<K, T><<<grid, K::THREADS, K::SMEM, stream>>>(p, m, p.z ? 1 : 0);
     ++*launches;
     return cudaGetLastError();
 }
@@ -904,25 +1074,42 @@ cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n
 {
     if constexpr (VEC == 1) {
         (void)npt; (void)sched;
-        return run<Cfg<T, 4, 0, 32, 64, 1>, T>(p, false, s, n);
+        return run<Cfg<T, 4, 0, 32, 64, 1>, T>(p, s, n);
     } else {
-        // TMA variants use shorter chunks: their raw tiles add shared memory,
-        // and without prefetch registers the CTA count per SM is set by it
         if (sched == 3 && p.tok > 0) {
             cudaError_t e = npt == 2 ? run_ts<TsCfg<T, 2, 4, 8, 8>, T>(p, s, n)
                                      : run_ts<TsCfg<T, 4, 4, 8, 8>, T>(p, s, n);
             if (e != cudaErrorNotSupported) return e;
         }
-        if (sched >= 2) {
-            if (npt == 16) return run<Cfg<T, 16, 0, 128, 16, VEC>, T>(p, true, s, n);
-            if (npt == 8) return run<Cfg<T, 8, 0, 64, 32, VEC>, T>(p, true, s, n);
-            if (npt == 2) return run<Cfg<T, 2, 0, 16, 64, VEC>, T>(p, true, s, n);
-            return run<Cfg<T, 4, 0, 32, 32, VEC>, T>(p, true, s, n);
+        if (sched == 4 || sched == 5) {
+            // one warp per CTA: a CTA barrier costs next to nothing and warps of
+            // different CTAs interleave freely
+            cudaError_t e = cudaErrorNotSupported;
+            if (p.tok > 0) {
+                if (sched == 4) {
+                    if (npt == 16) e = run_tma<TmaCfg<T, 16, 32, 32>, T>(p, s, n);
+                    else if (npt == 8) e = run_tma<TmaCfg<T, 8, 16, 32>, T>(p, s, n);
+                    else e = run_tma<TmaCfg<T, 4, 8, 32>, T>(p, s, n);
+                } else {
+                    if (npt == 16) e = run_tma<TmaCfg<T, 16, 32, 64>, T>(p, s, n);
+                    else if (npt == 8) e = run_tma<TmaCfg<T, 8, 16, 64>, T>(p, s, n);
+                    else e = run_tma<TmaCfg<T, 4, 8, 64>, T>(p, s, n);
+                }
+            }
+            if (e != cudaErrorNotSupported) return e;
         }
-        if (npt == 16) return run<Cfg<T, 16, 0, 128, 32, VEC>, T>(p, false, s, n);
-        if (npt == 8) return run<Cfg<T, 8, 0, 64, 64, VEC>, T>(p, false, s, n);
-        if (npt == 2) return run<Cfg<T, 2, 0, 16, 64, VEC>, T>(p, false, s, n);
-        return run<Cfg<T, 4, 0, 32, 64, VEC>, T>(p, false, s, n);
+        if (sched >= 2 && p.tok > 0) {
+            cudaError_t e = cudaErrorNotSupported;
+            if (npt == 16) e = run_tma<TmaCfg<T, 16, 128, 16>, T>(p, s, n);
+            else if (npt == 8) e = run_tma<TmaCfg<T, 8, 64, 16>, T>(p, s, n);
+            else if (npt == 2) e = run_tma<TmaCfg<T, 2, 16, 32>, T>(p, s, n);
+            else e = run_tma<TmaCfg<T, 4, 32, 16>, T>(p, s, n);
+            if (e != cudaErrorNotSupported) return e;
+        }
+        if (npt == 16) return run<Cfg<T, 16, 0, 128, 32, VEC>, T>(p, s, n);
+        if (npt == 8) return run<Cfg<T, 8, 0, 64, 64, VEC>, T>(p, s, n);
+        if (npt == 2) return run<Cfg<T, 2, 0, 16, 64, VEC>, T>(p, s, n);
+        return run<Cfg<T, 4, 0, 32, 64, VEC>, T>(p, s, n);
     }
 }
 
@@ -942,7 +1129,7 @@ void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
 void set_scan_variant(int npt, int sched)
 {
     g_forced_npt = (npt == 2 || npt == 4 || npt == 8 || npt == 16) ? npt : 0;
-    g_forced_sched = (sched >= 1 && sched <= 3) ? sched : 0;
+    g_forced_sched = (sched >= 1 && sched <= 5) ? sched : 0;
 }
 
 size_t scan_order_bytes(int64_t S) { return (size_t)((S * 4 + 255) / 256) * 256; }
