@@ -85,9 +85,15 @@ unsigned long long ssm_launch_count(void);
  * channel per lane (2, 4, 8 or 16; 16 / value lanes then share a channel) and
  * the schedule (1: next chunk prefetched into registers; 2: tiles staged by
  * TMA; 3: TMA staging with each chunk split in time over four warps, which
- * combine their segments through a carry step; only 2 or 4 states per lane).
- * 0 lets the library choose. Applies to the 16-byte vector path; the scalar
- * path always uses 4 states per lane and register prefetch. Process-wide; not thread-safe against concurrent scan calls.
+ * combine their segments through a carry step, only 2 or 4 states per lane;
+ * 4 and 5: one-warp CTAs with 32- and 64-token chunks; 6: warp-specialised,
+ * helper warps run the per-token work beside the recurrence warps;
+ * 7: one-warp CTAs that each own their channels and stage their own tiles,
+ * 4, 8 or 16 states per lane). 0 lets the library choose. Applies to the
+ * 16-byte vector path; the scalar path always uses 4 states per lane and
+ * register prefetch. A variant whose alignment needs the inputs do not meet
+ * falls back to schedule 2, then 1. Process-wide; not thread-safe against
+ * concurrent scan calls.
  * Returns SSM_OK or SSM_ERR_INVALID_ARGUMENT. Results differ between variants
  * only in the order of the readout sum.
  */

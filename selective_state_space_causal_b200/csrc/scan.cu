@@ -695,6 +695,546 @@ scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
 }
 
 // ---------------------------------------------------------------------------
+// Warp-specialized variant (TMA staging). REC threads run the recurrence; HELP
+// helper threads run, for the same CTA, the per-token pre-pass one chunk ahead
+// and the output pass one chunk behind, so the recurrence warps keep the
+// special-function unit busy while the helpers unpack, softplus, gate and
+// store. The two roles hand chunks over through double-buffered shared
+// arrays and mbarriers; the raw TMA tiles are triple-buffered so each load is
+// issued a full chunk before it is needed. Every wait is bounded.
+//   raw_full[3] : TMA landed           (count 1 + transaction bytes)
+//   dd_full[2]  : pre-pass written     (count HELP)
+//   rec_done[2] : recurrence finished  (count REC; sDD free, sYP written)
+//   out_done[2] : output finished      (count HELP; sYP and the raw stage free)
+// ---------------------------------------------------------------------------
+template <typename T, int NPT_, int CH_, int TCH_, int HELP_>
+struct WsCfg {
+    static constexpr int NPT = NPT_, CH = CH_, TCH = TCH_, HELP = HELP_;
+    static constexpr int TPC = kN / NPT, NP = NPT / 2;
+    static constexpr int REC = CH * TPC;
+    static constexpr int THREADS = REC + HELP;
+    static constexpr int VEC = 16 / sizeof(T);
+    static constexpr int CV = CH / VEC;
+    static constexpr int ITEMS = TCH * CV;
+    static constexpr int IPT = (ITEMS + HELP - 1) / HELP;
+    static constexpr int ROWP = CH + CH / 8;
+    static constexpr int ROWY = CH * TPC + (CH / 8) * 4;
+    static constexpr int BCN = TCH * kN / VEC;
+    static constexpr size_t DD = 16 * (size_t)TCH * ROWP;
+    static constexpr size_t YP = 4 * (size_t)TCH * ROWY;
+    static constexpr size_t BC = 4 * (size_t)TCH * kN;
+    static constexpr size_t RAW_ACT = sizeof(T) * TCH * CH;
+    static constexpr size_t RAW_BC = sizeof(T) * TCH * kN;
+    static constexpr size_t RAWSTAGE = 3 * align128(RAW_ACT) + 2 * align128(RAW_BC);
+    static constexpr size_t OFF_DD = 0;
+    static constexpr size_t OFF_YP = OFF_DD + 2 * align128(DD);
+    static constexpr size_t OFF_B = OFF_YP + 2 * align128(YP);
+    static constexpr size_t OFF_C = OFF_B + 2 * align128(BC);
+    static constexpr size_t OFF_RAW = OFF_C + 2 * align128(BC);
+    static constexpr size_t OFF_BAR = OFF_RAW + 3 * RAWSTAGE;
+    static constexpr size_t SMEM = OFF_BAR + 128;
+    static_assert(NPT % 2 == 0 && CH % 8 == 0, "shape");
+    static_assert(HELP % 32 == 0 && REC % 32 == 0 && THREADS <= 1024, "roles are whole warps");
+    static_assert(HELP % CV == 0, "each helper keeps one channel vector");
+};
+
+__device__ __forceinline__ void mbar_init_n(uint64_t *bar, int count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(saddr(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(saddr(bar)) : "memory");
+}
+
+template <class K, typename T>
+__global__ void __launch_bounds__(K::THREADS)
+scan_ws_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
+{
+    constexpr int NPT = K::NPT, NP = K::NP, TPC = K::TPC, CH = K::CH, TCH = K::TCH;
+    constexpr int VEC = K::VEC, CV = K::CV, IPT = K::IPT, REC = K::REC, HELP = K::HELP;
+    constexpr int ROWP = K::ROWP, ROWY = K::ROWY;
+    extern __shared__ __align__(128) unsigned char smem[];
+    auto sDD = [&](int s) { return reinterpret_cast<float4 *>(smem + K::OFF_DD + s * align128(K::DD)); };
+    auto sYP = [&](int s) { return reinterpret_cast<float *>(smem + K::OFF_YP + s * align128(K::YP)); };
+    auto sB = [&](int s) { return reinterpret_cast<float *>(smem + K::OFF_B + s * align128(K::BC)); };
+    auto sC = [&](int s) { return reinterpret_cast<float *>(smem + K::OFF_C + s * align128(K::BC)); };
+    auto raw = [&](int stage, int which) -> T * {
+        size_t off = K::OFF_RAW + (size_t)stage * K::RAWSTAGE;
+        off += which < 3 ? (size_t)which * align128(K::RAW_ACT)
+                         : 3 * align128(K::RAW_ACT) + (size_t)(which - 3) * align128(K::RAW_BC);
+        return reinterpret_cast<T *>(smem + off);
+    };  // which: 0 u, 1 dt, 2 z, 3 B, 4 C
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+    uint64_t *raw_full = bars, *dd_full = bars + 3, *rec_done = bars + 5, *out_done = bars + 7;
+
+    const int tid = threadIdx.x;
+    const int64_t cbase = (int64_t)blockIdx.x * CH;
+    int64_t seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
+    int64_t start, end;
+    if (p.cu) {
+        start = clamp_off(p.cu[seq], p.tok);
+        end = max(clamp_off(p.cu[seq + 1], p.tok), start);
+    } else {
+        start = seq * p.L;
+        end = start + p.L;
+    }
+    const int nchunks = (int)((end - start + TCH - 1) / TCH);
+
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) mbar_init_n(&raw_full[i], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init_n(&dd_full[i], HELP);
+            mbar_init_n(&rec_done[i], REC);
+            mbar_init_n(&out_done[i], HELP);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    bool failed = false;
+
+    if (tid >= REC) {
+        // ================= helpers: TMA, pre-pass, output =================
+        const int hid = tid - REC;
+        const uint32_t tx_bytes = (uint32_t)((has_z ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
+        auto issue = [&](int j) {
+            const int st = j % 3;
+            mbar_expect_tx(&raw_full[st], tx_bytes);
+            const int x = (int)cbase, y = (int)(start + (int64_t)j * TCH);
+            tma_2d(raw(st, 0), &m.u, &raw_full[st], x, y);
+            tma_2d(raw(st, 1), &m.dt, &raw_full[st], x, y);
+            if (has_z) tma_2d(raw(st, 2), &m.z, &raw_full[st], x, y);
+            tma_2d(raw(st, 3), &m.b, &raw_full[st], 0, y);
+            tma_2d(raw(st, 4), &m.c, &raw_full[st], 0, y);
+        };
+        if (hid == 0)
+            for (int j = 0; j < 3 && j < nchunks; ++j) issue(j);
+
+        const int cvl = hid % CV;
+        const int64_t cg = cbase + (int64_t)cvl * VEC;
+        const bool vvalid = cg < p.D;
+        float dtb[VEC], dsk[VEC];
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) {
+            dtb[i] = (vvalid && p.dt_bias) ? __ldg(p.dt_bias + cg + i) : 0.f;
+            dsk[i] = (vvalid && p.Dskip) ? __ldg(p.Dskip + cg + i) : 0.f;
+        }
+        const int vcol = col4(cvl * VEC);
+        const int vy = coly<TPC>(cvl * VEC, 0);
+        T *Y = static_cast<T *>(p.y);
+
+        auto output = [&](int j) {
+            const int s = j & 1, st = j % 3;
+            const int64_t t0 = start + (int64_t)j * TCH;
+            const int nt = (int)min((int64_t)TCH, end - t0);
+            mbar_wait(&rec_done[s], (uint32_t)((j >> 1) & 1), failed, &g_scan_status, 1);
+            const T *rU = raw(st, 0), *rZ = raw(st, 2);
+            const float *yp0 = sYP(s);
+#pragma unroll
+            for (int i = 0; i < IPT; ++i) {
+                const int it = hid + i * HELP;
+                if (it >= K::ITEMS) break;
+                const int tl = it / CV;
+                if (tl < nt && vvalid) {
+                    float fu[VEC], fz[VEC], out[VEC];
+                    unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rU + tl * CH + cvl * VEC), fu);
+                    if (has_z) unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rZ + tl * CH + cvl * VEC), fz);
+                    const float *yp = yp0 + tl * ROWY + vy;
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) {
+                        float sum = 0.f;
+                        if constexpr (TPC >= 4) {
+#pragma unroll
+                            for (int q = 0; q < TPC; q += 4) {
+                                const float4 v4 = *reinterpret_cast<const float4 *>(yp + e * TPC + q);
+                                sum += (v4.x + v4.y) + (v4.z + v4.w);
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < TPC; ++q) sum += yp[e * TPC + q];
+                        }
+                        out[e] = fmaf(dsk[e], fu[e], sum);
+                    }
+                    if (has_z) {
+#pragma unroll
+                        for (int e = 0; e < VEC; e += 2) {
+                            float g0, g1;
+                            silu2(fz[e], fz[e + 1], g0, g1);
+                            out[e] *= g0;
+                            out[e + 1] *= g1;
+                        }
+                    }
+                    store_vec<T, VEC>(Y + (t0 + tl) * p.D + cg, out);
+                }
+            }
+            mbar_arrive(&out_done[s]);
+            if (hid == 0 && j + 3 < nchunks) {
+                // every helper has finished with raw stage j % 3
+                mbar_wait(&out_done[s], (uint32_t)((j >> 1) & 1), failed, &g_scan_status, 1);
+                fence_proxy_async();
+                issue(j + 3);
+            }
+        };
+
+        for (int k = 0; k < nchunks; ++k) {
+            const int s = k & 1, st = k % 3;
+            const int64_t t0 = start + (int64_t)k * TCH;
+            const int nt = (int)min((int64_t)TCH, end - t0);
+            mbar_wait(&raw_full[st], (uint32_t)((k / 3) & 1), failed, &g_scan_status, 1);
+            // sDD/sB/sC stage s were released by the recurrence of chunk k-2,
+            // which output(k-2) waited for before this iteration
+            const T *rU = raw(st, 0), *rDT = raw(st, 1);
+            float4 *dd = sDD(s);
+#pragma unroll
+            for (int i = 0; i < IPT; ++i) {
+                const int it = hid + i * HELP;
+                if (it >= K::ITEMS) break;
+                const int tl = it / CV;
+                const bool live = tl < nt && vvalid;
+                float fdt[VEC], fu[VEC];
+                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rDT + tl * CH + cvl * VEC), fdt);
+                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rU + tl * CH + cvl * VEC), fu);
+                float4 *dst = dd + tl * ROWP + vcol;
+#pragma unroll
+                for (int e = 0; e < VEC; e += 2) {
+                    float d0 = fdt[e] + dtb[e], d1 = fdt[e + 1] + dtb[e + 1];
+                    if (p.delta_softplus) softplus2(d0, d1, d0, d1);
+                    d0 = live ? d0 : 0.f;
+                    d1 = live ? d1 : 0.f;
+                    float x0, x1;
+                    upk2(mul2(pk2(d0, d1), pk2(fu[e], fu[e + 1])), x0, x1);
+                    dst[e] = make_float4(d0, d0, x0, x0);
+                    dst[e + 1] = make_float4(d1, d1, x1, x1);
+                }
+            }
+            {
+                const T *rB = raw(st, 3), *rC = raw(st, 4);
+                float *b = sB(s), *c = sC(s);
+                for (int q = hid; q < K::BCN; q += HELP) {
+                    const int e0 = q * VEC;
+                    const bool live = e0 / kN < nt;
+                    float fb[VEC], fc[VEC];
+                    unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rB + e0), fb);
+                    unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rC + e0), fc);
+#pragma unroll
+                    for (int e = 0; e < VEC; e += 4) {
+                        *reinterpret_cast<float4 *>(b + e0 + e) = live
+                            ? make_float4(fb[e], fb[e + 1], fb[e + 2], fb[e + 3])
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                        *reinterpret_cast<float4 *>(c + e0 + e) = live
+                            ? make_float4(fc[e], fc[e + 1], fc[e + 2], fc[e + 3])
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                }
+            }
+            mbar_arrive(&dd_full[s]);
+            if (k >= 1) output(k - 1);
+        }
+        if (nchunks >= 1) output(nchunks - 1);
+    } else {
+        // ================= recurrence =================
+        const int cl = tid / TPC, sub = tid % TPC;
+        const int64_t c0 = cbase + cl;
+        const bool cvalid = c0 < p.D;
+        f32x2 A2p[NP], hp[NP];
+#pragma unroll
+        for (int j = 0; j < NPT; j += 2) {
+            const int64_t ai = c0 * kN + sub * NPT + j;
+            const int64_t hi = (seq * p.D + c0) * kN + sub * NPT + j;
+            A2p[j / 2] = cvalid ? pk2(__ldg(p.A + ai) * kLog2e, __ldg(p.A + ai + 1) * kLog2e) : 0ull;
+            hp[j / 2] = (cvalid && p.h0) ? pk2(p.h0[hi], p.h0[hi + 1]) : 0ull;
+        }
+        const int mycol = col4(cl);
+        const int myy = coly<TPC>(cl, sub);
+        for (int k = 0; k < nchunks; ++k) {
+            const int s = k & 1;
+            const int64_t t0 = start + (int64_t)k * TCH;
+            const int nt = (int)min((int64_t)TCH, end - t0);
+            mbar_wait(&dd_full[s], (uint32_t)((k >> 1) & 1), failed, &g_scan_status, 1);
+            if (k >= 2) mbar_wait(&out_done[s], (uint32_t)(((k - 2) >> 1) & 1), failed, &g_scan_status, 1);
+            const float4 *dd = sDD(s);
+            const float *b = sB(s), *c = sC(s);
+            float *yp = sYP(s);
+#pragma unroll 4
+            for (int tq = 0; tq < nt; ++tq) {
+                const float4 v = dd[tq * ROWP + mycol];
+                const f32x2 ddv = pk2(v.x, v.y), xx = pk2(v.z, v.w);
+                f32x2 acc = 0ull;
+#pragma unroll
+                for (int j = 0; j + 1 < NP; j += 2) {
+                    const float4 b4 = *reinterpret_cast<const float4 *>(b + tq * kN + sub * NPT + 2 * j);
+                    const float4 c4 = *reinterpret_cast<const float4 *>(c + tq * kN + sub * NPT + 2 * j);
+                    float a0, a1, a2, a3;
+                    upk2(mul2(ddv, A2p[j]), a0, a1);
+                    upk2(mul2(ddv, A2p[j + 1]), a2, a3);
+                    const f32x2 dA0 = pk2(ex2_approx(a0), ex2_approx(a1));
+                    const f32x2 dA1 = pk2(ex2_approx(a2), ex2_approx(a3));
+                    hp[j] = fma2(dA0, hp[j], mul2(xx, pk2(b4.x, b4.y)));
+                    hp[j + 1] = fma2(dA1, hp[j + 1], mul2(xx, pk2(b4.z, b4.w)));
+                    acc = fma2(pk2(c4.x, c4.y), hp[j], acc);
+                    acc = fma2(pk2(c4.z, c4.w), hp[j + 1], acc);
+                }
+                if constexpr (NP % 2 == 1) {
+                    const float2 b2 = *reinterpret_cast<const float2 *>(b + tq * kN + sub * NPT);
+                    const float2 c2 = *reinterpret_cast<const float2 *>(c + tq * kN + sub * NPT);
+                    float a0, a1;
+                    upk2(mul2(ddv, A2p[NP - 1]), a0, a1);
+                    const f32x2 dA = pk2(ex2_approx(a0), ex2_approx(a1));
+                    hp[NP - 1] = fma2(dA, hp[NP - 1], mul2(xx, pk2(b2.x, b2.y)));
+                    acc = fma2(pk2(c2.x, c2.y), hp[NP - 1], acc);
+                }
+                float s0, s1;
+                upk2(acc, s0, s1);
+                yp[tq * ROWY + myy] = s0 + s1;
+            }
+            mbar_arrive(&rec_done[s]);
+        }
+        if (p.h_final && cvalid) {
+#pragma unroll
+            for (int j = 0; j < NPT; j += 2) {
+                float lo, hi;
+                upk2(hp[j / 2], lo, hi);
+                const int64_t o = (seq * p.D + c0) * kN + sub * NPT + j;
+                p.h_final[o] = lo;
+                p.h_final[o + 1] = hi;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Warp-autonomous variant. A CTA is one warp that owns CPW = 32 / TPC channels
+// of one sequence; nothing is shared between warps, so there is no CTA-wide
+// barrier and the warps of an SM drift into different phases: while some run
+// the exponential-heavy recurrence, others unpack, softplus, gate and store,
+// and the special-function unit stays busy. Per chunk of TCH tokens:
+//   1. TMA has landed the raw u, dt, z (TCH x CPW) and B, C (TCH x 16) tiles
+//      (two stages, issued two chunks ahead by lane 0; bounded mbarrier wait).
+//   2. B and C are widened to fp32; lane (channel, sub) computes delta and
+//      delta*u for tokens sub, sub + TPC, ... of its channel into sDX, and
+//      keeps D*u and silu(z) of those tokens in registers.
+//   3. Recurrence over the chunk (fully unrolled); the lane's partial readout
+//      of each token goes to the raw stage, which is dead by then.
+//   4. The lane that owns a token sums its channel's TPC partials, applies
+//      skip and gate and stores y.
+// ---------------------------------------------------------------------------
+template <typename T, int NPT_, int TCH_>
+struct WarpCfg {
+    static constexpr int NPT = NPT_, TCH = TCH_;
+    static constexpr int TPC = kN / NPT;            // lanes per channel
+    static constexpr int CPW = 32 / TPC;            // channels per warp
+    static constexpr int TPL = TCH / TPC;           // tokens per lane in steps 2 and 4
+    static constexpr int VEC = 16 / sizeof(T);
+    static constexpr size_t RAW_ACT = sizeof(T) * TCH * CPW;
+    static constexpr size_t RAW_BC = sizeof(T) * TCH * kN;
+    static constexpr size_t RAW = 3 * align128(RAW_ACT) + 2 * align128(RAW_BC);
+    static constexpr size_t YP = sizeof(float) * TCH * 32;
+    static constexpr size_t STAGE = align128(RAW > YP ? RAW : YP);
+    static constexpr size_t OFF_B = 2 * STAGE;
+    static constexpr size_t OFF_C = OFF_B + align128(sizeof(float) * TCH * kN);
+    static constexpr size_t OFF_DX = OFF_C + align128(sizeof(float) * TCH * kN);
+    static constexpr size_t OFF_BAR = OFF_DX + align128(sizeof(float2) * TCH * CPW);
+    static constexpr size_t SMEM = OFF_BAR + 16;
+    static_assert(NPT % 4 == 0, "states are read four at a time");
+    static_assert(TPL % 2 == 0, "per-token work goes in packed pairs");
+    static_assert((CPW * sizeof(T)) % 16 == 0, "TMA rows are whole 16-byte pieces");
+    static_assert((TCH * kN) % VEC == 0, "B and C tiles are whole 16-byte pieces");
+};
+
+template <class K, typename T>
+__global__ void __launch_bounds__(32)
+scan_warp_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
+{
+    constexpr int NPT = K::NPT, TPC = K::TPC, CPW = K::CPW, TCH = K::TCH, TPL = K::TPL;
+    constexpr int VEC = K::VEC;
+    extern __shared__ __align__(128) unsigned char smem[];
+    float *sB = reinterpret_cast<float *>(smem + K::OFF_B);
+    float *sC = reinterpret_cast<float *>(smem + K::OFF_C);
+    float2 *sDX = reinterpret_cast<float2 *>(smem + K::OFF_DX);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+    auto raw = [&](int st, int which) -> T * {
+        size_t off = (size_t)st * K::STAGE;
+        off += which < 3 ? (size_t)which * align128(K::RAW_ACT)
+                         : 3 * align128(K::RAW_ACT) + (size_t)(which - 3) * align128(K::RAW_BC);
+        return reinterpret_cast<T *>(smem + off);
+    };  // which: 0 u, 1 dt, 2 z, 3 B, 4 C
+
+    const int lane = threadIdx.x;
+    const int cl = lane / TPC, sub = lane % TPC;
+    const int64_t cbase = (int64_t)blockIdx.x * CPW;
+    const int64_t c = cbase + cl;
+    const bool cvalid = c < p.D;
+    int64_t seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
+    int64_t start, end;
+    if (p.cu) {
+        start = clamp_off(p.cu[seq], p.tok);
+        end = max(clamp_off(p.cu[seq + 1], p.tok), start);
+    } else {
+        start = seq * p.L;
+        end = start + p.L;
+    }
+    const int nchunks = (int)((end - start + TCH - 1) / TCH);
+
+    if (lane == 0) {
+        mbar_init_n(&bar[0], 1);
+        mbar_init_n(&bar[1], 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    const uint32_t tx_bytes = (uint32_t)((has_z ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
+    auto issue = [&](int j) {
+        const int st = j & 1;
+        mbar_expect_tx(&bar[st], tx_bytes);
+        const int x = (int)cbase, y = (int)(start + (int64_t)j * TCH);
+        tma_2d(raw(st, 0), &m.u, &bar[st], x, y);
+        tma_2d(raw(st, 1), &m.dt, &bar[st], x, y);
+        if (has_z) tma_2d(raw(st, 2), &m.z, &bar[st], x, y);
+        tma_2d(raw(st, 3), &m.b, &bar[st], 0, y);
+        tma_2d(raw(st, 4), &m.c, &bar[st], 0, y);
+    };
+    if (lane == 0) {
+        if (nchunks > 0) issue(0);
+        if (nchunks > 1) issue(1);
+    }
+
+    f32x2 A2p[NPT / 2], hp[NPT / 2];
+#pragma unroll
+    for (int j = 0; j < NPT; j += 4) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), h = a;
+        if (cvalid) {
+            a = __ldg(reinterpret_cast<const float4 *>(p.A + c * kN + sub * NPT + j));
+            if (p.h0) h = *reinterpret_cast<const float4 *>(p.h0 + (seq * p.D + c) * kN + sub * NPT + j);
+        }
+        A2p[j / 2] = pk2(a.x * kLog2e, a.y * kLog2e);
+        A2p[j / 2 + 1] = pk2(a.z * kLog2e, a.w * kLog2e);
+        hp[j / 2] = pk2(h.x, h.y);
+        hp[j / 2 + 1] = pk2(h.z, h.w);
+    }
+    const float dtb = (cvalid && p.dt_bias) ? __ldg(p.dt_bias + c) : 0.f;
+    const float dsk = (cvalid && p.Dskip) ? __ldg(p.Dskip + c) : 0.f;
+    T *Y = static_cast<T *>(p.y);
+
+    bool failed = false;
+    for (int k = 0; k < nchunks; ++k) {
+        const int st = k & 1;
+        const int64_t t0 = start + (int64_t)k * TCH;
+        const int nt = (int)min((int64_t)TCH, end - t0);
+        mbar_wait(&bar[st], (uint32_t)((k >> 1) & 1), failed, &g_scan_status, 1);
+
+        // ---- step 2: widen B, C; delta, delta*u, D*u, silu(z) of this lane's tokens ----
+        {
+            const T *rB = raw(st, 3), *rC = raw(st, 4);
+#pragma unroll
+            for (int q = lane; q < TCH * kN / VEC; q += 32) {
+                float fb[VEC], fc[VEC];
+                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rB + q * VEC), fb);
+                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rC + q * VEC), fc);
+#pragma unroll
+                for (int e = 0; e < VEC; e += 4) {
+                    *reinterpret_cast<float4 *>(sB + q * VEC + e) =
+                        make_float4(fb[e], fb[e + 1], fb[e + 2], fb[e + 3]);
+                    *reinterpret_cast<float4 *>(sC + q * VEC + e) =
+                        make_float4(fc[e], fc[e + 1], fc[e + 2], fc[e + 3]);
+                }
+            }
+        }
+        float skip[TPL], gate[TPL];
+        {
+            const T *rU = raw(st, 0), *rDT = raw(st, 1), *rZ = raw(st, 2);
+#pragma unroll
+            for (int i = 0; i < TPL; i += 2) {
+                const int ta = sub + TPC * i, tb = ta + TPC;
+                float da = to_f32(rDT[ta * CPW + cl]) + dtb, db = to_f32(rDT[tb * CPW + cl]) + dtb;
+                if (p.delta_softplus) softplus2(da, db, da, db);
+                const float ua = to_f32(rU[ta * CPW + cl]), ub = to_f32(rU[tb * CPW + cl]);
+                float xa, xb;
+                upk2(mul2(pk2(da, db), pk2(ua, ub)), xa, xb);
+                sDX[ta * CPW + cl] = make_float2(da, xa);
+                sDX[tb * CPW + cl] = make_float2(db, xb);
+                skip[i] = dsk * ua;
+                skip[i + 1] = dsk * ub;
+                if (has_z) {
+                    silu2(to_f32(rZ[ta * CPW + cl]), to_f32(rZ[tb * CPW + cl]), gate[i], gate[i + 1]);
+                } else {
+                    gate[i] = gate[i + 1] = 1.f;
+                }
+            }
+        }
+        __syncwarp();
+
+        // ---- step 3: recurrence; partial readouts into the (now dead) raw stage ----
+        float *sYP = reinterpret_cast<float *>(smem + (size_t)st * K::STAGE);
+#pragma unroll
+        for (int t = 0; t < TCH; ++t) {
+            if (t >= nt) break;
+            const float2 v = sDX[t * CPW + cl];
+            const f32x2 dd = pk2(v.x, v.x), xx = pk2(v.y, v.y);
+            f32x2 acc = 0ull;
+#pragma unroll
+            for (int q = 0; q < NPT / 4; ++q) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(sB + t * kN + sub * NPT + 4 * q);
+                const float4 c4 = *reinterpret_cast<const float4 *>(sC + t * kN + sub * NPT + 4 * q);
+                float a0, a1, a2, a3;
+                upk2(mul2(dd, A2p[2 * q]), a0, a1);
+                upk2(mul2(dd, A2p[2 * q + 1]), a2, a3);
+                const f32x2 dA0 = pk2(ex2_approx(a0), ex2_approx(a1));
+                const f32x2 dA1 = pk2(ex2_approx(a2), ex2_approx(a3));
+                hp[2 * q] = fma2(dA0, hp[2 * q], mul2(xx, pk2(b4.x, b4.y)));
+                hp[2 * q + 1] = fma2(dA1, hp[2 * q + 1], mul2(xx, pk2(b4.z, b4.w)));
+                acc = fma2(pk2(c4.x, c4.y), hp[2 * q], acc);
+                acc = fma2(pk2(c4.z, c4.w), hp[2 * q + 1], acc);
+            }
+            float s0, s1;
+            upk2(acc, s0, s1);
+            sYP[t * 32 + lane] = s0 + s1;
+        }
+        __syncwarp();
+
+        // ---- step 4: sum partials, skip, gate, store ----
+#pragma unroll
+        for (int i = 0; i < TPL; ++i) {
+            const int t = sub + TPC * i;
+            if (t < nt && cvalid) {
+                const float *yp = sYP + t * 32 + cl * TPC;
+                float sum = 0.f;
+                if constexpr (TPC >= 4) {
+#pragma unroll
+                    for (int q = 0; q < TPC; q += 4) {
+                        const float4 v4 = *reinterpret_cast<const float4 *>(yp + q);
+                        sum += (v4.x + v4.y) + (v4.z + v4.w);
+                    }
+                } else if constexpr (TPC == 2) {
+                    const float2 v2 = *reinterpret_cast<const float2 *>(yp);
+                    sum = v2.x + v2.y;
+                } else {
+                    sum = yp[0];
+                }
+                Y[(t0 + t) * p.D + c] = from_f32<T>((sum + skip[i]) * gate[i]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0 && k + 2 < nchunks) {
+            // every lane's reads of this stage (raw tiles, then partials) are done
+            fence_proxy_async();
+            issue(k + 2);
+        }
+    }
+    if (p.h_final && cvalid) {
+        float *hf = p.h_final + (seq * p.D + c) * kN + sub * NPT;
+#pragma unroll
+        for (int j = 0; j < NPT; j += 4) {
+            float x0, x1, x2, x3;
+            upk2(hp[j / 2], x0, x1);
+            upk2(hp[j / 2 + 1], x2, x3);
+            *reinterpret_cast<float4 *>(hf + j) = make_float4(x0, x1, x2, x3);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Variant 3: time-split chunks (TMA staging). A chunk of SEG x TS tokens is
 // cut into SEG segments handled by different warps, which multiplies the
 // warps available to sequences x channels pairs that are too few to fill the
@@ -1041,6 +1581,58 @@ cudaError_t run_tma(const Params &p, cudaStream_t stream, int *launches)
 }
 
 template <class K, typename T>
+cudaError_t run_ws(const Params &p, cudaStream_t stream, int *launches)
+{
+    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
+    Maps m;
+    const bool bf = sizeof(T) == 2;
+    bool ok = p.tok > 0 && encode_2d(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+              encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+    if (ok) {
+        if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+        else m.z = m.u;  // never loaded
+    }
+    if (!ok) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(scan_ws_kernel<K, T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)K::SMEM);
+    if (e != cudaSuccess) return e;
+    scan_ws_kernel<K, T><<<grid, K::THREADS, K::SMEM, stream>>>(p, m, p.z ? 1 : 0);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+template <class K, typename T>
+cudaError_t run_warp(const Params &p, cudaStream_t stream, int *launches)
+{
+    const dim3 grid((unsigned)((p.D + K::CPW - 1) / K::CPW), (unsigned)p.S);
+    Maps m;
+    const bool bf = sizeof(T) == 2;
+    const bool aligned = ((uintptr_t)p.A % 16 == 0) &&
+                         (!p.h0 || (uintptr_t)p.h0 % 16 == 0) &&
+                         (!p.h_final || (uintptr_t)p.h_final % 16 == 0);
+    bool ok = aligned && p.tok > 0 &&
+              encode_2d(&m.u, p.u, bf, p.D, p.tok, K::CPW, K::TCH) &&
+              encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CPW, K::TCH) &&
+              encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+              encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+    if (ok) {
+        if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CPW, K::TCH);
+        else m.z = m.u;  // never loaded
+    }
+    if (!ok) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(scan_warp_kernel<K, T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)K::SMEM);
+    if (e != cudaSuccess) return e;
+    scan_warp_kernel<K, T><<<grid, 32, K::SMEM, stream>>>(p, m, p.z ? 1 : 0);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+template <class K, typename T>
 cudaError_t run_ts(const Params &p, cudaStream_t stream, int *launches)
 {
     const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
@@ -1079,6 +1671,21 @@ cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n
         if (sched == 3 && p.tok > 0) {
             cudaError_t e = npt == 2 ? run_ts<TsCfg<T, 2, 4, 8, 8>, T>(p, s, n)
                                      : run_ts<TsCfg<T, 4, 4, 8, 8>, T>(p, s, n);
+            if (e != cudaErrorNotSupported) return e;
+        }
+        if (sched == 6 && p.tok > 0) {
+            cudaError_t e;
+            if (npt == 16) e = run_ws<WsCfg<T, 16, 64, 8, 64>, T>(p, s, n);
+            else if (npt == 8) e = run_ws<WsCfg<T, 8, 64, 8, 64>, T>(p, s, n);
+            else if (npt == 2) e = run_ws<WsCfg<T, 2, 16, 16, 64>, T>(p, s, n);
+            else e = run_ws<WsCfg<T, 4, 32, 16, 64>, T>(p, s, n);
+            if (e != cudaErrorNotSupported) return e;
+        }
+        if (sched == 7 && p.tok > 0) {
+            cudaError_t e;
+            if (npt == 16) e = run_warp<WarpCfg<T, 16, 16>, T>(p, s, n);
+            else if (npt == 8) e = run_warp<WarpCfg<T, 8, 16>, T>(p, s, n);
+            else e = run_warp<WarpCfg<T, 4, 16>, T>(p, s, n);
             if (e != cudaErrorNotSupported) return e;
         }
         if (sched == 4 || sched == 5) {
@@ -1129,7 +1736,7 @@ void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
 void set_scan_variant(int npt, int sched)
 {
     g_forced_npt = (npt == 2 || npt == 4 || npt == 8 || npt == 16) ? npt : 0;
-    g_forced_sched = (sched >= 1 && sched <= 5) ? sched : 0;
+    g_forced_sched = (sched >= 1 && sched <= 7) ? sched : 0;
 }
 
 size_t scan_order_bytes(int64_t S) { return (size_t)((S * 4 + 255) / 256) * 256; }

@@ -12,9 +12,11 @@
 
 namespace ssm {
 
-// Non-blocking polls before a wait gives up (about 0.2 s with the back-off;
-// a tile normally lands within microseconds).
-constexpr unsigned kTmaSpinLimit = 1u << 21;
+// Bounded waits: each try suspends the thread in hardware until the phase
+// completes or about kSuspendNs nanoseconds pass, so a waiting warp takes no
+// issue slots; after kWaitTries tries (about half a second) the wait gives up.
+constexpr unsigned kWaitTries = 1u << 17;
+constexpr uint32_t kSuspendNs = 4096;
 
 __device__ __forceinline__ uint32_t saddr(const void *p)
 {
@@ -50,21 +52,20 @@ __device__ __forceinline__ void fence_proxy_async()
 }
 
 // Waits for phase `parity` of the barrier with a bounded number of
-// non-blocking polls. On timeout it sets bit `code` of *status and marks
+// suspending tries. On timeout it sets bit `code` of *status and marks
 // `failed`, after which this thread no longer waits at all, so a kernel
 // always terminates.
 __device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &failed,
                                           int *status, int code)
 {
     if (failed) return;
-    for (unsigned i = 0; i < kTmaSpinLimit; ++i) {
+    for (unsigned i = 0; i < kWaitTries; ++i) {
         uint32_t done;
         asm volatile(
-            "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
             " selp.u32 %0, 1, 0, p;\n}\n"
-            : "=r"(done) : "r"(saddr(bar)), "r"(parity) : "memory");
+            : "=r"(done) : "r"(saddr(bar)), "r"(parity), "r"(kSuspendNs) : "memory");
         if (done) return;
-        if (i >= 32) __nanosleep(64);
     }
     failed = true;
     atomicOr(status, code);
