@@ -42,6 +42,10 @@ N_STATE = 16
 SMS = 148
 MUFU_PER_CLK_PER_SM = 16  # ex2 results per clock per SM (special-function unit)
 FALLBACK_HBM_GBS = 6650.0
+# kernel that each scan schedule launches (ssm_set_scan_variant numbering)
+SCAN_KERNELS = {1: "scan_kernel", 2: "scan_tma_kernel", 3: "scan_ts_kernel", 4: "scan_tma_kernel",
+                5: "scan_tma_kernel", 6: "scan_ws_kernel", 7: "scan_warp_kernel",
+                8: "scan_staged_kernel"}
 
 
 # ---------------------------------------------------------------------------
@@ -273,8 +277,11 @@ def bench_headline(args, world, peaks, rank_dev):
     mufu = mufu_peak_gexp(peaks["sm_max_mhz"])
     achieved = st.scan_exps() / (scan_ms * 1e-3) / 1e9
     sha = source_sha("scan.cu", "common.cuh")
-    traffic = recorded_traffic("scan_kernel", sha)
-    roofline = {"kernel": "scan_kernel (scan_tma_kernel)", "bound": "alu", "unit": "Gexp/s",
+    npt, sched = st.ssm.ssm_scan_variant_for(st.Bn, st.D)
+    kernel = SCAN_KERNELS.get(sched, "scan_tma_kernel")
+    traffic = recorded_traffic(kernel, sha)
+    roofline = {"kernel": kernel, "variant": {"states_per_lane": npt, "schedule": sched},
+                "bound": "alu", "unit": "Gexp/s",
                 "achieved": round(achieved, 1), "peak": round(mufu, 1),
                 "frac": round(achieved / mufu, 4), "traffic": traffic,
                 "kernel_ms": round(scan_ms, 5),

@@ -89,7 +89,8 @@ unsigned long long ssm_launch_count(void);
  * 4 and 5: one-warp CTAs with 32- and 64-token chunks; 6: warp-specialised,
  * helper warps run the per-token work beside the recurrence warps;
  * 7: one-warp CTAs that each own their channels and stage their own tiles,
- * 4, 8 or 16 states per lane). 0 lets the library choose. Applies to the
+ * 4, 8 or 16 states per lane; 8: the layout of schedule 1 with TMA staging).
+ * 0 lets the library choose. Applies to the
  * 16-byte vector path; the scalar path always uses 4 states per lane and
  * register prefetch. A variant whose alignment needs the inputs do not meet
  * falls back to schedule 2, then 1. Process-wide; not thread-safe against
@@ -98,6 +99,19 @@ unsigned long long ssm_launch_count(void);
  * only in the order of the readout sum.
  */
 int ssm_set_scan_variant(int states_per_lane, int schedule);
+
+/*
+ * Reports the kernel variant ssm_selective_scan_fwd picks on its 16-byte
+ * vector path for S sequences of D channels on the current device: states
+ * per lane and schedule, as ssm_set_scan_variant names them (a forced
+ * variant is reported as forced). A variant whose alignment needs the
+ * inputs do not meet still falls back at call time. Host-only; launches
+ * nothing. The writes to *states_per_lane and *schedule are the only
+ * effects. Returns SSM_OK, or SSM_ERR_INVALID_ARGUMENT for S < 1, D < 1 or
+ * a NULL pointer. An introspection call of this library; the method has no
+ * counterpart.
+ */
+int ssm_scan_variant_for(int64_t S, int64_t D, int *states_per_lane, int *schedule);
 
 /*
  * Device-side status of the library's kernels on the current device: 0 while

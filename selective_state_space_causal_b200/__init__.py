@@ -19,6 +19,7 @@ from ._lib import (  # noqa: F401
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_noalloc,
     ssm_selective_state_update,
+    ssm_scan_variant_for,
     ssm_set_scan_variant,
     ssm_version,
 )

@@ -27,6 +27,7 @@ SIGNATURES = [
     ("ssm_version", _int, []),
     ("ssm_launch_count", ctypes.c_ulonglong, []),
     ("ssm_set_scan_variant", _int, [_int, _int]),
+    ("ssm_scan_variant_for", _int, [_i64, _i64, ctypes.POINTER(_int), ctypes.POINTER(_int)]),
     ("ssm_device_status", _int, [_int]),
     ("ssm_check_cu_seqlens", _int, [_vp, _i64, _i64]),
     ("ssm_causal_conv1d", _int, [_vp, _vp, _vp, _vp, _i64, _i64, _int, _vp, _i64, _vp, _vp, _int,
@@ -109,6 +110,13 @@ def ssm_launch_count() -> int:
 
 def ssm_set_scan_variant(states_per_lane: int, schedule: int = 0) -> None:
     _check(lib.ssm_set_scan_variant(int(states_per_lane), int(schedule)))
+
+
+def ssm_scan_variant_for(S: int, D: int) -> tuple[int, int]:
+    """(states per lane, schedule) the scan picks for S sequences of D channels."""
+    npt, sched = _int(0), _int(0)
+    _check(lib.ssm_scan_variant_for(int(S), int(D), ctypes.byref(npt), ctypes.byref(sched)))
+    return npt.value, sched.value
 
 
 def ssm_device_status(clear: bool = False) -> int:

@@ -15,6 +15,7 @@
 
 namespace ssm {
 void set_scan_variant(int npt, int sched);
+void scan_variant_for(int64_t S, int64_t D, int *npt, int *sched);
 size_t scan_order_bytes(int64_t S);
 int read_scan_status(bool clear);
 int read_conv_status(bool clear);
@@ -90,11 +91,20 @@ unsigned long long ssm_launch_count(void) { return g_launches.load(std::memory_o
 int ssm_set_scan_variant(int npt, int sched)
 {
     const bool npt_ok = npt == 0 || npt == 2 || npt == 4 || npt == 8 || npt == 16;
-    const bool sched_ok = sched >= 0 && sched <= 7;
+    const bool sched_ok = sched >= 0 && sched <= 8;
     if (!npt_ok || !sched_ok)
         return fail(SSM_ERR_INVALID_ARGUMENT,
-                    "ssm_set_scan_variant: states per lane 0, 2, 4, 8 or 16; schedule 0..7");
+                    "ssm_set_scan_variant: states per lane 0, 2, 4, 8 or 16; schedule 0..8");
     ssm::set_scan_variant(npt, sched);
+    return ok();
+}
+
+int ssm_scan_variant_for(int64_t S, int64_t D, int *states_per_lane, int *schedule)
+{
+    if (S < 1 || D < 1 || !states_per_lane || !schedule)
+        return fail(SSM_ERR_INVALID_ARGUMENT,
+                    "ssm_scan_variant_for: S >= 1, D >= 1 and two output pointers required");
+    ssm::scan_variant_for(S, D, states_per_lane, schedule);
     return ok();
 }
 

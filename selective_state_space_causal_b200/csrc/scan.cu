@@ -31,6 +31,7 @@
 // * Tokens past a sequence's end are padded with delta = 0 (dA = 1, no input),
 //   which leaves h unchanged, so the inner loop needs no tail branch.
 // * Packed sequences are scheduled longest-first when scratch is supplied.
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -431,6 +432,105 @@ struct Maps {
     CUtensorMap u, dt, z, b, c;
 };
 
+// ---------------------------------------------------------------------------
+// Schedule 8: the layout and readout of schedule 1 (per-token float2 arrays,
+// shuffle-butterfly readout into the gate slot) with the raw tiles brought in
+// by TMA instead of register prefetch: one stage, issued as soon as the
+// pre-pass has read the previous one. Fewest registers of the staged kernels,
+// which suits shapes with few (sequence, channel) pairs.
+// ---------------------------------------------------------------------------
+template <class K, typename T>
+__global__ void __launch_bounds__(K::THREADS)
+scan_staged_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
+{
+    constexpr int VEC = K::VEC, IPT = K::IPT, THREADS = K::THREADS, CV = K::CV, TCH = K::TCH;
+    constexpr int CH = K::CH;
+    extern __shared__ __align__(128) unsigned char smem[];
+    float2 *sDX = reinterpret_cast<float2 *>(smem + K::OFF_DX);
+    float2 *sUG = reinterpret_cast<float2 *>(smem + K::OFF_UG);
+    float *sB = reinterpret_cast<float *>(smem + K::OFF_B);
+    float *sC = reinterpret_cast<float *>(smem + K::OFF_C);
+    T *rU = reinterpret_cast<T *>(smem + K::OFF_RU);
+    T *rDT = reinterpret_cast<T *>(smem + K::OFF_RDT);
+    T *rZ = reinterpret_cast<T *>(smem + K::OFF_RZ);
+    T *rB = reinterpret_cast<T *>(smem + K::OFF_RB);
+    T *rC = reinterpret_cast<T *>(smem + K::OFF_RC);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+
+    const int tid = threadIdx.x;
+    const Lane l = lane_setup<K>(p);
+    const uint32_t tx_bytes = (uint32_t)((has_z ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
+
+    if (tid == 0) mbar_init(bar);
+    __syncthreads();
+    auto issue = [&](int64_t t0) {
+        mbar_expect_tx(bar, tx_bytes);
+        const int x = (int)l.cbase, y = (int)t0;
+        tma_2d(rU, &m.u, bar, x, y);
+        tma_2d(rDT, &m.dt, bar, x, y);
+        if (has_z) tma_2d(rZ, &m.z, bar, x, y);
+        tma_2d(rB, &m.b, bar, 0, y);
+        tma_2d(rC, &m.c, bar, 0, y);
+    };
+    if (tid == 0 && l.start < l.end) issue(l.start);
+
+    f32x2 A2p[K::NPT / 2], hp[K::NPT / 2];
+    load_state<K>(p, l, A2p, hp);
+    const float dsk = (l.cvalid && p.Dskip) ? __ldg(p.Dskip + l.c0) : 0.f;
+    float dtb[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) dtb[i] = (l.vvalid && p.dt_bias) ? __ldg(p.dt_bias + l.cg + i) : 0.f;
+
+    uint32_t parity = 0;
+    bool failed = false;
+    for (int64_t t0 = l.start; t0 < l.end; t0 += TCH) {
+        const int nt = (int)min((int64_t)TCH, l.end - t0);
+        mbar_wait(bar, parity, failed, &g_scan_status, 1);
+        parity ^= 1u;
+#pragma unroll
+        for (int i = 0; i < IPT; ++i) {
+            const int tl = (tid + i * THREADS) / CV;
+            const int ro = tl * CH + l.cvl * VEC;
+            float fdt[VEC], fu[VEC], fz[VEC];
+            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rDT + ro), fdt);
+            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rU + ro), fu);
+            if (has_z) unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(rZ + ro), fz);
+            prepass_item<VEC>(sDX + tl * K::ROW2 + l.vcol, sUG + tl * K::ROW2 + l.vcol,
+                              tl < nt && l.vvalid, fdt, fu, fz, has_z != 0, dtb,
+                              p.delta_softplus);
+        }
+#pragma unroll
+        for (int i = 0; i < K::BPT; ++i) {
+            const int q = tid + i * THREADS;
+            if (q < K::BCN) {
+                const int e0 = q * K::BCVEC;
+                const bool live = e0 / kN < nt;
+                float fb[K::BCVEC], fc[K::BCVEC];
+                unpack16<T, K::BCVEC>(*reinterpret_cast<const uint4 *>(rB + e0), fb);
+                unpack16<T, K::BCVEC>(*reinterpret_cast<const uint4 *>(rC + e0), fc);
+#pragma unroll
+                for (int e = 0; e < K::BCVEC; ++e) {
+                    sB[e0 + e] = live ? fb[e] : 0.f;
+                    sC[e0 + e] = live ? fc[e] : 0.f;
+                }
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && t0 + TCH < l.end) {
+            // the raw tiles were read through the generic proxy; order those
+            // reads before the next asynchronous-proxy writes into them
+            fence_proxy_async();
+            issue(t0 + TCH);
+        }
+        const int ntr = ((nt + K::TPC - 1) / K::TPC) * K::TPC;
+        recur_chunk<K>(sDX, sUG, sB, sC, ntr, l.mycol, l.sub, A2p, hp, dsk);
+        __syncthreads();
+        store_y<K, T>(static_cast<T *>(p.y), sUG, tid, nt, l.vvalid, l.vcol, t0, p.D, l.cg);
+    }
+    save_state<K>(p, l, hp);
+}
+
+
 // Shapes of the TMA-staged kernel. Per (token, channel) shared memory holds
 // (delta, delta, delta*u, delta*u) as one float4, so a lane gets both packed
 // operands of its recurrence from one 16-byte load, and TPC partial readouts.
@@ -606,8 +706,7 @@ scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
         }
 
         // ---- recurrence: packed fp32x2, one ex2 per state and token ----
-#pragma unroll 4
-        for (int tq = 0; tq < nt; ++tq) {
+        auto step = [&](const int tq) {
             const float4 v = sDD[tq * ROWP + mycol];
             const f32x2 dd = pk2(v.x, v.y), xx = pk2(v.z, v.w);
             f32x2 acc = 0ull;
@@ -637,6 +736,15 @@ scan_tma_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
             float s0, s1;
             upk2(acc, s0, s1);
             sYP[tq * ROWY + myy] = s0 + s1;
+        };
+        // full chunks run fully unrolled, so every shared-memory offset is an
+        // immediate; only a sequence's ragged last chunk takes the plain loop
+        if (nt == TCH) {
+#pragma unroll
+            for (int tq = 0; tq < TCH; ++tq) step(tq);
+        } else {
+#pragma unroll 1
+            for (int tq = 0; tq < nt; ++tq) step(tq);
         }
         __syncthreads();
 
@@ -1581,6 +1689,30 @@ cudaError_t run_tma(const Params &p, cudaStream_t stream, int *launches)
 }
 
 template <class K, typename T>
+cudaError_t run_staged(const Params &p, cudaStream_t stream, int *launches)
+{
+    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
+    Maps m;
+    const bool bf = sizeof(T) == 2;
+    bool ok = p.tok > 0 && encode_2d(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+              encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+    if (ok) {
+        if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+        else m.z = m.u;  // never loaded
+    }
+    if (!ok) return cudaErrorNotSupported;
+    cudaError_t e = cudaFuncSetAttribute(scan_staged_kernel<K, T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)K::SMEM_TMA);
+    if (e != cudaSuccess) return e;
+    scan_staged_kernel<K, T><<<grid, K::THREADS, K::SMEM_TMA, stream>>>(p, m, p.z ? 1 : 0);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+template <class K, typename T>
 cudaError_t run_ws(const Params &p, cudaStream_t stream, int *launches)
 {
     const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
@@ -1681,6 +1813,14 @@ cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n
             else e = run_ws<WsCfg<T, 4, 32, 16, 64>, T>(p, s, n);
             if (e != cudaErrorNotSupported) return e;
         }
+        if (sched == 8 && p.tok > 0) {
+            cudaError_t e;
+            if (npt == 16) e = run_staged<Cfg<T, 16, 0, 128, 16, VEC>, T>(p, s, n);
+            else if (npt == 8) e = run_staged<Cfg<T, 8, 0, 64, 32, VEC>, T>(p, s, n);
+            else if (npt == 2) e = run_staged<Cfg<T, 2, 0, 16, 64, VEC>, T>(p, s, n);
+            else e = run_staged<Cfg<T, 4, 0, 32, 32, VEC>, T>(p, s, n);
+            if (e != cudaErrorNotSupported) return e;
+        }
         if (sched == 7 && p.tok > 0) {
             cudaError_t e;
             if (npt == 16) e = run_warp<WarpCfg<T, 16, 16>, T>(p, s, n);
@@ -1720,23 +1860,58 @@ cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n
     }
 }
 
-// Measured on B200: with few (sequence, channel) pairs, splitting a channel's
-// states over more lanes wins (more warps); with many, fewer lanes per channel
-// win (fewer instructions per exponential). TMA staging throughout.
+// SM count of the current device, looked up once per device.
+int sm_count()
+{
+    static std::atomic<int> cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < 64) {
+        const int v = cache[dev].load(std::memory_order_relaxed);
+        if (v > 0) return v;
+    }
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+        n = 148;
+    if (dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
+}
+
+// Measured on B200 (exponential rate against the special-function peak):
+// 8 states per lane with double-buffered TMA staging has the fewest
+// instructions per exponential and wins once the GPU holds about 20 warps per
+// SM of it (packed 65536 x 5120: 0.60 against 0.53 for the next best); below
+// that, latency decides and thinner lanes win: 2 states per lane in the
+// single-stage layout of schedule 8 (8 x 2048 x 1536: 0.345 against 0.33 for 4
+// states with register prefetch; 1 x 8192 x 8192: 0.33 against 0.31), with 4
+// states per lane in between.
 void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
 {
-    const int64_t pairs = S * D;
-    const int npt_auto = pairs < (1 << 15) ? 2 : (pairs < (1 << 17) ? 4 : 8);
+    const int64_t chains = S * D * kN;            // (sequence, channel, state) recurrences
+    const int64_t per_sm = chains / sm_count();
+    int npt_auto, sched_auto;
+    if (per_sm >= 8 * 640) {
+        npt_auto = 8;
+        sched_auto = 2;
+    } else if (per_sm >= 4 * 640) {
+        npt_auto = 4;
+        sched_auto = 8;
+    } else {
+        npt_auto = 2;
+        sched_auto = 8;
+    }
     *npt = g_forced_npt ? g_forced_npt : npt_auto;
-    *sched = g_forced_sched ? g_forced_sched : 2;
+    *sched = g_forced_sched ? g_forced_sched : sched_auto;
 }
 
 }  // namespace
 
+void scan_variant_for(int64_t S, int64_t D, int *npt, int *sched) { pick_variant(S, D, npt, sched); }
+
 void set_scan_variant(int npt, int sched)
 {
     g_forced_npt = (npt == 2 || npt == 4 || npt == 8 || npt == 16) ? npt : 0;
-    g_forced_sched = (sched >= 1 && sched <= 7) ? sched : 0;
+    g_forced_sched = (sched >= 1 && sched <= 8) ? sched : 0;
 }
 
 size_t scan_order_bytes(int64_t S) { return (size_t)((S * 4 + 255) / 256) * 256; }

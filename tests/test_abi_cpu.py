@@ -132,7 +132,28 @@ def test_check_cu_seqlens_host():
 def test_tuning_knob():
     for n, c in ((0, 0), (2, 1), (4, 1), (4, 2), (4, 3), (8, 2), (16, 1), (16, 2)):
         ssm.ssm_set_scan_variant(n, c)
-    for n, c in ((3, 1), (16, 8), (4, -1)):
+    for n, c in ((3, 1), (16, 9), (4, -1)):
         with pytest.raises(ssm.SsmError):
             ssm.ssm_set_scan_variant(n, c)
     ssm.ssm_set_scan_variant(0, 0)
+
+
+def test_variant_choice():
+    """The automatic choice follows (sequence, channel, state) recurrences per
+    SM (148 SMs when no device is visible): 8 states per lane with TMA staging
+    when the GPU holds about 20 warps per SM of them, else 4 and then 2 states
+    per lane in the single-stage TMA layout. A forced variant is reported as
+    forced."""
+    ssm.ssm_set_scan_variant(0, 0)
+    assert ssm.ssm_scan_variant_for(8, 1536) == (2, 8)      # 8 x 2048 x 1536 layer
+    assert ssm.ssm_scan_variant_for(43, 5120) == (8, 2)     # packed 65536 x 5120
+    assert ssm.ssm_scan_variant_for(1, 8192) == (2, 8)      # one 8192-channel sequence
+    assert ssm.ssm_scan_variant_for(4, 8192) == (4, 8)
+    assert ssm.ssm_scan_variant_for(1, 32) == (2, 8)
+    ssm.ssm_set_scan_variant(16, 7)
+    assert ssm.ssm_scan_variant_for(1, 32) == (16, 7)
+    ssm.ssm_set_scan_variant(0, 0)
+    for S, D in ((0, 16), (4, 0)):
+        with pytest.raises(ssm.SsmError) as ei:
+            ssm.ssm_scan_variant_for(S, D)
+        assert ei.value.code == -1
