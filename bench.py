@@ -13,6 +13,7 @@ Each step reads a different one of 4 input sets (about 600 MB together),
 so no step finds its inputs in the 126 MB L2.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --scan-sweep [NPT,SCHED ...]   # scan alone per kernel variant
 
 With N > 1 (torchrun) every rank runs the same workload on its own GPU (the
 path shards with no exchange: replicas), and the value counts every rank's
@@ -61,6 +62,10 @@ def parse_args():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the packed, long-context and decode workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scan-sweep", nargs="*", metavar="NPT,SCHED", default=None,
+                    help="instead of the step: time the scan alone for each variant "
+                         "(states per lane, schedule; default: a standard list) on the "
+                         "four prefill shapes and print one JSON line per measurement")
     return ap.parse_args()
 
 
@@ -560,10 +565,75 @@ def bench_reference(args):
 
 # ---------------------------------------------------------------------------
 
+SWEEP_VARIANTS = [(0, 0), (2, 8), (4, 8), (8, 2), (4, 1), (8, 7), (8, 6), (2, 3)]
+
+
+def scan_sweep(variants, peaks):
+    """Scan alone per variant on the prefill shapes; one JSON line each."""
+    import torch
+
+    import selective_state_space_causal_b200 as ssm
+    from selective_state_space_causal_b200 import synth
+
+    mufu = mufu_peak_gexp(peaks["sm_max_mhz"])
+    lens = synth.sample_lengths(0, 65536)
+    shapes = [("mamba130m_layer_b8_l2048", 16384, 1536, None, 8),
+              ("packmamba_2p8b_varlen_65536", 65536, 5120, synth.cu_from_lengths(lens), len(lens)),
+              ("falcon_mamba7b_longctx_131072 (one 8192-token call)", 8192, 8192, None, 1),
+              ("uniform_32x2048_d5120", 65536, 5120, synth.cu_from_lengths([2048] * 32), 32)]
+    for name, tok, D, cu, S in shapes:
+        prm = synth.make_params(0, D)
+        A, Dk, dtb = (torch.from_numpy(v).cuda() for v in (prm.A, prm.Dskip, prm.dt_bias))
+        cu_d = torch.from_numpy(cu).cuda() if cu is not None else None
+        sets = [synth.device_activations(i, tok, D) for i in range(3)]
+        y = torch.empty((tok, D), dtype=torch.bfloat16, device="cuda")
+        h = torch.empty((S, D, N_STATE), device="cuda")
+        ws = torch.empty(max(1, ssm.ssm_scan_workspace_size(tok, D, N_STATE, S)),
+                         dtype=torch.uint8, device="cuda")
+        for npt, sched in variants:
+            ssm.ssm_set_scan_variant(npt, sched)
+            picked = ssm.ssm_scan_variant_for(S, D)
+
+            def call(a):
+                ssm.ssm_selective_scan_fwd(a["x"], a["dt"], A, a["B"], a["C"], y, Dskip=Dk,
+                                           z=a["z"], dt_bias=dtb, h_final=h, cu_seqlens=cu_d,
+                                           S=S, workspace=ws if cu_d is not None else None)
+
+            for i in range(3):
+                call(sets[i % 3])
+            torch.cuda.synchronize()
+            n = 30 if tok * D < 1e9 else 10
+            e0, e1 = _events(2)
+            e0.record()
+            for i in range(n):
+                call(sets[i % 3])
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / n
+            gexp = tok * D * N_STATE / (ms * 1e-3) / 1e9
+            print(json.dumps({"workload": name, "states_per_lane": picked[0], "schedule": picked[1],
+                              "auto": npt == 0 and sched == 0, "scan_ms": round(ms, 4),
+                              "gexp_per_s": round(gexp, 1), "mufu_frac": round(gexp / mufu, 4)}),
+                  flush=True)
+        ssm.ssm_set_scan_variant(0, 0)
+        del sets
+        torch.cuda.empty_cache()
+    if ssm.ssm_device_status() != 0:
+        raise RuntimeError("a bounded device wait timed out during the sweep")
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return bench_reference(args)
+    if args.scan_sweep is not None:
+        import torch
+
+        torch.cuda.set_device(0)
+        variants = ([tuple(int(x) for x in v.split(",")) for v in args.scan_sweep]
+                    if args.scan_sweep else SWEEP_VARIANTS)
+        return scan_sweep(variants, load_peaks())
     rank, local, world = dist_info()
     import torch
 
