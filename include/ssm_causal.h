@@ -115,9 +115,10 @@ int ssm_scan_variant_for(int64_t S, int64_t D, int *states_per_lane, int *schedu
 
 /*
  * Device-side status of the library's kernels on the current device: 0 while
- * every bounded wait for a TMA tile completed; bit 0 set once a scan kernel's
- * wait gave up, bit 1 once a conv kernel's did (the results of that call are
- * then unspecified; the kernel still terminates). Synchronises the device.
+ * every bounded wait for a TMA tile or bulk copy completed; bit 0 set once a
+ * scan kernel's wait gave up, bit 1 once a conv kernel's did, bit 2 once a
+ * decode kernel's did (the results of that call are then unspecified; the
+ * kernel still terminates). Synchronises the device.
  * clear != 0 resets the flags. Returns SSM_ERR_CUDA if the query itself fails.
  */
 int ssm_device_status(int clear);

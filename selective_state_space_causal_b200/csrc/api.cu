@@ -19,6 +19,7 @@ void scan_variant_for(int64_t S, int64_t D, int *npt, int *sched);
 size_t scan_order_bytes(int64_t S);
 int read_scan_status(bool clear);
 int read_conv_status(bool clear);
+int read_decode_status(bool clear);
 cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
 int64_t noalloc_max_sequences();
 }  // namespace ssm
@@ -112,9 +113,10 @@ int ssm_device_status(int clear)
 {
     const int a = ssm::read_scan_status(clear != 0);
     const int b = ssm::read_conv_status(clear != 0);
-    if (a < 0 || b < 0) return fail(SSM_ERR_CUDA, "ssm_device_status: CUDA query failed");
+    const int d = ssm::read_decode_status(clear != 0);
+    if (a < 0 || b < 0 || d < 0) return fail(SSM_ERR_CUDA, "ssm_device_status: CUDA query failed");
     g_error.clear();
-    return (a ? 1 : 0) | (b ? 2 : 0);
+    return (a ? 1 : 0) | (b ? 2 : 0) | (d ? 4 : 0);
 }
 
 int ssm_check_cu_seqlens(const int32_t *cu, int64_t S, int64_t tok)

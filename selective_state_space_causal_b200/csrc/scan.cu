@@ -846,16 +846,6 @@ struct WsCfg {
     static_assert(HELP % CV == 0, "each helper keeps one channel vector");
 };
 
-__device__ __forceinline__ void mbar_init_n(uint64_t *bar, int count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(saddr(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(saddr(bar)) : "memory");
-}
-
 template <class K, typename T>
 __global__ void __launch_bounds__(K::THREADS)
 scan_ws_kernel(const Params p, const __grid_constant__ Maps m, const int has_z)
