@@ -67,7 +67,7 @@ struct Cfg {
     static constexpr int THREADS = CH * TPC;
     static constexpr int CV = CH / VEC;                   // channel vectors per row
     static constexpr int ITEMS = TCH * CV;                // (token, vector) items per chunk
-    static constexpr int IPT = ITEMS / THREADS;           // items per thread
+    static constexpr int IPT = (ITEMS + THREADS - 1) / THREADS;  // items per thread (last partial)
     static constexpr int ROW2 = CH + 2 * (CH / 16);       // padded smem row, in float2
     static constexpr int BCVEC = 16 / sizeof(T);          // B/C elements per 16 bytes
     static constexpr int BCN = TCH * kN / BCVEC;          // 16-byte B (or C) pieces per chunk
@@ -89,7 +89,6 @@ struct Cfg {
     static constexpr size_t SMEM_TMA = OFF_BAR + 128;
     static_assert(CH % 16 == 0, "channel tile is a multiple of 16");
     static_assert(NPT % 2 == 0, "states come in packed pairs");
-    static_assert(ITEMS % THREADS == 0, "items must divide evenly");
     static_assert(THREADS % CV == 0, "each thread keeps one channel vector");
     static_assert(TCH % TPC == 0, "chunk must hold whole token groups");
     static_assert(THREADS <= 1024 && (THREADS % 32) == 0, "block size");
@@ -126,7 +125,7 @@ __device__ __forceinline__ void prepass_item(float2 *dx_row, float2 *ug_row, boo
 #pragma unroll
     for (int e = 0; e < VEC; ++e) {
         float d = fdt[e] + dtb[e];
-        if (softplus) d = softplus_f(d);
+        if (softplus) d = softplus_fast(d);
         vd[e] = live ? d : 0.f;
         vdx[e] = live ? d * fu[e] : 0.f;
         vu[e] = live ? fu[e] : 0.f;
@@ -226,6 +225,7 @@ __device__ __forceinline__ void store_y(T *Y, const float2 *sUG, int tid, int nt
     constexpr int VEC = K::VEC;
 #pragma unroll
     for (int i = 0; i < K::IPT; ++i) {
+        if (tid + i * K::THREADS >= K::ITEMS) break;
         const int tl = (tid + i * K::THREADS) / K::CV;
         if (tl < nt && vvalid) {
             float out[VEC];
@@ -361,6 +361,7 @@ scan_kernel(const Params p)
     auto prefetch = [&](int64_t t0) {
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
+            if (tid + i * THREADS >= K::ITEMS) break;
             const int64_t row = t0 + (tid + i * THREADS) / CV;
             if (row < l.end && l.vvalid) {
                 const int64_t off = row * p.D + l.cg;
@@ -386,6 +387,7 @@ scan_kernel(const Params p)
         const int nt = (int)min((int64_t)TCH, l.end - t0);
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
+            if (tid + i * THREADS >= K::ITEMS) break;
             const int tl = (tid + i * THREADS) / CV;
             float fdt[VEC], fu[VEC], fz[VEC];
             const bool live = tl < nt && l.vvalid;
@@ -489,6 +491,7 @@ scan_staged_kernel(const Params p, const __grid_constant__ Maps m, const int has
         parity ^= 1u;
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
+            if (tid + i * THREADS >= K::ITEMS) break;
             const int tl = (tid + i * THREADS) / CV;
             const int ro = tl * CH + l.cvl * VEC;
             float fdt[VEC], fu[VEC], fz[VEC];
