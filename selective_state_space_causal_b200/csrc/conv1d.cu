@@ -54,6 +54,21 @@ struct Seqs {
     }
 };
 
+__device__ __forceinline__ float rcp_approx(float x)
+{
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// SiLU as z * 1/(1 + 2^(-z log2 e)) on the special-function unit; every conv
+// path (and the packed one below) uses exactly these operations, so a token
+// gets the same bits whichever path computes it.
+__device__ __forceinline__ float conv_silu(float z)
+{
+    return z * rcp_approx(ex2_approx(z * -kLog2e) + 1.f);
+}
+
 template <typename T, int VEC, int K>
 __device__ __forceinline__ void conv_out(const float (&wk)[K][VEC], const float (&bv)[VEC],
                                          const float (&win)[K][VEC], int apply_silu,
@@ -64,7 +79,7 @@ __device__ __forceinline__ void conv_out(const float (&wk)[K][VEC], const float 
         float acc = bv[i];
 #pragma unroll
         for (int k = 0; k < K; ++k) acc = fmaf(wk[k][i], win[k][i], acc);
-        out[i] = apply_silu ? silu_f(acc) : acc;
+        out[i] = apply_silu ? conv_silu(acc) : acc;
     }
 }
 
@@ -164,16 +179,73 @@ conv1d_kernel(const T *__restrict__ x, T *__restrict__ xc, const float *__restri
     }
 }
 
+// Packed-pair helpers of the TMA path: 8 bytes of channels (4 bf16 or 2 fp32)
+// as VEC/2 fp32x2 pairs, the K-tap window in packed FFMA and conv_silu per half.
+template <typename T, int VEC>
+__device__ __forceinline__ void unpack8_pk(const uint2 &raw, f32x2 (&o)[VEC / 2])
+{
+    static_assert(VEC * sizeof(T) == 8, "8-byte vectors");
+    if constexpr (sizeof(T) == 2) {
+        o[0] = pk2(__uint_as_float(raw.x << 16), __uint_as_float(raw.x & 0xffff0000u));
+        o[1] = pk2(__uint_as_float(raw.y << 16), __uint_as_float(raw.y & 0xffff0000u));
+    } else {
+        o[0] = pk2(__uint_as_float(raw.x), __uint_as_float(raw.y));
+    }
+}
+
+template <typename T, int VEC>
+__device__ __forceinline__ void store8_pk(T *p, const f32x2 (&v)[VEC / 2])
+{
+    uint2 raw;
+    if constexpr (sizeof(T) == 2) {
+        float a, b, c, d;
+        upk2(v[0], a, b);
+        upk2(v[1], c, d);
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
+        raw.x = *reinterpret_cast<const uint32_t *>(&lo);
+        raw.y = *reinterpret_cast<const uint32_t *>(&hi);
+    } else {
+        float a, b;
+        upk2(v[0], a, b);
+        raw.x = __float_as_uint(a);
+        raw.y = __float_as_uint(b);
+    }
+    *reinterpret_cast<uint2 *>(p) = raw;
+}
+
+template <int VEC, int K>
+__device__ __forceinline__ void conv_out_pk(const f32x2 (&wk)[K][VEC / 2], const f32x2 (&bv)[VEC / 2],
+                                            const f32x2 (&win)[K][VEC / 2], int apply_silu,
+                                            f32x2 (&out)[VEC / 2])
+{
+#pragma unroll
+    for (int i = 0; i < VEC / 2; ++i) {
+        f32x2 acc = bv[i];
+#pragma unroll
+        for (int k = 0; k < K; ++k) acc = fma2(wk[k][i], win[k][i], acc);
+        if (apply_silu) {  // conv_silu on both halves
+            float a0, a1;
+            upk2(mul2(acc, pk2(-kLog2e, -kLog2e)), a0, a1);
+            float d0, d1;
+            upk2(add2(pk2(ex2_approx(a0), ex2_approx(a1)), pk2(1.f, 1.f)), d0, d1);
+            acc = mul2(acc, pk2(rcp_approx(d0), rcp_approx(d1)));
+        }
+        out[i] = acc;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // TMA-tiled variant (16-byte aligned rows). A CTA owns kTileT tokens x one
 // 128-byte row of channels: one TMA box of kTileT + K - 1 rows (the K - 1 halo
 // rows may start before token 0 or run past the last token; those read zeros)
 // lands in shared memory, then each thread slides the K-tap window over its
-// kTileG tokens of one 16-byte channel vector and writes 16-byte outputs.
-// Many small CTAs per SM overlap one CTA's load with another's arithmetic.
+// kTileG tokens of one 8-byte channel vector and writes 8-byte outputs (a warp
+// still writes whole 128-byte rows). 8-byte vectors keep the weights and window
+// in few registers, so many CTAs fit per SM and overlap one CTA's load with
+// another's arithmetic.
 // ---------------------------------------------------------------------------
 constexpr int kTileT = 128;      // tokens per CTA
-constexpr int kTileG = 8;        // tokens per thread
+constexpr int kTileG = 16;       // tokens per thread
 constexpr int kTileThreads = 128;
 
 template <typename T, typename TS, int K>
@@ -182,7 +254,7 @@ conv1d_tma_kernel(const __grid_constant__ CUtensorMap xmap, T *__restrict__ xc,
                   const float *__restrict__ w, const float *__restrict__ bias, Seqs sq, int64_t D,
                   const TS *__restrict__ state_in, int apply_silu)
 {
-    constexpr int VEC = 16 / sizeof(T);        // channels per 16-byte vector
+    constexpr int VEC = 8 / sizeof(T);         // channels per 8-byte vector
     constexpr int CW = 128 / sizeof(T);        // channels per tile row (128 bytes)
     constexpr int NV = CW / VEC;               // vectors per row
     constexpr int ROWS = kTileT + K - 1;
@@ -211,6 +283,13 @@ conv1d_tma_kernel(const __grid_constant__ CUtensorMap xmap, T *__restrict__ xc,
         for (int k = 0; k < K; ++k) wk[k][i] = active ? __ldg(w + (c0 + i) * K + k) : 0.f;
         bv[i] = (active && bias) ? __ldg(bias + c0 + i) : 0.f;
     }
+    f32x2 wk2[K][VEC / 2], bv2[VEC / 2];
+#pragma unroll
+    for (int i = 0; i < VEC / 2; ++i) {
+#pragma unroll
+        for (int k = 0; k < K; ++k) wk2[k][i] = pk2(wk[k][2 * i], wk[k][2 * i + 1]);
+        bv2[i] = pk2(bv[2 * i], bv[2 * i + 1]);
+    }
     // every thread waits, so no thread leaves while the copy is in flight
     bool failed = false;
     mbar_wait(&bar, 0, failed, &g_conv_status, 1);
@@ -224,20 +303,22 @@ conv1d_tma_kernel(const __grid_constant__ CUtensorMap xmap, T *__restrict__ xc,
     auto row = [&](int64_t pos) { return (int)(pos - (t0 - (K - 1))); };
 
     if (ta - (K - 1) >= s_start && ta + kTileG <= s_end) {
-        float win[K][VEC];
+        f32x2 win[K][VEC / 2];
 #pragma unroll
         for (int k = 0; k < K - 1; ++k)
-            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(tile + row(ta - (K - 1) + k) * CW + v * VEC), win[k]);
+            unpack8_pk<T, VEC>(*reinterpret_cast<const uint2 *>(tile + row(ta - (K - 1) + k) * CW + v * VEC), win[k]);
+        T *dst = xc + ta * D + c0;
 #pragma unroll
         for (int t = 0; t < kTileG; ++t) {
-            unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(tile + row(ta + t) * CW + v * VEC), win[K - 1]);
-            float out[VEC];
-            conv_out<T, VEC, K>(wk, bv, win, apply_silu, out);
-            store_vec<T, VEC>(xc + (ta + t) * D + c0, out);
+            unpack8_pk<T, VEC>(*reinterpret_cast<const uint2 *>(tile + row(ta + t) * CW + v * VEC), win[K - 1]);
+            f32x2 out[VEC / 2];
+            conv_out_pk<VEC, K>(wk2, bv2, win, apply_silu, out);
+            store8_pk<T, VEC>(dst, out);
+            dst += D;
 #pragma unroll
             for (int k = 0; k < K - 1; ++k)
 #pragma unroll
-                for (int i = 0; i < VEC; ++i) win[k][i] = win[k + 1][i];
+                for (int i = 0; i < VEC / 2; ++i) win[k][i] = win[k + 1][i];
         }
         return;
     }
@@ -255,7 +336,8 @@ conv1d_tma_kernel(const __grid_constant__ CUtensorMap xmap, T *__restrict__ xc,
         for (int k = 0; k < K; ++k) {
             const int64_t pos = t - (K - 1) + k;
             if (pos >= s_start) {
-                unpack16<T, VEC>(*reinterpret_cast<const uint4 *>(tile + row(pos) * CW + v * VEC), win[k]);
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) win[k][i] = to_f32(tile[row(pos) * CW + v * VEC + i]);
             } else {
 #pragma unroll
                 for (int i = 0; i < VEC; ++i)

@@ -145,7 +145,7 @@ __device__ __forceinline__ void recur_chunk(const float2 *__restrict__ sDX, floa
                                             f32x2 (&hp)[K::NPT / 2], float dsk)
 {
     constexpr int NPT = K::NPT, TPC = K::TPC, ROW2 = K::ROW2, NP = K::NPT / 2;
-    for (int tt = 0; tt < ntr; tt += TPC) {
+    auto group = [&](const int tt) {
         float yp[TPC];
         if constexpr (K::BATCH) {
             // all exponentials of the group first, then the dependent FMAs
@@ -214,6 +214,14 @@ __device__ __forceinline__ void recur_chunk(const float2 *__restrict__ sDX, floa
         float2 *q2 = sUG + (tt + sub) * ROW2 + mycol;
         const float2 ug = *q2;
         q2->x = (yp[0] + dsk * ug.x) * ug.y;
+    };
+    // full chunks run fully unrolled, so one group's loads and exponentials
+    // can overlap the previous group's readout butterfly
+    if (ntr == K::TCH) {
+#pragma unroll
+        for (int tt = 0; tt < K::TCH; tt += TPC) group(tt);
+    } else {
+        for (int tt = 0; tt < ntr; tt += TPC) group(tt);
     }
 }
 
@@ -1873,11 +1881,12 @@ int sm_count()
 // Measured on B200 (exponential rate against the special-function peak):
 // 8 states per lane with double-buffered TMA staging has the fewest
 // instructions per exponential and wins once the GPU holds about 20 warps per
-// SM of it (packed 65536 x 5120: 0.60 against 0.53 for the next best); below
-// that, latency decides and thinner lanes win: 2 states per lane in the
-// single-stage layout of schedule 8 (8 x 2048 x 1536: 0.345 against 0.33 for 4
-// states with register prefetch; 1 x 8192 x 8192: 0.33 against 0.31), with 4
-// states per lane in between.
+// SM of it (packed 65536 x 5120: 0.60 against 0.52 for the next best); below
+// that, latency decides and thinner lanes win: 4 states per lane with register
+// prefetch while that still gives about 10 warps per SM (8 x 2048 x 1536:
+// 0.366 against 0.356 for 2 states in schedule 8), else 2 states per lane in
+// the single-stage TMA layout of schedule 8 (1 x 8192 x 8192: 0.353 against
+// 0.31 for 4 states).
 void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
 {
     const int64_t chains = S * D * kN;            // (sequence, channel, state) recurrences
@@ -1886,9 +1895,9 @@ void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
     if (per_sm >= 8 * 640) {
         npt_auto = 8;
         sched_auto = 2;
-    } else if (per_sm >= 4 * 640) {
+    } else if (per_sm >= 4 * 320) {
         npt_auto = 4;
-        sched_auto = 8;
+        sched_auto = 1;
     } else {
         npt_auto = 2;
         sched_auto = 8;
