@@ -8,7 +8,8 @@ and returns new arrays; the wrappers do data marshalling only.
 
 Parity pins: the closed-form geometric series, the brute-force unrolled sum,
 ``numpy.correlate`` for the convolution, the packing, chunking and decode
-invariants and a hand-worked dyadic example all pin these routines (see the
+invariants, the equality of replay decode with eager decode, bit-level bf16
+rounding and a hand-worked dyadic example all pin these routines (see the
 ``tests/test_oracle_*.py`` files). No function here is "parity unpinned".
 """
 
@@ -86,6 +87,15 @@ class Oracle:
                                             _dp, _dp, _int, _ip, _i64, _dp, _i64, _i64, _int,
                                             _int]
         lib.oracle_state_update.restype = None
+        lib.oracle_round_bf16.argtypes = [_dp, _dp, _i64]
+        lib.oracle_round_bf16.restype = None
+        lib.oracle_replay_state.argtypes = [_dp, _dp, _dp, _dp, _ip, _dp, _i64, _int, _i64, _int,
+                                            _dp]
+        lib.oracle_replay_state.restype = None
+        lib.oracle_replay_step.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _ip, _int, _dp, _dp, _dp,
+                                           _dp, _dp, _dp, _dp, _dp, _dp, _dp, _int, _ip, _i64, _dp,
+                                           _i64, _i64, _int, _int]
+        lib.oracle_replay_step.restype = None
         lib.oracle_num_threads.restype = _int
         lib.oracle_set_num_threads.argtypes = [_int]
         self.lib = lib
@@ -154,6 +164,56 @@ class Oracle:
                                      _ptr(A), _ptr(args[6]), _ptr(args[7]), int(delta_softplus),
                                      _iptr(idx), cs.shape[0], _ptr(y), Bt, D, N, K)
         return y, cs, ss
+
+    # -- replay decode -------------------------------------------------------
+    def round_bf16(self, v):
+        """Nearest bf16 value of each element (ties to even), as float64."""
+        v = _f64(v)
+        out = np.empty_like(v)
+        self.lib.oracle_round_bf16(_ptr(v), _ptr(out), v.size)
+        return out
+
+    def replay_init(self, ck, W, keep_lo=True):
+        """A replay representation starting at state ck (n_slots, D, N): a dict
+        with the checkpoint, its bf16 copy (or None), empty buffers and lengths."""
+        ck = _f64(ck).copy()
+        n_slots, D, N = ck.shape
+        return {"ck": ck, "ck_lo": self.round_bf16(ck) if keep_lo else None, "W": int(W),
+                "bd": np.zeros((n_slots, W, D)), "bx": np.zeros((n_slots, W, D)),
+                "bB": np.zeros((n_slots, W, N)), "len": np.zeros(n_slots, np.int64)}
+
+    def replay_state(self, rep, A):
+        """The state each slot of a replay representation stands for (n_slots, D, N)."""
+        ck = rep["ck"]
+        n_slots, D, N = ck.shape
+        h = np.zeros_like(ck)
+        self.lib.oracle_replay_state(_ptr(ck), _ptr(rep["bd"]), _ptr(rep["bx"]), _ptr(rep["bB"]),
+                                     _iptr(rep["len"]), _ptr(_f64(A)), n_slots, rep["W"], D, N,
+                                     _ptr(h))
+        return h
+
+    def replay_step(self, conv_state, rep, x, dt, B, C, z, conv_w, conv_b, A, Dskip, dt_bias,
+                    delta_softplus=True, state_indices=None, y_init=None):
+        """One replay decode step. Returns (y, conv_state', rep'); inputs are not modified."""
+        cs = _f64(conv_state).copy()
+        lo = rep["ck_lo"]
+        new = {"ck": rep["ck"].copy(), "ck_lo": None if lo is None else lo.copy(),
+               "W": rep["W"], "bd": rep["bd"].copy(), "bx": rep["bx"].copy(),
+               "bB": rep["bB"].copy(), "len": rep["len"].copy()}
+        x = _f64(x)
+        Bt, D = x.shape
+        A = _f64(A)
+        N = A.shape[1]
+        K = cs.shape[2] + 1
+        idx = None if state_indices is None else np.ascontiguousarray(state_indices, np.int64)
+        y = np.zeros((Bt, D)) if y_init is None else _f64(y_init).copy()
+        args = [_f64(a) for a in (dt, B, C, z, conv_w, conv_b, Dskip, dt_bias)]
+        self.lib.oracle_replay_step(
+            _ptr(cs), _ptr(new["ck"]), _ptr(new["ck_lo"]), _ptr(new["bd"]), _ptr(new["bx"]),
+            _ptr(new["bB"]), _iptr(new["len"]), new["W"], _ptr(x), _ptr(args[0]), _ptr(args[1]),
+            _ptr(args[2]), _ptr(args[3]), _ptr(args[4]), _ptr(args[5]), _ptr(A), _ptr(args[6]),
+            _ptr(args[7]), int(delta_softplus), _iptr(idx), cs.shape[0], _ptr(y), Bt, D, N, K)
+        return y, cs, new
 
 
 _DEFAULT = None

@@ -30,6 +30,12 @@
  *             (tp_builder.py: present_conv / present_ssm outputs; "Scaling
  *             State-Space Models...", abstract: SSM cache across prefill and
  *             decode).
+ *   replay:   the SSM state of a slot is kept as a checkpoint plus the SSM
+ *             inputs (delta, xc, B) of the tokens since it; outputs come from
+ *             unrolling the recurrence from the checkpoint, and the checkpoint
+ *             is rewritten once every W tokens; an optional bf16 copy of the
+ *             checkpoint serves the outputs of the other steps ("ReplaySSM:
+ *             Cache SSM Inputs, Not State", abstract).
  *
  * Channels are independent, so the outer (sequence, channel) loops may run on
  * several OpenMP threads; each (sequence, channel) is computed by one thread in
@@ -192,5 +198,133 @@ void oracle_state_update(double *conv_state, double *ssm_state, const double *x,
             if (z) yt *= silu(z[b * D + c]);
             y[b * D + c] = yt;
         }
+    }
+}
+
+/*
+ * Round to the nearest bf16 value (8 significant bits), ties to even. The
+ * value is split as m * 2^e with 0.5 <= |m| < 1; m * 2^8 is rounded to an
+ * integer in the current (round-to-nearest-even) mode and scaled back. Values
+ * are assumed inside bf16's normal range.
+ */
+static double round_bf16(double v)
+{
+    if (v == 0.0 || !isfinite(v)) return v;
+    int e;
+    const double m = frexp(v, &e);
+    return ldexp(nearbyint(ldexp(m, 8)), e - 8);
+}
+
+void oracle_round_bf16(const double *in, double *out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = round_bf16(in[i]);
+}
+
+/*
+ * The state a replay slot stands for, written as the unrolled recurrence
+ * (the product of the decays of the tokens after i is the exponential of A
+ * times the sum of their deltas):
+ *   h[n] = exp(A[n] * sum_{i<len} delta_i) * base[n]
+ *        + sum_{i<len} exp(A[n] * sum_{i<r<len} delta_r) * delta_i * xc_i * B_i[n].
+ * base: (D, N); bd, bx: (W, D) deltas and conv outputs of the buffered
+ * tokens, oldest first; bB: (W, N); out: (D, N).
+ */
+static void replay_unroll(const double *base, const double *bd, const double *bx,
+                          const double *bB, int64_t len, const double *A, int64_t D, int N,
+                          int64_t c, double *out_c)
+{
+    for (int n = 0; n < N; ++n) {
+        const double a = A[c * N + n];
+        double total = 0.0;
+        for (int64_t i = 0; i < len; ++i) total += bd[i * D + c];
+        double h = exp(a * total) * base[c * N + n];
+        for (int64_t i = 0; i < len; ++i) {
+            double after = 0.0;
+            for (int64_t r = i + 1; r < len; ++r) after += bd[r * D + c];
+            h += exp(a * after) * bd[i * D + c] * bx[i * D + c] * bB[i * N + n];
+        }
+        out_c[n] = h;
+    }
+}
+
+/*
+ * Materialise the current state of every slot: ck (n_slots, D, N) replayed
+ * over the slot's len[s] buffered tokens. bd, bx: (n_slots, W, D);
+ * bB: (n_slots, W, N); h: (n_slots, D, N).
+ */
+void oracle_replay_state(const double *ck, const double *bd, const double *bx, const double *bB,
+                         const int64_t *len, const double *A, int64_t n_slots, int W,
+                         int64_t D, int N, double *h)
+{
+    if (N > ORACLE_MAX_N) return;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t s = 0; s < n_slots; ++s)
+        for (int64_t c = 0; c < D; ++c)
+            replay_unroll(ck + s * D * N, bd + s * W * D, bx + s * W * D, bB + s * W * N, len[s],
+                          A, D, N, c, h + (s * D + c) * N);
+}
+
+/*
+ * One replay decode token per row b, slot s = idx[b] (or b); rows with s < 0
+ * or s >= n_slots are skipped (their y row, buffers and checkpoint untouched).
+ * With j = len[s] tokens already buffered:
+ *   conv exactly as oracle_state_update (the conv state is kept eagerly);
+ *   delta = softplus(dt + dt_bias) (flag);
+ *   the token's (delta, xc, B) becomes buffered token j (j + 1 tokens now);
+ *   if j + 1 == W (a checkpoint step): h = replay of ck over the j + 1 tokens;
+ *     ck = h, ck_lo = round_bf16(h) (if kept), len = 0;
+ *   else: h = replay of ck_lo (or ck when no copy is kept) over the j + 1
+ *     tokens; len = j + 1;
+ *   y = (C.h + Dskip*xc) * silu(z).
+ * conv_state (n_slots, D, K-1); ck, ck_lo (n_slots, D, N) (ck_lo may be NULL);
+ * bd, bx (n_slots, W, D); bB (n_slots, W, N); len (n_slots); all updated in place.
+ */
+void oracle_replay_step(double *conv_state, double *ck, double *ck_lo, double *bd, double *bx,
+                        double *bB, int64_t *len, int W, const double *x, const double *dt,
+                        const double *B, const double *C, const double *z, const double *conv_w,
+                        const double *conv_b, const double *A, const double *Dskip,
+                        const double *dt_bias, int delta_softplus, const int64_t *idx,
+                        int64_t n_slots, double *y, int64_t Bt, int64_t D, int N, int K)
+{
+    if (N > ORACLE_MAX_N || K > ORACLE_MAX_K || W < 1) return;
+    /* rows are independent (distinct slots); each row's channels share its buffer length */
+    for (int64_t b = 0; b < Bt; ++b) {
+        const int64_t s = idx ? idx[b] : b;
+        if (s < 0 || s >= n_slots) continue;
+        const int64_t j = len[s];
+        const int flush = (j + 1 == W);
+        double *sbd = bd + s * W * D, *sbx = bx + s * W * D, *sbB = bB + s * W * N;
+        for (int n = 0; n < N; ++n) sbB[j * N + n] = B[b * N + n];
+#pragma omp parallel for schedule(static)
+        for (int64_t c = 0; c < D; ++c) {
+            double win[ORACLE_MAX_K];
+            for (int i = 0; i < K - 1; ++i) win[i] = conv_state[(s * D + c) * (K - 1) + i];
+            win[K - 1] = x[b * D + c];
+            double acc = conv_b ? conv_b[c] : 0.0;
+            for (int k = 0; k < K; ++k) acc += conv_w[c * K + k] * win[k];
+            const double xcv = silu(acc);
+            for (int i = 0; i < K - 1; ++i) conv_state[(s * D + c) * (K - 1) + i] = win[i + 1];
+
+            double d = dt[b * D + c] + (dt_bias ? dt_bias[c] : 0.0);
+            if (delta_softplus) d = softplus(d);
+            sbd[j * D + c] = d;
+            sbx[j * D + c] = xcv;
+
+            const double *base = (flush || ck_lo == NULL) ? ck : ck_lo;
+            double h[ORACLE_MAX_N];
+            replay_unroll(base + s * D * N, sbd, sbx, sbB, j + 1, A, D, N, c, h);
+            double sum = 0.0;
+            for (int n = 0; n < N; ++n) sum += C[b * N + n] * h[n];
+            double yt = sum + (Dskip ? Dskip[c] : 0.0) * xcv;
+            if (z) yt *= silu(z[b * D + c]);
+            y[b * D + c] = yt;
+            if (flush) {
+                for (int n = 0; n < N; ++n) {
+                    ck[(s * D + c) * N + n] = h[n];
+                    if (ck_lo) ck_lo[(s * D + c) * N + n] = round_bf16(h[n]);
+                }
+            }
+        }
+        len[s] = flush ? 0 : j + 1;
     }
 }

@@ -13,7 +13,11 @@ AssertionError when the oracle disagrees with the fact it is pinned to:
   in two with the state carried equals the one-shot prefill; prefill followed
   by k decode steps equals prefill over the extended sequence; permuted state
   indices with -1 padding touch exactly the named slots;
-* a hand-worked dyadic example stored under tests/golden/.
+* a hand-worked dyadic example stored under tests/golden/;
+* replay decode (checkpoint plus buffered inputs) against eager decode: equal
+  outputs and states, the bf16 checkpoint copy entering exactly the outputs
+  of non-checkpoint steps (a linearity identity), and bf16 rounding against a
+  bit-level round-to-nearest-even of float32 values and torch's conversion.
 
 The same checks run against deliberately broken copies of the oracle in
 test_oracle_mutants.py, which shows that each plausible slip is caught.
@@ -344,9 +348,163 @@ def check_golden_dyadic(orc):
     assert np.array_equal(so.reshape(-1), gc["state_out"])
 
 
+# ---------------------------------------------------------------------------
+# replay decode ("ReplaySSM: Cache SSM Inputs, Not State", abstract)
+# ---------------------------------------------------------------------------
+
+def _bf16_bits_rne(v32):
+    """Round float32 values to bf16 on their bit patterns (round to nearest, ties to even)."""
+    bits = np.asarray(v32, np.float32).view(np.uint32).astype(np.uint64)
+    lsb = (bits >> 16) & 1
+    out = ((bits + 0x7FFF + lsb) & 0xFFFF0000).astype(np.uint32)
+    return out.view(np.float32).astype(np.float64)
+
+
+def check_round_bf16(orc):
+    import torch
+
+    rng = np.random.default_rng(71)
+    v = (rng.standard_normal(4000) * np.exp(rng.uniform(-30, 30, 4000))).astype(np.float32)
+    # exact ties between two bf16 values: the even neighbour wins
+    ties = np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 3 * 2.0 ** -9 + 2.0 ** -9,
+                     (1 + 2.0 ** -7 + 2.0 ** -8) * 2.0 ** 20], dtype=np.float32)
+    v = np.concatenate([v, ties, np.float32([0.0, 1.0, -2.5, 65280.0, 1e-30])])
+    got = orc.round_bf16(v.astype(np.float64))
+    assert np.array_equal(got, _bf16_bits_rne(v))
+    lib = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(got, lib)
+    assert got[4000] == 1.0 and got[4001] == 1 + 2.0 ** -6
+
+
+def _replay_setup(seed, n_slots, D, N, K):
+    rng = np.random.default_rng(seed)
+    p, _ = _rand_layer(seed + 1, 1, D, N, K)
+    cs = rng.standard_normal((n_slots, D, K - 1))
+    h = rng.standard_normal((n_slots, D, N))
+    return p, cs, h, rng
+
+
+def _step_inputs(rng, Bt, D, N):
+    return {"x": rng.standard_normal((Bt, D)), "dt": 0.3 * rng.standard_normal((Bt, D)),
+            "z": rng.standard_normal((Bt, D)), "B": rng.standard_normal((Bt, N)),
+            "C": rng.standard_normal((Bt, N))}
+
+
+def check_replay_equals_eager(orc):
+    n_slots, D, N, K = 3, 5, 4, 4
+    for W in (1, 2, 3, 5):
+        p, cs0, h0, rng = _replay_setup(81 + W, n_slots, D, N, K)
+        rep = orc.replay_init(h0, W, keep_lo=False)
+        cs_e, h_e, cs_r = cs0, h0, cs0
+        for t in range(11):
+            a = _step_inputs(rng, n_slots, D, N)
+            args = (a["x"], a["dt"], a["B"], a["C"], a["z"], p["w"], p["b"], p["A"], p["D"],
+                    p["dtb"])
+            y_e, cs_e, h_e = orc.state_update(cs_e, h_e, *args)
+            y_r, cs_r, rep = orc.replay_step(cs_r, rep, *args)
+            assert _rel_err(y_r, y_e) <= 1e-12, (W, t)
+            assert np.array_equal(cs_r, cs_e), (W, t)
+            assert np.all(rep["len"] == (t + 1) % W), (W, t, rep["len"])
+            assert _rel_err(orc.replay_state(rep, p["A"]), h_e) <= 1e-12, (W, t)
+            if (t + 1) % W == 0:
+                assert _rel_err(rep["ck"], h_e) <= 1e-12, (W, t)
+
+
+def check_replay_low_precision(orc):
+    """With a bf16 copy, a non-checkpoint step's output differs from eager by
+    exactly the copy's rounding carried through the decay of the buffered
+    tokens (the output is linear in the checkpoint); checkpoint steps use the
+    fp64 checkpoint and match eager."""
+    from scipy.special import expit
+
+    n_slots, D, N, K, W = 2, 6, 5, 4, 4
+    p, cs0, h0, rng = _replay_setup(91, n_slots, D, N, K)
+    rep = orc.replay_init(h0, W, keep_lo=True)
+    assert np.array_equal(rep["ck_lo"], orc.round_bf16(h0))
+    cs_e, h_e, cs_r = cs0, h0, cs0
+    dsum = np.zeros((n_slots, D))
+    for t in range(10):
+        a = _step_inputs(rng, n_slots, D, N)
+        args = (a["x"], a["dt"], a["B"], a["C"], a["z"], p["w"], p["b"], p["A"], p["D"], p["dtb"])
+        ck_before, lo_before = rep["ck"].copy(), rep["ck_lo"].copy()
+        y_e, cs_e, h_e = orc.state_update(cs_e, h_e, *args)
+        y_r, cs_r, rep = orc.replay_step(cs_r, rep, *args)
+        dsum += np.logaddexp(0.0, a["dt"] + p["dtb"][None, :])
+        if (t + 1) % W == 0:
+            assert _rel_err(y_r, y_e) <= 1e-12, t
+            assert _rel_err(rep["ck"], h_e) <= 1e-12, t
+            assert np.array_equal(rep["ck_lo"], orc.round_bf16(rep["ck"])), t
+            dsum[:] = 0.0
+        else:
+            decay = np.exp(p["A"][None, :, :] * dsum[:, :, None])
+            corr = np.sum(a["C"][:, None, :] * decay * (lo_before - ck_before), axis=2)
+            want = y_e + corr * a["z"] * expit(a["z"])
+            assert _rel_err(y_r, want) <= 1e-12, t
+            assert not np.allclose(y_r, y_e, rtol=0, atol=1e-9 * np.abs(y_e).max()), t
+            assert np.array_equal(rep["ck"], ck_before) and np.array_equal(rep["ck_lo"], lo_before)
+
+
+def check_replay_state_indices(orc):
+    n_slots, Bt, D, N, K, W = 7, 4, 3, 4, 4, 3
+    p, cs, h, rng = _replay_setup(101, n_slots, D, N, K)
+    rep = orc.replay_init(h, W, keep_lo=True)
+    rep["len"][:] = [0, 1, 2, 1, 0, 2, 1]  # slots at different points of their windows
+    rep["bd"][:] = np.abs(rng.standard_normal(rep["bd"].shape)) * 0.05
+    rep["bx"][:] = rng.standard_normal(rep["bx"].shape)
+    rep["bB"][:] = rng.standard_normal(rep["bB"].shape)
+    a = _step_inputs(rng, Bt, D, N)
+    idx = np.array([5, -1, 0, 3], dtype=np.int64)
+    sentinel = np.full((Bt, D), 123.5)
+    args = (a["x"], a["dt"], a["B"], a["C"], a["z"], p["w"], p["b"], p["A"], p["D"], p["dtb"])
+    y, cs2, rep2 = orc.replay_step(cs, rep, *args, state_indices=idx, y_init=sentinel)
+    untouched = [s for s in range(n_slots) if s not in idx]
+    for key in ("ck", "ck_lo", "bd", "bx", "bB", "len"):
+        assert np.array_equal(rep2[key][untouched], rep[key][untouched]), key
+    assert np.array_equal(cs2[untouched], cs[untouched])
+    assert np.array_equal(y[1], sentinel[1])
+    assert list(rep2["len"][[5, 0, 3]]) == [0, 1, 2]  # slot 5 reached W tokens: checkpoint step
+    # the touched slots equal a run over the gathered slots, and eager decode of
+    # their materialised states
+    rows, slots = [0, 2, 3], idx[[0, 2, 3]]
+    sub = {k: (v[slots] if isinstance(v, np.ndarray) else v) for k, v in rep.items()}
+    sub_args = tuple(v[rows] for v in args[:5]) + args[5:]
+    yd, csd, repd = orc.replay_step(cs[slots], sub, *sub_args)
+    assert np.array_equal(y[rows], yd)
+    assert np.array_equal(cs2[slots], csd)
+    for key in ("ck", "ck_lo", "bd", "bx", "bB", "len"):
+        assert np.array_equal(rep2[key][slots], repd[key]), key
+    h_now = orc.replay_state(rep, p["A"])[slots]
+    ye, _, he = orc.state_update(cs[slots], h_now, *sub_args)
+    nolo = dict(sub, ck_lo=None)
+    yn, _, repn = orc.replay_step(cs[slots], nolo, *sub_args)
+    assert _rel_err(yn, ye) <= 1e-12
+    assert _rel_err(orc.replay_state(repn, p["A"]), he) <= 1e-12
+
+
+def check_replay_after_prefill(orc):
+    """Prefill, then k replay steps from its final state, equals prefill over
+    the extended sequence (outputs and state)."""
+    D, N, K, L0, k, W = 4, 4, 4, 9, 7, 3
+    L = L0 + k
+    p, a = _rand_layer(111, L, D, N, K)
+    y, hf, cs = _layer(orc, a["x"], a["dt"], a["z"], a["B"], a["C"], p,
+                       np.array([0, L], dtype=np.int64))
+    _, h, c = _layer(orc, a["x"][:L0], a["dt"][:L0], a["z"][:L0], a["B"][:L0], a["C"][:L0], p,
+                     np.array([0, L0], dtype=np.int64))
+    rep = orc.replay_init(h, W, keep_lo=False)
+    for t in range(L0, L):
+        sl = slice(t, t + 1)
+        yt, c, rep = orc.replay_step(c, rep, a["x"][sl], a["dt"][sl], a["B"][sl], a["C"][sl],
+                                     a["z"][sl], p["w"], p["b"], p["A"], p["D"], p["dtb"])
+        assert _rel_err(yt[0], y[t]) <= 1e-12, t
+    assert _rel_err(orc.replay_state(rep, p["A"]), hf) <= 1e-12
+    assert np.array_equal(c, cs)
+
+
 ALL_CHECKS = [
     check_softplus_spot, check_silu_spot, check_conv_identity_tap, check_closed_form,
     check_bruteforce, check_conv_correlate, check_pack_equals_separate,
     check_chunked_equals_oneshot, check_decode_invariant, check_state_indices,
-    check_golden_dyadic,
+    check_golden_dyadic, check_round_bf16, check_replay_equals_eager,
+    check_replay_low_precision, check_replay_state_indices, check_replay_after_prefill,
 ]

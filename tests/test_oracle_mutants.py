@@ -51,6 +51,25 @@ MUTANTS = {
                                  "double yt = sum + (Dskip ? Dskip[c] : 0.0) * x[b * D + c];", 0),
     "decode_wrong_slot": ("const int64_t s = idx ? idx[b] : b;",
                           "const int64_t s = b < n_slots ? b : -1;", 0),
+    "replay_base_not_decayed": ("double h = exp(a * total) * base[c * N + n];",
+                                "double h = base[c * N + n];", 0),
+    "replay_input_decayed_by_own_step": ("for (int64_t r = i + 1; r < len; ++r)",
+                                         "for (int64_t r = i; r < len; ++r)", 0),
+    "replay_B_of_newest_token": ("* bx[i * D + c] * bB[i * N + n];",
+                                 "* bx[i * D + c] * bB[(len - 1) * N + n];", 0),
+    "replay_checkpoint_step_reads_low_copy": (
+        "const double *base = (flush || ck_lo == NULL) ? ck : ck_lo;",
+        "const double *base = (ck_lo == NULL) ? ck : ck_lo;", 0),
+    "replay_never_reads_low_copy": ("const double *base = (flush || ck_lo == NULL) ? ck : ck_lo;",
+                                    "const double *base = ck;", 0),
+    "replay_length_not_reset": ("len[s] = flush ? 0 : j + 1;", "len[s] = flush ? j : j + 1;", 0),
+    "replay_checkpoint_every_step": ("const int flush = (j + 1 == W);", "const int flush = 1;", 0),
+    "replay_low_copy_not_refreshed": ("if (ck_lo) ck_lo[(s * D + c) * N + n] = round_bf16(h[n]);",
+                                      "(void)0;", 0),
+    "round_bf16_truncates": ("ldexp(nearbyint(ldexp(m, 8)), e - 8)",
+                             "ldexp(trunc(ldexp(m, 8)), e - 8)", 0),
+    "round_bf16_seven_bits": ("ldexp(nearbyint(ldexp(m, 8)), e - 8)",
+                              "ldexp(nearbyint(ldexp(m, 7)), e - 7)", 0),
 }
 
 
