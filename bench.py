@@ -62,6 +62,12 @@ def parse_args():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the packed, long-context and decode workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--replay-windows", type=int, nargs="+", default=[3], metavar="W",
+                    help="checkpoint intervals of the replay decode measurement")
+    ap.add_argument("--profile-decode", type=int, default=None, metavar="W",
+                    help="instead of the step: run 3 windows of replay decode steps (checkpoint "
+                         "every W tokens, bf16 copy) and 3 eager decode steps at 256 x 8192 from "
+                         "random states, untimed, as a small case for ncu captures")
     ap.add_argument("--scan-sweep", nargs="*", metavar="NPT,SCHED", default=None,
                     help="instead of the step: time the scan alone for each variant "
                          "(states per lane, schedule; default: a standard list) on the "
@@ -336,7 +342,7 @@ def bench_headline(args, world, peaks, rank_dev):
     return res
 
 
-def bench_secondary(peaks, world, steps_scale=1.0):
+def bench_secondary(peaks, world, steps_scale=1.0, replay_windows=(3,)):
     """Packed varlen prefill, chunked long-context prefill and batch-256 decode."""
     import torch
 
@@ -475,9 +481,87 @@ def bench_secondary(peaks, world, steps_scale=1.0):
         "algorithmic_bytes_per_step": bytes_step,
         "hbm_frac": round(bytes_step / (per * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "step": "ssm_selective_state_update, 256 rows x 8192 channels, fresh inputs per step"}
+    for W in replay_windows:
+        out[f"decode_b256_d8192_replay_w{W}"] = bench_replay(peaks, world, ly, cs, h, W, steps,
+                                                             mufu)
     del cs, h
     torch.cuda.empty_cache()
     return out
+
+
+def replay_bytes_per_step(Bt, D, W, keep_lo=True):
+    """Algorithmic HBM bytes of one replay decode step, averaged over a window of
+    W steps taken in lockstep by every row (buffer lengths 0, 1, ..., W-1).
+
+    Per (row, channel): conv state 6 B in and out, x, dt, z in and y out (2 B
+    each); a step with j buffered tokens reads the checkpoint copy (32 B bf16,
+    or 64 B fp32 without the copy), j buffered (delta, delta*xc) pairs (8 B
+    each) and writes its own pair (8 B); the checkpoint step (j = W-1) instead
+    reads the fp32 checkpoint (64 B), the W-1 pairs, and writes the checkpoint
+    (64 B) and its copy (32 B). Per row: B and C (bf16, 32 B each), buffered B
+    rows (64 B each), the new B row (64 B). Per channel: A, conv weight and
+    biases, Dskip (92 B)."""
+    per_ch = 0
+    per_row = 0
+    for j in range(W):
+        per_ch += 12 + 8
+        per_row += 2 * N_STATE * 2 + 64 * j
+        if j == W - 1:
+            per_ch += 64 + 8 * j + 64 + (32 if keep_lo else 0)
+        else:
+            per_ch += (32 if keep_lo else 64) + 8 * j + 8
+            per_row += 64
+    total = Bt * D * per_ch + Bt * per_row + W * D * (4 * 4 + 3 * 4 + N_STATE * 4)
+    return total / W
+
+
+def bench_replay(peaks, world, ly, cs, h, W, steps, mufu):
+    """Batch-256 decode through the replay kernels (checkpoint + input buffer,
+    bf16 checkpoint copy), on the same prefill states and the same kind of
+    fresh per-step inputs as the eager decode measurement."""
+    import torch
+
+    import selective_state_space_causal_b200 as ssm
+    from selective_state_space_causal_b200 import synth
+
+    Bt, D = h.shape[0], h.shape[1]
+    rep = ssm.replay_buffers(Bt, D, W, "cuda", keep_lo=True)
+    rep["ckpt"].copy_(h)
+    csr = cs.clone()
+    ssm.ssm_replay_reset(rep)
+    yd = torch.empty((Bt, D), dtype=torch.bfloat16, device="cuda")
+    s0, s1 = _events(2)
+    block = 100
+    total_ms = 0.0
+    done = 0
+    l0 = ssm.ssm_launch_count()
+    for b0 in range(0, steps, block):
+        blk = [synth.device_activations(5000 + b0 + i, Bt, D) for i in range(block)]
+        _barrier_sync(world)
+        s0.record()
+        for s in blk:
+            ssm.ssm_replay_state_update(csr, rep, s["x"], s["dt"], s["B"], s["C"], yd, ly.w, ly.A,
+                                        z=s["z"], conv_b=ly.b, Dskip=ly.Dskip,
+                                        dt_bias=ly.dt_bias)
+        s1.record()
+        _barrier_sync(world)
+        total_ms += _max_over_ranks(s0.elapsed_time(s1), world)
+        done += block
+        del blk
+    launches = ssm.ssm_launch_count() - l0
+    per = total_ms / done
+    bytes_step = replay_bytes_per_step(Bt, D, W)
+    exps_step = Bt * D * N_STATE * (W + 1) / 2
+    res = {
+        "steps_per_s": 1e3 / per * world, "ms_per_step": per, "steps": done, "window": W,
+        "algorithmic_bytes_per_step": int(bytes_step),
+        "hbm_frac": round(bytes_step / (per * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "mufu_frac": round(exps_step / (per * 1e-3) / 1e9 / mufu, 4),
+        "gpu_launches_per_step": launches / done,
+        "step": f"ssm_replay_state_update (checkpoint every {W} tokens, bf16 copy for outputs), "
+                "256 rows x 8192 channels, fresh inputs per step"}
+    del rep, csr
+    return res
 
 
 # ---------------------------------------------------------------------------
@@ -623,8 +707,43 @@ def scan_sweep(variants, peaks):
     return 0
 
 
+def profile_decode(W):
+    """A few replay and eager decode steps at 256 x 8192 from random states
+    (about 0.5 GB on the device), for profiler captures; prints nothing timed."""
+    import torch
+
+    import selective_state_space_causal_b200 as ssm
+    from selective_state_space_causal_b200 import synth
+
+    Bt, D = 256, 8192
+    ly = Layer(D)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1)
+    h = 0.3 * torch.randn((Bt, D, N_STATE), device="cuda", generator=g)
+    cs = torch.randn((Bt, D, 3), device="cuda", generator=g).to(torch.bfloat16)
+    rep = ssm.replay_buffers(Bt, D, W, "cuda", keep_lo=True)
+    rep["ckpt"].copy_(h)
+    ssm.ssm_replay_reset(rep)
+    ins = [synth.device_activations(10 + i, Bt, D) for i in range(4)]
+    y = torch.empty((Bt, D), dtype=torch.bfloat16, device="cuda")
+    for i in range(3 * W):
+        s = ins[i % 4]
+        ssm.ssm_replay_state_update(cs, rep, s["x"], s["dt"], s["B"], s["C"], y, ly.w, ly.A,
+                                    z=s["z"], conv_b=ly.b, Dskip=ly.Dskip, dt_bias=ly.dt_bias)
+    for i in range(3):
+        s = ins[i % 4]
+        ssm.ssm_selective_state_update(cs, h, s["x"], s["dt"], s["B"], s["C"], y, ly.w, ly.A,
+                                       z=s["z"], conv_b=ly.b, Dskip=ly.Dskip, dt_bias=ly.dt_bias)
+    torch.cuda.synchronize()
+    assert ssm.ssm_device_status() == 0
+    print(json.dumps({"profile_decode": {"window": W, "replay_steps": 3 * W, "eager_steps": 3}}))
+
+
 def main():
     args = parse_args()
+    if args.profile_decode is not None:
+        profile_decode(args.profile_decode)
+        return
     if args.impl == "reference":
         return bench_reference(args)
     if args.scan_sweep is not None:
@@ -647,7 +766,7 @@ def main():
                                 device_id=torch.device("cuda", local))
     peaks = load_peaks()
     res = bench_headline(args, world, peaks, local)
-    secondary = None if args.no_secondary else bench_secondary(peaks, world)
+    secondary = None if args.no_secondary else bench_secondary(peaks, world, replay_windows=tuple(args.replay_windows))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline()

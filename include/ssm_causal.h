@@ -44,6 +44,9 @@
  * - "PackMamba: Efficient Processing of Variable-Length Sequences in Mamba
  *   training", abstract: packed sequences with no information passed between
  *   sequences.
+ * - "ReplaySSM: Cache SSM Inputs, Not State", abstract: decode with the state
+ *   kept as a checkpoint plus the SSM inputs of recent tokens
+ *   (ssm_replay_state_update, ssm_replay_reset, ssm_replay_flush).
  */
 #ifndef SSM_CAUSAL_H
 #define SSM_CAUSAL_H
@@ -117,8 +120,8 @@ int ssm_scan_variant_for(int64_t S, int64_t D, int *states_per_lane, int *schedu
  * Device-side status of the library's kernels on the current device: 0 while
  * every bounded wait for a TMA tile or bulk copy completed; bit 0 set once a
  * scan kernel's wait gave up, bit 1 once a conv kernel's did, bit 2 once a
- * decode kernel's did (the results of that call are then unspecified; the
- * kernel still terminates). Synchronises the device.
+ * decode kernel's did, bit 3 once a replay decode kernel's did (the results
+ * of that call are then unspecified; the kernel still terminates). Synchronises the device.
  * clear != 0 resets the flags. Returns SSM_ERR_CUDA if the query itself fails.
  */
 int ssm_device_status(int clear);
@@ -227,6 +230,92 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
                                const int32_t *state_indices, int64_t n_slots, void *y,
                                int64_t Bt, int64_t D, int N, int K, ssm_dtype act_dtype,
                                ssm_dtype conv_state_dtype, ssm_stream_t stream);
+
+/*
+ * Replay decode: one token per row, with each slot's SSM state kept as a
+ * checkpoint plus the SSM inputs of the tokens since it.
+ * Follows "ReplaySSM: Cache SSM Inputs, Not State" (abstract): the recurrence
+ * is unrolled so that outputs are computed by replaying the buffered inputs
+ * from the checkpoint, the checkpoint is rewritten only once every W tokens,
+ * and a low-precision copy of the checkpoint serves the outputs of the other
+ * steps while the fp32 checkpoint alone feeds the recurrent update. The
+ * per-token math is that of ssm_selective_state_update (tp_builder.py,
+ * _add_mamba_tp_layer), computed with the same operations in the same order.
+ *
+ * For row b with slot s = state_indices[b] (or b) and j = buf_len[s] tokens
+ * buffered:
+ *   conv, conv-state shift, delta exactly as ssm_selective_state_update;
+ *   if j + 1 == W (a checkpoint step): h = ckpt[s] replayed over the j
+ *     buffered tokens and this one; ckpt[s] = h; ckpt_lo[s] = bf16(h);
+ *     buf_len[s] = 0;
+ *   else: h = ckpt_lo[s] (or ckpt[s] when ckpt_lo is NULL) replayed over the
+ *     j buffered tokens and this one; this token's (delta, delta*xc) becomes
+ *     buffer entry j and its B entry j; buf_len[s] = j + 1;
+ *   y[b] = (C[b].h + Dskip*xc) * silu(z[b]).
+ * Replaying a token is h = exp(delta*A)*h + (delta*xc)*B with that token's
+ * values. After a checkpoint step ckpt[s] holds bit-for-bit the state that
+ * ssm_selective_state_update would hold after the same tokens.
+ *
+ *   conv_state     (n_slots, D, K-1) of conv_state_dtype, updated in place
+ *   ckpt           (n_slots, D, N) fp32 checkpoint, rewritten on checkpoint steps
+ *   ckpt_lo        (n_slots, D, N) bf16 copy of ckpt, or NULL (outputs then read
+ *                  ckpt on every step)
+ *   buf            (n_slots, W-1, D, 2) fp32: (delta, delta*xc) of buffered
+ *                  tokens, oldest first; NULL allowed when W == 1
+ *   buf_B          (n_slots, W-1, N) fp32: B of buffered tokens; NULL when W == 1
+ *   buf_len        (n_slots) int32: tokens buffered per slot, 0..W-1 (a value
+ *                  outside is clamped into that range)
+ *   tickets        (n_slots) uint32 scratch: all zero before the first call
+ *                  (ssm_replay_reset zeroes them); every call leaves them zero.
+ *                  The channel blocks of a row count themselves here, and the
+ *                  last one advances buf_len.
+ *   W              checkpoint interval, 1..8 (W == 1 is eager decode plus the
+ *                  bf16 copy)
+ *   x, dt, z, B, C, conv_w, conv_b, A, Dskip, dt_bias, delta_softplus,
+ *   state_indices, n_slots, y, Bt, D, N, K, dtypes: as ssm_selective_state_update
+ * All of conv_state, ckpt, ckpt_lo, buf, buf_B, x, dt, z, B, C and A must be
+ * 16-byte aligned and D * element size of x (and D * (K-1) * element size of
+ * the conv state) a multiple of 16 bytes, else SSM_ERR_MISALIGNED. Two rows
+ * naming the same slot race (undefined result). Before the first step of a
+ * window, ckpt must hold the state and ssm_replay_reset must have run.
+ */
+int ssm_replay_state_update(void *conv_state, float *ckpt, void *ckpt_lo, float *buf,
+                            float *buf_B, int32_t *buf_len, uint32_t *tickets, int W,
+                            const void *x, const void *dt, const void *B, const void *C,
+                            const void *z, const float *conv_w, const float *conv_b,
+                            const float *A, const float *Dskip, const float *dt_bias,
+                            int delta_softplus, const int32_t *state_indices, int64_t n_slots,
+                            void *y, int64_t Bt, int64_t D, int N, int K, ssm_dtype act_dtype,
+                            ssm_dtype conv_state_dtype, ssm_stream_t stream);
+
+/*
+ * Starts the replay window of each listed slot at the state held in ckpt
+ * (for example a prefill's final state): ckpt_lo[s] = bf16(ckpt[s]) when
+ * ckpt_lo is not NULL, buf_len[s] = 0, tickets[s] = 0.
+ * ("ReplaySSM: Cache SSM Inputs, Not State", abstract: checkpoint plus input
+ * buffer.)
+ *   slots  (n) int32 slot numbers, or NULL for slots 0..n-1; entries outside
+ *          [0, n_slots) are skipped
+ *   ckpt (n_slots, D, N) fp32; ckpt_lo (n_slots, D, N) bf16 or NULL; both
+ *   16-byte aligned. N must be 16.
+ */
+int ssm_replay_reset(const float *ckpt, void *ckpt_lo, int32_t *buf_len, uint32_t *tickets,
+                     const int32_t *slots, int64_t n, int64_t n_slots, int64_t D, int N,
+                     ssm_stream_t stream);
+
+/*
+ * Replays every buffered token of each listed slot into its fp32 checkpoint,
+ * refreshes the bf16 copy and empties the buffer (buf_len[s] = 0), with the
+ * arithmetic of a checkpoint step. Afterwards ckpt[s] is the slot's current
+ * state, as ssm_selective_state_update would hold it; use it to hand a slot
+ * back to eager decode or to read its state. Two launches (the lengths are
+ * cleared after every channel has read them).
+ *   Arguments as ssm_replay_state_update and ssm_replay_reset.
+ */
+int ssm_replay_flush(float *ckpt, void *ckpt_lo, const float *buf, const float *buf_B,
+                     int32_t *buf_len, uint32_t *tickets, const float *A, int W,
+                     const int32_t *slots, int64_t n, int64_t n_slots, int64_t D, int N,
+                     ssm_stream_t stream);
 
 /*
  * ssm_selective_scan_fwd without a workspace, for callers that cannot

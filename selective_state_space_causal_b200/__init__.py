@@ -10,11 +10,15 @@ from ._lib import (  # noqa: F401
     SSM_F32,
     SsmError,
     lib,
+    replay_buffers,
     ssm_causal_conv1d,
     ssm_check_cu_seqlens,
     ssm_last_error,
     ssm_launch_count,
     ssm_device_status,
+    ssm_replay_flush,
+    ssm_replay_reset,
+    ssm_replay_state_update,
     ssm_scan_workspace_size,
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_noalloc,

@@ -40,6 +40,12 @@ SIGNATURES = [
     ("ssm_selective_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _int, _vp, _i64, _vp, _i64, _i64, _int, _int, _int,
                                           _int, _vp]),
+    ("ssm_replay_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
+                                       _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _i64, _vp, _i64,
+                                       _i64, _int, _int, _int, _int, _vp]),
+    ("ssm_replay_reset", _int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp]),
+    ("ssm_replay_flush", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _i64, _i64, _i64,
+                                _int, _vp]),
 ]
 
 
@@ -196,3 +202,61 @@ def ssm_selective_state_update(conv_state, ssm_state, x, dt, B, C, y, conv_w, A,
         _ptr(conv_w), _ptr(conv_b), _ptr(A), _ptr(Dskip), _ptr(dt_bias), int(bool(delta_softplus)),
         _ptr(state_indices), ssm_state.shape[0], _ptr(y), Bt, D, N, K, _dtype(x),
         _dtype(conv_state), _stream(stream)))
+
+
+def replay_buffers(n_slots: int, D: int, W: int, device, N: int = 16, keep_lo: bool = True):
+    """Allocate the replay representation's tensors (torch, on `device`) in the
+    layouts ssm_replay_state_update documents: ckpt (n_slots, D, N) fp32,
+    ckpt_lo (n_slots, D, N) bf16 or None, buf (n_slots, W-1, D, 2) fp32,
+    buf_B (n_slots, W-1, N) fp32, buf_len (n_slots) int32, tickets (n_slots)
+    int32 used as uint32. Values are zero; fill ckpt, then call ssm_replay_reset."""
+    import torch
+
+    e = max(W - 1, 1)
+    return {
+        "ckpt": torch.zeros((n_slots, D, N), dtype=torch.float32, device=device),
+        "ckpt_lo": torch.zeros((n_slots, D, N), dtype=torch.bfloat16, device=device)
+        if keep_lo else None,
+        "buf": torch.zeros((n_slots, e, D, 2), dtype=torch.float32, device=device),
+        "buf_B": torch.zeros((n_slots, e, N), dtype=torch.float32, device=device),
+        "buf_len": torch.zeros(n_slots, dtype=torch.int32, device=device),
+        "tickets": torch.zeros(n_slots, dtype=torch.int32, device=device),
+        "W": int(W),
+    }
+
+
+def ssm_replay_state_update(conv_state, rep, x, dt, B, C, y, conv_w, A, z=None, conv_b=None,
+                            Dskip=None, dt_bias=None, delta_softplus=True, state_indices=None,
+                            stream=None):
+    """One replay decode step; `rep` holds the tensors of replay_buffers()."""
+    Bt, D = x.shape
+    N = A.shape[1]
+    K = conv_w.shape[1]
+    ck = rep["ckpt"]
+    _check(lib.ssm_replay_state_update(
+        _ptr(conv_state), _ptr(ck), _ptr(rep["ckpt_lo"]), _ptr(rep["buf"]), _ptr(rep["buf_B"]),
+        _ptr(rep["buf_len"]), _ptr(rep["tickets"]), int(rep["W"]), _ptr(x), _ptr(dt), _ptr(B),
+        _ptr(C), _ptr(z), _ptr(conv_w), _ptr(conv_b), _ptr(A), _ptr(Dskip), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(state_indices), ck.shape[0], _ptr(y), Bt, D, N, K,
+        _dtype(x), _dtype(conv_state), _stream(stream)))
+
+
+def ssm_replay_reset(rep, slots=None, n=None, stream=None):
+    """Start the listed slots' windows (all slots if None) at the states in rep['ckpt']."""
+    ck = rep["ckpt"]
+    n_slots, D, N = ck.shape
+    n = (slots.numel() if slots is not None else n_slots) if n is None else n
+    _check(lib.ssm_replay_reset(_ptr(ck), _ptr(rep["ckpt_lo"]), _ptr(rep["buf_len"]),
+                                _ptr(rep["tickets"]), _ptr(slots), n, n_slots, D, N,
+                                _stream(stream)))
+
+
+def ssm_replay_flush(rep, A, slots=None, n=None, stream=None):
+    """Replay the listed slots' buffers into rep['ckpt'] and empty them."""
+    ck = rep["ckpt"]
+    n_slots, D, N = ck.shape
+    n = (slots.numel() if slots is not None else n_slots) if n is None else n
+    _check(lib.ssm_replay_flush(_ptr(ck), _ptr(rep["ckpt_lo"]), _ptr(rep["buf"]),
+                                _ptr(rep["buf_B"]), _ptr(rep["buf_len"]), _ptr(rep["tickets"]),
+                                _ptr(A), int(rep["W"]), _ptr(slots), n, n_slots, D, N,
+                                _stream(stream)))

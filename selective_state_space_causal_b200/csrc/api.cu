@@ -22,6 +22,34 @@ int read_conv_status(bool clear);
 int read_decode_status(bool clear);
 cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
 int64_t noalloc_max_sequences();
+int read_replay_status(bool clear);
+
+struct ReplayStepArgs {
+    void *conv_state;
+    float *ckpt;
+    void *ckpt_lo;
+    float *buf, *bufB;
+    int32_t *len;
+    uint32_t *tickets;
+    int W;
+    const void *x, *dt, *B, *C, *z;
+    const float *conv_w, *conv_b, *A, *Dskip, *dt_bias;
+    int delta_softplus;
+    const int32_t *idx;
+    int64_t n_slots;
+    void *y;
+    int64_t Bt, D;
+    int K;
+    bool act_bf16, conv_bf16;
+};
+cudaError_t launch_replay_step(const ReplayStepArgs &a, cudaStream_t stream, int *launches);
+cudaError_t launch_replay_reset(const float *ckpt, void *ckpt_lo, int32_t *len, uint32_t *tickets,
+                                const int32_t *slots, int64_t n, int64_t n_slots, int64_t D,
+                                cudaStream_t stream, int *launches);
+cudaError_t launch_replay_flush(float *ckpt, void *ckpt_lo, const float *buf, const float *bufB,
+                                int32_t *len, uint32_t *tickets, const float *A, int W,
+                                const int32_t *slots, int64_t n, int64_t n_slots, int64_t D,
+                                cudaStream_t stream, int *launches);
 }  // namespace ssm
 
 namespace {
@@ -114,9 +142,11 @@ int ssm_device_status(int clear)
     const int a = ssm::read_scan_status(clear != 0);
     const int b = ssm::read_conv_status(clear != 0);
     const int d = ssm::read_decode_status(clear != 0);
-    if (a < 0 || b < 0 || d < 0) return fail(SSM_ERR_CUDA, "ssm_device_status: CUDA query failed");
+    const int r = ssm::read_replay_status(clear != 0);
+    if (a < 0 || b < 0 || d < 0 || r < 0)
+        return fail(SSM_ERR_CUDA, "ssm_device_status: CUDA query failed");
     g_error.clear();
-    return (a ? 1 : 0) | (b ? 2 : 0) | (d ? 4 : 0);
+    return (a ? 1 : 0) | (b ? 2 : 0) | (d ? 4 : 0) | (r ? 8 : 0);
 }
 
 int ssm_check_cu_seqlens(const int32_t *cu, int64_t S, int64_t tok)
@@ -256,6 +286,104 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
                       dt(conv_state_dtype)};
     int launched = 0;
     cudaError_t e = ssm::launch_decode(a, reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
+// Shared checks of a replay slot list (NULL = slots 0..n-1).
+static int check_replay_slots(const char *fn, const int32_t *slots, int64_t n, int64_t n_slots,
+                              int64_t D, int N)
+{
+    if (N != 16) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: N must be 16 (got %d)", fn, N);
+    if (D < 1 || n < 0 || n > 65535 || n_slots < 0)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: bad sizes (D=%lld, n=%lld, n_slots=%lld)", fn,
+                    (long long)D, (long long)n, (long long)n_slots);
+    if (!slots && n > n_slots)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: without a slot list, n must be <= n_slots", fn);
+    if (!aligned(slots, 4)) return fail(SSM_ERR_MISALIGNED, "%s: slots misaligned", fn);
+    return SSM_OK;
+}
+
+int ssm_replay_state_update(void *conv_state, float *ckpt, void *ckpt_lo, float *buf,
+                            float *buf_B, int32_t *buf_len, uint32_t *tickets, int W,
+                            const void *x, const void *dt_, const void *B, const void *C,
+                            const void *z, const float *conv_w, const float *conv_b,
+                            const float *A, const float *Dskip, const float *dt_bias,
+                            int delta_softplus, const int32_t *state_indices, int64_t n_slots,
+                            void *y, int64_t Bt, int64_t D, int N, int K, ssm_dtype act_dtype,
+                            ssm_dtype conv_state_dtype, ssm_stream_t stream)
+{
+    const char *fn = "ssm_replay_state_update";
+    if (!valid_dtype(act_dtype) || !valid_dtype(conv_state_dtype))
+        return fail(SSM_ERR_UNSUPPORTED_DTYPE, "%s: unknown dtype", fn);
+    if (N != 16) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: N must be 16 (got %d)", fn, N);
+    if (K < 2 || K > 4) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: K must be 2..4 (got %d)", fn, K);
+    if (W < 1 || W > 8) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: W must be 1..8 (got %d)", fn, W);
+    if (D < 1 || Bt < 0 || Bt > 65535 || n_slots < 0)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: bad sizes (D=%lld, Bt=%lld, n_slots=%lld)", fn,
+                    (long long)D, (long long)Bt, (long long)n_slots);
+    if (!state_indices && n_slots < Bt)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: identity slots need n_slots >= Bt", fn);
+    if (Bt > 0 && (!conv_state || !ckpt || !buf_len || !tickets || !x || !dt_ || !B || !C ||
+                   !conv_w || !A || !y))
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: a required pointer is NULL", fn);
+    if (Bt > 0 && W > 1 && (!buf || !buf_B))
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: W > 1 needs buf and buf_B", fn);
+    const size_t es = esize(act_dtype), cs = esize(conv_state_dtype);
+    if (!aligned(conv_w, 4) || !aligned(conv_b, 4) || !aligned(Dskip, 4) ||
+        !aligned(dt_bias, 4) || !aligned(state_indices, 4) || !aligned(buf_len, 4) ||
+        !aligned(tickets, 4) || !aligned(y, es))
+        return fail(SSM_ERR_MISALIGNED, "%s: a pointer is not aligned to its element size", fn);
+    if (!aligned(conv_state, 16) || !aligned(ckpt, 16) || !aligned(ckpt_lo, 16) ||
+        !aligned(buf, 16) || !aligned(buf_B, 16) || !aligned(x, 16) || !aligned(dt_, 16) ||
+        !aligned(z, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(A, 16) ||
+        (D * (int64_t)es) % 16 != 0 || (D * (K - 1) * (int64_t)cs) % 16 != 0)
+        return fail(SSM_ERR_MISALIGNED,
+                    "%s: conv_state, ckpt, ckpt_lo, buf, buf_B, x, dt, z, B, C and A must be "
+                    "16-byte aligned, and D * element size (and D * (K-1) * conv-state element "
+                    "size) multiples of 16 bytes", fn);
+    ssm::ReplayStepArgs a{conv_state, ckpt, ckpt_lo, buf, buf_B, buf_len, tickets, W, x, dt_, B,
+                          C, z, conv_w, conv_b, A, Dskip, dt_bias, delta_softplus,
+                          state_indices, n_slots, y, Bt, D, K, act_dtype == SSM_BF16,
+                          conv_state_dtype == SSM_BF16};
+    int launched = 0;
+    cudaError_t e = ssm::launch_replay_step(a, reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
+int ssm_replay_reset(const float *ckpt, void *ckpt_lo, int32_t *buf_len, uint32_t *tickets,
+                     const int32_t *slots, int64_t n, int64_t n_slots, int64_t D, int N,
+                     ssm_stream_t stream)
+{
+    const char *fn = "ssm_replay_reset";
+    if (int r = check_replay_slots(fn, slots, n, n_slots, D, N)) return r;
+    if (n > 0 && (!buf_len || !tickets || (ckpt_lo && !ckpt)))
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: a required pointer is NULL", fn);
+    if (!aligned(ckpt, 16) || !aligned(ckpt_lo, 16) || !aligned(buf_len, 4) || !aligned(tickets, 4))
+        return fail(SSM_ERR_MISALIGNED, "%s: ckpt and ckpt_lo must be 16-byte aligned", fn);
+    int launched = 0;
+    cudaError_t e = ssm::launch_replay_reset(ckpt, ckpt_lo, buf_len, tickets, slots, n, n_slots,
+                                             D, reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
+int ssm_replay_flush(float *ckpt, void *ckpt_lo, const float *buf, const float *buf_B,
+                     int32_t *buf_len, uint32_t *tickets, const float *A, int W,
+                     const int32_t *slots, int64_t n, int64_t n_slots, int64_t D, int N,
+                     ssm_stream_t stream)
+{
+    const char *fn = "ssm_replay_flush";
+    if (W < 1 || W > 8) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: W must be 1..8 (got %d)", fn, W);
+    if (int r = check_replay_slots(fn, slots, n, n_slots, D, N)) return r;
+    if (n > 0 && (!ckpt || !buf_len || !tickets || !A || (W > 1 && (!buf || !buf_B))))
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: a required pointer is NULL", fn);
+    if (!aligned(ckpt, 16) || !aligned(ckpt_lo, 16) || !aligned(buf, 16) || !aligned(buf_B, 16) ||
+        !aligned(A, 16) || !aligned(buf_len, 4) || !aligned(tickets, 4))
+        return fail(SSM_ERR_MISALIGNED,
+                    "%s: ckpt, ckpt_lo, buf, buf_B and A must be 16-byte aligned", fn);
+    int launched = 0;
+    cudaError_t e = ssm::launch_replay_flush(ckpt, ckpt_lo, buf, buf_B, buf_len, tickets, A, W,
+                                             slots, n, n_slots, D,
+                                             reinterpret_cast<cudaStream_t>(stream), &launched);
     return finish(e, launched, fn);
 }
 

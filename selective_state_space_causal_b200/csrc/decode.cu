@@ -157,7 +157,7 @@ decode_kernel(const Params p, const int64_t Bt)
             for (int k = 0; k < K; ++k) acc = fmaf(wk[k], win[r][k], acc);
             xcv = silu_f(acc);
             float d = dtv[r] + dtb;
-            if (p.delta_softplus) d = softplus_f(d);
+            if (p.delta_softplus) d = softplus_fast(d);
             const float dx = d * xcv;
             float hv[8] = {ha[r].x, ha[r].y, ha[r].z, ha[r].w, hb[r].x, hb[r].y, hb[r].z, hb[r].w};
 #pragma unroll
@@ -325,7 +325,7 @@ decode_bulk_kernel(const Params p, const int64_t Bt)
 #pragma unroll
             for (int k = 0; k < K; ++k) acc = fmaf(w[k], win[k], acc);
             const float xcv = silu_f(acc);
-            if (p.delta_softplus) d = softplus_f(d);
+            if (p.delta_softplus) d = softplus_fast(d);
             const float dx = d * xcv;
             const f32x2 dd = pk2(d, d), xx = pk2(dx, dx);
             const T *Bp = static_cast<const T *>(p.B) + b * kN;

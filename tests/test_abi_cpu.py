@@ -158,3 +158,53 @@ def test_variant_choice():
         with pytest.raises(ssm.SsmError) as ei:
             ssm.ssm_scan_variant_for(S, D)
         assert ei.value.code == -1
+
+
+def replay(**kw):
+    a = dict(cs=A16, ck=A16, lo=A16, buf=A16, bB=A16, ln=A16, tk=A16, W=4, x=A16, dt=A16, B=A16,
+             C=A16, z=None, w=A16, b=None, A=A16, Dsk=None, dtb=None, sp=1, idx=None, slots=8,
+             y=A16, Bt=8, D=32, N=16, K=4, adt=1, cdt=1)
+    a.update(kw)
+    return L.ssm_replay_state_update(a["cs"], a["ck"], a["lo"], a["buf"], a["bB"], a["ln"], a["tk"],
+                                     a["W"], a["x"], a["dt"], a["B"], a["C"], a["z"], a["w"],
+                                     a["b"], a["A"], a["Dsk"], a["dtb"], a["sp"], a["idx"],
+                                     a["slots"], a["y"], a["Bt"], a["D"], a["N"], a["K"], a["adt"],
+                                     a["cdt"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(W=0), -1), (dict(W=9), -1), (dict(N=8), -1), (dict(K=5), -1), (dict(slots=4), -1),
+    (dict(ck=None), -1), (dict(tk=None), -1), (dict(ln=None), -1), (dict(buf=None), -1),
+    (dict(bB=None), -1), (dict(ck=A16 + 4), -3), (dict(lo=A16 + 8), -3), (dict(buf=A16 + 8), -3),
+    (dict(D=36), -3), (dict(D=4, adt=0, cdt=1, K=4), -3), (dict(x=A16 + 2), -3), (dict(adt=4), -2),
+    (dict(Bt=70000, slots=70000), -1),
+])
+def test_replay_rejects(kw, code):
+    assert replay(**kw) == code
+    assert _err()
+
+
+def test_replay_window_one_needs_no_buffer():
+    # W == 1 takes no buffer; with Bt == 0 nothing is launched, so this runs without a GPU
+    assert replay(W=1, buf=None, bB=None, Bt=0) == 0
+
+
+@pytest.mark.parametrize("fn,kw,code", [
+    ("reset", dict(N=8), -1), ("reset", dict(n=9, slots_ptr=None), -1),
+    ("reset", dict(ln=None), -1), ("reset", dict(lo=A16 + 8), -3),
+    ("reset", dict(slots_ptr=A16 + 2), -3),
+    ("flush", dict(W=0), -1), ("flush", dict(A=None), -1), ("flush", dict(buf=None), -1),
+    ("flush", dict(ck=A16 + 4), -3), ("flush", dict(n=-1), -1),
+])
+def test_replay_reset_flush_reject(fn, kw, code):
+    a = dict(ck=A16, lo=A16, buf=A16, bB=A16, ln=A16, tk=A16, A=A16, W=4, slots_ptr=None, n=8,
+             n_slots=8, D=32, N=16)
+    a.update(kw)
+    if fn == "reset":
+        rc = L.ssm_replay_reset(a["ck"], a["lo"], a["ln"], a["tk"], a["slots_ptr"], a["n"],
+                                a["n_slots"], a["D"], a["N"], None)
+    else:
+        rc = L.ssm_replay_flush(a["ck"], a["lo"], a["buf"], a["bB"], a["ln"], a["tk"], a["A"],
+                                a["W"], a["slots_ptr"], a["n"], a["n_slots"], a["D"], a["N"], None)
+    assert rc == code
+    assert _err()
