@@ -242,19 +242,21 @@ class HeadlineStep:
     def scan_exps(self):
         return self.tok * self.D * N_STATE
 
-    def run(self, i, ev=None, inputs=None, dec_inputs=None):
+    def run(self, i, ev=None, inputs=None, dec_inputs=None, y=None, yd=None):
         ssm, ly = self.ssm, self.layer
         a = inputs if inputs is not None else self.sets[i % self.SETS]
         d = dec_inputs if dec_inputs is not None else self.dec[i % self.SETS]
+        y = self.y if y is None else y
+        yd = self.yd if yd is None else yd
         ssm.ssm_causal_conv1d(a["x"], self.xc, ly.w, bias=ly.b, S=self.Bn,
                               conv_state_out=self.cs)
         if ev is not None:
             ev[0].record()
-        ssm.ssm_selective_scan_fwd(self.xc, a["dt"], ly.A, a["B"], a["C"], self.y, Dskip=ly.Dskip,
+        ssm.ssm_selective_scan_fwd(self.xc, a["dt"], ly.A, a["B"], a["C"], y, Dskip=ly.Dskip,
                                    z=a["z"], dt_bias=ly.dt_bias, h_final=self.h, S=self.Bn)
         if ev is not None:
             ev[1].record()
-        ssm.ssm_selective_state_update(self.cs, self.h, d["x"], d["dt"], d["B"], d["C"], self.yd,
+        ssm.ssm_selective_state_update(self.cs, self.h, d["x"], d["dt"], d["B"], d["C"], yd,
                                        ly.w, ly.A, z=d["z"], conv_b=ly.b, Dskip=ly.Dskip,
                                        dt_bias=ly.dt_bias)
 
@@ -333,10 +335,66 @@ def bench_headline(args, world, peaks, rank_dev):
         e2e_step(i)
     stop.record()
     _barrier_sync(world)
+    ems_serial = _max_over_ranks(start.elapsed_time(stop) / Ke, world)
+
+    # The same steps pipelined the way a serving loop runs them: step i+1's
+    # inputs are copied in (one stream) while step i computes (a second) and
+    # step i-1's outputs are copied out (a third), with double-buffered device
+    # inputs and outputs; every step still copies its own inputs in and its
+    # own outputs out inside the timed region.
+    s_in, s_cmp, s_out = (torch.cuda.Stream() for _ in range(3))
+    dev_in2 = [dev_in, {k: torch.empty_like(v) for k, v in dev_in.items()}]
+    dev_dec2 = [dev_dec, {k: torch.empty_like(v) for k, v in dev_dec.items()}]
+    y2 = [st.y, torch.empty_like(st.y)]
+    yd2 = [st.yd, torch.empty_like(st.yd)]
+    y_host2 = [y_host, torch.empty_like(y_host).pin_memory()]
+    yd_host2 = [yd_host, torch.empty_like(yd_host).pin_memory()]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def pipelined(n):
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_cmp[b])  # step i-2 has read these inputs
+                for k in dev_in2[b]:
+                    dev_in2[b][k].copy_(host_in[k], non_blocking=True)
+                for k in dev_dec2[b]:
+                    dev_dec2[b][k].copy_(host_dec[k], non_blocking=True)
+                ev_in[b].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(ev_in[b])
+                if i >= 2:
+                    s_cmp.wait_event(ev_out[b])  # step i-2's outputs are copied out
+                st.run(i, inputs=dev_in2[b], dec_inputs=dev_dec2[b], y=y2[b], yd=yd2[b])
+                ev_cmp[b].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_cmp[b])
+                y_host2[b].copy_(y2[b], non_blocking=True)
+                yd_host2[b].copy_(yd2[b], non_blocking=True)
+                ev_out[b].record(s_out)
+
+    torch.cuda.synchronize()
+    pipelined(max(3, args.warmup // 4))
+    torch.cuda.synchronize()
+    _barrier_sync(world)
+    start.record(s_in)
+    pipelined(Ke)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cmp)
+    stop.record(s_out)
+    torch.cuda.synchronize()
+    _barrier_sync(world)
     ems = _max_over_ranks(start.elapsed_time(stop) / Ke, world)
     res["e2e"] = {"value": whole_job_rate(st.units(), world, ems), "unit": UNIT,
                   "ms_per_step": ems, "h2d_bytes_per_step": int(h2d),
-                  "d2h_bytes_per_step": int(d2h)}
+                  "d2h_bytes_per_step": int(d2h),
+                  "how": "pipelined: copy-in, compute and copy-out streams, double-buffered"}
+    res["e2e_serial"] = {"value": whole_job_rate(st.units(), world, ems_serial), "unit": UNIT,
+                         "ms_per_step": ems_serial,
+                         "how": "copy in, compute, copy out, one step after another"}
     del st
     torch.cuda.empty_cache()
     return res
@@ -782,7 +840,7 @@ def main():
                        "l2": "4 rotating input sets (~600 MB) larger than L2",
                        "parallelism": f"replicas x{world}"},
             "roofline": res["roofline"], "clocks": res["clocks"], "e2e": res["e2e"],
-            "gpu_launches": res["gpu_launches"], "cpu_baseline": cpu, "workloads": secondary,
+            "e2e_serial": res["e2e_serial"], "gpu_launches": res["gpu_launches"], "cpu_baseline": cpu, "workloads": secondary,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
