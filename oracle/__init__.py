@@ -9,7 +9,8 @@ and returns new arrays; the wrappers do data marshalling only.
 Parity pins: the closed-form geometric series, the brute-force unrolled sum,
 ``numpy.correlate`` for the convolution, the packing, chunking and decode
 invariants, the equality of replay decode with eager decode, bit-level bf16
-rounding and a hand-worked dyadic example all pin these routines (see the
+rounding, central finite differences of the forward scan (for its backward) and
+a hand-worked dyadic example all pin these routines (see the
 ``tests/test_oracle_*.py`` files). No function here is "parity unpinned".
 """
 
@@ -96,6 +97,11 @@ class Oracle:
                                            _dp, _dp, _dp, _dp, _dp, _dp, _dp, _int, _ip, _i64, _dp,
                                            _i64, _i64, _int, _int]
         lib.oracle_replay_step.restype = None
+        lib.oracle_selective_scan_bwd.argtypes = [_dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _int,
+                                                  _dp, _ip, _i64, _i64, _i64, _int, _dp, _dp,
+                                                  _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp, _dp,
+                                                  _dp]
+        lib.oracle_selective_scan_bwd.restype = None
         lib.oracle_num_threads.restype = _int
         lib.oracle_set_num_threads.argtypes = [_int]
         self.lib = lib
@@ -144,6 +150,32 @@ class Oracle:
                                        _ptr(args[5]), int(delta_softplus), _ptr(args[6]),
                                        _iptr(cu), S, tok, D, N, _ptr(y), _ptr(hf))
         return (y, hf) if want_state else y
+
+    def selective_scan_bwd(self, u, delta, A, B, C, dy, Dskip=None, z=None, dt_bias=None,
+                           delta_softplus=True, h0=None, cu_seqlens=None, S=None,
+                           dh_final=None):
+        """Gradients of sum(dy * y) + sum(dh_final * h_final) with respect to every
+        input of selective_scan. Returns a dict: du, ddt, dz (or None), dB, dC, dA,
+        dDskip, ddt_bias, dh0."""
+        u = _f64(u)
+        tok, D = u.shape
+        A = _f64(A)
+        N = A.shape[1]
+        cu = _cu(cu_seqlens, tok, S)
+        S = len(cu) - 1
+        out = {"du": np.zeros((tok, D)), "ddt": np.zeros((tok, D)),
+               "dz": np.zeros((tok, D)) if z is not None else None,
+               "dB": np.zeros((tok, N)), "dC": np.zeros((tok, N)), "dA": np.zeros((D, N)),
+               "dDskip": np.zeros(D), "ddt_bias": np.zeros(D), "dh0": np.zeros((S, D, N))}
+        work = np.zeros(((tok + S + 1) * N,))
+        args = [_f64(a) for a in (delta, B, C, Dskip, z, dt_bias, h0, dy, dh_final)]
+        self.lib.oracle_selective_scan_bwd(
+            _ptr(u), _ptr(args[0]), _ptr(A), _ptr(args[1]), _ptr(args[2]), _ptr(args[3]),
+            _ptr(args[4]), _ptr(args[5]), int(delta_softplus), _ptr(args[6]), _iptr(cu), S, tok,
+            D, N, _ptr(args[7]), _ptr(args[8]), _ptr(out["du"]), _ptr(out["ddt"]),
+            _ptr(out["dz"]), _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dA"]),
+            _ptr(out["dDskip"]), _ptr(out["ddt_bias"]), _ptr(out["dh0"]), _ptr(work))
+        return out
 
     # -- decode ------------------------------------------------------------
     def state_update(self, conv_state, ssm_state, x, dt, B, C, z, conv_w, conv_b, A, Dskip,

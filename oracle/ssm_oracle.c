@@ -328,3 +328,99 @@ void oracle_replay_step(double *conv_state, double *ck, double *ck_lo, double *b
         len[s] = flush ? 0 : j + 1;
     }
 }
+
+/*
+ * Gradients of the selective scan (the training backward pass that PackMamba's
+ * packed sequences need: "PackMamba: Efficient Processing of Variable-Length
+ * Sequences in Mamba training", abstract), written from the chain rule of the
+ * forward definition above, sequence by sequence, with no flow across a
+ * cu_seqlens boundary. For each (sequence, channel), with v_t = dt_t + dt_bias,
+ * D_t = softplus(v_t) (or v_t), a_t[n] = exp(D_t A[n]), h_t = a_t h_{t-1} +
+ * D_t u_t B_t, q_t = sum_n C_t[n] h_t[n] + Dskip u_t, g_t = silu(z_t) (or 1),
+ * y_t = q_t g_t, and an upstream gradient dy_t (plus dh_final for the last
+ * state):
+ *   dq_t = dy_t g_t;  dz_t = dy_t q_t silu'(z_t);  dDskip += dq_t u_t;
+ *   G_t[n] = dq_t C_t[n] + a_{t+1}[n] G_{t+1}[n]   (G after the last token =
+ *            dh_final, carried backwards; it is dL/dh_t)
+ *   dC_t[n] += dq_t h_t[n];   dB_t[n] += G_t[n] D_t u_t;
+ *   du_t = dq_t Dskip + sum_n G_t[n] D_t B_t[n];
+ *   dD_t = sum_n G_t[n] (u_t B_t[n] + A[n] a_t[n] h_{t-1}[n]);
+ *   dA[n] += G_t[n] D_t a_t[n] h_{t-1}[n];
+ *   ddt_t = dD_t softplus'(v_t) (= dD_t when the softplus is off);
+ *   ddt_bias += ddt_t;   dh0[n] = a_{t0}[n] G_{t0}[n] for the first token t0.
+ * The forward states h_t are recomputed and kept for the whole sequence.
+ * Outputs: du, ddt, dz (tok, D) (dz only with z); dB, dC (tok, N) summed over
+ * channels; dA (D, N), dDskip, ddt_bias (D) summed over sequences; dh0 (S, D, N).
+ * Every output array is written (overwritten), not accumulated into.
+ */
+void oracle_selective_scan_bwd(const double *u, const double *delta, const double *A,
+                               const double *B, const double *C, const double *Dskip,
+                               const double *z, const double *dt_bias, int delta_softplus,
+                               const double *h0, const int64_t *cu, int64_t S, int64_t tok,
+                               int64_t D, int N, const double *dy, const double *dh_final,
+                               double *du, double *ddt, double *dz, double *dB, double *dC,
+                               double *dA, double *dDskip, double *ddt_bias, double *dh0,
+                               double *work)
+{
+    if (N > ORACLE_MAX_N) return;
+    /* work: (tok + S) * N doubles of state history, one channel at a time */
+    for (int64_t i = 0; i < tok * N; ++i) dB[i] = dC[i] = 0.0;
+    for (int64_t i = 0; i < D * N; ++i) dA[i] = 0.0;
+    for (int64_t c = 0; c < D; ++c) {
+        if (dDskip) dDskip[c] = 0.0;
+        if (ddt_bias) ddt_bias[c] = 0.0;
+    }
+    for (int64_t s = 0; s < S; ++s) {
+        const int64_t t0 = cu[s], t1 = cu[s + 1], len = t1 - t0;
+        for (int64_t c = 0; c < D; ++c) {
+            /* hist[k] = h after k tokens of the sequence (hist[0] = h0) */
+            double *hist = work;
+            for (int n = 0; n < N; ++n) hist[n] = h0 ? h0[(s * D + c) * N + n] : 0.0;
+            for (int64_t k = 0; k < len; ++k) {
+                const int64_t t = t0 + k;
+                double d = delta[t * D + c] + (dt_bias ? dt_bias[c] : 0.0);
+                if (delta_softplus) d = softplus(d);
+                for (int n = 0; n < N; ++n)
+                    hist[(k + 1) * N + n] = exp(d * A[c * N + n]) * hist[k * N + n] +
+                                            d * u[t * D + c] * B[t * N + n];
+            }
+            double G[ORACLE_MAX_N];
+            for (int n = 0; n < N; ++n) G[n] = dh_final ? dh_final[(s * D + c) * N + n] : 0.0;
+            for (int64_t k = len - 1; k >= 0; --k) {
+                const int64_t t = t0 + k;
+                const double v = delta[t * D + c] + (dt_bias ? dt_bias[c] : 0.0);
+                const double d = delta_softplus ? softplus(v) : v;
+                const double dsp = delta_softplus ? 1.0 / (1.0 + exp(-v)) : 1.0;
+                const double ut = u[t * D + c];
+                const double *h = hist + (k + 1) * N, *hp = hist + k * N;
+                double q = (Dskip ? Dskip[c] : 0.0) * ut;
+                for (int n = 0; n < N; ++n) q += C[t * N + n] * h[n];
+                double g = 1.0, dg = 0.0;
+                if (z) {
+                    const double zt = z[t * D + c], sg = 1.0 / (1.0 + exp(-zt));
+                    g = zt * sg;
+                    dg = sg * (1.0 + zt * (1.0 - sg));
+                }
+                const double dq = dy[t * D + c] * g;
+                if (dz) dz[t * D + c] = z ? dy[t * D + c] * q * dg : 0.0;
+                if (dDskip) dDskip[c] += dq * ut;
+                double dut = dq * (Dskip ? Dskip[c] : 0.0), dd = 0.0;
+                for (int n = 0; n < N; ++n) {
+                    const double a = exp(d * A[c * N + n]);
+                    G[n] += dq * C[t * N + n];
+                    dC[t * N + n] += dq * h[n];
+                    dB[t * N + n] += G[n] * d * ut;
+                    dut += G[n] * d * B[t * N + n];
+                    dd += G[n] * (ut * B[t * N + n] + A[c * N + n] * a * hp[n]);
+                    dA[c * N + n] += G[n] * d * a * hp[n];
+                    G[n] *= a;
+                }
+                du[t * D + c] = dut;
+                ddt[t * D + c] = dd * dsp;
+                if (ddt_bias) ddt_bias[c] += dd * dsp;
+            }
+            if (dh0)
+                for (int n = 0; n < N; ++n) dh0[(s * D + c) * N + n] = G[n];
+        }
+    }
+}

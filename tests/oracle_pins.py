@@ -501,10 +501,97 @@ def check_replay_after_prefill(orc):
     assert np.array_equal(c, cs)
 
 
+# ---------------------------------------------------------------------------
+# backward scan (training): chain rule against finite differences
+# ---------------------------------------------------------------------------
+
+def _bwd_case(seed, lens, D, N, gate=True, softplus=True):
+    rng = np.random.default_rng(seed)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int64)
+    tok, S = int(cu[-1]), len(lens)
+    # the step size must stay positive: raw values through the softplus, or
+    # positive values directly when it is off
+    delta = 0.4 * rng.standard_normal((tok, D)) if softplus else 0.1 * np.abs(
+        rng.standard_normal((tok, D)))
+    f = {"u": rng.standard_normal((tok, D)), "delta": delta,
+         "A": -np.exp(rng.uniform(-1, 1, (D, N))), "B": rng.standard_normal((tok, N)),
+         "C": rng.standard_normal((tok, N)), "Dskip": rng.standard_normal(D),
+         "z": rng.standard_normal((tok, D)) if gate else None,
+         "dt_bias": rng.uniform(-2, -0.5, D) if softplus else rng.uniform(0.05, 0.3, D),
+         "h0": rng.standard_normal((S, D, N))}
+    w = {"dy": rng.standard_normal((tok, D)), "dh_final": rng.standard_normal((S, D, N))}
+    return f, w, cu, softplus
+
+
+def _loss(orc, f, w, cu, softplus):
+    y, hf = orc.selective_scan(f["u"], f["delta"], f["A"], f["B"], f["C"], Dskip=f["Dskip"],
+                               z=f["z"], dt_bias=f["dt_bias"], delta_softplus=softplus,
+                               h0=f["h0"], cu_seqlens=cu, want_state=True)
+    return float(np.sum(w["dy"] * y) + np.sum(w["dh_final"] * hf))
+
+
+def check_bwd_finite_differences(orc):
+    """Every gradient of the backward scan equals the central difference of the
+    forward scan's loss sum(dy*y) + sum(dh_final*h_final), element by element."""
+    names = {"u": "du", "delta": "ddt", "z": "dz", "B": "dB", "C": "dC", "A": "dA",
+             "Dskip": "dDskip", "dt_bias": "ddt_bias", "h0": "dh0"}
+    for gate, softplus, lens in ((True, True, [3, 0, 5]), (False, False, [4, 2])):
+        f, w, cu, sp = _bwd_case(121 + len(lens), lens, 2, 3, gate, softplus)
+        g = orc.selective_scan_bwd(f["u"], f["delta"], f["A"], f["B"], f["C"], w["dy"],
+                                   Dskip=f["Dskip"], z=f["z"], dt_bias=f["dt_bias"],
+                                   delta_softplus=sp, h0=f["h0"], cu_seqlens=cu,
+                                   dh_final=w["dh_final"])
+        eps = 1e-6
+        for name, gname in names.items():
+            if f[name] is None:
+                assert g[gname] is None
+                continue
+            arr = f[name]
+            num = np.zeros(arr.shape)
+            for idx in np.ndindex(arr.shape):
+                keep = arr[idx]
+                arr[idx] = keep + eps
+                lp = _loss(orc, f, w, cu, sp)
+                arr[idx] = keep - eps
+                lm = _loss(orc, f, w, cu, sp)
+                arr[idx] = keep
+                num[idx] = (lp - lm) / (2 * eps)
+            scale = max(np.max(np.abs(num)), 1.0)
+            err = np.max(np.abs(g[gname] - num)) / scale
+            assert err <= 1e-6, (name, gate, softplus, err)
+
+
+def check_bwd_pack_equals_separate(orc):
+    """A packed backward equals its sequences' backwards: per-token gradients
+    and dh0 exactly, the per-channel sums (dA, dDskip, ddt_bias) as the sum of
+    the separate runs."""
+    lens = [5, 1, 0, 7]
+    f, w, cu, sp = _bwd_case(131, lens, 3, 4)
+    g = orc.selective_scan_bwd(f["u"], f["delta"], f["A"], f["B"], f["C"], w["dy"],
+                               Dskip=f["Dskip"], z=f["z"], dt_bias=f["dt_bias"], h0=f["h0"],
+                               cu_seqlens=cu, dh_final=w["dh_final"])
+    tot = {k: np.zeros_like(g[k]) for k in ("dA", "dDskip", "ddt_bias")}
+    for s in range(len(lens)):
+        a, b = cu[s], cu[s + 1]
+        gs = orc.selective_scan_bwd(f["u"][a:b], f["delta"][a:b], f["A"], f["B"][a:b],
+                                    f["C"][a:b], w["dy"][a:b], Dskip=f["Dskip"],
+                                    z=f["z"][a:b], dt_bias=f["dt_bias"], h0=f["h0"][s:s + 1],
+                                    cu_seqlens=np.array([0, b - a]),
+                                    dh_final=w["dh_final"][s:s + 1])
+        for k in ("du", "ddt", "dz", "dB", "dC"):
+            assert np.array_equal(g[k][a:b], gs[k]), (s, k)
+        assert np.array_equal(g["dh0"][s], gs["dh0"][0]), s
+        for k in tot:
+            tot[k] += gs[k]
+    for k in tot:
+        assert _rel_err(g[k], tot[k]) <= 1e-14, k
+
+
 ALL_CHECKS = [
     check_softplus_spot, check_silu_spot, check_conv_identity_tap, check_closed_form,
     check_bruteforce, check_conv_correlate, check_pack_equals_separate,
     check_chunked_equals_oneshot, check_decode_invariant, check_state_indices,
     check_golden_dyadic, check_round_bf16, check_replay_equals_eager,
     check_replay_low_precision, check_replay_state_indices, check_replay_after_prefill,
+    check_bwd_finite_differences, check_bwd_pack_equals_separate,
 ]

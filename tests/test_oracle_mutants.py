@@ -70,6 +70,22 @@ MUTANTS = {
                              "ldexp(trunc(ldexp(m, 8)), e - 8)", 0),
     "round_bf16_seven_bits": ("ldexp(nearbyint(ldexp(m, 8)), e - 8)",
                               "ldexp(nearbyint(ldexp(m, 7)), e - 7)", 0),
+    "bwd_gradient_not_decayed": ("G[n] *= a;", "G[n] *= 1.0;", 0),
+    "bwd_readout_term_dropped": ("G[n] += dq * C[t * N + n];", "G[n] += 0.0 * C[t * N + n];", 0),
+    "bwd_softplus_derivative_dropped": (
+        "const double dsp = delta_softplus ? 1.0 / (1.0 + exp(-v)) : 1.0;",
+        "const double dsp = 1.0;", 0),
+    "bwd_dA_with_current_state": ("dA[c * N + n] += G[n] * d * a * hp[n];",
+                                  "dA[c * N + n] += G[n] * d * a * h[n];", 0),
+    "bwd_dB_without_u": ("dB[t * N + n] += G[n] * d * ut;", "dB[t * N + n] += G[n] * d;", 0),
+    "bwd_gate_derivative_wrong": ("dg = sg * (1.0 + zt * (1.0 - sg));", "dg = sg;", 0),
+    "bwd_skip_term_dropped": ("double dut = dq * (Dskip ? Dskip[c] : 0.0), dd = 0.0;",
+                              "double dut = 0.0, dd = 0.0;", 0),
+    "bwd_ddelta_state_term_dropped": (
+        "dd += G[n] * (ut * B[t * N + n] + A[c * N + n] * a * hp[n]);",
+        "dd += G[n] * (ut * B[t * N + n]);", 0),
+    "bwd_dC_with_state_gradient": ("dC[t * N + n] += dq * h[n];", "dC[t * N + n] += G[n] * h[n];",
+                                   0),
 }
 
 
