@@ -64,6 +64,9 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--replay-windows", type=int, nargs="+", default=[3], metavar="W",
                     help="checkpoint intervals of the replay decode measurement")
+    ap.add_argument("--profile-scan-bwd", action="store_true",
+                    help="instead of the step: run 3 backward scans over 16384 packed tokens of "
+                         "5120 channels (about 1.5 GB), untimed, for ncu captures")
     ap.add_argument("--profile-decode", type=int, default=None, metavar="W",
                     help="instead of the step: run 3 windows of replay decode steps (checkpoint "
                          "every W tokens, bf16 copy) and 3 eager decode steps at 256 x 8192 from "
@@ -452,7 +455,13 @@ def bench_secondary(peaks, world, steps_scale=1.0, replay_windows=(3,)):
         "gtoken_ch_per_s": tot * D * world / (ms * 1e-3) / 1e9, "ms_per_step": ms,
         "scan_ms": scan_ms, "scan_mufu_frac": round(tot * D * N_STATE / (scan_ms * 1e-3) / 1e9 / mufu, 4),
         "sequences": S, "step": "conv1d+selective_scan (packed, longest-first schedule)"}
-    del a, xc, y, cs, h, ws
+    del xc, y, cs, h, ws
+    torch.cuda.empty_cache()
+
+    # -- backward of the packed prefill's scan (PackMamba training) ---------
+    out["packmamba_2p8b_varlen_65536_scan_bwd"] = bench_scan_bwd(peaks, world, ly, a, cu, S,
+                                                                steps_scale)
+    del a
     torch.cuda.empty_cache()
 
     # -- long-context chunked prefill --------------------------------------
@@ -545,6 +554,56 @@ def bench_secondary(peaks, world, steps_scale=1.0, replay_windows=(3,)):
     del cs, h
     torch.cuda.empty_cache()
     return out
+
+
+def bench_scan_bwd(peaks, world, ly, a, cu, S, steps_scale=1.0):
+    """Backward of the selective scan on the packed prefill's inputs (bf16
+    activations, upstream gradient dy drawn like x). Algorithmic work per
+    (token, channel): 2 x 16 exponentials (the decays of one forward pass to
+    produce the states and of the reverse pass; the kernel executes 3 x 16, as
+    it recomputes the states chunk by chunk from checkpoints instead of storing
+    them) and 14 bytes (u, dt, z, dy in; du, ddelta, dz out)."""
+    import torch
+
+    import selective_state_space_causal_b200 as ssm
+    from selective_state_space_causal_b200 import synth
+
+    tok, D = a["x"].shape
+    dy = synth.device_activations(77, tok, D)["x"]
+    f32 = dict(device="cuda", dtype=torch.float32)
+    g = {"du": torch.empty_like(a["x"]), "ddelta": torch.empty_like(a["x"]),
+         "dz": torch.empty_like(a["x"]), "dB": torch.empty((tok, N_STATE), **f32),
+         "dC": torch.empty((tok, N_STATE), **f32), "dA": torch.empty((D, N_STATE), **f32),
+         "dDskip": torch.empty((D,), **f32), "ddt_bias": torch.empty((D,), **f32),
+         "dh0": torch.empty((S, D, N_STATE), **f32)}
+    ws = torch.empty(ssm.ssm_scan_bwd_workspace_size(tok, D, N_STATE, S), dtype=torch.uint8,
+                     device="cuda")
+
+    def call():
+        ssm.ssm_selective_scan_bwd(a["x"], a["dt"], ly.A, a["B"], a["C"], dy, g, Dskip=ly.Dskip,
+                                   z=a["z"], dt_bias=ly.dt_bias, cu_seqlens=cu, workspace=ws)
+
+    for _ in range(2):
+        call()
+    n = max(3, int(10 * steps_scale))
+    s0, s1 = _events(2)
+    _barrier_sync(world)
+    s0.record()
+    for _ in range(n):
+        call()
+    s1.record()
+    _barrier_sync(world)
+    ms = _max_over_ranks(s0.elapsed_time(s1) / n, world)
+    mufu = mufu_peak_gexp(peaks["sm_max_mhz"])
+    units = tok * D
+    res = {"gtoken_ch_per_s": units * world / (ms * 1e-3) / 1e9, "ms_per_call": ms,
+           "mufu_frac": round(units * 2 * N_STATE / (ms * 1e-3) / 1e9 / mufu, 4),
+           "executed_exp_frac": round(units * 3 * N_STATE / (ms * 1e-3) / 1e9 / mufu, 4),
+           "hbm_frac": round(units * 14 / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+           "workspace_bytes": ws.numel(), "sequences": S,
+           "step": "ssm_selective_scan_bwd over the packed 65536 x 5120 prefill, all gradients"}
+    del g, ws, dy
+    return res
 
 
 def replay_bytes_per_step(Bt, D, W, keep_lo=True):
@@ -765,6 +824,35 @@ def scan_sweep(variants, peaks):
     return 0
 
 
+def profile_scan_bwd():
+    """Three backward scans on a quarter of the packed workload, for profiler captures."""
+    import torch
+
+    import selective_state_space_causal_b200 as ssm
+    from selective_state_space_causal_b200 import synth
+
+    D, tot = 5120, 16384
+    lens = synth.sample_lengths(0, tot, 128, 8192)
+    cu = torch.from_numpy(synth.cu_from_lengths(lens)).cuda()
+    ly = Layer(D)
+    a = synth.device_activations(0, tot, D)
+    dy = synth.device_activations(1, tot, D)["x"]
+    f32 = dict(device="cuda", dtype=torch.float32)
+    g = {"du": torch.empty_like(a["x"]), "ddelta": torch.empty_like(a["x"]),
+         "dz": torch.empty_like(a["x"]), "dB": torch.empty((tot, N_STATE), **f32),
+         "dC": torch.empty((tot, N_STATE), **f32), "dA": torch.empty((D, N_STATE), **f32),
+         "dDskip": torch.empty((D,), **f32), "ddt_bias": torch.empty((D,), **f32),
+         "dh0": torch.empty((len(lens), D, N_STATE), **f32)}
+    ws = torch.empty(ssm.ssm_scan_bwd_workspace_size(tot, D, N_STATE, len(lens)),
+                     dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        ssm.ssm_selective_scan_bwd(a["x"], a["dt"], ly.A, a["B"], a["C"], dy, g, Dskip=ly.Dskip,
+                                   z=a["z"], dt_bias=ly.dt_bias, cu_seqlens=cu, workspace=ws)
+    torch.cuda.synchronize()
+    assert ssm.ssm_device_status() == 0
+    print(json.dumps({"profile_scan_bwd": {"tokens": tot, "d_inner": D, "sequences": len(lens)}}))
+
+
 def profile_decode(W):
     """A few replay and eager decode steps at 256 x 8192 from random states
     (about 0.5 GB on the device), for profiler captures; prints nothing timed."""
@@ -801,6 +889,9 @@ def main():
     args = parse_args()
     if args.profile_decode is not None:
         profile_decode(args.profile_decode)
+        return
+    if args.profile_scan_bwd:
+        profile_scan_bwd()
         return
     if args.impl == "reference":
         return bench_reference(args)

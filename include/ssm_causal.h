@@ -29,7 +29,8 @@
  *   be empty. cu_seqlens == NULL means a dense batch of S rows of tok/S tokens.
  * - Floating-point work is fp32 throughout (fp32 state, fp32 accumulation);
  *   bf16 tensors are converted on load and rounded to nearest even on store.
- * - Results are deterministic: no atomics take part in the arithmetic.
+ * - Results are deterministic: no atomics take part in the arithmetic, except
+ *   in the channel- and sequence-sums of ssm_selective_scan_bwd (see there).
  * - Every call returns SSM_OK (0) or a negative status and then launches
  *   nothing; ssm_last_error() gives a message for the calling thread.
  *
@@ -44,6 +45,9 @@
  * - "PackMamba: Efficient Processing of Variable-Length Sequences in Mamba
  *   training", abstract: packed sequences with no information passed between
  *   sequences.
+ * - The backward pass of the selective scan (ssm_selective_scan_bwd) is the
+ *   chain rule of the forward above, for training on packed sequences
+ *   (PackMamba abstract).
  * - "ReplaySSM: Cache SSM Inputs, Not State", abstract: decode with the state
  *   kept as a checkpoint plus the SSM inputs of recent tokens
  *   (ssm_replay_state_update, ssm_replay_reset, ssm_replay_flush).
@@ -230,6 +234,57 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
                                const int32_t *state_indices, int64_t n_slots, void *y,
                                int64_t Bt, int64_t D, int N, int K, ssm_dtype act_dtype,
                                ssm_dtype conv_state_dtype, ssm_stream_t stream);
+
+/*
+ * Workspace bytes ssm_selective_scan_bwd needs for `tok` packed tokens of D
+ * channels in S sequences (N must be 16; 0 for invalid sizes): one fp32 state
+ * checkpoint per 16 tokens of each sequence and channel, about 4 bytes per
+ * token and channel.
+ */
+size_t ssm_scan_bwd_workspace_size(int64_t tok, int64_t D, int N, int64_t S);
+
+/*
+ * Backward of ssm_selective_scan_fwd: gradients of the loss L through
+ * sum(dy * y) + sum(dh_final * h_final) with respect to every input, for
+ * training on packed sequences ("PackMamba: Efficient Processing of
+ * Variable-Length Sequences in Mamba training", abstract: no information
+ * passes between sequences, forwards or backwards). The forward is the one
+ * of ssm_selective_scan_fwd (tp_builder.py, _add_mamba_tp_layer); with
+ * G_t = dL/dh_t = dy_t silu(z_t) C_t + exp(delta_{t+1} A) G_{t+1}:
+ *   du_t = dy_t silu(z_t) Dskip + delta_t (G_t . B_t)
+ *   ddelta_t = [G_t . (u_t B_t + A exp(delta_t A) h_{t-1})] softplus'(dt_t + dt_bias)
+ *   dz_t = dy_t (C_t . h_t + Dskip u_t) silu'(z_t)
+ *   dB_t = sum_c delta_t u_t G_t,  dC_t = sum_c dy_t silu(z_t) h_t
+ *   dA = sum_t G_t delta_t exp(delta_t A) h_{t-1},  dDskip = sum_t dy_t silu(z_t) u_t
+ *   ddt_bias = sum_t ddelta_t,  dh0 = exp(delta_{t0} A) G_{t0} (first token t0)
+ * (softplus' = 1 and no bias when delta_softplus = 0; silu(z) = 1 and
+ * silu' = 0 without z). The forward states are recomputed, not stored.
+ *
+ *   u, delta, B, C, Dskip, z, dt_bias, delta_softplus, h0, cu_seqlens, S,
+ *   tok, D, N, act_dtype: exactly the forward call's arguments
+ *   dy             (tok, D) act_dtype: gradient of y
+ *   dh_final       (S, D, N) fp32 or NULL (= 0): gradient of h_final
+ *   du, ddelta     (tok, D) act_dtype, written; ddelta is the gradient of the
+ *                  raw `delta` input (before dt_bias and the softplus)
+ *   dz             (tok, D) act_dtype or NULL; written (zeros when z is NULL)
+ *   dB, dC         (tok, N) fp32, written (summed over channels)
+ *   dA             (D, N) fp32, written (summed over sequences and tokens)
+ *   dDskip, ddt_bias (D) fp32 or NULL, written
+ *   dh0            (S, D, N) fp32 or NULL, written
+ *   workspace      >= ssm_scan_bwd_workspace_size() bytes, 256-byte aligned;
+ *                  required; its contents are overwritten
+ * dB, dC, dA, dDskip and ddt_bias are sums over CTAs taken with fp32 atomics,
+ * so their last bits may differ from run to run; every other output is
+ * deterministic. Outputs must not overlap the inputs.
+ */
+int ssm_selective_scan_bwd(const void *u, const void *delta, const float *A, const void *B,
+                           const void *C, const float *Dskip, const void *z,
+                           const float *dt_bias, int delta_softplus, const float *h0,
+                           const int32_t *cu_seqlens, int64_t S, const void *dy,
+                           const float *dh_final, void *du, void *ddelta, void *dz, float *dB,
+                           float *dC, float *dA, float *dDskip, float *ddt_bias, float *dh0,
+                           int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
+                           size_t workspace_bytes, ssm_stream_t stream);
 
 /*
  * Replay decode: one token per row, with each slot's SSM state kept as a

@@ -19,7 +19,9 @@ from ._lib import (  # noqa: F401
     ssm_replay_flush,
     ssm_replay_reset,
     ssm_replay_state_update,
+    ssm_scan_bwd_workspace_size,
     ssm_scan_workspace_size,
+    ssm_selective_scan_bwd,
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_noalloc,
     ssm_selective_state_update,

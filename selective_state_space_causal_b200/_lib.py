@@ -40,6 +40,10 @@ SIGNATURES = [
     ("ssm_selective_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _int, _vp, _i64, _vp, _i64, _i64, _int, _int, _int,
                                           _int, _vp]),
+    ("ssm_scan_bwd_workspace_size", _sz, [_i64, _i64, _int, _i64]),
+    ("ssm_selective_scan_bwd", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64,
+                                      _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
+                                      _i64, _int, _int, _vp, _sz, _vp]),
     ("ssm_replay_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _i64, _vp, _i64,
                                        _i64, _int, _int, _int, _int, _vp]),
@@ -260,3 +264,28 @@ def ssm_replay_flush(rep, A, slots=None, n=None, stream=None):
                                 _ptr(rep["buf_B"]), _ptr(rep["buf_len"]), _ptr(rep["tickets"]),
                                 _ptr(A), int(rep["W"]), _ptr(slots), n, n_slots, D, N,
                                 _stream(stream)))
+
+
+def ssm_scan_bwd_workspace_size(tok: int, D: int, N: int, S: int) -> int:
+    return int(lib.ssm_scan_bwd_workspace_size(tok, D, N, S))
+
+
+def ssm_selective_scan_bwd(u, delta, A, B, C, dy, grads, Dskip=None, z=None, dt_bias=None,
+                           delta_softplus=True, h0=None, dh_final=None, cu_seqlens=None, S=None,
+                           workspace=None, stream=None):
+    """Backward of ssm_selective_scan_fwd. `grads` holds the output tensors:
+    du, ddelta (like u), dz (like u, or None), dB, dC (tok, N) fp32, dA (D, N)
+    fp32, dDskip, ddt_bias (D) fp32 or None, dh0 (S, D, N) fp32 or None.
+    `workspace` is a device byte tensor of ssm_scan_bwd_workspace_size() bytes."""
+    tok, D = u.shape
+    N = A.shape[1]
+    if S is None:
+        S = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
+    g = grads
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib.ssm_selective_scan_bwd(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(cu_seqlens), S, _ptr(dy), _ptr(dh_final),
+        _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g.get("dz")), _ptr(g["dB"]), _ptr(g["dC"]),
+        _ptr(g["dA"]), _ptr(g.get("dDskip")), _ptr(g.get("ddt_bias")), _ptr(g.get("dh0")), tok, D,
+        N, _dtype(u), _ptr(workspace), ws_bytes, _stream(stream)))

@@ -24,6 +24,21 @@ cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
 int64_t noalloc_max_sequences();
 int read_replay_status(bool clear);
 
+struct ScanBwdArgs {
+    const void *u, *dt, *B, *C, *z, *dy;
+    const float *A, *Dskip, *dt_bias, *h0, *dh_final;
+    const int32_t *cu;
+    int64_t S;
+    void *du, *ddt, *dz;
+    float *dB, *dC, *dA, *dDskip, *ddt_bias, *dh0;
+    float *ckpt;
+    int64_t tok, D;
+    int softplus;
+    bool bf16;
+};
+size_t scan_bwd_ckpt_floats(int64_t tok, int64_t D, int64_t S);
+cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *launches);
+
 struct ReplayStepArgs {
     void *conv_state;
     float *ckpt;
@@ -286,6 +301,66 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
                       dt(conv_state_dtype)};
     int launched = 0;
     cudaError_t e = ssm::launch_decode(a, reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
+size_t ssm_scan_bwd_workspace_size(int64_t tok, int64_t D, int N, int64_t S)
+{
+    if (tok < 0 || D < 1 || N != 16 || S < 1) return 0;
+    return (ssm::scan_bwd_ckpt_floats(tok, D, S) * sizeof(float) + 255) / 256 * 256;
+}
+
+int ssm_selective_scan_bwd(const void *u, const void *delta, const float *A, const void *B,
+                           const void *C, const float *Dskip, const void *z,
+                           const float *dt_bias, int delta_softplus, const float *h0,
+                           const int32_t *cu_seqlens, int64_t S, const void *dy,
+                           const float *dh_final, void *du, void *ddelta, void *dz, float *dB,
+                           float *dC, float *dA, float *dDskip, float *ddt_bias, float *dh0,
+                           int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
+                           size_t workspace_bytes, ssm_stream_t stream)
+{
+    const char *fn = "ssm_selective_scan_bwd";
+    if (!valid_dtype(act_dtype)) return fail(SSM_ERR_UNSUPPORTED_DTYPE, "%s: unknown dtype", fn);
+    if (N != 16) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: N must be 16 (got %d)", fn, N);
+    if (D < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: D must be >= 1", fn);
+    if (int r = check_seqs(fn, cu_seqlens, S, tok)) return r;
+    if (!A || !dA || !dB || !dC) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: A, dA, dB and dC are required", fn);
+    if (tok > 0 && (!u || !delta || !B || !C || !dy || !du || !ddelta))
+        return fail(SSM_ERR_INVALID_ARGUMENT,
+                    "%s: u, delta, B, C, dy, du and ddelta are required", fn);
+    const size_t es = esize(act_dtype);
+    const void *acts[] = {u, delta, z, dy, du, ddelta, dz, B, C};
+    for (const void *q : acts)
+        if (!aligned(q, es)) return fail(SSM_ERR_MISALIGNED, "%s: a pointer is not aligned to its element size", fn);
+    const void *f32s[] = {A, Dskip, dt_bias, h0, dh_final, dB, dC, dA, dDskip, ddt_bias, dh0};
+    for (const void *q : f32s)
+        if (!aligned(q, 4)) return fail(SSM_ERR_MISALIGNED, "%s: an fp32 pointer is misaligned", fn);
+    const size_t need = ssm_scan_bwd_workspace_size(tok, D, N, S);
+    if (!workspace || workspace_bytes < need)
+        return fail(SSM_ERR_WORKSPACE, "%s: workspace has %zu bytes, needs %zu", fn,
+                    workspace ? workspace_bytes : (size_t)0, need);
+    if (!aligned(workspace, 256))
+        return fail(SSM_ERR_MISALIGNED, "%s: workspace must be 256-byte aligned", fn);
+    if (tok > 0) {
+        const size_t bytes = (size_t)tok * D * es;
+        const void *outs[] = {du, ddelta, dz};
+        const void *ins[] = {u, delta, z, dy, B, C};
+        for (const void *o : outs) {
+            if (!o) continue;
+            for (const void *in : ins) {
+                if (!in) continue;
+                const char *a = static_cast<const char *>(o), *b = static_cast<const char *>(in);
+                if (a < b + bytes && b < a + bytes)
+                    return fail(SSM_ERR_INVALID_ARGUMENT, "%s: a gradient overlaps an input", fn);
+            }
+        }
+    }
+    ssm::ScanBwdArgs a{u, delta, B, C, z, dy, A, Dskip, dt_bias, h0, dh_final, cu_seqlens, S,
+                       du, ddelta, dz, dB, dC, dA, dDskip, ddt_bias, dh0,
+                       static_cast<float *>(workspace), tok, D, delta_softplus,
+                       act_dtype == SSM_BF16};
+    int launched = 0;
+    cudaError_t e = ssm::launch_scan_bwd(a, reinterpret_cast<cudaStream_t>(stream), &launched);
     return finish(e, launched, fn);
 }
 

@@ -208,3 +208,33 @@ def test_replay_reset_flush_reject(fn, kw, code):
                                 a["W"], a["slots_ptr"], a["n"], a["n_slots"], a["D"], a["N"], None)
     assert rc == code
     assert _err()
+
+
+def bwd(**kw):
+    a = dict(u=A16, dt=A16 + 0x200000, A=A16, B=A16, C=A16, Dsk=None, z=None, dtb=None, sp=1,
+             h0=None, cu=None, S=1, dy=A16 + 0x400000, dhf=None, du=A16 + 0x600000,
+             ddt=A16 + 0x800000, dz=None, dB=A16, dC=A16, dA=A16, dDsk=None, ddtb=None,
+             dh0=None, tok=64, D=32, N=16, adt=1, ws=A16, wsb=1 << 30)
+    a.update(kw)
+    return L.ssm_selective_scan_bwd(a["u"], a["dt"], a["A"], a["B"], a["C"], a["Dsk"], a["z"],
+                                    a["dtb"], a["sp"], a["h0"], a["cu"], a["S"], a["dy"],
+                                    a["dhf"], a["du"], a["ddt"], a["dz"], a["dB"], a["dC"],
+                                    a["dA"], a["dDsk"], a["ddtb"], a["dh0"], a["tok"], a["D"],
+                                    a["N"], a["adt"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=8), -1), (dict(dA=None), -1), (dict(dB=None), -1), (dict(dy=None), -1),
+    (dict(du=None), -1), (dict(ws=None), -5), (dict(wsb=64), -5), (dict(ws=A16 + 16), -3),
+    (dict(u=A16 + 1), -3), (dict(dA=A16 + 2), -3), (dict(adt=5), -2), (dict(S=0), -1),
+    (dict(du=A16 + 0x200000), -1), (dict(tok=63, S=2), -1),
+])
+def test_scan_bwd_rejects(kw, code):
+    assert bwd(**kw) == code
+    assert _err()
+
+
+def test_scan_bwd_workspace_size():
+    n = ssm.ssm_scan_bwd_workspace_size(16384, 1536, 16, 8)
+    assert n % 256 == 0 and n >= (16384 // 16 + 8) * 1536 * 64
+    assert ssm.ssm_scan_bwd_workspace_size(100, 64, 8, 1) == 0

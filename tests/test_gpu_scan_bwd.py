@@ -1,0 +1,147 @@
+"""Backward of the selective scan on the GPU against the fp64 oracle's
+backward (itself pinned to finite differences of the forward), for training on
+packed sequences (PackMamba abstract).
+
+Tolerances follow gpu_helpers: outputs stored in the activation dtype (du,
+ddelta, dz) take the bf16 bound with one bf16 step of slack for bf16
+activations and 1e-4 rms for fp32; the fp32 outputs (dB, dC, dA, dDskip,
+ddt_bias, dh0) take the bare bound of the activation dtype.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import selective_state_space_causal_b200 as ssm
+from selective_state_space_causal_b200 import synth
+from gpu_helpers import TOL_BF16, TOL_F32, act_dtype, assert_close, cu_tensor, dev, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_bwd(u, dt, A, B, C, dy, Dskip, z, dt_bias, h0, dh_final, cu, S, softplus=True):
+    tok, D = u.shape
+    N = A.shape[1]
+    f32 = dict(device="cuda", dtype=torch.float32)
+    g = {"du": torch.full_like(u, 7.0), "ddelta": torch.full_like(u, 7.0),
+         "dz": torch.full_like(u, 7.0) if z is not None else None,
+         "dB": torch.full((tok, N), 7.0, **f32), "dC": torch.full((tok, N), 7.0, **f32),
+         "dA": torch.full((D, N), 7.0, **f32), "dDskip": torch.full((D,), 7.0, **f32),
+         "ddt_bias": torch.full((D,), 7.0, **f32), "dh0": torch.full((S, D, N), 7.0, **f32)}
+    ws = torch.empty(max(1, ssm.ssm_scan_bwd_workspace_size(tok, D, N, S)), dtype=torch.uint8,
+                     device="cuda")
+    ssm.ssm_selective_scan_bwd(u, dt, A, B, C, dy, g, Dskip=Dskip, z=z, dt_bias=dt_bias,
+                               delta_softplus=softplus, h0=h0, dh_final=dh_final, cu_seqlens=cu,
+                               S=S, workspace=ws)
+    torch.cuda.synchronize()
+    return g
+
+
+def _check(orc, bf16, lens, D, gate=True, softplus=True, dense_rows=None, seed=0):
+    dt_ = act_dtype(bf16)
+    if dense_rows:
+        tok = dense_rows[0] * dense_rows[1]
+        cu_d, cu_h, S = None, None, dense_rows[0]
+    else:
+        cu_d, cu_h = cu_tensor(lens)
+        tok, S = int(cu_h[-1]), len(lens)
+    prm = synth.make_params(seed, D, random_bias=True, random_A=True, random_D=True)
+    act = synth.make_activations(seed, tok, D, bf16=bf16)
+    rng = np.random.default_rng(seed + 7)
+    dy = rng.standard_normal((tok, D)).astype(np.float32)
+    if bf16:
+        dy = synth.round_bf16(dy)
+    st = synth.make_states(seed + 1, S, D, bf16=bf16, scale=0.3)
+    dhf = (0.3 * rng.standard_normal((S, D, 16))).astype(np.float32)
+    z = act["z"] if gate else None
+    delta, dtb = act["dt"], prm.dt_bias
+    if not softplus:
+        # without the softplus the input is the step size itself: positive values
+        delta = np.logaddexp(0.0, act["dt"].astype(np.float64) + prm.dt_bias[None, :])
+        delta = synth.round_bf16(delta.astype(np.float32)) if bf16 else delta.astype(np.float32)
+        dtb = None
+    g = _run_bwd(dev(act["x"], dt_), dev(delta, dt_), dev(prm.A), dev(act["B"], dt_),
+                 dev(act["C"], dt_), dev(dy, dt_), dev(prm.Dskip), dev(z, dt_) if gate else None,
+                 dev(dtb), dev(st["h0"]), dev(dhf), cu_d, S, softplus)
+    r = orc.selective_scan_bwd(act["x"], delta, prm.A, act["B"], act["C"], dy,
+                               Dskip=prm.Dskip, z=z, dt_bias=dtb, delta_softplus=softplus,
+                               h0=st["h0"], cu_seqlens=None if dense_rows else cu_h,
+                               S=S if dense_rows else None, dh_final=dhf)
+    tol = TOL_BF16 if bf16 else TOL_F32
+    assert_close(host(g["du"]), r["du"], bf16, tol, "du")
+    assert_close(host(g["ddelta"]), r["ddt"], bf16, tol, "ddelta")
+    if gate:
+        assert_close(host(g["dz"]), r["dz"], bf16, tol, "dz")
+    for k, rk in (("dB", "dB"), ("dC", "dC"), ("dA", "dA"), ("dDskip", "dDskip"),
+                  ("ddt_bias", "ddt_bias"), ("dh0", "dh0")):
+        if k == "ddt_bias" and dtb is None:
+            continue
+        assert_close(host(g[k]), r[rk], False, tol, k)
+    assert ssm.ssm_device_status() == 0
+    return g
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_bwd_packed_matches_oracle(orc, bf16):
+    # chunk edges at 16 tokens: lengths below, at, across and far beyond them;
+    # an empty and a one-token sequence; a partial 8-channel block
+    _check(orc, bf16, [37, 0, 1, 130, 16, 17, 5], 40)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_bwd_no_gate_no_softplus(orc, bf16):
+    _check(orc, bf16, [20, 3, 48], 64, gate=False, softplus=False, seed=3)
+
+
+def test_bwd_dense_rows(orc):
+    _check(orc, True, None, 96, dense_rows=(3, 80), seed=5)
+
+
+def test_bwd_deterministic_outputs():
+    """Two runs agree bit for bit on the per-token gradients and dh0; the
+    atomically summed ones agree to fp32 rounding."""
+    lens = [300, 77, 1000]
+    cu_d, cu_h = cu_tensor(lens)
+    tok, S, D = int(cu_h[-1]), len(lens), 256
+    prm = synth.make_params(9, D, random_bias=True)
+    a = synth.device_activations(9, tok, D)
+    dy = synth.device_activations(10, tok, D)["x"]
+    p = {k: dev(getattr(prm, k)) for k in ("A", "Dskip", "dt_bias")}
+    runs = [_run_bwd(a["x"], a["dt"], p["A"], a["B"], a["C"], dy, p["Dskip"], a["z"],
+                     p["dt_bias"], None, None, cu_d, S) for _ in range(2)]
+    for k in ("du", "ddelta", "dz", "dh0"):
+        assert torch.equal(runs[0][k], runs[1][k]), k
+    for k in ("dB", "dC", "dA", "dDskip", "ddt_bias"):
+        x, y = runs[0][k], runs[1][k]
+        assert torch.allclose(x, y, rtol=1e-5, atol=1e-5 * float(y.abs().max())), k
+
+
+def test_bwd_packmamba_workload_sampled(orc):
+    """The packed 65536-token, 5120-channel training shape: per-token gradients,
+    dA, dDskip, ddt_bias and dh0 of sampled channels against the oracle run on
+    those channels alone (channels are independent for these)."""
+    w = synth.WORKLOADS["packmamba_2p8b_varlen_65536"]
+    D, tot = w["D"], w["total"]
+    lens = synth.sample_lengths(0, tot, w["len_lo"], w["len_hi"])
+    cu_d, cu_h = cu_tensor(lens)
+    S = len(lens)
+    prm = synth.make_params(0, D)
+    p = {k: dev(getattr(prm, k)) for k in ("A", "Dskip", "dt_bias")}
+    a = synth.device_activations(0, tot, D)
+    dy = synth.device_activations(1, tot, D)["x"]
+    g = _run_bwd(a["x"], a["dt"], p["A"], a["B"], a["C"], dy, p["Dskip"], a["z"], p["dt_bias"],
+                 None, None, cu_d, S)
+    rng = np.random.default_rng(0)
+    ch = np.sort(rng.choice(D, size=6, replace=False))
+    chd = torch.from_numpy(ch).cuda()
+    sel = lambda t: host(t.index_select(1, chd))  # noqa: E731
+    r = orc.selective_scan_bwd(sel(a["x"]), sel(a["dt"]), prm.A[ch], host(a["B"]), host(a["C"]),
+                               sel(dy), Dskip=prm.Dskip[ch], z=sel(a["z"]),
+                               dt_bias=prm.dt_bias[ch], cu_seqlens=cu_h)
+    for k, rk in (("du", "du"), ("ddelta", "ddt"), ("dz", "dz")):
+        assert_close(sel(g[k]), r[rk], True, TOL_BF16, k)
+    assert_close(host(g["dA"])[ch], r["dA"], False, TOL_BF16, "dA")
+    assert_close(host(g["dDskip"])[ch], r["dDskip"], False, TOL_BF16, "dDskip")
+    assert_close(host(g["ddt_bias"])[ch], r["ddt_bias"], False, TOL_BF16, "ddt_bias")
+    assert_close(host(g["dh0"])[:, ch], r["dh0"], False, TOL_BF16, "dh0")
+    assert ssm.ssm_device_status() == 0
