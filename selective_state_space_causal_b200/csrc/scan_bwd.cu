@@ -67,6 +67,48 @@ struct Smem {
     float out[3][kTS][kCh];      // du, ddt, dz of the chunk
 };
 
+// Raw chunk inputs as they sit in global memory, copied in one chunk ahead.
+template <typename T>
+struct RawChunk {
+    T act[4][kTS][kCh];  // dt, u, z, dy
+    T bc[2][kTS][kN];    // B, C
+};
+
+// 16-byte asynchronous copy from global to shared memory (completion through
+// the issuing thread's cp.async groups).
+__device__ __forceinline__ void cp16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 :: "r"((uint32_t)__cvta_generic_to_shared(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
+// Issue the copies of chunk [t0, t0 + nt): dt and u (and z, dy when `full`)
+// rows of the CTA's channels, and the B (and C) rows. Needs D * sizeof(T) and
+// every base a multiple of 16 bytes (the host checks).
+template <typename T>
+__device__ __forceinline__ void issue_chunk(const BwdParams &p, RawChunk<T> &r, int64_t t0, int nt,
+                                            int64_t cbase, int nch, bool full)
+{
+    constexpr int V = 16 / sizeof(T), VR = kCh / V, VB = kN / V;
+    const T *src_act[4] = {static_cast<const T *>(p.dt), static_cast<const T *>(p.u),
+                           static_cast<const T *>(p.z), static_cast<const T *>(p.dy)};
+    const int narr = full ? 4 : 2, nvr = nch / V;
+    for (int e = threadIdx.x; e < narr * kTS * VR; e += kThreads) {
+        const int arr = e / (kTS * VR), rem = e % (kTS * VR), tl = rem / VR, v = rem % VR;
+        if (tl >= nt || v >= nvr || src_act[arr] == nullptr) continue;
+        cp16(&r.act[arr][tl][v * V], src_act[arr] + (t0 + tl) * p.D + cbase + v * V);
+    }
+    const T *src_bc[2] = {static_cast<const T *>(p.B), static_cast<const T *>(p.C)};
+    for (int e = threadIdx.x; e < (full ? 2 : 1) * kTS * VB; e += kThreads) {
+        const int arr = e / (kTS * VB), rem = e % (kTS * VB), tl = rem / VB, v = rem % VB;
+        if (tl >= nt) continue;
+        cp16(&r.bc[arr][tl][v * V], src_bc[arr] + (t0 + tl) * kN + v * V);
+    }
+}
+
 __device__ __forceinline__ float sigmoid_f(float v) { return __fdividef(1.0f, 1.0f + __expf(-v)); }
 
 template <typename T>
@@ -119,6 +161,48 @@ __device__ __forceinline__ void stage_chunk(const BwdParams &p, Smem &sm, int64_
     }
 }
 
+// The same staging from the raw shared-memory copy of the chunk.
+template <typename T>
+__device__ __forceinline__ void stage_from_raw(const BwdParams &p, Smem &sm, const RawChunk<T> &r,
+                                               int nt, int64_t cbase, bool full)
+{
+    const int tid = threadIdx.x;
+    const bool has_z = p.z != nullptr;
+    for (int e = tid; e < kTS * kCh; e += kThreads) {
+        const int tl = e / kCh, cl = e % kCh;
+        const int64_t c = cbase + cl;
+        float d = 0.f, dsp = 0.f, u = 0.f, dq = 0.f, dzf = 0.f;
+        if (tl < nt && c < p.D) {
+            const float v = to_f32(r.act[0][tl][cl]) + (p.dt_bias ? __ldg(p.dt_bias + c) : 0.f);
+            d = p.softplus ? softplus_fast(v) : v;
+            dsp = p.softplus ? sigmoid_f(v) : 1.f;
+            u = to_f32(r.act[1][tl][cl]);
+            if (full) {
+                const float dy = to_f32(r.act[3][tl][cl]);
+                float g = 1.f, dg = 0.f;
+                if (has_z) {
+                    const float zt = to_f32(r.act[2][tl][cl]), sg = sigmoid_f(zt);
+                    g = zt * sg;
+                    dg = sg * (1.f + zt * (1.f - sg));
+                }
+                dq = dy * g;
+                dzf = dy * dg;
+            }
+        }
+        sm.d[tl][cl] = d;
+        sm.dsp[tl][cl] = dsp;
+        sm.u[tl][cl] = u;
+        sm.dq[tl][cl] = dq;
+        sm.dzf[tl][cl] = dzf;
+    }
+    for (int e = tid; e < kTS * kN; e += kThreads) {
+        const int tl = e / kN, n = e % kN;
+        const bool live = tl < nt;
+        sm.B[tl][n] = live ? to_f32(r.bc[0][tl][n]) : 0.f;
+        if (full) sm.C[tl][n] = live ? to_f32(r.bc[1][tl][n]) : 0.f;
+    }
+}
+
 // h <- a * h + (d u) * B for this lane's 4 states; returns a.
 __device__ __forceinline__ void fwd_token(f32x2 (&h)[2], const f32x2 (&A2)[2], float d, float u,
                                           const float *Bn, f32x2 (&a)[2])
@@ -133,14 +217,16 @@ __device__ __forceinline__ void fwd_token(f32x2 (&h)[2], const f32x2 (&A2)[2], f
     }
 }
 
-template <typename T>
+template <typename T, bool ASYNC>
 __global__ void __launch_bounds__(kThreads)
 scan_bwd_kernel(const BwdParams p)
 {
     __shared__ Smem sm;
+    __shared__ __align__(16) RawChunk<T> raw[ASYNC ? 2 : 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sub = tid % kTPC, cl = tid / kTPC;
     const int64_t cbase = (int64_t)blockIdx.x * kCh, c = cbase + cl;
+    const int nch = (int)min((int64_t)kCh, p.D - cbase);
     const bool cvalid = c < p.D;
     const int64_t s = blockIdx.y;
     int64_t start, end;
@@ -174,6 +260,10 @@ scan_bwd_kernel(const BwdParams p)
         const int64_t o = (s * p.D + c) * kN + sub * kNPT + 2 * j;
         h[j] = (cvalid && p.h0) ? pk2(p.h0[o], p.h0[o + 1]) : 0ull;
     }
+    if (ASYNC && nchunks > 0) {
+        issue_chunk<T>(p, raw[0], start, (int)min((int64_t)kTS, len), cbase, nch, false);
+        cp_commit();
+    }
     for (int64_t k = 0; k < nchunks; ++k) {
         const int64_t t0 = start + k * kTS;
         const int nt = (int)min((int64_t)kTS, end - t0);
@@ -183,8 +273,24 @@ scan_bwd_kernel(const BwdParams p)
             upk2(h[1], v.z, v.w);
             *reinterpret_cast<float4 *>(ck + k * p.D * kN) = v;
         }
-        __syncthreads();  // the previous chunk's values are no longer read
-        stage_chunk<T>(p, sm, t0, nt, cbase, false);
+        if constexpr (ASYNC) {
+            // the next chunk's copies go out before this one is staged; the
+            // buffer they fill was last read before the previous barrier
+            if (k + 1 < nchunks) {
+                const int64_t t1 = t0 + kTS;
+                issue_chunk<T>(p, raw[(k + 1) & 1], t1, (int)min((int64_t)kTS, end - t1), cbase,
+                               nch, false);
+                cp_commit();
+                cp_wait<1>();
+            } else {
+                cp_wait<0>();
+            }
+            __syncthreads();  // every thread's copies have landed; the previous chunk is done
+            stage_from_raw<T>(p, sm, raw[k & 1], nt, cbase, false);
+        } else {
+            __syncthreads();  // the previous chunk's values are no longer read
+            stage_chunk<T>(p, sm, t0, nt, cbase, false);
+        }
         __syncthreads();
         for (int tl = 0; tl < nt; ++tl) {
             f32x2 a[2];
@@ -201,11 +307,30 @@ scan_bwd_kernel(const BwdParams p)
     }
     float dDsk = 0.f, ddtb = 0.f;
     T *DU = static_cast<T *>(p.du), *DDT = static_cast<T *>(p.ddt), *DZ = static_cast<T *>(p.dz);
+    __syncthreads();  // phase A's last chunk is no longer read
+    if (ASYNC && nchunks > 0) {
+        const int64_t tl0 = start + (nchunks - 1) * kTS;
+        issue_chunk<T>(p, raw[0], tl0, (int)(end - tl0), cbase, nch, true);
+        cp_commit();
+    }
     for (int64_t k = nchunks - 1; k >= 0; --k) {
         const int64_t t0 = start + k * kTS;
         const int nt = (int)min((int64_t)kTS, end - t0);
-        __syncthreads();  // the previous chunk's shared values are no longer read
-        stage_chunk<T>(p, sm, t0, nt, cbase, true);
+        const int buf = (int)((nchunks - 1 - k) & 1);
+        if constexpr (ASYNC) {
+            if (k > 0) {
+                issue_chunk<T>(p, raw[buf ^ 1], t0 - kTS, kTS, cbase, nch, true);
+                cp_commit();
+                cp_wait<1>();
+            } else {
+                cp_wait<0>();
+            }
+            __syncthreads();  // copies landed; the previous chunk's shared values are no longer read
+            stage_from_raw<T>(p, sm, raw[buf], nt, cbase, true);
+        } else {
+            __syncthreads();  // the previous chunk's shared values are no longer read
+            stage_chunk<T>(p, sm, t0, nt, cbase, true);
+        }
         __syncthreads();
         // recompute this lane's states over the chunk from its checkpoint
         f32x2 hc[2], hist[kTS][2];
@@ -411,10 +536,17 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *laun
     p.dh0 = a.dh0; p.ckpt = a.ckpt;
     p.S = a.S; p.tok = a.tok; p.D = a.D; p.L = a.cu ? 0 : a.tok / a.S; p.softplus = a.softplus;
     const dim3 grid((unsigned)((a.D + kCh - 1) / kCh), (unsigned)a.S);
-    if (a.bf16)
-        scan_bwd_kernel<__nv_bfloat16><<<grid, kThreads, 0, stream>>>(p);
-    else
-        scan_bwd_kernel<float><<<grid, kThreads, 0, stream>>>(p);
+    const size_t es = a.bf16 ? 2 : 4;
+    const uintptr_t mis = (uintptr_t)a.u | (uintptr_t)a.dt | (uintptr_t)a.z | (uintptr_t)a.dy |
+                          (uintptr_t)a.B | (uintptr_t)a.C;
+    const bool async_ok = (mis % 16 == 0) && ((size_t)a.D * es) % 16 == 0;
+    if (a.bf16) {
+        if (async_ok) scan_bwd_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, stream>>>(p);
+        else scan_bwd_kernel<__nv_bfloat16, false><<<grid, kThreads, 0, stream>>>(p);
+    } else {
+        if (async_ok) scan_bwd_kernel<float, true><<<grid, kThreads, 0, stream>>>(p);
+        else scan_bwd_kernel<float, false><<<grid, kThreads, 0, stream>>>(p);
+    }
     ++*launches;
     return cudaGetLastError();
 }
