@@ -274,3 +274,62 @@ def test_replay_many_rows_per_cta_bitwise():
     assert torch.equal(cs_r, cs_e)
     assert bool((rep["tickets"] == 0).all())
     assert ssm.ssm_device_status() == 0
+
+
+@pytest.mark.parametrize("K", [3, 4])
+def test_replay_mixed_dtypes_and_bare_options(orc, K):
+    """bf16 activations with an fp32 conv state; no gate, no Dskip, no conv
+    bias, no dt_bias and the softplus off (the raw input is the step size)."""
+    n_slots, Bt, D, W, steps = 5, 5, 64, 3, 7
+    prm = _params(70 + K, D, K)
+    p = _dev_params(prm)
+    st = synth.make_states(71, n_slots, D, K=K, bf16=False, scale=0.3)
+    cs = dev(st["conv_state"])  # fp32 conv state
+    rep = ssm.replay_buffers(n_slots, D, W, "cuda", keep_lo=False)
+    rep["ckpt"].copy_(dev(st["h0"]))
+    ssm.ssm_replay_reset(rep)
+    rcs = np.asarray(st["conv_state"], np.float64)
+    rrep = orc.replay_init(st["h0"], W, keep_lo=False)
+    y = torch.empty((Bt, D), device="cuda", dtype=BF)
+    for t in range(steps):
+        s = synth.make_activations(400 + t, Bt, D, bf16=True)
+        delta = synth.round_bf16(np.logaddexp(0.0, s["dt"].astype(np.float64)
+                                              + prm.dt_bias[None, :]).astype(np.float32))
+        ssm.ssm_replay_state_update(cs, rep, dev(s["x"], BF), dev(delta, BF), dev(s["B"], BF),
+                                    dev(s["C"], BF), y, p["conv_w"], p["A"],
+                                    delta_softplus=False)
+        ry, rcs, rrep = orc.replay_step(rcs, rrep, s["x"], delta, s["B"], s["C"], None,
+                                        prm.conv_w, None, prm.A, None, None,
+                                        delta_softplus=False)
+        assert_close(host(y), ry, True, TOL_BF16, f"y at step {t}")
+        assert_close(host(cs), rcs, False, TOL_F32, f"fp32 conv state at step {t}")
+        assert np.array_equal(host(rep["buf_len"]), rrep["len"])
+    ssm.ssm_replay_flush(rep, p["A"])
+    assert_close(host(rep["ckpt"]), orc.replay_state(rrep, prm.A), False, TOL_BF16, "state")
+
+
+def test_replay_skips_out_of_range_slots_and_clamps_lengths(orc):
+    """A slot index >= n_slots skips its row like -1; a buffer length outside
+    0..W-1 (corrupt) is clamped into range, so the call stays in bounds."""
+    n_slots, Bt, D, W = 4, 3, 128, 3
+    prm = _params(80, D, 4)
+    p = _dev_params(prm)
+    st = synth.make_states(81, n_slots, D, bf16=True, scale=0.3)
+    cs = dev(st["conv_state"], BF)
+    rep = ssm.replay_buffers(n_slots, D, W, "cuda", keep_lo=True)
+    rep["ckpt"].copy_(dev(st["h0"]))
+    ssm.ssm_replay_reset(rep)
+    rep["buf_len"][2] = 100  # corrupt: clamped to W-1, a checkpoint step
+    idx = torch.tensor([2, 9, 0], dtype=torch.int32, device="cuda")
+    s = synth.make_activations(500, Bt, D, bf16=True)
+    y = torch.full((Bt, D), 5.0, device="cuda", dtype=BF)
+    before = {k: rep[k].clone() for k in ("ckpt", "ckpt_lo", "buf")}
+    _step(cs, rep, s, y, p, BF, idx)
+    torch.cuda.synchronize()
+    assert bool((y[1] == 5.0).all()), "the out-of-range row keeps its y"
+    lens = host(rep["buf_len"])
+    assert lens[2] == 0 and lens[0] == 1 and lens[1] == 0 and lens[3] == 0
+    assert torch.equal(rep["ckpt"][1], before["ckpt"][1])
+    assert torch.equal(rep["ckpt"][3], before["ckpt"][3])
+    assert not torch.equal(rep["ckpt"][2], before["ckpt"][2]), "slot 2 took a checkpoint step"
+    assert ssm.ssm_device_status() == 0

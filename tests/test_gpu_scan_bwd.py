@@ -145,3 +145,40 @@ def test_bwd_packmamba_workload_sampled(orc):
     assert_close(host(g["ddt_bias"])[ch], r["ddt_bias"], False, TOL_BF16, "ddt_bias")
     assert_close(host(g["dh0"])[:, ch], r["dh0"], False, TOL_BF16, "dh0")
     assert ssm.ssm_device_status() == 0
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_bwd_unaligned_rows_scalar_staging(orc, bf16):
+    """D = 36: bf16 rows are not a multiple of 16 bytes, so the chunk inputs are
+    staged with scalar loads (fp32 rows of 144 bytes still take the copies)."""
+    _check(orc, bf16, [19, 40, 2], 36, seed=11)
+
+
+def test_bwd_optional_inputs_absent(orc):
+    """No Dskip, dt_bias, h0, dh_final and no dz output: the remaining gradients
+    still match the oracle, which takes the same absences as zeros."""
+    lens = [33, 9]
+    cu_d, cu_h = cu_tensor(lens)
+    tok, S, D = int(cu_h[-1]), len(lens), 48
+    prm = synth.make_params(12, D, random_A=True)
+    act = synth.make_activations(12, tok, D, bf16=True)
+    dy = synth.round_bf16(np.random.default_rng(13).standard_normal((tok, D)).astype(np.float32))
+    BF = torch.bfloat16
+    f32 = dict(device="cuda", dtype=torch.float32)
+    u = dev(act["x"], BF)
+    g = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u), "dz": None,
+         "dB": torch.empty((tok, 16), **f32), "dC": torch.empty((tok, 16), **f32),
+         "dA": torch.empty((D, 16), **f32)}
+    ws = torch.empty(ssm.ssm_scan_bwd_workspace_size(tok, D, 16, S), dtype=torch.uint8,
+                     device="cuda")
+    ssm.ssm_selective_scan_bwd(u, dev(act["dt"], BF), dev(prm.A), dev(act["B"], BF),
+                               dev(act["C"], BF), dev(dy, BF), g, z=dev(act["z"], BF),
+                               cu_seqlens=cu_d, workspace=ws)
+    torch.cuda.synchronize()
+    r = orc.selective_scan_bwd(act["x"], act["dt"], prm.A, act["B"], act["C"], dy,
+                               z=act["z"], cu_seqlens=cu_h)
+    assert_close(host(g["du"]), r["du"], True, TOL_BF16, "du")
+    assert_close(host(g["ddelta"]), r["ddt"], True, TOL_BF16, "ddelta")
+    for k in ("dB", "dC", "dA"):
+        assert_close(host(g[k]), r[k], False, TOL_BF16, k)
+    assert ssm.ssm_device_status() == 0
