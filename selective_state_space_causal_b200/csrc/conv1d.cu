@@ -234,6 +234,37 @@ __device__ __forceinline__ void conv_out_pk(const f32x2 (&wk)[K][VEC / 2], const
     }
 }
 
+// conv_state_out[s, c, :] = last K-1 entries of [conv_state_in[s, c, :] || x_seq[:, c]].
+// One thread per (sequence, channel) reads everything it needs before writing,
+// so the output may be the same buffer as the input state.
+template <typename T, typename TS, int K>
+__device__ __forceinline__ void state_out_one(const T *__restrict__ x, const Seqs &sq, int64_t D,
+                                              const TS *state_in, TS *state_out, int64_t s,
+                                              int64_t c)
+{
+    const int64_t s_start = sq.off(s);
+    const int64_t len = max(sq.off(s + 1), s_start) - s_start;
+    float v[K - 1];
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) {
+        const int64_t pos = len - (K - 1) + j;
+        v[j] = pos >= 0 ? to_f32(x[(s_start + pos) * D + c])
+                        : (state_in ? to_f32(state_in[(s * D + c) * (K - 1) + (K - 1) + pos]) : 0.f);
+    }
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) state_out[(s * D + c) * (K - 1) + j] = from_f32<TS>(v[j]);
+}
+
+template <typename T, typename TS, int K>
+__global__ void __launch_bounds__(kThreads)
+conv_state_out_kernel(const T *__restrict__ x, Seqs sq, int64_t D, const TS *state_in,
+                      TS *state_out)
+{
+    const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    if (gid >= sq.S * D) return;
+    state_out_one<T, TS, K>(x, sq, D, state_in, state_out, gid / D, gid % D);
+}
+
 // ---------------------------------------------------------------------------
 // TMA-tiled variant (16-byte aligned rows). A CTA owns kTileT tokens x one
 // 128-byte row of channels: one TMA box of kTileT + K - 1 rows (the K - 1 halo
@@ -242,7 +273,9 @@ __device__ __forceinline__ void conv_out_pk(const f32x2 (&wk)[K][VEC / 2], const
 // kTileG tokens of one 8-byte channel vector and writes 8-byte outputs (a warp
 // still writes whole 128-byte rows). 8-byte vectors keep the weights and window
 // in few registers, so many CTAs fit per SM and overlap one CTA's load with
-// another's arithmetic.
+// another's arithmetic. When the conv-state output does not overlap the input
+// state, CTAs past the n_tiles token tiles of each channel row write it (one
+// (sequence, channel) per thread), which saves a launch.
 // ---------------------------------------------------------------------------
 constexpr int kTileT = 128;      // tokens per CTA
 constexpr int kTileG = 16;       // tokens per thread
@@ -252,7 +285,8 @@ template <typename T, typename TS, int K>
 __global__ void __launch_bounds__(kTileThreads)
 conv1d_tma_kernel(const __grid_constant__ CUtensorMap xmap, T *__restrict__ xc,
                   const float *__restrict__ w, const float *__restrict__ bias, Seqs sq, int64_t D,
-                  const TS *__restrict__ state_in, int apply_silu)
+                  const TS *__restrict__ state_in, int apply_silu, const T *__restrict__ x,
+                  TS *__restrict__ state_out, unsigned n_tiles)
 {
     constexpr int VEC = 8 / sizeof(T);         // channels per 8-byte vector
     constexpr int CW = 128 / sizeof(T);        // channels per tile row (128 bytes)
@@ -265,6 +299,12 @@ conv1d_tma_kernel(const __grid_constant__ CUtensorMap xmap, T *__restrict__ xc,
     const int tid = threadIdx.x;
     const int64_t t0 = (int64_t)blockIdx.x * kTileT;
     const int64_t cbase = (int64_t)blockIdx.y * CW;
+    if (blockIdx.x >= n_tiles) {  // conv-state output of this channel row
+        const int64_t idx = (int64_t)(blockIdx.x - n_tiles) * kTileThreads + tid;
+        const int64_t ss = idx / CW, cc = cbase + idx % CW;
+        if (ss < sq.S && cc < D) state_out_one<T, TS, K>(x, sq, D, state_in, state_out, ss, cc);
+        return;
+    }
     if (tid == 0) mbar_init(&bar);
     __syncthreads();
     if (tid == 0) {
@@ -352,36 +392,13 @@ conv1d_tma_kernel(const __grid_constant__ CUtensorMap xmap, T *__restrict__ xc,
     }
 }
 
-// conv_state_out[s, c, :] = last K-1 entries of [conv_state_in[s, c, :] || x_seq[:, c]].
-// One thread per (sequence, channel) reads everything it needs before writing,
-// so the output may be the same buffer as the input state.
-template <typename T, typename TS, int K>
-__global__ void __launch_bounds__(kThreads)
-conv_state_out_kernel(const T *__restrict__ x, Seqs sq, int64_t D, const TS *state_in,
-                      TS *state_out)
-{
-    const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    if (gid >= sq.S * D) return;
-    const int64_t s = gid / D, c = gid % D;
-    const int64_t s_start = sq.off(s);
-    const int64_t len = max(sq.off(s + 1), s_start) - s_start;
-    float v[K - 1];
-#pragma unroll
-    for (int j = 0; j < K - 1; ++j) {
-        const int64_t pos = len - (K - 1) + j;
-        v[j] = pos >= 0 ? to_f32(x[(s_start + pos) * D + c])
-                        : (state_in ? to_f32(state_in[(s * D + c) * (K - 1) + (K - 1) + pos]) : 0.f);
-    }
-#pragma unroll
-    for (int j = 0; j < K - 1; ++j) state_out[(s * D + c) * (K - 1) + j] = from_f32<TS>(v[j]);
-}
-
 template <typename T, typename TS, int K>
 cudaError_t run(const ConvArgs &a, cudaStream_t stream, int *launches)
 {
     Seqs sq{a.cu, a.S, a.tok, a.cu ? 0 : a.tok / a.S};
     const T *x = static_cast<const T *>(a.x);
     const TS *st_in = static_cast<const TS *>(a.state_in);
+    bool state_done = false;  // the state output rode along with the tile kernel
     if (a.tok > 0) {
         constexpr int V = 16 / sizeof(T);
         const bool vec = a.vec && (a.D % V == 0);
@@ -391,10 +408,21 @@ cudaError_t run(const ConvArgs &a, cudaStream_t stream, int *launches)
         CUtensorMap map;
         if (vec && encode_2d(&map, a.x, sizeof(T) == 2, a.D, a.tok, 128 / sizeof(T),
                              kTileT + K - 1)) {
-            const dim3 grid((unsigned)((a.tok + kTileT - 1) / kTileT),
-                            (unsigned)((a.D * sizeof(T) + 127) / 128));
+            // the state output rides along unless it overlaps the input state,
+            // whose reads by the tile CTAs must all come first
+            const size_t sbytes = (size_t)a.S * a.D * (K - 1) * sizeof(TS);
+            const char *si = static_cast<const char *>(a.state_in);
+            const char *so = static_cast<const char *>(a.state_out);
+            const bool ride = a.state_out && (!si || si + sbytes <= so || so + sbytes <= si);
+            constexpr int CW = 128 / sizeof(T);
+            const unsigned n_tiles = (unsigned)((a.tok + kTileT - 1) / kTileT);
+            const unsigned extra =
+                ride ? (unsigned)((a.S * CW + kTileThreads - 1) / kTileThreads) : 0u;
+            const dim3 grid(n_tiles + extra, (unsigned)((a.D * sizeof(T) + 127) / 128));
             conv1d_tma_kernel<T, TS, K><<<grid, kTileThreads, 0, stream>>>(
-                map, static_cast<T *>(a.xc), a.w, a.bias, sq, a.D, st_in, a.apply_silu);
+                map, static_cast<T *>(a.xc), a.w, a.bias, sq, a.D, st_in, a.apply_silu, x,
+                static_cast<TS *>(a.state_out), n_tiles);
+            state_done = ride;
         } else if (vec)
             conv1d_kernel<T, TS, V, K><<<blocks, kThreads, 0, stream>>>(
                 x, static_cast<T *>(a.xc), a.w, a.bias, sq, a.D, st_in, a.apply_silu);
@@ -405,7 +433,7 @@ cudaError_t run(const ConvArgs &a, cudaStream_t stream, int *launches)
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    if (a.state_out) {
+    if (a.state_out && !state_done) {
         const int64_t n = a.S * a.D;
         const unsigned blocks = (unsigned)((n + kThreads - 1) / kThreads);
         conv_state_out_kernel<T, TS, K><<<blocks, kThreads, 0, stream>>>(
