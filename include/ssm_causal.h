@@ -236,6 +236,36 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
                                ssm_dtype conv_state_dtype, ssm_stream_t stream);
 
 /*
+ * Causal depthwise conv1d + SiLU fused into the selective scan: the result of
+ * ssm_causal_conv1d (apply_silu = 1) feeding ssm_selective_scan_fwd as u, in
+ * one kernel that never writes the conv output to memory (it stays in fp32,
+ * where the two-call path stores it in act_dtype between the calls). Follows
+ * the mixer dataflow of "Scaling State-Space Models on Multiple GPUs with
+ * Tensor Parallelism", Fig. 1 (conv, then the state update), with the math of
+ * tp_builder.py, _add_mamba_tp_layer, over packed sequences (PackMamba,
+ * abstract).
+ *
+ *   x, conv_w, conv_b, conv_state_in, conv_state_out, K, conv_state_dtype:
+ *                  as ssm_causal_conv1d (conv_state_out may be conv_state_in)
+ *   xc             (tok, D) act_dtype or NULL: if given, the conv output is also
+ *                  written there (rounded to act_dtype)
+ *   delta, A, B, C, Dskip, z, dt_bias, delta_softplus, h0, cu_seqlens, S, y,
+ *   h_final, tok, D, N, act_dtype: as ssm_selective_scan_fwd (u is the conv
+ *                  output); y must not overlap x, delta or z
+ * Always one kernel: the scan's register-prefetch layout (4 or 8 states per
+ * lane as ssm_scan_variant_for reports it, 4 when rows are not 16-byte
+ * aligned), sequences in index order. Where the scan alone would pick a TMA
+ * schedule (many sequence-channel pairs) the two-call path can be faster.
+ */
+int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
+                      const void *conv_state_in, void *conv_state_out, void *xc, int K,
+                      ssm_dtype conv_state_dtype, const void *delta, const float *A,
+                      const void *B, const void *C, const float *Dskip, const void *z,
+                      const float *dt_bias, int delta_softplus, const float *h0,
+                      const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
+                      int64_t tok, int64_t D, int N, ssm_dtype act_dtype, ssm_stream_t stream);
+
+/*
  * Workspace bytes ssm_selective_scan_bwd needs for `tok` packed tokens of D
  * channels in S sequences (N must be 16; 0 for invalid sizes): one fp32 state
  * checkpoint per 16 tokens of each sequence and channel, about 4 bytes per

@@ -12,6 +12,7 @@ from ._lib import (  # noqa: F401
     lib,
     replay_buffers,
     ssm_causal_conv1d,
+    ssm_conv_scan_fwd,
     ssm_check_cu_seqlens,
     ssm_last_error,
     ssm_launch_count,

@@ -40,6 +40,9 @@ SIGNATURES = [
     ("ssm_selective_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                           _vp, _int, _vp, _i64, _vp, _i64, _i64, _int, _int, _int,
                                           _int, _vp]),
+    ("ssm_conv_scan_fwd", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _vp, _vp, _vp, _vp,
+                                 _vp, _vp, _vp, _int, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _int,
+                                 _int, _vp]),
     ("ssm_scan_bwd_workspace_size", _sz, [_i64, _i64, _int, _i64]),
     ("ssm_selective_scan_bwd", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64,
                                       _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
@@ -289,3 +292,23 @@ def ssm_selective_scan_bwd(u, delta, A, B, C, dy, grads, Dskip=None, z=None, dt_
         _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g.get("dz")), _ptr(g["dB"]), _ptr(g["dC"]),
         _ptr(g["dA"]), _ptr(g.get("dDskip")), _ptr(g.get("ddt_bias")), _ptr(g.get("dh0")), tok, D,
         N, _dtype(u), _ptr(workspace), ws_bytes, _stream(stream)))
+
+
+def ssm_conv_scan_fwd(x, conv_w, delta, A, B, C, y, conv_b=None, conv_state_in=None,
+                      conv_state_out=None, xc=None, Dskip=None, z=None, dt_bias=None,
+                      delta_softplus=True, h0=None, h_final=None, cu_seqlens=None, S=None,
+                      stream=None):
+    """Fused conv1d + SiLU -> selective scan. x, delta, z, y, xc: (tok, D);
+    conv_w (D, K) fp32; conv states (S, D, K-1); A (D, N); B, C (tok, N)."""
+    tok, D = x.shape
+    N = A.shape[1]
+    K = conv_w.shape[1]
+    if S is None:
+        S = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
+    st = conv_state_in if conv_state_in is not None else conv_state_out
+    sdt = _dtype(st) if st is not None else _dtype(x)
+    _check(lib.ssm_conv_scan_fwd(
+        _ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(conv_state_in), _ptr(conv_state_out), _ptr(xc),
+        K, sdt, _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(cu_seqlens), S, _ptr(y), _ptr(h_final), tok, D,
+        N, _dtype(x), _stream(stream)))

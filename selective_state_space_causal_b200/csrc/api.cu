@@ -37,6 +37,18 @@ struct ScanBwdArgs {
     bool bf16;
 };
 size_t scan_bwd_ckpt_floats(int64_t tok, int64_t D, int64_t S);
+
+struct ConvScanArgs {
+    const void *x;
+    const float *w, *bias;
+    const void *state_in;
+    void *state_out;
+    void *xc;
+    int K;
+    DType state_dtype;
+    ScanArgs scan;
+};
+cudaError_t launch_conv_scan(const ConvScanArgs &a, int npt, cudaStream_t stream, int *launches);
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *launches);
 
 struct ReplayStepArgs {
@@ -301,6 +313,63 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
                       dt(conv_state_dtype)};
     int launched = 0;
     cudaError_t e = ssm::launch_decode(a, reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
+int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
+                      const void *conv_state_in, void *conv_state_out, void *xc, int K,
+                      ssm_dtype conv_state_dtype, const void *delta, const float *A,
+                      const void *B, const void *C, const float *Dskip, const void *z,
+                      const float *dt_bias, int delta_softplus, const float *h0,
+                      const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
+                      int64_t tok, int64_t D, int N, ssm_dtype act_dtype, ssm_stream_t stream)
+{
+    const char *fn = "ssm_conv_scan_fwd";
+    if (!valid_dtype(act_dtype) || !valid_dtype(conv_state_dtype))
+        return fail(SSM_ERR_UNSUPPORTED_DTYPE, "%s: unknown dtype", fn);
+    if (N != 16) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: N must be 16 (got %d)", fn, N);
+    if (K < 2 || K > 4) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: K must be 2..4 (got %d)", fn, K);
+    if (D < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: D must be >= 1", fn);
+    if (int r = check_seqs(fn, cu_seqlens, S, tok)) return r;
+    if (!A || !conv_w) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: A and conv_w are required", fn);
+    if (tok > 0 && (!x || !delta || !B || !C || !y))
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: x, delta, B, C and y are required", fn);
+    const size_t es = esize(act_dtype), ss = esize(conv_state_dtype);
+    if (!aligned(x, es) || !aligned(delta, es) || !aligned(z, es) || !aligned(y, es) ||
+        !aligned(xc, es) || !aligned(conv_state_in, ss) || !aligned(conv_state_out, ss) ||
+        !aligned(A, 4) || !aligned(conv_w, 4) || !aligned(conv_b, 4) || !aligned(Dskip, 4) ||
+        !aligned(dt_bias, 4) || !aligned(h0, 4) || !aligned(h_final, 4))
+        return fail(SSM_ERR_MISALIGNED, "%s: a pointer is not aligned to its element size", fn);
+    if (!aligned(B, 16) || !aligned(C, 16))
+        return fail(SSM_ERR_MISALIGNED, "%s: B and C must be 16-byte aligned", fn);
+    if (tok > 0) {
+        const size_t bytes = (size_t)tok * D * es;
+        const void *outs[2] = {y, xc};
+        const void *ins[4] = {x, delta, z, nullptr};
+        for (const void *o : outs) {
+            if (!o) continue;
+            for (const void *in : ins) {
+                if (!in) continue;
+                const char *a = static_cast<const char *>(in), *b = static_cast<const char *>(o);
+                if (a < b + bytes && b < a + bytes)
+                    return fail(SSM_ERR_INVALID_ARGUMENT, "%s: an output overlaps an input", fn);
+            }
+        }
+        if (xc) {
+            const char *a = static_cast<const char *>(xc), *b = static_cast<const char *>(y);
+            if (a < b + bytes && b < a + bytes)
+                return fail(SSM_ERR_INVALID_ARGUMENT, "%s: xc overlaps y", fn);
+        }
+    }
+    int npt = 4, sched = 1;
+    ssm::scan_variant_for(S, D, &npt, &sched);
+    ssm::ScanArgs sa{x, delta, A, B, C, Dskip, z, dt_bias, delta_softplus, h0, cu_seqlens, S, y,
+                     h_final, tok, D, N, dt(act_dtype), nullptr, true};
+    ssm::ConvScanArgs a{x, conv_w, conv_b, conv_state_in, conv_state_out, xc, K,
+                        dt(conv_state_dtype), sa};
+    int launched = 0;
+    cudaError_t e = ssm::launch_conv_scan(a, npt == 8 ? 8 : 4,
+                                          reinterpret_cast<cudaStream_t>(stream), &launched);
     return finish(e, launched, fn);
 }
 

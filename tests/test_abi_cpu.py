@@ -238,3 +238,24 @@ def test_scan_bwd_workspace_size():
     n = ssm.ssm_scan_bwd_workspace_size(16384, 1536, 16, 8)
     assert n % 256 == 0 and n >= (16384 // 16 + 8) * 1536 * 64
     assert ssm.ssm_scan_bwd_workspace_size(100, 64, 8, 1) == 0
+
+
+def conv_scan(**kw):
+    a = dict(x=A16, w=A16, b=None, si=None, so=None, xc=None, K=4, sdt=1, dt=A16 + 0x200000,
+             A=A16, B=A16, C=A16, Dsk=None, z=None, dtb=None, sp=1, h0=None, cu=None, S=1,
+             y=A16 + 0x400000, hf=None, tok=64, D=32, N=16, adt=1)
+    a.update(kw)
+    return L.ssm_conv_scan_fwd(a["x"], a["w"], a["b"], a["si"], a["so"], a["xc"], a["K"], a["sdt"],
+                               a["dt"], a["A"], a["B"], a["C"], a["Dsk"], a["z"], a["dtb"],
+                               a["sp"], a["h0"], a["cu"], a["S"], a["y"], a["hf"], a["tok"],
+                               a["D"], a["N"], a["adt"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(K=5), -1), (dict(N=8), -1), (dict(w=None), -1), (dict(x=None), -1), (dict(y=None), -1),
+    (dict(B=A16 + 8), -3), (dict(x=A16 + 1), -3), (dict(adt=7), -2), (dict(sdt=7), -2),
+    (dict(y=A16), -1), (dict(xc=A16 + 0x400000), -1), (dict(S=3, tok=64), -1),
+])
+def test_conv_scan_rejects(kw, code):
+    assert conv_scan(**kw) == code
+    assert _err()
