@@ -292,7 +292,7 @@ def bench_headline(args, world, peaks, rank_dev):
 
     mufu = mufu_peak_gexp(peaks["sm_max_mhz"])
     achieved = st.scan_exps() / (scan_ms * 1e-3) / 1e9
-    sha = source_sha("scan.cu", "common.cuh")
+    sha = source_sha("scan.cu", "scan_parts.cuh", "common.cuh")
     npt, sched = st.ssm.ssm_scan_variant_for(st.Bn, st.D)
     kernel = SCAN_KERNELS.get(sched, "scan_tma_kernel")
     traffic = recorded_traffic(kernel, sha)
@@ -308,6 +308,40 @@ def bench_headline(args, world, peaks, rank_dev):
                                  / 1e9 / peaks["hbm_gbs"], 4)
     res = {"value": value, "ms_per_step": ms_max, "roofline": roofline, "clocks": clk,
            "gpu_launches": int(launches), "step_ms_this_rank": ms}
+
+    # the same step with the fused conv -> scan kernel
+    def fused_step(i, ev=None):
+        ssm_, ly = st.ssm, st.layer
+        a = st.sets[i % st.SETS]
+        d = st.dec[i % st.SETS]
+        if ev is not None:
+            ev[0].record()
+        ssm_.ssm_conv_scan_fwd(a["x"], ly.w, a["dt"], ly.A, a["B"], a["C"], st.y, conv_b=ly.b,
+                               conv_state_out=st.cs, Dskip=ly.Dskip, z=a["z"],
+                               dt_bias=ly.dt_bias, h_final=st.h, S=st.Bn)
+        if ev is not None:
+            ev[1].record()
+        ssm_.ssm_selective_state_update(st.cs, st.h, d["x"], d["dt"], d["B"], d["C"], st.yd, ly.w,
+                                        ly.A, z=d["z"], conv_b=ly.b, Dskip=ly.Dskip,
+                                        dt_bias=ly.dt_bias)
+
+    for i in range(args.warmup):
+        fused_step(i)
+    Kf = max(10, K // 4)
+    fevs = [_events(2) for _ in range(Kf)]
+    _barrier_sync(world)
+    start.record()
+    for i in range(Kf):
+        fused_step(i, fevs[i])
+    stop.record()
+    _barrier_sync(world)
+    fms = _max_over_ranks(start.elapsed_time(stop) / Kf, world)
+    f_kernel_ms = sum(e[0].elapsed_time(e[1]) for e in fevs) / Kf
+    res["fused_step"] = {
+        "value": whole_job_rate(st.units(), world, fms), "unit": UNIT, "ms_per_step": fms,
+        "conv_scan_kernel_ms": round(f_kernel_ms, 5),
+        "mufu_frac": round(st.scan_exps() / (f_kernel_ms * 1e-3) / 1e9 / mufu, 4),
+        "step": "ssm_conv_scan_fwd (fused conv1d+silu -> selective_scan) -> 1 decode step"}
 
     # end to end through the public API with pinned host buffers
     host_in = {k: v.cpu().pin_memory() for k, v in st.sets[0].items()}
@@ -931,7 +965,8 @@ def main():
                        "l2": "4 rotating input sets (~600 MB) larger than L2",
                        "parallelism": f"replicas x{world}"},
             "roofline": res["roofline"], "clocks": res["clocks"], "e2e": res["e2e"],
-            "e2e_serial": res["e2e_serial"], "gpu_launches": res["gpu_launches"], "cpu_baseline": cpu, "workloads": secondary,
+            "e2e_serial": res["e2e_serial"], "fused_step": res["fused_step"],
+            "gpu_launches": res["gpu_launches"], "cpu_baseline": cpu, "workloads": secondary,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

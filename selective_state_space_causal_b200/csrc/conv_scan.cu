@@ -51,7 +51,7 @@ __device__ __forceinline__ float conv_silu_f(float z)
 template <class K, int KW>
 struct ConvSmem {
     static constexpr int ROWS = K::TCH + KW - 1;
-    static constexpr int RS = K::CH + 1;  // row stride: one float of padding per row
+    static constexpr int RS = K::CH + 4;  // row stride: 16 bytes of padding per row
     static constexpr size_t OFF_X = K::SMEM;                          // fp32 [ROWS][RS]
     static constexpr size_t OFF_W = align128(OFF_X + sizeof(float) * ROWS * RS);
     static constexpr size_t OFF_BIAS = OFF_W + sizeof(float) * K::CH * KW;
@@ -72,7 +72,7 @@ conv_scan_kernel(const Params p, const ConvParams cp)
     float *sB = reinterpret_cast<float *>(smem + K::OFF_B);
     float *sC = reinterpret_cast<float *>(smem + K::OFF_C);
     // tile row r holds position t0 - (KW-1) + r; rows are RS floats apart so
-    // that items of different tokens read different banks
+    // that the 16-byte reads of items of different tokens hit different banks
     float *sX = reinterpret_cast<float *>(smem + G::OFF_X);
     float *sW = reinterpret_cast<float *>(smem + G::OFF_W);   // [KW][CH], tap-major
     constexpr int RS = G::RS;
@@ -112,6 +112,14 @@ conv_scan_kernel(const Params p, const ConvParams cp)
 #pragma unroll
     for (int i = 0; i < VEC; ++i) dtb[i] = (l.vvalid && p.dt_bias) ? __ldg(p.dt_bias + l.cg + i) : 0.f;
     const int cvl = l.cvl * VEC;  // this thread's first channel within the CTA
+    __syncthreads();  // taps and bias staged
+    float wr[KW][VEC], br[VEC];  // this thread's taps and bias (its channel vector is fixed)
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        br[e] = sBias[cvl + e];
+#pragma unroll
+        for (int k = 0; k < KW; ++k) wr[k][e] = sW[k * CH + cvl + e];
+    }
 
     RawT rdt[IPT], rx[IPT], rz[IPT];
     uint4 rb[K::BPT], rc[K::BPT];
@@ -155,8 +163,15 @@ conv_scan_kernel(const Params p, const ConvParams cp)
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) fx[e] = 0.f;
             }
+            float *dst = sX + (KW - 1 + tl) * RS + cvl;
+            if constexpr (VEC % 4 == 0) {
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) sX[(KW - 1 + tl) * RS + cvl + e] = fx[e];
+                for (int e = 0; e < VEC; e += 4)
+                    *reinterpret_cast<float4 *>(dst + e) = make_float4(fx[e], fx[e + 1], fx[e + 2], fx[e + 3]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) dst[e] = fx[e];
+            }
         }
         __syncthreads();  // tile complete (and the previous chunk's readers are done)
 #pragma unroll
@@ -168,12 +183,27 @@ conv_scan_kernel(const Params p, const ConvParams cp)
             if (live) {
                 unpack<T, VEC>(rdt[i], fdt);
                 if (Z) unpack<T, VEC>(rz[i], fz);
+                float win[KW][VEC];
+#pragma unroll
+                for (int k = 0; k < KW; ++k) {
+                    const float *src = sX + (tl + k) * RS + cvl;
+                    if constexpr (VEC % 4 == 0) {
+#pragma unroll
+                        for (int e = 0; e < VEC; e += 4) {
+                            const float4 v4 = *reinterpret_cast<const float4 *>(src + e);
+                            win[k][e] = v4.x; win[k][e + 1] = v4.y;
+                            win[k][e + 2] = v4.z; win[k][e + 3] = v4.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < VEC; ++e) win[k][e] = src[e];
+                    }
+                }
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) {
-                    float acc = sBias[cvl + e];
+                    float acc = br[e];
 #pragma unroll
-                    for (int k = 0; k < KW; ++k)
-                        acc = fmaf(sW[k * CH + cvl + e], sX[(tl + k) * RS + cvl + e], acc);
+                    for (int k = 0; k < KW; ++k) acc = fmaf(wr[k][e], win[k][e], acc);
                     fu[e] = conv_silu_f(acc);
                 }
                 if (XC) store_vec<T, VEC>(XC + (t0 + tl) * p.D + l.cg, fu);
