@@ -10,13 +10,14 @@
 // state (or zeros), and the sequence's last K-1 inputs become its new conv
 // state.
 //
-// The kernel is the register-prefetch scan (schedule 1) with one more stage in
-// its per-chunk pre-pass: the chunk's raw x rows (prefetched into registers one
-// chunk ahead, as u is in the plain scan) are written as fp32 into a
-// shared-memory tile below K-1 halo rows (the previous chunk's last inputs, or
-// the carried state at a sequence start); after a barrier each pre-pass item
-// forms its conv output from the tile, applies SiLU and proceeds as the plain
-// scan's pre-pass with that value as u. The conv takes the same operations in
+// The kernel is the register-prefetch scan (schedule 1) with the conv in its
+// per-chunk pre-pass: the chunk's raw x rows (prefetched into registers one
+// chunk ahead, as u is in the plain scan) sit as fp32 in a shared-memory tile
+// below K-1 halo rows (the previous chunk's last inputs, or the carried state
+// at a sequence start); each pre-pass item forms its conv output from the
+// tile, applies SiLU and proceeds as the plain scan's pre-pass with that value
+// as u. Two tiles alternate, so the next chunk's tile is filled during this
+// chunk and no extra barrier is needed. The conv takes the same operations in
 // the same order as the conv kernel (taps oldest first, bias first, SiLU as
 // x * 1/(1 + 2^(-x log2 e))), and xc stays in fp32.
 #include "common.cuh"
@@ -52,8 +53,8 @@ template <class K, int KW>
 struct ConvSmem {
     static constexpr int ROWS = K::TCH + KW - 1;
     static constexpr int RS = K::CH + 4;  // row stride: 16 bytes of padding per row
-    static constexpr size_t OFF_X = K::SMEM;                          // fp32 [ROWS][RS]
-    static constexpr size_t OFF_W = align128(OFF_X + sizeof(float) * ROWS * RS);
+    static constexpr size_t OFF_X = K::SMEM;                          // fp32 [2][ROWS][RS]
+    static constexpr size_t OFF_W = align128(OFF_X + sizeof(float) * 2 * ROWS * RS);
     static constexpr size_t OFF_BIAS = OFF_W + sizeof(float) * K::CH * KW;
     static constexpr size_t SMEM = align128(OFF_BIAS + sizeof(float) * K::CH);
 };
@@ -112,14 +113,6 @@ conv_scan_kernel(const Params p, const ConvParams cp)
 #pragma unroll
     for (int i = 0; i < VEC; ++i) dtb[i] = (l.vvalid && p.dt_bias) ? __ldg(p.dt_bias + l.cg + i) : 0.f;
     const int cvl = l.cvl * VEC;  // this thread's first channel within the CTA
-    __syncthreads();  // taps and bias staged
-    float wr[KW][VEC], br[VEC];  // this thread's taps and bias (its channel vector is fixed)
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-        br[e] = sBias[cvl + e];
-#pragma unroll
-        for (int k = 0; k < KW; ++k) wr[k][e] = sW[k * CH + cvl + e];
-    }
 
     RawT rdt[IPT], rx[IPT], rz[IPT];
     uint4 rb[K::BPT], rc[K::BPT];
@@ -147,33 +140,59 @@ conv_scan_kernel(const Params p, const ConvParams cp)
         }
     };
 
-    int nt_last = 0;
-    if (l.start < l.end) prefetch(l.start);
-    for (int64_t t0 = l.start; t0 < l.end; t0 += TCH) {
-        const int nt = (int)min((int64_t)TCH, l.end - t0);
-        nt_last = nt;
-        // raw x of the chunk into the tile, below the halo rows
+    // Two tiles: chunk k convolves from tile k mod 2 and fills tile (k+1) mod 2
+    // for the next chunk (its halo rows from chunk k's last inputs during the
+    // pre-pass, its own rows from the prefetched registers after the
+    // recurrence), so the chunk needs no barrier beyond the scan's own.
+    float *const tile0 = sX, *const tile1 = sX + G::ROWS * RS;
+    auto put = [&](float *row, const float (&fx)[VEC]) {
+        if constexpr (VEC % 4 == 0) {
+#pragma unroll
+            for (int e = 0; e < VEC; e += 4)
+                *reinterpret_cast<float4 *>(row + e) = make_float4(fx[e], fx[e + 1], fx[e + 2], fx[e + 3]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) row[e] = fx[e];
+        }
+    };
+    // the raw x rows of the chunk starting at t1 (prefetched) into a tile
+    auto put_chunk = [&](float *tile, int64_t t1) {
+        const int n1 = (int)min((int64_t)TCH, l.end - t1);
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
             if (tid + i * THREADS >= K::ITEMS) break;
             const int tl = (tid + i * THREADS) / CV;
             float fx[VEC];
-            if (tl < nt && l.vvalid) unpack<T, VEC>(rx[i], fx);
+            if (tl < n1 && l.vvalid) unpack<T, VEC>(rx[i], fx);
             else {
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) fx[e] = 0.f;
             }
-            float *dst = sX + (KW - 1 + tl) * RS + cvl;
-            if constexpr (VEC % 4 == 0) {
-#pragma unroll
-                for (int e = 0; e < VEC; e += 4)
-                    *reinterpret_cast<float4 *>(dst + e) = make_float4(fx[e], fx[e + 1], fx[e + 2], fx[e + 3]);
-            } else {
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) dst[e] = fx[e];
-            }
+            put(tile + (KW - 1 + tl) * RS + cvl, fx);
         }
-        __syncthreads();  // tile complete (and the previous chunk's readers are done)
+    };
+
+    int nt_last = 0;
+    float *tile_last = tile0;
+    if (l.start < l.end) {
+        prefetch(l.start);
+        put_chunk(tile0, l.start);
+    }
+    __syncthreads();  // taps, bias, carried state and the first chunk's rows are staged
+    float wr[KW][VEC], br[VEC];  // this thread's taps and bias (its channel vector is fixed)
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+        br[e] = sBias[cvl + e];
+#pragma unroll
+        for (int k = 0; k < KW; ++k) wr[k][e] = sW[k * CH + cvl + e];
+    }
+    int cur = 0;
+    for (int64_t t0 = l.start; t0 < l.end; t0 += TCH) {
+        const int nt = (int)min((int64_t)TCH, l.end - t0);
+        const bool more = t0 + TCH < l.end;  // then this chunk is full (nt = TCH >= KW - 1)
+        float *tc = cur ? tile1 : tile0, *tn = cur ? tile0 : tile1;
+        nt_last = nt;
+        tile_last = tc;
 #pragma unroll
         for (int i = 0; i < IPT; ++i) {
             if (tid + i * THREADS >= K::ITEMS) break;
@@ -186,7 +205,7 @@ conv_scan_kernel(const Params p, const ConvParams cp)
                 float win[KW][VEC];
 #pragma unroll
                 for (int k = 0; k < KW; ++k) {
-                    const float *src = sX + (tl + k) * RS + cvl;
+                    const float *src = tc + (tl + k) * RS + cvl;
                     if constexpr (VEC % 4 == 0) {
 #pragma unroll
                         for (int e = 0; e < VEC; e += 4) {
@@ -207,6 +226,13 @@ conv_scan_kernel(const Params p, const ConvParams cp)
                     fu[e] = conv_silu_f(acc);
                 }
                 if (XC) store_vec<T, VEC>(XC + (t0 + tl) * p.D + l.cg, fu);
+                // the next chunk's halo rows: this chunk's last KW-1 inputs
+                if (more && tl >= nt - (KW - 1)) put(tn + (tl - (nt - (KW - 1))) * RS + cvl, win[KW - 1]);
+            } else if (more && tl >= nt - (KW - 1)) {
+                float zero[VEC];
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) zero[e] = 0.f;
+                put(tn + (tl - (nt - (KW - 1))) * RS + cvl, zero);
             }
             prepass_item<VEC>(sDX + tl * K::ROW2 + l.vcol, sUG + tl * K::ROW2 + l.vcol, live, fdt,
                               fu, fz, Z != nullptr, dtb, p.delta_softplus);
@@ -228,29 +254,26 @@ conv_scan_kernel(const Params p, const ConvParams cp)
             }
         }
         __syncthreads();
-        // the next chunk's halo: this chunk's last KW-1 inputs (a full chunk,
-        // so source and destination rows do not overlap)
-        if (t0 + TCH < l.end) {
-            for (int e = tid; e < (KW - 1) * CH; e += THREADS)
-                sX[(e / CH) * RS + e % CH] = sX[(nt + e / CH) * RS + e % CH];
-            prefetch(t0 + TCH);
-        }
+        if (more) prefetch(t0 + TCH);
         const int ntr = ((nt + K::TPC - 1) / K::TPC) * K::TPC;
         recur_chunk<K>(sDX, sUG, sB, sC, ntr, l.mycol, l.sub, A2p, hp, dsk);
+        if (more) put_chunk(tn, t0 + TCH);  // the loads have had the recurrence to land
         __syncthreads();
         store_y<K, T>(static_cast<T *>(p.y), sUG, tid, nt, l.vvalid, l.vcol, t0, p.D, l.cg);
+        cur ^= 1;
     }
     save_state<K>(p, l, hp);
     // new conv state: the last KW-1 positions of [carried state || x_seq], which
-    // sit in tile rows nt_last .. nt_last + KW-2 (rows 0.. when the sequence is
-    // empty)
+    // sit in rows nt_last .. nt_last + KW-2 of the last chunk's tile (rows 0.. of
+    // the first tile when the sequence is empty); every write to it preceded a
+    // barrier
     if (SOUT) {
-        __syncthreads();  // the empty sequence's halo rows were written by other threads
         for (int e = tid; e < (KW - 1) * CH; e += THREADS) {
             const int j = e / CH, cl = e % CH;
             const int64_t c = l.cbase + cl;
             if (c < p.D)
-                SOUT[(l.seq * p.D + c) * (KW - 1) + j] = from_f32<TS>(sX[(nt_last + j) * RS + cl]);
+                SOUT[(l.seq * p.D + c) * (KW - 1) + j] =
+                    from_f32<TS>(tile_last[(nt_last + j) * RS + cl]);
         }
     }
 }
