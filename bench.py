@@ -617,23 +617,31 @@ def bench_scan_bwd(peaks, world, ly, a, cu, S, steps_scale=1.0):
         ssm.ssm_selective_scan_bwd(a["x"], a["dt"], ly.A, a["B"], a["C"], dy, g, Dskip=ly.Dskip,
                                    z=a["z"], dt_bias=ly.dt_bias, cu_seqlens=cu, workspace=ws)
 
-    for _ in range(2):
-        call()
-    n = max(3, int(10 * steps_scale))
-    s0, s1 = _events(2)
-    _barrier_sync(world)
-    s0.record()
-    for _ in range(n):
-        call()
-    s1.record()
-    _barrier_sync(world)
-    ms = _max_over_ranks(s0.elapsed_time(s1) / n, world)
+    def timed(variant):
+        ssm.ssm_set_scan_bwd_variant(variant)
+        for _ in range(2):
+            call()
+        n = max(3, int(10 * steps_scale))
+        s0, s1 = _events(2)
+        _barrier_sync(world)
+        s0.record()
+        for _ in range(n):
+            call()
+        s1.record()
+        _barrier_sync(world)
+        return _max_over_ranks(s0.elapsed_time(s1) / n, world)
+
+    # both kernels (4 lanes per channel; one thread per channel), then the
+    # library's own choice, which is the reported figure
+    per_variant = {str(v): round(timed(v), 4) for v in (1, 2)}
+    ms = timed(0)
     mufu = mufu_peak_gexp(peaks["sm_max_mhz"])
     units = tok * D
     res = {"gtoken_ch_per_s": units * world / (ms * 1e-3) / 1e9, "ms_per_call": ms,
            "mufu_frac": round(units * 2 * N_STATE / (ms * 1e-3) / 1e9 / mufu, 4),
            "executed_exp_frac": round(units * 3 * N_STATE / (ms * 1e-3) / 1e9 / mufu, 4),
            "hbm_frac": round(units * 14 / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+           "variant": ssm.ssm_scan_bwd_variant_for(S, D), "ms_per_variant": per_variant,
            "workspace_bytes": ws.numel(), "sequences": S,
            "step": "ssm_selective_scan_bwd over the packed 65536 x 5120 prefill, all gradients"}
     del g, ws, dy
@@ -884,7 +892,8 @@ def profile_scan_bwd():
                                    z=a["z"], dt_bias=ly.dt_bias, cu_seqlens=cu, workspace=ws)
     torch.cuda.synchronize()
     assert ssm.ssm_device_status() == 0
-    print(json.dumps({"profile_scan_bwd": {"tokens": tot, "d_inner": D, "sequences": len(lens)}}))
+    print(json.dumps({"profile_scan_bwd": {"tokens": tot, "d_inner": D, "sequences": len(lens),
+                                           "variant": ssm.ssm_scan_bwd_variant_for(len(lens), D)}}))
 
 
 def profile_decode(W):

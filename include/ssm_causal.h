@@ -267,11 +267,33 @@ int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
 
 /*
  * Workspace bytes ssm_selective_scan_bwd needs for `tok` packed tokens of D
- * channels in S sequences (N must be 16; 0 for invalid sizes): one fp32 state
- * checkpoint per 16 tokens of each sequence and channel, about 4 bytes per
- * token and channel.
+ * channels in S sequences (N must be 16; 0 for invalid sizes): room for one
+ * fp32 state checkpoint per 8 tokens of each sequence and channel (about 8
+ * bytes per token and channel) and the sequences' longest-first order.
  */
 size_t ssm_scan_bwd_workspace_size(int64_t tok, int64_t D, int N, int64_t S);
+
+/*
+ * Tuning knob for ssm_selective_scan_bwd's kernel: 1 splits each channel's
+ * 16 states over 4 lanes (16-token chunks, per-token sums over states and
+ * channels by shuffles); 2 gives each channel one thread with all 16 states
+ * (8-token chunks whose states are summed over channels from shared memory;
+ * about half of variant 1's instructions per token and channel, a quarter of
+ * its threads); 0 lets the library choose (2 once S * ceil(D / 128) reaches
+ * twice the SM count, else 1). Process-wide; not
+ * thread-safe against concurrent backward calls. Returns SSM_OK or
+ * SSM_ERR_INVALID_ARGUMENT. The variants differ only in the order of their
+ * floating-point sums.
+ */
+int ssm_set_scan_bwd_variant(int variant);
+
+/*
+ * The kernel (1 or 2, as ssm_set_scan_bwd_variant names them) that
+ * ssm_selective_scan_bwd uses for S sequences of D channels on the current
+ * device, written to *variant. Host-only; launches nothing. Returns SSM_OK,
+ * or SSM_ERR_INVALID_ARGUMENT for S < 1, D < 1 or a NULL pointer.
+ */
+int ssm_scan_bwd_variant_for(int64_t S, int64_t D, int *variant);
 
 /*
  * Backward of ssm_selective_scan_fwd: gradients of the loss L through

@@ -44,6 +44,8 @@ SIGNATURES = [
                                  _vp, _vp, _vp, _int, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _int,
                                  _int, _vp]),
     ("ssm_scan_bwd_workspace_size", _sz, [_i64, _i64, _int, _i64]),
+    ("ssm_set_scan_bwd_variant", _int, [_int]),
+    ("ssm_scan_bwd_variant_for", _int, [_i64, _i64, ctypes.POINTER(_int)]),
     ("ssm_selective_scan_bwd", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64,
                                       _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                       _i64, _int, _int, _vp, _sz, _vp]),
@@ -271,6 +273,17 @@ def ssm_replay_flush(rep, A, slots=None, n=None, stream=None):
 
 def ssm_scan_bwd_workspace_size(tok: int, D: int, N: int, S: int) -> int:
     return int(lib.ssm_scan_bwd_workspace_size(tok, D, N, S))
+
+
+def ssm_set_scan_bwd_variant(variant: int) -> None:
+    """0: library's choice; 1: four lanes per channel; 2: one thread per channel."""
+    _check(lib.ssm_set_scan_bwd_variant(int(variant)))
+
+
+def ssm_scan_bwd_variant_for(S: int, D: int) -> int:
+    v = ctypes.c_int(0)
+    _check(lib.ssm_scan_bwd_variant_for(int(S), int(D), ctypes.byref(v)))
+    return v.value
 
 
 def ssm_selective_scan_bwd(u, delta, A, B, C, dy, grads, Dskip=None, z=None, dt_bias=None,

@@ -36,7 +36,9 @@ struct ScanBwdArgs {
     int softplus;
     bool bf16;
 };
-size_t scan_bwd_ckpt_floats(int64_t tok, int64_t D, int64_t S);
+size_t scan_bwd_workspace_bytes(int64_t tok, int64_t D, int64_t S);
+void set_scan_bwd_variant(int v);
+int scan_bwd_variant_for(int64_t S, int64_t D);
 
 struct ConvScanArgs {
     const void *x;
@@ -376,7 +378,24 @@ int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
 size_t ssm_scan_bwd_workspace_size(int64_t tok, int64_t D, int N, int64_t S)
 {
     if (tok < 0 || D < 1 || N != 16 || S < 1) return 0;
-    return (ssm::scan_bwd_ckpt_floats(tok, D, S) * sizeof(float) + 255) / 256 * 256;
+    return ssm::scan_bwd_workspace_bytes(tok, D, S);
+}
+
+int ssm_set_scan_bwd_variant(int variant)
+{
+    if (variant < 0 || variant > 2)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "ssm_set_scan_bwd_variant: variant 0, 1 or 2");
+    ssm::set_scan_bwd_variant(variant);
+    return ok();
+}
+
+int ssm_scan_bwd_variant_for(int64_t S, int64_t D, int *variant)
+{
+    if (S < 1 || D < 1 || !variant)
+        return fail(SSM_ERR_INVALID_ARGUMENT,
+                    "ssm_scan_bwd_variant_for: S >= 1, D >= 1 and an output pointer required");
+    *variant = ssm::scan_bwd_variant_for(S, D);
+    return ok();
 }
 
 int ssm_selective_scan_bwd(const void *u, const void *delta, const float *A, const void *B,

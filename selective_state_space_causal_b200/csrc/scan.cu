@@ -1630,6 +1630,17 @@ void set_scan_variant(int npt, int sched)
 
 size_t scan_order_bytes(int64_t S) { return (size_t)((S * 4 + 255) / 256) * 256; }
 
+// Longest-first order of packed sequences (as the scan uses it), for the
+// library's other kernels over packed sequences.
+cudaError_t launch_seq_order(const int32_t *cu, int64_t S, int64_t tok, int32_t *order,
+                             cudaStream_t stream)
+{
+    order_kernel<<<1, 1024, 0, stream>>>(cu, S, tok, order);
+    return cudaGetLastError();
+}
+
+int device_sm_count() { return sm_count(); }
+
 int read_scan_status(bool clear)
 {
     int v = 0;

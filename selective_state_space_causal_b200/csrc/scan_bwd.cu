@@ -29,6 +29,9 @@
 // state) and CTA. dA, dDskip and ddt_bias (summed over sequences) take one
 // atomic per CTA and channel. The atomics make the last bits of those sums
 // depend on the order in which CTAs finish; everything else is deterministic.
+#include <atomic>
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace ssm {
@@ -49,9 +52,11 @@ struct BwdParams {
     const int32_t *cu;
     void *du, *ddt, *dz;
     float *dB, *dC, *dA, *dDskip, *ddt_bias, *dh0;
-    float *ckpt;  // workspace: (tok / kTS + S + 1, D, 16)
+    float *ckpt;  // workspace: one state per chunk start of each sequence and channel
+    const int32_t *order;  // longest-first sequence order, or NULL
     int64_t S, tok, D, L;
     int softplus;
+    int vec_atomics;  // dB and dC are 16-byte aligned: sums go out as float4 atomics
 };
 
 // Shared memory of one CTA.
@@ -93,19 +98,20 @@ __device__ __forceinline__ void issue_chunk(const BwdParams &p, RawChunk<T> &r, 
                                             int64_t cbase, int nch, bool full)
 {
     constexpr int V = 16 / sizeof(T), VR = kCh / V, VB = kN / V;
-    const T *src_act[4] = {static_cast<const T *>(p.dt), static_cast<const T *>(p.u),
-                           static_cast<const T *>(p.z), static_cast<const T *>(p.dy)};
+    const T *DT = static_cast<const T *>(p.dt), *U = static_cast<const T *>(p.u);
+    const T *Z = static_cast<const T *>(p.z), *DY = static_cast<const T *>(p.dy);
     const int narr = full ? 4 : 2, nvr = nch / V;
     for (int e = threadIdx.x; e < narr * kTS * VR; e += kThreads) {
         const int arr = e / (kTS * VR), rem = e % (kTS * VR), tl = rem / VR, v = rem % VR;
-        if (tl >= nt || v >= nvr || src_act[arr] == nullptr) continue;
-        cp16(&r.act[arr][tl][v * V], src_act[arr] + (t0 + tl) * p.D + cbase + v * V);
+        const T *src = arr == 0 ? DT : arr == 1 ? U : arr == 2 ? Z : DY;  // selects: no local array
+        if (tl >= nt || v >= nvr || src == nullptr) continue;
+        cp16(&r.act[arr][tl][v * V], src + (t0 + tl) * p.D + cbase + v * V);
     }
-    const T *src_bc[2] = {static_cast<const T *>(p.B), static_cast<const T *>(p.C)};
     for (int e = threadIdx.x; e < (full ? 2 : 1) * kTS * VB; e += kThreads) {
         const int arr = e / (kTS * VB), rem = e % (kTS * VB), tl = rem / VB, v = rem % VB;
         if (tl >= nt) continue;
-        cp16(&r.bc[arr][tl][v * V], src_bc[arr] + (t0 + tl) * kN + v * V);
+        const T *src = static_cast<const T *>(arr ? p.C : p.B);
+        cp16(&r.bc[arr][tl][v * V], src + (t0 + tl) * kN + v * V);
     }
 }
 
@@ -228,7 +234,7 @@ scan_bwd_kernel(const BwdParams p)
     const int64_t cbase = (int64_t)blockIdx.x * kCh, c = cbase + cl;
     const int nch = (int)min((int64_t)kCh, p.D - cbase);
     const bool cvalid = c < p.D;
-    const int64_t s = blockIdx.y;
+    const int64_t s = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
     int64_t start, end;
     if (p.cu) {
         start = clamp_off(p.cu[s], p.tok);
@@ -476,6 +482,482 @@ scan_bwd_kernel(const BwdParams p)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Thread-per-channel variant. One thread owns one (sequence, channel) with
+// all 16 states in registers (eight packed fp32x2 pairs): sums over states
+// take no shuffles, and the CTA's 128 channels share each token's B and C. Chunks of kWTS tokens, one
+// checkpoint each. Phase A is as above; phase B, per chunk, last first:
+//   1. recompute the chunk's states from its checkpoint into shared memory,
+//      with dz on the way (C . h_t is at hand), keeping each token's delta,
+//      delta u, u, dy silu(z) and softplus' in registers;
+//   2. dC_t = sum_c dy silu(z) h_t over the CTA's channels, from shared
+//      memory (below);
+//   3. walk the chunk backwards with G in registers; the states of token t
+//      give way to its dB terms G_t delta_t u_t in shared memory;
+//   4. dB_t, summed over channels as in 2.
+// A channel sum (2, 4) gives each warp 8 (token, 4-state) items: lane
+// (k, i) = (lane / 8, lane % 8) of warp w adds item 8 w + i over channels
+// 32 k .. 32 k + 31, two shuffles join the four quarters, and one 16-byte
+// atomic per item and CTA adds the result. Rows of the state buffer are padded by 16 bytes, so the 8
+// lanes of a 16-byte load phase, on 8 consecutive rows, hit 8 different
+// banks; rows of dy silu(z) are padded by 4 bytes per group and 32 bytes per
+// token, so all 32 lanes' 4-byte loads do too.
+// ---------------------------------------------------------------------------
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr int kWCh = 128;              // channels (= threads) per CTA
+constexpr int kWTS = 8;                // tokens per chunk and per checkpoint
+constexpr int kWRow = kWCh + 1;        // float4 per padded state row
+constexpr int kWQRow = 136;            // floats per padded dy silu(z) row
+
+constexpr int kWGCh = 32;              // channels per lane quarter of a channel sum
+static_assert(3 * (kWGCh + 1) + kWGCh <= kWQRow, "dy silu(z) row");
+
+template <typename T>
+struct WRaw {
+    T act[4][kWTS][kWCh];  // dt, u, z, dy
+    T bc[2][kWTS][kN];     // B, C
+};
+
+struct WSmem {
+    // row (slot * 4 + q): states 4q .. 4q + 3 of every channel; slot 0 holds
+    // the checkpoint, slot tl + 1 the states after token tl, later its dB terms
+    float4 hist[(kWTS + 1) * 4][kWRow];
+    float dq[kWTS][kWQRow];
+    float B[kWTS][kN];
+    float C[kWTS][kN];
+};
+
+__device__ __forceinline__ int wq_col(int c) { return (c / kWGCh) * (kWGCh + 1) + c % kWGCh; }
+
+template <typename T>
+__device__ __forceinline__ void w_issue(const BwdParams &p, WRaw<T> &r, int64_t t0, int nt,
+                                        int64_t cbase, int nch, bool full)
+{
+    constexpr int V = 16 / sizeof(T), VR = kWCh / V, VB = kN / V;
+    const T *DT = static_cast<const T *>(p.dt), *U = static_cast<const T *>(p.u);
+    const T *Z = static_cast<const T *>(p.z), *DY = static_cast<const T *>(p.dy);
+    const int narr = full ? 4 : 2, nvr = nch / V;
+    for (int e = threadIdx.x; e < narr * kWTS * VR; e += kWCh) {
+        const int arr = e / (kWTS * VR), rem = e % (kWTS * VR), tl = rem / VR, v = rem % VR;
+        const T *src = arr == 0 ? DT : arr == 1 ? U : arr == 2 ? Z : DY;  // selects: no local array
+        if (tl >= nt || v >= nvr || src == nullptr) continue;
+        cp16(&r.act[arr][tl][v * V], src + (t0 + tl) * p.D + cbase + v * V);
+    }
+    for (int e = threadIdx.x; e < (full ? 2 : 1) * kWTS * VB; e += kWCh) {
+        const int arr = e / (kWTS * VB), rem = e % (kWTS * VB), tl = rem / VB, v = rem % VB;
+        if (tl >= nt) continue;
+        const T *src = static_cast<const T *>(arr ? p.C : p.B);
+        cp16(&r.bc[arr][tl][v * V], src + (t0 + tl) * kN + v * V);
+    }
+}
+
+// Sum over the CTA's channels of the chunk's state rows (weighted by dy
+// silu(z) when `weighted`), added into dst (tok, 16) at tokens t0 .. t0 + nt.
+__device__ __forceinline__ void w_channel_sum(const BwdParams &p, const WSmem &sm, bool weighted,
+                                              float *dst, int64_t t0, int nt)
+{
+    const int lane = threadIdx.x & 31, k = lane >> 3;
+    const int item = (threadIdx.x >> 5) * 8 + (lane & 7), tl = item >> 2, q = item & 3;
+    f32x2 s01 = 0ull, s23 = 0ull;
+    if (tl < nt) {
+        const float4 *row = &sm.hist[(tl + 1) * 4 + q][k * kWGCh];
+        if (weighted) {
+            const float *wt = &sm.dq[tl][k * (kWGCh + 1)];
+#pragma unroll 8
+            for (int j = 0; j < kWGCh; ++j) {
+                const float4 v = row[j];
+                const f32x2 c = pk2(wt[j], wt[j]);
+                s01 = fma2(c, pk2(v.x, v.y), s01);
+                s23 = fma2(c, pk2(v.z, v.w), s23);
+            }
+        } else {
+#pragma unroll 8
+            for (int j = 0; j < kWGCh; ++j) {
+                const float4 v = row[j];
+                s01 = add2(s01, pk2(v.x, v.y));
+                s23 = add2(s23, pk2(v.z, v.w));
+            }
+        }
+    }
+    float4 acc;
+    upk2(s01, acc.x, acc.y);
+    upk2(s23, acc.z, acc.w);
+#pragma unroll
+    for (int m = 8; m <= 16; m <<= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, m);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, m);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, m);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, m);
+    }
+    if (k == 0 && tl < nt) {
+        float *o = dst + (t0 + tl) * kN + 4 * q;
+        if (p.vec_atomics) {
+            atomicAdd(reinterpret_cast<float4 *>(o), acc);
+        } else {
+            atomicAdd(o, acc.x);
+            atomicAdd(o + 1, acc.y);
+            atomicAdd(o + 2, acc.z);
+            atomicAdd(o + 3, acc.w);
+        }
+    }
+}
+
+constexpr size_t w_smem_bytes(size_t raw_bytes) { return sizeof(WSmem) + 2 * raw_bytes; }
+
+template <typename T, bool ASYNC>
+__global__ void __launch_bounds__(kWCh, 2)
+scan_bwd_wide_kernel(const BwdParams p)
+{
+    constexpr int NP = 8, NQ = 4;  // packed state pairs, state quads
+    extern __shared__ __align__(128) unsigned char w_smem[];
+    WSmem &sm = *reinterpret_cast<WSmem *>(w_smem);
+    WRaw<T> *raw = reinterpret_cast<WRaw<T> *>(w_smem + sizeof(WSmem));
+    const int tid = threadIdx.x, cl = tid;
+    const int64_t cbase = (int64_t)blockIdx.x * kWCh, c = cbase + cl;
+    const int nch = (int)min((int64_t)kWCh, p.D - cbase);
+    const bool cvalid = c < p.D;
+    const int64_t s = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    int64_t start, end;
+    if (p.cu) {
+        start = clamp_off(p.cu[s], p.tok);
+        end = max(clamp_off(p.cu[s + 1], p.tok), start);
+    } else {
+        start = s * p.L;
+        end = start + p.L;
+    }
+    const int64_t len = end - start;
+    const int64_t nchunks = (len + kWTS - 1) / kWTS;
+    // checkpoint slots of this sequence: floor(start / kWTS) + s + k never collide
+    float *ck = p.ckpt + ((start / kWTS + s) * p.D + c) * kN;
+    const int64_t ck_stride = p.D * kN;
+
+    f32x2 A2[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int n = 2 * j;
+        const float a0 = cvalid ? __ldg(p.A + c * kN + n) : 0.f;
+        const float a1 = cvalid ? __ldg(p.A + c * kN + n + 1) : 0.f;
+        A2[j] = pk2(a0 * kLog2e, a1 * kLog2e);
+    }
+    const float dsk = (cvalid && p.Dskip) ? __ldg(p.Dskip + c) : 0.f;
+    const float dtb = (cvalid && p.dt_bias) ? __ldg(p.dt_bias + c) : 0.f;
+    const T *DT = static_cast<const T *>(p.dt), *U = static_cast<const T *>(p.u);
+    const T *Z = static_cast<const T *>(p.z), *DY = static_cast<const T *>(p.dy);
+    const T *Bp = static_cast<const T *>(p.B), *Cp = static_cast<const T *>(p.C);
+    const bool has_z = Z != nullptr;
+
+    // the chunk's B (and C) rows in fp32: one (token, state) per thread
+    auto fill_bc = [&](const WRaw<T> &r, int64_t t0, int nt, bool with_c) {
+        if (tid >= kWTS * kN) return;
+        const int tl = tid >> 4, n = tid & 15;
+        float b = 0.f, cc = 0.f;
+        if (tl < nt) {
+            if constexpr (ASYNC) {
+                b = to_f32(r.bc[0][tl][n]);
+                if (with_c) cc = to_f32(r.bc[1][tl][n]);
+            } else {
+                b = ld1(Bp + (t0 + tl) * kN + n);
+                if (with_c) cc = ld1(Cp + (t0 + tl) * kN + n);
+            }
+        }
+        sm.B[tl][n] = b;
+        if (with_c) sm.C[tl][n] = cc;
+    };
+    // this channel's value of activation `arr` at chunk token tl (channel valid)
+    auto act = [&](const WRaw<T> &r, int arr, int tl, int64_t t) -> float {
+        if constexpr (ASYNC) {
+            return to_f32(r.act[arr][tl][cl]);
+        } else {
+            const T *src = arr == 0 ? DT : arr == 1 ? U : arr == 2 ? Z : DY;
+            return ld1(src + t * p.D + c);
+        }
+    };
+    // this thread's state rows: one base address, constant offsets after
+    const float *Bq = &sm.B[0][0], *Cq = &sm.C[0][0];
+    float4 *Hq = &sm.hist[0][cl];
+    auto bquad = [&](int tl, int qq) { return *reinterpret_cast<const float4 *>(Bq + tl * kN + 4 * qq); };
+    auto cquad = [&](int tl, int qq) { return *reinterpret_cast<const float4 *>(Cq + tl * kN + 4 * qq); };
+    auto hist = [&](int slot, int qq) -> float4 & { return Hq[(slot * 4 + qq) * kWRow]; };
+
+    // ---- phase A: forward, checkpoint at every chunk start ----------------
+    f32x2 h[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int64_t o = (s * p.D + c) * kN + 2 * j;
+        h[j] = (cvalid && p.h0) ? pk2(p.h0[o], p.h0[o + 1]) : 0ull;
+    }
+    if (ASYNC && nchunks > 0) {
+        w_issue<T>(p, raw[0], start, (int)min((int64_t)kWTS, len), cbase, nch, false);
+        cp_commit();
+    }
+    for (int64_t k = 0; k < nchunks; ++k) {
+        const int64_t t0 = start + k * kWTS;
+        const int nt = (int)min((int64_t)kWTS, end - t0);
+        if (cvalid) {
+            float4 *dst = reinterpret_cast<float4 *>(ck + k * ck_stride);
+#pragma unroll
+            for (int qq = 0; qq < NQ; ++qq) {
+                float4 v;
+                upk2(h[2 * qq], v.x, v.y);
+                upk2(h[2 * qq + 1], v.z, v.w);
+                dst[qq] = v;
+            }
+        }
+        if constexpr (ASYNC) cp_wait<0>();
+        __syncthreads();  // chunk k has landed; chunk k - 1 is no longer read
+        if (ASYNC && k + 1 < nchunks) {
+            const int64_t t1 = t0 + kWTS;
+            w_issue<T>(p, raw[(k + 1) & 1], t1, (int)min((int64_t)kWTS, end - t1),
+                                   cbase, nch, false);
+            cp_commit();
+        }
+        fill_bc(raw[k & 1], t0, nt, false);
+        __syncthreads();
+        // full chunks take a copy of the token loop without per-token guards,
+        // so the compiler can overlap neighbouring tokens' work
+        auto walk = [&](auto full) {
+            constexpr bool kFull = decltype(full)::value;
+#pragma unroll
+            for (int tl = 0; tl < kWTS; ++tl) {
+                if (kFull || tl < nt) {
+                    const float v = act(raw[k & 1], 0, tl, t0 + tl) + dtb;
+                    const float d = p.softplus ? softplus_fast(v) : v;
+                    const float x = d * act(raw[k & 1], 1, tl, t0 + tl);
+                    const f32x2 dd = pk2(d, d), xx = pk2(x, x);
+#pragma unroll
+                    for (int qq = 0; qq < NQ; ++qq) {
+                        const float4 b4 = bquad(tl, qq);
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 2 * qq + e;
+                            float e0, e1;
+                            upk2(mul2(dd, A2[j]), e0, e1);
+                            const f32x2 a = pk2(ex2_approx(e0), ex2_approx(e1));
+                            const f32x2 b2 = e ? pk2(b4.z, b4.w) : pk2(b4.x, b4.y);
+                            h[j] = fma2(a, h[j], mul2(xx, b2));
+                        }
+                    }
+                }
+            }
+        };
+        if (cvalid) {
+            if (nt == kWTS) walk(std::true_type{});
+            else walk(std::false_type{});
+        }
+    }
+
+    // ---- phase B: reverse -----------------------------------------------------
+    f32x2 G[NP], dAacc[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int64_t o = (s * p.D + c) * kN + 2 * j;
+        G[j] = (cvalid && p.dh_final) ? pk2(p.dh_final[o], p.dh_final[o + 1]) : 0ull;
+        dAacc[j] = 0ull;
+    }
+    float dDsk = 0.f, ddtb = 0.f;
+    T *DU = static_cast<T *>(p.du), *DDT = static_cast<T *>(p.ddt), *DZ = static_cast<T *>(p.dz);
+    if constexpr (ASYNC) cp_wait<0>();
+    __syncthreads();  // phase A's last chunk is no longer read
+    if (ASYNC && nchunks > 0) {
+        const int64_t tl0 = start + (nchunks - 1) * kWTS;
+        w_issue<T>(p, raw[0], tl0, (int)(end - tl0), cbase, nch, true);
+        cp_commit();
+    }
+    for (int64_t k = nchunks - 1; k >= 0; --k) {
+        const int64_t t0 = start + k * kWTS;
+        const int nt = (int)min((int64_t)kWTS, end - t0);
+        const int buf = (int)((nchunks - 1 - k) & 1);
+        f32x2 hc[NP];
+        if (cvalid) {
+            const float4 *src = reinterpret_cast<const float4 *>(ck + k * ck_stride);
+#pragma unroll
+            for (int qq = 0; qq < NQ; ++qq) {
+                const float4 v = src[qq];
+                hc[2 * qq] = pk2(v.x, v.y);
+                hc[2 * qq + 1] = pk2(v.z, v.w);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < NP; ++j) hc[j] = 0ull;
+        }
+        if constexpr (ASYNC) cp_wait<0>();
+        __syncthreads();  // chunk k has landed; the previous chunk's dB sum is done
+        if (ASYNC && k > 0) {
+            w_issue<T>(p, raw[buf ^ 1], t0 - kWTS, kWTS, cbase, nch, true);
+            cp_commit();
+        }
+        fill_bc(raw[buf], t0, nt, true);
+#pragma unroll
+        for (int qq = 0; qq < NQ; ++qq) {
+            float4 v;
+            upk2(hc[2 * qq], v.x, v.y);
+            upk2(hc[2 * qq + 1], v.z, v.w);
+            hist(0, qq) = v;
+        }
+        __syncthreads();  // B and C rows staged
+
+        // 1. recompute the chunk's states; dz
+        float dr[kWTS], xr[kWTS], ur[kWTS], qr[kWTS], sr[kWTS];
+        auto recompute = [&](auto full) {
+            constexpr bool kFull = decltype(full)::value;
+#pragma unroll
+            for (int tl = 0; tl < kWTS; ++tl) {
+                // staged values are read for every lane (shared memory holds
+                // some value for each) and masked afterwards, so the token
+                // loop has no divergent branch; direct loads stay guarded
+                const bool live = (kFull || tl < nt) && cvalid;
+                float vdt = 0.f, vu = 0.f, vdy = 0.f, vz = 0.f;
+                if (ASYNC || live) {
+                    vdt = act(raw[buf], 0, tl, t0 + tl);
+                    vu = act(raw[buf], 1, tl, t0 + tl);
+                    vdy = act(raw[buf], 3, tl, t0 + tl);
+                    if (has_z) vz = act(raw[buf], 2, tl, t0 + tl);
+                }
+                const float v = vdt + dtb;
+                float d = p.softplus ? softplus_fast(v) : v;
+                float sp = p.softplus ? sigmoid_f(v) : 1.f;
+                float g = 1.f, dg = 0.f;
+                if (has_z) {
+                    const float sg = sigmoid_f(vz);
+                    g = vz * sg;
+                    dg = sg * (1.f + vz * (1.f - sg));
+                }
+                d = live ? d : 0.f;
+                sp = live ? sp : 0.f;
+                const float u = live ? vu : 0.f;
+                const float x = d * u;
+                const float dq = live ? vdy * g : 0.f;
+                const float dzf = live ? vdy * dg : 0.f;
+                dr[tl] = d;
+                xr[tl] = x;
+                ur[tl] = u;
+                qr[tl] = dq;
+                sr[tl] = sp;
+                sm.dq[tl][wq_col(cl)] = dq;
+                if (kFull || tl < nt) {
+                    const f32x2 dd = pk2(d, d), xx = pk2(x, x);
+                    f32x2 qp = 0ull, qp1 = 0ull;
+#pragma unroll
+                    for (int qq = 0; qq < NQ; ++qq) {
+                        const float4 b4 = bquad(tl, qq);
+                        const float4 c4 = cquad(tl, qq);
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 2 * qq + e;
+                            float e0, e1;
+                            upk2(mul2(dd, A2[j]), e0, e1);
+                            const f32x2 a = pk2(ex2_approx(e0), ex2_approx(e1));
+                            const f32x2 b2 = e ? pk2(b4.z, b4.w) : pk2(b4.x, b4.y);
+                            const f32x2 c2 = e ? pk2(c4.z, c4.w) : pk2(c4.x, c4.y);
+                            hc[j] = fma2(a, hc[j], mul2(xx, b2));
+                            if (e) qp1 = fma2(c2, hc[j], qp1);
+                            else qp = fma2(c2, hc[j], qp);
+                        }
+                        float4 v;
+                        upk2(hc[2 * qq], v.x, v.y);
+                        upk2(hc[2 * qq + 1], v.z, v.w);
+                        hist(tl + 1, qq) = v;
+                    }
+                    float q0s, q1s;
+                    upk2(add2(qp, qp1), q0s, q1s);
+                    const float qs = q0s + q1s;
+                    if (cvalid && DZ)
+                        DZ[(t0 + tl) * p.D + c] = from_f32<T>(has_z ? dzf * (qs + dsk * u) : 0.f);
+                }
+            }
+        };
+        if (nt == kWTS) recompute(std::true_type{});
+        else recompute(std::false_type{});
+        __syncthreads();  // the chunk's states and dy silu(z) are in shared memory
+
+        // 2. dC over the CTA's channels
+        w_channel_sum(p, sm, true, p.dC, t0, nt);
+        __syncthreads();  // the states are no longer read by other threads
+
+        // 3. reverse walk
+        auto reverse = [&](auto full) {
+            constexpr bool kFull = decltype(full)::value;
+#pragma unroll
+            for (int tl = kWTS - 1; tl >= 0; --tl) {
+                if (kFull || tl < nt) {
+                    const float d = dr[tl], x = xr[tl], dq = qr[tl];
+                    const f32x2 dd = pk2(d, d), xx = pk2(x, x), dqq = pk2(dq, dq);
+                    f32x2 dup = 0ull, ddp = 0ull, dup1 = 0ull, ddp1 = 0ull;
+#pragma unroll
+                    for (int qq = 0; qq < NQ; ++qq) {
+                        const float4 b4 = bquad(tl, qq);
+                        const float4 c4 = cquad(tl, qq);
+                        const float4 hp = hist(tl, qq);  // h_{t-1}
+                        float4 gx;
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 2 * qq + e;
+                            float e0, e1;
+                            upk2(mul2(dd, A2[j]), e0, e1);
+                            const f32x2 a = pk2(ex2_approx(e0), ex2_approx(e1));
+                            const f32x2 b2 = e ? pk2(b4.z, b4.w) : pk2(b4.x, b4.y);
+                            const f32x2 c2 = e ? pk2(c4.z, c4.w) : pk2(c4.x, c4.y);
+                            const f32x2 h2 = e ? pk2(hp.z, hp.w) : pk2(hp.x, hp.y);
+                            G[j] = fma2(dqq, c2, G[j]);         // G_t = dq C + a_{t+1} G_{t+1}
+                            const f32x2 g2 = mul2(G[j], xx);    // dB terms
+                            if (e) {
+                                dup1 = fma2(G[j], b2, dup1);    // G . B
+                                upk2(g2, gx.z, gx.w);
+                            } else {
+                                dup = fma2(G[j], b2, dup);
+                                upk2(g2, gx.x, gx.y);
+                            }
+                            G[j] = mul2(a, G[j]);               // a G_t: dL/dh_{t-1} so far
+                            const f32x2 gah = mul2(G[j], h2);   // G a h_{t-1}
+                            if (e) ddp1 = fma2(gah, A2[j], ddp1);  // G A a h_{t-1} / ln 2
+                            else ddp = fma2(gah, A2[j], ddp);
+                            dAacc[j] = fma2(gah, dd, dAacc[j]);
+                        }
+                        hist(tl + 1, qq) = gx;
+                    }
+                    float u0, u1, x0, x1;
+                    upk2(add2(dup, dup1), u0, u1);
+                    upk2(add2(ddp, ddp1), x0, x1);
+                    const float us = u0 + u1;
+                    const float xs = x0 + x1;
+                    // the per-token values are zero for a channel beyond D
+                    const float ddt = (ur[tl] * us + kLn2 * xs) * sr[tl];
+                    dDsk += dq * ur[tl];
+                    ddtb += ddt;
+                    if (cvalid) {
+                        const int64_t o = (t0 + tl) * p.D + c;
+                        DU[o] = from_f32<T>(dq * dsk + d * us);
+                        DDT[o] = from_f32<T>(ddt);
+                    }
+                }
+            }
+        };
+        if (nt == kWTS) reverse(std::true_type{});
+        else reverse(std::false_type{});
+        __syncthreads();  // the chunk's dB terms are in shared memory
+
+        // 4. dB over the CTA's channels
+        w_channel_sum(p, sm, false, p.dB, t0, nt);
+    }
+    if (cvalid) {
+#pragma unroll
+        for (int j = 0; j < NP; ++j) {
+            const int n = 2 * j;
+            float g0, g1, a0, a1;
+            upk2(G[j], g0, g1);
+            upk2(dAacc[j], a0, a1);
+            if (p.dh0) {
+                p.dh0[(s * p.D + c) * kN + n] = g0;
+                p.dh0[(s * p.D + c) * kN + n + 1] = g1;
+            }
+            atomicAdd(p.dA + c * kN + n, a0);
+            atomicAdd(p.dA + c * kN + n + 1, a1);
+        }
+        if (p.dDskip) atomicAdd(p.dDskip + c, dDsk);
+        if (p.ddt_bias) atomicAdd(p.ddt_bias + c, ddtb);
+    }
+}
+
 __global__ void zero_kernel(float *a, int64_t na, float *b, int64_t nb)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -500,9 +982,53 @@ struct ScanBwdArgs {
     bool bf16;
 };
 
-size_t scan_bwd_ckpt_floats(int64_t tok, int64_t D, int64_t S)
+cudaError_t launch_seq_order(const int32_t *cu, int64_t S, int64_t tok, int32_t *order,
+                             cudaStream_t stream);
+int device_sm_count();
+
+// Checkpoint floats of the thread-per-channel kernel (one state per kWTS
+// tokens); the lane-split kernel's one per kTS tokens fits in the same area.
+static size_t ckpt_floats(int64_t tok, int64_t D, int64_t S)
 {
-    return (size_t)(tok / kTS + S + 1) * (size_t)D * kN;
+    return (size_t)(tok / kWTS + S + 1) * (size_t)D * kN;
+}
+
+static size_t order_offset(int64_t tok, int64_t D, int64_t S)
+{
+    return (ckpt_floats(tok, D, S) * sizeof(float) + 255) / 256 * 256;
+}
+
+size_t scan_bwd_workspace_bytes(int64_t tok, int64_t D, int64_t S)
+{
+    return order_offset(tok, D, S) + (size_t)((S * 4 + 255) / 256) * 256;
+}
+
+static std::atomic<int> g_bwd_forced{0};
+
+void set_scan_bwd_variant(int v) { g_bwd_forced.store(v, std::memory_order_relaxed); }
+
+// 1: four lanes per channel (kTS-token chunks); 2: one thread per channel.
+// The thread-per-channel kernel executes about half the instructions per
+// (token, channel) (14 against 28 warp instructions, measured) but has a
+// quarter of the threads; it is chosen once its CTAs fill every SM twice
+// (two CTAs are resident per SM).
+int scan_bwd_variant_for(int64_t S, int64_t D)
+{
+    const int f = g_bwd_forced.load(std::memory_order_relaxed);
+    if (f) return f;
+    const int64_t ctas = S * ((D + kWCh - 1) / kWCh);
+    return ctas >= 2 * (int64_t)device_sm_count() ? 2 : 1;
+}
+
+template <typename T, bool ASYNC>
+static cudaError_t run_wide(const BwdParams &p, dim3 grid, cudaStream_t stream)
+{
+    const size_t smem = w_smem_bytes(sizeof(WRaw<T>));
+    cudaError_t e = cudaFuncSetAttribute(scan_bwd_wide_kernel<T, ASYNC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    scan_bwd_wide_kernel<T, ASYNC><<<grid, kWCh, smem, stream>>>(p);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *launches)
@@ -533,22 +1059,44 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *laun
     p.A = a.A; p.Dskip = a.Dskip; p.dt_bias = a.dt_bias; p.h0 = a.h0; p.dh_final = a.dh_final;
     p.cu = a.cu; p.du = a.du; p.ddt = a.ddt; p.dz = a.dz;
     p.dB = a.dB; p.dC = a.dC; p.dA = a.dA; p.dDskip = a.dDskip; p.ddt_bias = a.ddt_bias;
-    p.dh0 = a.dh0; p.ckpt = a.ckpt;
+    p.dh0 = a.dh0; p.ckpt = a.ckpt; p.order = nullptr;
     p.S = a.S; p.tok = a.tok; p.D = a.D; p.L = a.cu ? 0 : a.tok / a.S; p.softplus = a.softplus;
-    const dim3 grid((unsigned)((a.D + kCh - 1) / kCh), (unsigned)a.S);
+    p.vec_atomics = ((uintptr_t)a.dB % 16 == 0) && ((uintptr_t)a.dC % 16 == 0);
+    if (a.cu && a.S > 1) {
+        // longest sequences first, so the longest chains do not start last
+        int32_t *order = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(a.ckpt) +
+                                                     order_offset(a.tok, a.D, a.S));
+        cudaError_t e = launch_seq_order(a.cu, a.S, a.tok, order, stream);
+        ++*launches;
+        if (e != cudaSuccess) return e;
+        p.order = order;
+    }
     const size_t es = a.bf16 ? 2 : 4;
     const uintptr_t mis = (uintptr_t)a.u | (uintptr_t)a.dt | (uintptr_t)a.z | (uintptr_t)a.dy |
                           (uintptr_t)a.B | (uintptr_t)a.C;
     const bool async_ok = (mis % 16 == 0) && ((size_t)a.D * es) % 16 == 0;
-    if (a.bf16) {
-        if (async_ok) scan_bwd_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, stream>>>(p);
-        else scan_bwd_kernel<__nv_bfloat16, false><<<grid, kThreads, 0, stream>>>(p);
+    cudaError_t e;
+    if (scan_bwd_variant_for(a.S, a.D) == 2) {
+        const dim3 grid((unsigned)((a.D + kWCh - 1) / kWCh), (unsigned)a.S);
+        if (a.bf16)
+            e = async_ok ? run_wide<__nv_bfloat16, true>(p, grid, stream)
+                         : run_wide<__nv_bfloat16, false>(p, grid, stream);
+        else
+            e = async_ok ? run_wide<float, true>(p, grid, stream)
+                         : run_wide<float, false>(p, grid, stream);
     } else {
-        if (async_ok) scan_bwd_kernel<float, true><<<grid, kThreads, 0, stream>>>(p);
-        else scan_bwd_kernel<float, false><<<grid, kThreads, 0, stream>>>(p);
+        const dim3 grid((unsigned)((a.D + kCh - 1) / kCh), (unsigned)a.S);
+        if (a.bf16) {
+            if (async_ok) scan_bwd_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, stream>>>(p);
+            else scan_bwd_kernel<__nv_bfloat16, false><<<grid, kThreads, 0, stream>>>(p);
+        } else {
+            if (async_ok) scan_bwd_kernel<float, true><<<grid, kThreads, 0, stream>>>(p);
+            else scan_bwd_kernel<float, false><<<grid, kThreads, 0, stream>>>(p);
+        }
+        e = cudaGetLastError();
     }
     ++*launches;
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace ssm

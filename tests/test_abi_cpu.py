@@ -138,6 +138,28 @@ def test_tuning_knob():
     ssm.ssm_set_scan_variant(0, 0)
 
 
+def test_bwd_variant_knob_and_choice():
+    """The backward takes one thread per channel once S * ceil(D / 128) CTAs
+    fill every SM twice (148 SMs when no device is visible), else four lanes
+    per channel; a forced kernel is reported as forced."""
+    ssm.ssm_set_scan_bwd_variant(0)
+    assert ssm.ssm_scan_bwd_variant_for(43, 5120) == 2    # packed 65536 x 5120
+    assert ssm.ssm_scan_bwd_variant_for(32, 5120) == 2    # 32 x 2048 x 5120
+    assert ssm.ssm_scan_bwd_variant_for(8, 1536) == 1     # 8 x 2048 x 1536 layer
+    assert ssm.ssm_scan_bwd_variant_for(1, 8192) == 1
+    for v in (1, 2):
+        ssm.ssm_set_scan_bwd_variant(v)
+        assert ssm.ssm_scan_bwd_variant_for(1, 16) == v
+    ssm.ssm_set_scan_bwd_variant(0)
+    for v in (-1, 3):
+        with pytest.raises(ssm.SsmError) as ei:
+            ssm.ssm_set_scan_bwd_variant(v)
+        assert ei.value.code == -1
+    for S, D in ((0, 16), (4, 0)):
+        with pytest.raises(ssm.SsmError):
+            ssm.ssm_scan_bwd_variant_for(S, D)
+
+
 def test_variant_choice():
     """The automatic choice follows (sequence, channel, state) recurrences per
     SM (148 SMs when no device is visible): 8 states per lane with TMA staging
@@ -236,7 +258,8 @@ def test_scan_bwd_rejects(kw, code):
 
 def test_scan_bwd_workspace_size():
     n = ssm.ssm_scan_bwd_workspace_size(16384, 1536, 16, 8)
-    assert n % 256 == 0 and n >= (16384 // 16 + 8) * 1536 * 64
+    # a 64-byte state per 8 tokens, sequence and channel, plus the sequence order
+    assert n % 256 == 0 and n >= (16384 // 8 + 8) * 1536 * 64 + 8 * 4
     assert ssm.ssm_scan_bwd_workspace_size(100, 64, 8, 1) == 0
 
 

@@ -19,6 +19,15 @@ from gpu_helpers import TOL_BF16, TOL_F32, act_dtype, assert_close, cu_tensor, d
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=[1, 2], ids=["lanes4", "thread"])
+def variant(request):
+    """Every test runs on both kernels: 4 lanes per channel, and one thread per
+    channel with all 16 states."""
+    ssm.ssm_set_scan_bwd_variant(request.param)
+    yield request.param
+    ssm.ssm_set_scan_bwd_variant(0)
+
+
 def _run_bwd(u, dt, A, B, C, dy, Dskip, z, dt_bias, h0, dh_final, cu, S, softplus=True):
     tok, D = u.shape
     N = A.shape[1]
@@ -82,22 +91,22 @@ def _check(orc, bf16, lens, D, gate=True, softplus=True, dense_rows=None, seed=0
 
 
 @pytest.mark.parametrize("bf16", [False, True])
-def test_bwd_packed_matches_oracle(orc, bf16):
-    # chunk edges at 16 tokens: lengths below, at, across and far beyond them;
-    # an empty and a one-token sequence; a partial 8-channel block
+def test_bwd_packed_matches_oracle(orc, bf16, variant):
+    # chunk edges at 8 and 16 tokens: lengths below, at, across and far beyond
+    # them; an empty and a one-token sequence; a partial channel block
     _check(orc, bf16, [37, 0, 1, 130, 16, 17, 5], 40)
 
 
 @pytest.mark.parametrize("bf16", [False, True])
-def test_bwd_no_gate_no_softplus(orc, bf16):
+def test_bwd_no_gate_no_softplus(orc, bf16, variant):
     _check(orc, bf16, [20, 3, 48], 64, gate=False, softplus=False, seed=3)
 
 
-def test_bwd_dense_rows(orc):
+def test_bwd_dense_rows(orc, variant):
     _check(orc, True, None, 96, dense_rows=(3, 80), seed=5)
 
 
-def test_bwd_deterministic_outputs():
+def test_bwd_deterministic_outputs(variant):
     """Two runs agree bit for bit on the per-token gradients and dh0; the
     atomically summed ones agree to fp32 rounding."""
     lens = [300, 77, 1000]
@@ -116,7 +125,7 @@ def test_bwd_deterministic_outputs():
         assert torch.allclose(x, y, rtol=1e-5, atol=1e-5 * float(y.abs().max())), k
 
 
-def test_bwd_packmamba_workload_sampled(orc):
+def test_bwd_packmamba_workload_sampled(orc, variant):
     """The packed 65536-token, 5120-channel training shape: per-token gradients,
     dA, dDskip, ddt_bias and dh0 of sampled channels against the oracle run on
     those channels alone (channels are independent for these)."""
@@ -148,13 +157,13 @@ def test_bwd_packmamba_workload_sampled(orc):
 
 
 @pytest.mark.parametrize("bf16", [False, True])
-def test_bwd_unaligned_rows_scalar_staging(orc, bf16):
+def test_bwd_unaligned_rows_scalar_staging(orc, bf16, variant):
     """D = 36: bf16 rows are not a multiple of 16 bytes, so the chunk inputs are
     staged with scalar loads (fp32 rows of 144 bytes still take the copies)."""
     _check(orc, bf16, [19, 40, 2], 36, seed=11)
 
 
-def test_bwd_optional_inputs_absent(orc):
+def test_bwd_optional_inputs_absent(orc, variant):
     """No Dskip, dt_bias, h0, dh_final and no dz output: the remaining gradients
     still match the oracle, which takes the same absences as zeros."""
     lens = [33, 9]
@@ -180,5 +189,41 @@ def test_bwd_optional_inputs_absent(orc):
     assert_close(host(g["du"]), r["du"], True, TOL_BF16, "du")
     assert_close(host(g["ddelta"]), r["ddt"], True, TOL_BF16, "ddelta")
     for k in ("dB", "dC", "dA"):
+        assert_close(host(g[k]), r[k], False, TOL_BF16, k)
+    assert ssm.ssm_device_status() == 0
+
+
+def test_bwd_many_channel_blocks_and_odd_sums(orc, variant):
+    """Several 128-channel blocks with a partial last one (D = 300), sequence
+    lengths around the 8- and 16-token chunks and an fp32 dB / dC pair that is
+    only 4-byte aligned (scalar atomics)."""
+    lens = [8, 7, 9, 64, 65, 3, 200]
+    cu_d, cu_h = cu_tensor(lens)
+    tok, S, D = int(cu_h[-1]), len(lens), 300
+    prm = synth.make_params(21, D, random_bias=True, random_A=True, random_D=True)
+    act = synth.make_activations(21, tok, D, bf16=True)
+    dy = synth.round_bf16(np.random.default_rng(22).standard_normal((tok, D)).astype(np.float32))
+    BF = torch.bfloat16
+    f32 = dict(device="cuda", dtype=torch.float32)
+    u = dev(act["x"], BF)
+    flat = torch.zeros(2 * tok * 16 + 2, **f32)
+    g = {"du": torch.empty_like(u), "ddelta": torch.empty_like(u), "dz": torch.empty_like(u),
+         "dB": flat[1:1 + tok * 16].view(tok, 16),
+         "dC": flat[2 + tok * 16:2 + 2 * tok * 16].view(tok, 16),
+         "dA": torch.empty((D, 16), **f32), "dDskip": torch.empty((D,), **f32),
+         "ddt_bias": torch.empty((D,), **f32), "dh0": torch.empty((S, D, 16), **f32)}
+    assert g["dB"].data_ptr() % 16 != 0 and g["dC"].data_ptr() % 16 != 0
+    ws = torch.empty(ssm.ssm_scan_bwd_workspace_size(tok, D, 16, S), dtype=torch.uint8,
+                     device="cuda")
+    ssm.ssm_selective_scan_bwd(u, dev(act["dt"], BF), dev(prm.A), dev(act["B"], BF),
+                               dev(act["C"], BF), dev(dy, BF), g, Dskip=dev(prm.Dskip),
+                               z=dev(act["z"], BF), dt_bias=dev(prm.dt_bias), cu_seqlens=cu_d,
+                               workspace=ws)
+    torch.cuda.synchronize()
+    r = orc.selective_scan_bwd(act["x"], act["dt"], prm.A, act["B"], act["C"], dy,
+                               Dskip=prm.Dskip, z=act["z"], dt_bias=prm.dt_bias, cu_seqlens=cu_h)
+    for k, rk in (("du", "du"), ("ddelta", "ddt"), ("dz", "dz")):
+        assert_close(host(g[k]), r[rk], True, TOL_BF16, k)
+    for k in ("dB", "dC", "dA", "dDskip", "ddt_bias", "dh0"):
         assert_close(host(g[k]), r[k], False, TOL_BF16, k)
     assert ssm.ssm_device_status() == 0
