@@ -602,7 +602,14 @@ __device__ __forceinline__ void w_channel_sum(const BwdParams &p, const WSmem &s
     }
 }
 
-constexpr size_t w_smem_bytes(size_t raw_bytes) { return sizeof(WSmem) + 2 * raw_bytes; }
+// Shared memory: the state rows, two raw chunk buffers and, with bf16
+// activations, the next chunk's checkpoint block (with fp32 activations it
+// would not leave room for two CTAs per SM, so those read it directly).
+constexpr size_t kWCkBytes = (size_t)kWCh * kN * sizeof(float);
+constexpr size_t w_smem_bytes(size_t raw_bytes, bool ck_async)
+{
+    return sizeof(WSmem) + 2 * raw_bytes + (ck_async ? kWCkBytes : 0);
+}
 
 template <typename T, bool ASYNC>
 __global__ void __launch_bounds__(kWCh, 2)
@@ -756,11 +763,20 @@ scan_bwd_wide_kernel(const BwdParams p)
     }
     float dDsk = 0.f, ddtb = 0.f;
     T *DU = static_cast<T *>(p.du), *DDT = static_cast<T *>(p.ddt), *DZ = static_cast<T *>(p.dz);
+    // with bf16 activations, chunk k - 1's checkpoint rows of the CTA's
+    // channels (contiguous, 64 bytes per channel) come in while chunk k runs
+    constexpr bool kCkAsync = ASYNC && sizeof(T) == 2;
+    float4 *ckb = reinterpret_cast<float4 *>(w_smem + sizeof(WSmem) + 2 * sizeof(WRaw<T>));
+    auto issue_ck = [&](int64_t kk) {
+        const float *src = p.ckpt + ((start / kWTS + s + kk) * p.D + cbase) * kN;
+        for (int e = tid; e < nch * 4; e += kWCh) cp16(&ckb[e], src + 4 * e);
+    };
     if constexpr (ASYNC) cp_wait<0>();
-    __syncthreads();  // phase A's last chunk is no longer read
+    __syncthreads();  // phase A's last chunk is no longer read; its checkpoints are visible
     if (ASYNC && nchunks > 0) {
         const int64_t tl0 = start + (nchunks - 1) * kWTS;
         w_issue<T>(p, raw[0], tl0, (int)(end - tl0), cbase, nch, true);
+        if constexpr (kCkAsync) issue_ck(nchunks - 1);
         cp_commit();
     }
     for (int64_t k = nchunks - 1; k >= 0; --k) {
@@ -768,7 +784,7 @@ scan_bwd_wide_kernel(const BwdParams p)
         const int nt = (int)min((int64_t)kWTS, end - t0);
         const int buf = (int)((nchunks - 1 - k) & 1);
         f32x2 hc[NP];
-        if (cvalid) {
+        if (!kCkAsync && cvalid) {
             const float4 *src = reinterpret_cast<const float4 *>(ck + k * ck_stride);
 #pragma unroll
             for (int qq = 0; qq < NQ; ++qq) {
@@ -776,9 +792,6 @@ scan_bwd_wide_kernel(const BwdParams p)
                 hc[2 * qq] = pk2(v.x, v.y);
                 hc[2 * qq + 1] = pk2(v.z, v.w);
             }
-        } else {
-#pragma unroll
-            for (int j = 0; j < NP; ++j) hc[j] = 0ull;
         }
         if constexpr (ASYNC) cp_wait<0>();
         __syncthreads();  // chunk k has landed; the previous chunk's dB sum is done
@@ -787,6 +800,18 @@ scan_bwd_wide_kernel(const BwdParams p)
             cp_commit();
         }
         fill_bc(raw[buf], t0, nt, true);
+        if (kCkAsync && cvalid) {
+#pragma unroll
+            for (int qq = 0; qq < NQ; ++qq) {
+                const float4 v = ckb[cl * 4 + qq];
+                hc[2 * qq] = pk2(v.x, v.y);
+                hc[2 * qq + 1] = pk2(v.z, v.w);
+            }
+        }
+        if (!cvalid) {
+#pragma unroll
+            for (int j = 0; j < NP; ++j) hc[j] = 0ull;
+        }
 #pragma unroll
         for (int qq = 0; qq < NQ; ++qq) {
             float4 v;
@@ -794,7 +819,11 @@ scan_bwd_wide_kernel(const BwdParams p)
             upk2(hc[2 * qq + 1], v.z, v.w);
             hist(0, qq) = v;
         }
-        __syncthreads();  // B and C rows staged
+        __syncthreads();  // B and C rows staged; the checkpoint block has been read
+        if (kCkAsync && k > 0) {
+            issue_ck(k - 1);
+            cp_commit();
+        }
 
         // 1. recompute the chunk's states; dz
         float dr[kWTS], xr[kWTS], ur[kWTS], qr[kWTS], sr[kWTS];
@@ -1023,7 +1052,7 @@ int scan_bwd_variant_for(int64_t S, int64_t D)
 template <typename T, bool ASYNC>
 static cudaError_t run_wide(const BwdParams &p, dim3 grid, cudaStream_t stream)
 {
-    const size_t smem = w_smem_bytes(sizeof(WRaw<T>));
+    const size_t smem = w_smem_bytes(sizeof(WRaw<T>), ASYNC && sizeof(T) == 2);
     cudaError_t e = cudaFuncSetAttribute(scan_bwd_wide_kernel<T, ASYNC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
