@@ -91,14 +91,34 @@ __device__ __forceinline__ void prepass_item(float2 *dx_row, float2 *ug_row, boo
                                              const float (&dtb)[VEC], int softplus)
 {
     float vd[VEC], vdx[VEC], vu[VEC], vg[VEC];
+    if constexpr (VEC % 2 == 0) {
+        // in pairs, with the exponentials on the FMA pipe: the special-function
+        // unit is left to the recurrence's decays
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-        float d = fdt[e] + dtb[e];
-        if (softplus) d = softplus_fast(d);
-        vd[e] = live ? d : 0.f;
-        vdx[e] = live ? d * fu[e] : 0.f;
-        vu[e] = live ? fu[e] : 0.f;
-        vg[e] = live ? (has_z ? silu_f(fz[e]) : 1.f) : 0.f;
+        for (int e = 0; e < VEC; e += 2) {
+            float d0 = fdt[e] + dtb[e], d1 = fdt[e + 1] + dtb[e + 1];
+            if (softplus) softplus2(d0, d1, d0, d1);
+            float g0 = 1.f, g1 = 1.f;
+            if (has_z) silu2(fz[e], fz[e + 1], g0, g1);
+            vd[e] = live ? d0 : 0.f;
+            vd[e + 1] = live ? d1 : 0.f;
+            vdx[e] = live ? d0 * fu[e] : 0.f;
+            vdx[e + 1] = live ? d1 * fu[e + 1] : 0.f;
+            vu[e] = live ? fu[e] : 0.f;
+            vu[e + 1] = live ? fu[e + 1] : 0.f;
+            vg[e] = live ? g0 : 0.f;
+            vg[e + 1] = live ? g1 : 0.f;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+            float d = fdt[e] + dtb[e];
+            if (softplus) d = softplus_fast(d);
+            vd[e] = live ? d : 0.f;
+            vdx[e] = live ? d * fu[e] : 0.f;
+            vu[e] = live ? fu[e] : 0.f;
+            vg[e] = live ? (has_z ? silu_f(fz[e]) : 1.f) : 0.f;
+        }
     }
     st_pairs<VEC>(dx_row, vd, vdx);
     st_pairs<VEC>(ug_row, vu, vg);
