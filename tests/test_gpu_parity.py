@@ -147,6 +147,16 @@ def test_scan_workspace_schedule_is_bit_identical(orc):
     assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
 
 
+def test_scan_many_short_sequences_past_the_sort_limit(orc):
+    """5000 packed sequences of 0 to 6 tokens: beyond the 4096 sequences the
+    longest-first sort handles, the schedule falls back to the given order; the
+    results are the same as without the schedule, and both match the oracle."""
+    lens = list(np.random.default_rng(16).integers(0, 7, size=5000))
+    y1, h1 = _scan_case(orc, 16, lens, 64, True, workspace=False)
+    y2, h2 = _scan_case(orc, 16, lens, 64, True, workspace=True)
+    assert np.array_equal(y1, y2) and np.array_equal(h1, h2)
+
+
 def test_scan_device_status_clean():
     """No bounded TMA wait gave up during the tests so far."""
     assert ssm.ssm_device_status(clear=True) == 0

@@ -227,3 +227,10 @@ def test_bwd_many_channel_blocks_and_odd_sums(orc, variant):
     for k in ("dB", "dC", "dA", "dDskip", "ddt_bias", "dh0"):
         assert_close(host(g[k]), r[k], False, TOL_BF16, k)
     assert ssm.ssm_device_status() == 0
+
+
+def test_bwd_many_short_sequences_past_the_sort_limit(orc, variant):
+    """5000 packed sequences of 0 to 6 tokens: more than the longest-first sort
+    handles (the order stays as given), with h0 and dh_final for each."""
+    lens = list(np.random.default_rng(23).integers(0, 7, size=5000))
+    _check(orc, True, lens, 128, seed=23)
