@@ -13,9 +13,14 @@
 //   dA += G_t D_t a_t h_{t-1};   dz_t = dy_t (C_t . h_t + Dskip u_t) silu'(z_t);
 //   dh0 = a_{t0} G_{t0}.
 //
-// One CTA owns one sequence and kCh channels; a channel's 16 states are split
-// over 4 adjacent lanes (4 states each, two packed fp32x2 registers), as in the
-// forward's register-prefetch schedule. Two phases:
+// Two kernels compute the same gradients; the host picks one by problem size
+// (scan_bwd_variant_for). Both recompute the forward states from checkpoints
+// rather than store them, and both run packed sequences longest first.
+//
+// scan_bwd_kernel (lane-split, for small S * D): one CTA owns one sequence and
+// kCh channels; a channel's 16 states are split over 4 adjacent lanes (4 states
+// each, two packed fp32x2 registers), as in the forward's register-prefetch
+// schedule. Two phases:
 //   A (forward): walk the sequence in kTS-token chunks and write the state at
 //     each chunk start to the workspace (4 bytes per token and channel);
 //   B (reverse): for each chunk, last first: a cooperative pre-pass stages the
@@ -29,6 +34,10 @@
 // state) and CTA. dA, dDskip and ddt_bias (summed over sequences) take one
 // atomic per CTA and channel. The atomics make the last bits of those sums
 // depend on the order in which CTAs finish; everything else is deterministic.
+//
+// scan_bwd_wide_kernel (thread-per-channel, for large S * D): one thread per
+// channel with all 16 states, 8-token chunks, dB and dC summed over channels
+// from shared memory; described above the kernel.
 #include <atomic>
 #include <type_traits>
 
