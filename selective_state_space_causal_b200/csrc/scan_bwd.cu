@@ -494,8 +494,9 @@ scan_bwd_kernel(const BwdParams p)
 // ---------------------------------------------------------------------------
 // Thread-per-channel variant. One thread owns one (sequence, channel) with
 // all 16 states in registers (eight packed fp32x2 pairs): sums over states
-// take no shuffles, and the CTA's 128 channels share each token's B and C. Chunks of kWTS tokens, one
-// checkpoint each. Phase A is as above; phase B, per chunk, last first:
+// take no shuffles, and the CTA's 128 channels share each token's B and C.
+// Chunks of kWTS tokens, one checkpoint each. Phase A is as above; phase B,
+// per chunk, last first:
 //   1. recompute the chunk's states from its checkpoint into shared memory,
 //      with dz on the way (C . h_t is at hand), keeping each token's delta,
 //      delta u, u, dy silu(z) and softplus' in registers;
@@ -504,22 +505,27 @@ scan_bwd_kernel(const BwdParams p)
 //   3. walk the chunk backwards with G in registers; the states of token t
 //      give way to its dB terms G_t delta_t u_t in shared memory;
 //   4. dB_t, summed over channels as in 2.
-// A channel sum (2, 4) gives each warp 8 (token, 4-state) items: lane
-// (k, i) = (lane / 8, lane % 8) of warp w adds item 8 w + i over channels
-// 32 k .. 32 k + 31, two shuffles join the four quarters, and one 16-byte
-// atomic per item and CTA adds the result. Rows of the state buffer are padded by 16 bytes, so the 8
-// lanes of a 16-byte load phase, on 8 consecutive rows, hit 8 different
-// banks; rows of dy silu(z) are padded by 4 bytes per group and 32 bytes per
-// token, so all 32 lanes' 4-byte loads do too.
+// A channel sum (2, 4) covers the chunk's 4 kWTS (token, 4-state) items: each
+// warp takes 8 items, and lane (k, i) = (lane / 8, lane % 8) of warp w adds
+// item 8 (w mod kWTS/2) + i over the kWGCh channels of group
+// 4 (w div kWTS/2) + k; two shuffles join a warp's four groups, and one
+// 16-byte atomic per item and warp adds the result. Rows of the state buffer
+// are padded by 16 bytes, so the 8 lanes of a 16-byte load phase, on 8
+// consecutive rows, hit 8 different banks; rows of dy silu(z) are padded by 4
+// bytes per group and 32 bytes per token, so all 32 lanes' 4-byte loads do
+// too.
 // ---------------------------------------------------------------------------
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kWCh = 128;              // channels (= threads) per CTA
 constexpr int kWTS = 8;                // tokens per chunk and per checkpoint
+constexpr int kWMinCtas = kWTS == 4 ? 3 : 2;  // CTAs per SM the shared memory allows
 constexpr int kWRow = kWCh + 1;        // float4 per padded state row
 constexpr int kWQRow = 136;            // floats per padded dy silu(z) row
 
-constexpr int kWGCh = 32;              // channels per lane quarter of a channel sum
-static_assert(3 * (kWGCh + 1) + kWGCh <= kWQRow, "dy silu(z) row");
+constexpr int kWItemWarps = kWTS / 2;  // warps that cover the chunk's items once
+constexpr int kWGCh = 4 * kWTS;        // channels per group of a channel sum
+static_assert(kWTS == 4 || kWTS == 8, "chunk of 4 or 8 tokens");
+static_assert((kWCh / kWGCh - 1) * (kWGCh + 1) + kWGCh <= kWQRow, "dy silu(z) row");
 
 template <typename T>
 struct WRaw {
@@ -565,13 +571,14 @@ __device__ __forceinline__ void w_issue(const BwdParams &p, WRaw<T> &r, int64_t 
 __device__ __forceinline__ void w_channel_sum(const BwdParams &p, const WSmem &sm, bool weighted,
                                               float *dst, int64_t t0, int nt)
 {
-    const int lane = threadIdx.x & 31, k = lane >> 3;
-    const int item = (threadIdx.x >> 5) * 8 + (lane & 7), tl = item >> 2, q = item & 3;
+    const int lane = threadIdx.x & 31, k = lane >> 3, w = threadIdx.x >> 5;
+    const int item = (w % kWItemWarps) * 8 + (lane & 7), tl = item >> 2, q = item & 3;
+    const int g = (w / kWItemWarps) * 4 + k;
     f32x2 s01 = 0ull, s23 = 0ull;
     if (tl < nt) {
-        const float4 *row = &sm.hist[(tl + 1) * 4 + q][k * kWGCh];
+        const float4 *row = &sm.hist[(tl + 1) * 4 + q][g * kWGCh];
         if (weighted) {
-            const float *wt = &sm.dq[tl][k * (kWGCh + 1)];
+            const float *wt = &sm.dq[tl][g * (kWGCh + 1)];
 #pragma unroll 8
             for (int j = 0; j < kWGCh; ++j) {
                 const float4 v = row[j];
@@ -621,7 +628,7 @@ constexpr size_t w_smem_bytes(size_t raw_bytes, bool ck_async)
 }
 
 template <typename T, bool ASYNC>
-__global__ void __launch_bounds__(kWCh, 2)
+__global__ void __launch_bounds__(kWCh, kWMinCtas)
 scan_bwd_wide_kernel(const BwdParams p)
 {
     constexpr int NP = 8, NQ = 4;  // packed state pairs, state quads
