@@ -168,7 +168,7 @@ constexpr int kComputeWarps = kCh / 32;
 constexpr int kThreads = kCh + 32;  // compute warps, then the producer warp
 
 template <typename T, typename TC, int K>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 4)  // 4 CTAs per SM: at most 102 registers
 replay_step_kernel(const RParams p)
 {
     using G = Stage<T, TC, K>;
@@ -243,17 +243,25 @@ replay_step_kernel(const RParams p)
             bulk_commit();
             held &= ~(1u << i);
         };
+        // the channel block's offsets, folded in once; the row's activations
+        // advance by rstep rows per row
+        const float *ck_c = p.ckpt + c0 * kN;
+        const __nv_bfloat16 *lo_c = p.ckpt_lo + c0 * kN;
+        const float *buf_c = p.buf + c0 * 2;
+        TC *cs_c = CS + c0 * (K - 1);
+        const int64_t wd = (int64_t)(W - 1) * D * 2;  // one slot's buffer, in floats
+        int64_t xoff = r0 * D + c0;
+        const int64_t xstep = rstep * D;
         for (int b0 = 0; b0 < nrows; b0 += kRowBatch) {
             const int nb = min(kRowBatch, nrows - b0);
             __syncthreads();  // the batch's metadata and B/C table are ready
             if (lead) {
-                for (int jj = 0; jj < nb; ++jj) {
+                for (int jj = 0; jj < nb; ++jj, xoff += xstep) {
                     if (held & (1u << st)) {
                         retire(st);
                         bulk_wait_read<0>();  // the stores have read the stage
                     }
                     const int64_t s = row_slot[jj];
-                    const int64_t b = r0 + (int64_t)(b0 + jj) * rstep;
                     held |= 1u << st;
                     held_ph = (held_ph & ~(1u << st)) | ((round & 1u) << st);
                     pend_slot[st] = (int)s;
@@ -269,20 +277,20 @@ replay_step_kernel(const RParams p)
                         mbar_expect_tx(&full[st],
                                        hb + (uint32_t)jl * (ent_b + G::BROW) + cs_b + io_b);
                         if (flush || !has_lo)
-                            bulk_g2s(dst, p.ckpt + s * DN + c0 * kN, hb, &full[st]);
+                            bulk_g2s(dst, ck_c + s * DN, hb, &full[st]);
                         else
-                            bulk_g2s(dst, p.ckpt_lo + s * DN + c0 * kN, hb, &full[st]);
-                        const float *bsrc = p.buf + (s * (W - 1) * D + c0) * 2;
+                            bulk_g2s(dst, lo_c + s * DN, hb, &full[st]);
+                        const float *bsrc = buf_c + s * wd;
                         for (int i = 0; i < jl; ++i)
                             bulk_g2s(dst + G::H + (uint32_t)i * G::ENTRY,
                                      bsrc + (int64_t)i * D * 2, ent_b, &full[st]);
                         if (jl > 0)
                             bulk_g2s(dst + g.off_bb, p.bufB + s * (int64_t)(W - 1) * kN,
                                      (uint32_t)jl * G::BROW, &full[st]);
-                        bulk_g2s(dst + g.off_cs, CS + (s * D + c0) * (K - 1), cs_b, &full[st]);
-                        bulk_g2s(dst + g.off_x, X + b * D + c0, a_b, &full[st]);
-                        bulk_g2s(dst + g.off_dt, DT + b * D + c0, a_b, &full[st]);
-                        if (has_z) bulk_g2s(dst + g.off_z, Z + b * D + c0, a_b, &full[st]);
+                        bulk_g2s(dst + g.off_cs, cs_c + s * D * (K - 1), cs_b, &full[st]);
+                        bulk_g2s(dst + g.off_x, X + xoff, a_b, &full[st]);
+                        bulk_g2s(dst + g.off_dt, DT + xoff, a_b, &full[st]);
+                        if (has_z) bulk_g2s(dst + g.off_z, Z + xoff, a_b, &full[st]);
                     }
                     if (++st == kStages) {
                         st = 0;
@@ -330,6 +338,9 @@ replay_step_kernel(const RParams p)
 
     int cons_st = 0;
     uint32_t cons_ph = 0;
+    unsigned char *sp_cur = smem;  // the stage of cons_st
+    T *yrow = y_t + r0 * D;        // this thread's y entry of the current row
+    const int64_t ystep = rstep * D;
     for (int b0 = 0; b0 < nrows; b0 += kRowBatch) {
         const int nb = min(kRowBatch, nrows - b0);
         // Every row's slot and length are read once, in parallel, before any
@@ -355,14 +366,13 @@ replay_step_kernel(const RParams p)
         }
         __syncthreads();
 
-        for (int jj = 0; jj < nb; ++jj) {
+        for (int jj = 0; jj < nb; ++jj, yrow += ystep) {
             const int st = cons_st;
             mbar_wait(&full[st], cons_ph, failed, &g_replay_status, 1);
             const int64_t s = row_slot[jj];
-            const int64_t b = r0 + (int64_t)(b0 + jj) * rstep;
             const int jl = row_len[jj];
             const bool flush = s >= 0 && jl + 1 == W;
-            unsigned char *sp = smem + (size_t)st * g.bytes;
+            unsigned char *sp = sp_cur;
             if (s >= 0 && cvalid) {
                 // the checkpoint: fp32, or the bf16 copy on the other steps
                 f32x2 h2[8];
@@ -454,7 +464,7 @@ replay_step_kernel(const RParams p)
                 upk2(yacc, y0, y1);
                 float yv = y0 + y1 + dsk * xcv;
                 if (has_z) yv *= silu_f(to_f32(reinterpret_cast<const T *>(sp + g.off_z)[t]));
-                y_t[b * D] = from_f32<T>(yv);
+                *yrow = from_f32<T>(yv);
             }
             // the row's B joins the buffer once (channel block 0)
             if (s >= 0 && !flush && blockIdx.x == 0 && t < kN)
@@ -463,9 +473,11 @@ replay_step_kernel(const RParams p)
             fence_proxy_async();
             __syncwarp();
             if ((t & 31) == 0) mbar_arrive(&done[st]);
+            sp_cur += g.bytes;
             if (++cons_st == kStages) {
                 cons_st = 0;
                 cons_ph ^= 1u;
+                sp_cur = smem;
             }
         }
         // The last channel block of a row to finish advances its length: one
