@@ -498,6 +498,15 @@ def bench_secondary(peaks, world, steps_scale=1.0, replay_windows=(3,)):
     del a
     torch.cuda.empty_cache()
 
+    # -- backward at the Mamba-130M layer shape (8 dense rows of 2048) -------
+    wl = synth.WORKLOADS["mamba130m_layer_b8_l2048"]
+    lyl = Layer(wl["D"])
+    al = synth.device_activations(0, wl["batch"] * wl["seqlen"], wl["D"])
+    out["mamba130m_layer_b8_l2048_scan_bwd"] = bench_scan_bwd(
+        peaks, world, lyl, al, None, wl["batch"], steps_scale, label="8 x 2048 x 1536 (dense rows)")
+    del al
+    torch.cuda.empty_cache()
+
     # -- long-context chunked prefill --------------------------------------
     w = synth.WORKLOADS["falcon_mamba7b_longctx_131072"]
     D, L, chunk = w["D"], w["seqlen"], w["chunk"]
@@ -590,9 +599,10 @@ def bench_secondary(peaks, world, steps_scale=1.0, replay_windows=(3,)):
     return out
 
 
-def bench_scan_bwd(peaks, world, ly, a, cu, S, steps_scale=1.0):
-    """Backward of the selective scan on the packed prefill's inputs (bf16
-    activations, upstream gradient dy drawn like x). Algorithmic work per
+def bench_scan_bwd(peaks, world, ly, a, cu, S, steps_scale=1.0, label="packed 65536 x 5120"):
+    """Backward of the selective scan on a prefill's inputs (bf16 activations,
+    upstream gradient dy drawn like x; packed when cu is given, else S dense
+    rows). Algorithmic work per
     (token, channel): 2 x 16 exponentials (the decays of one forward pass to
     produce the states and of the reverse pass; the kernel executes 3 x 16, as
     it recomputes the states chunk by chunk from checkpoints instead of storing
@@ -615,7 +625,8 @@ def bench_scan_bwd(peaks, world, ly, a, cu, S, steps_scale=1.0):
 
     def call():
         ssm.ssm_selective_scan_bwd(a["x"], a["dt"], ly.A, a["B"], a["C"], dy, g, Dskip=ly.Dskip,
-                                   z=a["z"], dt_bias=ly.dt_bias, cu_seqlens=cu, workspace=ws)
+                                   z=a["z"], dt_bias=ly.dt_bias, cu_seqlens=cu, S=S,
+                                   workspace=ws)
 
     def timed(variant):
         ssm.ssm_set_scan_bwd_variant(variant)
@@ -643,7 +654,7 @@ def bench_scan_bwd(peaks, world, ly, a, cu, S, steps_scale=1.0):
            "hbm_frac": round(units * 14 / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
            "variant": ssm.ssm_scan_bwd_variant_for(S, D), "ms_per_variant": per_variant,
            "workspace_bytes": ws.numel(), "sequences": S,
-           "step": "ssm_selective_scan_bwd over the packed 65536 x 5120 prefill, all gradients"}
+           "step": f"ssm_selective_scan_bwd over the {label} prefill, all gradients"}
     del g, ws, dy
     return res
 
