@@ -35,9 +35,10 @@
 // atomic per CTA and channel. The atomics make the last bits of those sums
 // depend on the order in which CTAs finish; everything else is deterministic.
 //
-// scan_bwd_wide_kernel (thread-per-channel, for large S * D): one thread per
-// channel with all 16 states, 8-token chunks, dB and dC summed over channels
-// from shared memory; described above the kernel.
+// scan_bwd_ckpt_kernel + scan_bwd_wide_kernel (thread-per-channel, for large
+// S * D): one thread per channel with all 16 states, 8-token chunks; the first
+// kernel writes the checkpoints, the second walks back, with dB and dC summed
+// over channels from shared memory; described above the kernels.
 #include <atomic>
 #include <type_traits>
 
@@ -495,7 +496,8 @@ scan_bwd_kernel(const BwdParams p)
 // Thread-per-channel variant. One thread owns one (sequence, channel) with
 // all 16 states in registers (eight packed fp32x2 pairs): sums over states
 // take no shuffles, and the CTA's 128 channels share each token's B and C.
-// Chunks of kWTS tokens, one checkpoint each. Phase A is as above; phase B,
+// Chunks of kWTS tokens, one checkpoint each. Phase A (the forward pass that
+// writes them) runs before, as scan_bwd_ckpt_kernel; this kernel is phase B,
 // per chunk, last first:
 //   1. recompute the chunk's states from its checkpoint into shared memory,
 //      with dz on the way (C . h_t is at hand), keeping each token's delta,
@@ -702,73 +704,6 @@ scan_bwd_wide_kernel(const BwdParams p)
     auto cquad = [&](int tl, int qq) { return *reinterpret_cast<const float4 *>(Cq + tl * kN + 4 * qq); };
     auto hist = [&](int slot, int qq) -> float4 & { return Hq[(slot * 4 + qq) * kWRow]; };
 
-    // ---- phase A: forward, checkpoint at every chunk start ----------------
-    f32x2 h[NP];
-#pragma unroll
-    for (int j = 0; j < NP; ++j) {
-        const int64_t o = (s * p.D + c) * kN + 2 * j;
-        h[j] = (cvalid && p.h0) ? pk2(p.h0[o], p.h0[o + 1]) : 0ull;
-    }
-    if (ASYNC && nchunks > 0) {
-        w_issue<T>(p, raw[0], start, (int)min((int64_t)kWTS, len), cbase, nch, false);
-        cp_commit();
-    }
-    for (int64_t k = 0; k < nchunks; ++k) {
-        const int64_t t0 = start + k * kWTS;
-        const int nt = (int)min((int64_t)kWTS, end - t0);
-        if (cvalid) {
-            float4 *dst = reinterpret_cast<float4 *>(ck + k * ck_stride);
-#pragma unroll
-            for (int qq = 0; qq < NQ; ++qq) {
-                float4 v;
-                upk2(h[2 * qq], v.x, v.y);
-                upk2(h[2 * qq + 1], v.z, v.w);
-                dst[qq] = v;
-            }
-        }
-        if constexpr (ASYNC) cp_wait<0>();
-        __syncthreads();  // chunk k has landed; chunk k - 1 is no longer read
-        if (ASYNC && k + 1 < nchunks) {
-            const int64_t t1 = t0 + kWTS;
-            w_issue<T>(p, raw[(k + 1) & 1], t1, (int)min((int64_t)kWTS, end - t1),
-                                   cbase, nch, false);
-            cp_commit();
-        }
-        fill_bc(raw[k & 1], t0, nt, false);
-        __syncthreads();
-        // full chunks take a copy of the token loop without per-token guards,
-        // so the compiler can overlap neighbouring tokens' work
-        auto walk = [&](auto full) {
-            constexpr bool kFull = decltype(full)::value;
-#pragma unroll
-            for (int tl = 0; tl < kWTS; ++tl) {
-                if (kFull || tl < nt) {
-                    const float v = act(raw[k & 1], 0, tl, t0 + tl) + dtb;
-                    const float d = p.softplus ? softplus_fast(v) : v;
-                    const float x = d * act(raw[k & 1], 1, tl, t0 + tl);
-                    const f32x2 dd = pk2(d, d), xx = pk2(x, x);
-#pragma unroll
-                    for (int qq = 0; qq < NQ; ++qq) {
-                        const float4 b4 = bquad(tl, qq);
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const int j = 2 * qq + e;
-                            float e0, e1;
-                            upk2(mul2(dd, A2[j]), e0, e1);
-                            const f32x2 a = pk2(ex2_approx(e0), ex2_approx(e1));
-                            const f32x2 b2 = e ? pk2(b4.z, b4.w) : pk2(b4.x, b4.y);
-                            h[j] = fma2(a, h[j], mul2(xx, b2));
-                        }
-                    }
-                }
-            }
-        };
-        if (cvalid) {
-            if (nt == kWTS) walk(std::true_type{});
-            else walk(std::false_type{});
-        }
-    }
-
     // ---- phase B: reverse -----------------------------------------------------
     f32x2 G[NP], dAacc[NP];
 #pragma unroll
@@ -787,8 +722,7 @@ scan_bwd_wide_kernel(const BwdParams p)
         const float *src = p.ckpt + ((start / kWTS + s + kk) * p.D + cbase) * kN;
         for (int e = tid; e < nch * 4; e += kWCh) cp16(&ckb[e], src + 4 * e);
     };
-    if constexpr (ASYNC) cp_wait<0>();
-    __syncthreads();  // phase A's last chunk is no longer read; its checkpoints are visible
+    // the checkpoints come from scan_bwd_ckpt_kernel, launched before on the stream
     if (ASYNC && nchunks > 0) {
         const int64_t tl0 = start + (nchunks - 1) * kWTS;
         w_issue<T>(p, raw[0], tl0, (int)(end - tl0), cbase, nch, true);
@@ -1003,6 +937,131 @@ scan_bwd_wide_kernel(const BwdParams p)
     }
 }
 
+// Phase A of the thread-per-channel backward as a kernel of its own: the
+// forward pass over each sequence that writes the state at every kWTS-token
+// chunk start (the checkpoint layout scan_bwd_wide_kernel reads). Without the
+// state buffer it needs 18 KB of shared memory (bf16) and few registers, so
+// several times as many warps per SM run it as would inside the reverse kernel.
+template <typename T, bool ASYNC>
+__global__ void __launch_bounds__(kWCh)
+scan_bwd_ckpt_kernel(const BwdParams p)
+{
+    constexpr int NP = 8, NQ = 4;  // packed state pairs, state quads
+    extern __shared__ __align__(128) unsigned char c_smem[];
+    WRaw<T> *raw = reinterpret_cast<WRaw<T> *>(c_smem);
+    float *sB = reinterpret_cast<float *>(c_smem + 2 * sizeof(WRaw<T>));  // [kWTS][kN]
+    const int tid = threadIdx.x, cl = tid;
+    const int64_t cbase = (int64_t)blockIdx.x * kWCh, c = cbase + tid;
+    const int nch = (int)min((int64_t)kWCh, p.D - cbase);
+    const bool cvalid = c < p.D;
+    const int64_t s = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    int64_t start, end;
+    if (p.cu) {
+        start = clamp_off(p.cu[s], p.tok);
+        end = max(clamp_off(p.cu[s + 1], p.tok), start);
+    } else {
+        start = s * p.L;
+        end = start + p.L;
+    }
+    const int64_t len = end - start;
+    const int64_t nchunks = (len + kWTS - 1) / kWTS;
+    float *ck = p.ckpt + ((start / kWTS + s) * p.D + c) * kN;
+    const int64_t ck_stride = p.D * kN;
+    f32x2 A2[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const float a0 = cvalid ? __ldg(p.A + c * kN + 2 * j) : 0.f;
+        const float a1 = cvalid ? __ldg(p.A + c * kN + 2 * j + 1) : 0.f;
+        A2[j] = pk2(a0 * kLog2e, a1 * kLog2e);
+    }
+    const float dtb = (cvalid && p.dt_bias) ? __ldg(p.dt_bias + c) : 0.f;
+    const T *DT = static_cast<const T *>(p.dt), *U = static_cast<const T *>(p.u);
+    const T *Bp = static_cast<const T *>(p.B);
+    // the chunk's B rows in fp32: one (token, state) per thread
+    auto fill_bc = [&](const WRaw<T> &r, int64_t t0, int nt, bool) {
+        if (tid >= kWTS * kN) return;
+        const int tl = tid >> 4, n = tid & 15;
+        float b = 0.f;
+        if (tl < nt) {
+            if constexpr (ASYNC) b = to_f32(r.bc[0][tl][n]);
+            else b = ld1(Bp + (t0 + tl) * kN + n);
+        }
+        sB[tl * kN + n] = b;
+    };
+    // this channel's dt (arr 0) or u (arr 1) at chunk token tl (channel valid)
+    auto act = [&](const WRaw<T> &r, int arr, int tl, int64_t t) -> float {
+        if constexpr (ASYNC) return to_f32(r.act[arr][tl][cl]);
+        else return ld1((arr == 0 ? DT : U) + t * p.D + c);
+    };
+    auto bquad = [&](int tl, int qq) { return *reinterpret_cast<const float4 *>(sB + tl * kN + 4 * qq); };
+
+    f32x2 h[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+        const int64_t o = (s * p.D + c) * kN + 2 * j;
+        h[j] = (cvalid && p.h0) ? pk2(p.h0[o], p.h0[o + 1]) : 0ull;
+    }
+    if (ASYNC && nchunks > 0) {
+        w_issue<T>(p, raw[0], start, (int)min((int64_t)kWTS, len), cbase, nch, false);
+        cp_commit();
+    }
+    for (int64_t k = 0; k < nchunks; ++k) {
+        const int64_t t0 = start + k * kWTS;
+        const int nt = (int)min((int64_t)kWTS, end - t0);
+        if (cvalid) {
+            float4 *dst = reinterpret_cast<float4 *>(ck + k * ck_stride);
+#pragma unroll
+            for (int qq = 0; qq < NQ; ++qq) {
+                float4 v;
+                upk2(h[2 * qq], v.x, v.y);
+                upk2(h[2 * qq + 1], v.z, v.w);
+                dst[qq] = v;
+            }
+        }
+        if constexpr (ASYNC) cp_wait<0>();
+        __syncthreads();  // chunk k has landed; chunk k - 1 is no longer read
+        if (ASYNC && k + 1 < nchunks) {
+            const int64_t t1 = t0 + kWTS;
+            w_issue<T>(p, raw[(k + 1) & 1], t1, (int)min((int64_t)kWTS, end - t1),
+                                   cbase, nch, false);
+            cp_commit();
+        }
+        fill_bc(raw[k & 1], t0, nt, false);
+        __syncthreads();
+        // full chunks take a copy of the token loop without per-token guards,
+        // so the compiler can overlap neighbouring tokens' work
+        auto walk = [&](auto full) {
+            constexpr bool kFull = decltype(full)::value;
+#pragma unroll
+            for (int tl = 0; tl < kWTS; ++tl) {
+                if (kFull || tl < nt) {
+                    const float v = act(raw[k & 1], 0, tl, t0 + tl) + dtb;
+                    const float d = p.softplus ? softplus_fast(v) : v;
+                    const float x = d * act(raw[k & 1], 1, tl, t0 + tl);
+                    const f32x2 dd = pk2(d, d), xx = pk2(x, x);
+#pragma unroll
+                    for (int qq = 0; qq < NQ; ++qq) {
+                        const float4 b4 = bquad(tl, qq);
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int j = 2 * qq + e;
+                            float e0, e1;
+                            upk2(mul2(dd, A2[j]), e0, e1);
+                            const f32x2 a = pk2(ex2_approx(e0), ex2_approx(e1));
+                            const f32x2 b2 = e ? pk2(b4.z, b4.w) : pk2(b4.x, b4.y);
+                            h[j] = fma2(a, h[j], mul2(xx, b2));
+                        }
+                    }
+                }
+            }
+        };
+        if (cvalid) {
+            if (nt == kWTS) walk(std::true_type{});
+            else walk(std::false_type{});
+        }
+    }
+}
+
 __global__ void zero_kernel(float *a, int64_t na, float *b, int64_t nb)
 {
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1066,11 +1125,20 @@ int scan_bwd_variant_for(int64_t S, int64_t D)
 }
 
 template <typename T, bool ASYNC>
-static cudaError_t run_wide(const BwdParams &p, dim3 grid, cudaStream_t stream)
+static cudaError_t run_wide(const BwdParams &p, dim3 grid, cudaStream_t stream, int *launches)
 {
+    // the forward pass that writes the checkpoints, then the reverse pass
+    const size_t ck_smem = 2 * sizeof(WRaw<T>) + sizeof(float) * kWTS * kN;
+    cudaError_t e = cudaFuncSetAttribute(scan_bwd_ckpt_kernel<T, ASYNC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ck_smem);
+    if (e != cudaSuccess) return e;
+    scan_bwd_ckpt_kernel<T, ASYNC><<<grid, kWCh, ck_smem, stream>>>(p);
+    ++*launches;
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     const size_t smem = w_smem_bytes(sizeof(WRaw<T>), ASYNC && sizeof(T) == 2);
-    cudaError_t e = cudaFuncSetAttribute(scan_bwd_wide_kernel<T, ASYNC>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(scan_bwd_wide_kernel<T, ASYNC>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     scan_bwd_wide_kernel<T, ASYNC><<<grid, kWCh, smem, stream>>>(p);
     return cudaGetLastError();
@@ -1124,11 +1192,11 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *laun
     if (scan_bwd_variant_for(a.S, a.D) == 2) {
         const dim3 grid((unsigned)((a.D + kWCh - 1) / kWCh), (unsigned)a.S);
         if (a.bf16)
-            e = async_ok ? run_wide<__nv_bfloat16, true>(p, grid, stream)
-                         : run_wide<__nv_bfloat16, false>(p, grid, stream);
+            e = async_ok ? run_wide<__nv_bfloat16, true>(p, grid, stream, launches)
+                         : run_wide<__nv_bfloat16, false>(p, grid, stream, launches);
         else
-            e = async_ok ? run_wide<float, true>(p, grid, stream)
-                         : run_wide<float, false>(p, grid, stream);
+            e = async_ok ? run_wide<float, true>(p, grid, stream, launches)
+                         : run_wide<float, false>(p, grid, stream, launches);
     } else {
         const dim3 grid((unsigned)((a.D + kCh - 1) / kCh), (unsigned)a.S);
         if (a.bf16) {
