@@ -546,7 +546,7 @@ struct WSmem {
 
 __device__ __forceinline__ int wq_col(int c) { return (c / kWGCh) * (kWGCh + 1) + c % kWGCh; }
 
-template <typename T>
+template <typename T, int NT = kWCh>  // NT: threads of the CTA that share the copies
 __device__ __forceinline__ void w_issue(const BwdParams &p, WRaw<T> &r, int64_t t0, int nt,
                                         int64_t cbase, int nch, bool full)
 {
@@ -554,13 +554,13 @@ __device__ __forceinline__ void w_issue(const BwdParams &p, WRaw<T> &r, int64_t 
     const T *DT = static_cast<const T *>(p.dt), *U = static_cast<const T *>(p.u);
     const T *Z = static_cast<const T *>(p.z), *DY = static_cast<const T *>(p.dy);
     const int narr = full ? 4 : 2, nvr = nch / V;
-    for (int e = threadIdx.x; e < narr * kWTS * VR; e += kWCh) {
+    for (int e = threadIdx.x; e < narr * kWTS * VR; e += NT) {
         const int arr = e / (kWTS * VR), rem = e % (kWTS * VR), tl = rem / VR, v = rem % VR;
         const T *src = arr == 0 ? DT : arr == 1 ? U : arr == 2 ? Z : DY;  // selects: no local array
         if (tl >= nt || v >= nvr || src == nullptr) continue;
         cp16(&r.act[arr][tl][v * V], src + (t0 + tl) * p.D + cbase + v * V);
     }
-    for (int e = threadIdx.x; e < (full ? 2 : 1) * kWTS * VB; e += kWCh) {
+    for (int e = threadIdx.x; e < (full ? 2 : 1) * kWTS * VB; e += NT) {
         const int arr = e / (kWTS * VB), rem = e % (kWTS * VB), tl = rem / VB, v = rem % VB;
         if (tl >= nt) continue;
         const T *src = static_cast<const T *>(arr ? p.C : p.B);
@@ -942,16 +942,21 @@ scan_bwd_wide_kernel(const BwdParams p)
 // chunk start (the checkpoint layout scan_bwd_wide_kernel reads). Without the
 // state buffer it needs 18 KB of shared memory (bf16) and few registers, so
 // several times as many warps per SM run it as would inside the reverse kernel.
+// Two adjacent lanes share a channel, 8 states each, which halves each thread's
+// serial chain: with packed sequences of mixed lengths the pass is bound by
+// its longest sequence.
+constexpr int kCkThreads = 2 * kWCh;
+
 template <typename T, bool ASYNC>
-__global__ void __launch_bounds__(kWCh)
+__global__ void __launch_bounds__(kCkThreads)
 scan_bwd_ckpt_kernel(const BwdParams p)
 {
-    constexpr int NP = 8, NQ = 4;  // packed state pairs, state quads
+    constexpr int NP = 4, NQ = 2;  // this lane's packed state pairs and state quads
     extern __shared__ __align__(128) unsigned char c_smem[];
     WRaw<T> *raw = reinterpret_cast<WRaw<T> *>(c_smem);
     float *sB = reinterpret_cast<float *>(c_smem + 2 * sizeof(WRaw<T>));  // [kWTS][kN]
-    const int tid = threadIdx.x, cl = tid;
-    const int64_t cbase = (int64_t)blockIdx.x * kWCh, c = cbase + tid;
+    const int tid = threadIdx.x, cl = tid >> 1, sub = tid & 1;
+    const int64_t cbase = (int64_t)blockIdx.x * kWCh, c = cbase + cl;
     const int nch = (int)min((int64_t)kWCh, p.D - cbase);
     const bool cvalid = c < p.D;
     const int64_t s = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
@@ -965,13 +970,13 @@ scan_bwd_ckpt_kernel(const BwdParams p)
     }
     const int64_t len = end - start;
     const int64_t nchunks = (len + kWTS - 1) / kWTS;
-    float *ck = p.ckpt + ((start / kWTS + s) * p.D + c) * kN;
+    float *ck = p.ckpt + ((start / kWTS + s) * p.D + c) * kN + 8 * sub;
     const int64_t ck_stride = p.D * kN;
     f32x2 A2[NP];
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
-        const float a0 = cvalid ? __ldg(p.A + c * kN + 2 * j) : 0.f;
-        const float a1 = cvalid ? __ldg(p.A + c * kN + 2 * j + 1) : 0.f;
+        const float a0 = cvalid ? __ldg(p.A + c * kN + 8 * sub + 2 * j) : 0.f;
+        const float a1 = cvalid ? __ldg(p.A + c * kN + 8 * sub + 2 * j + 1) : 0.f;
         A2[j] = pk2(a0 * kLog2e, a1 * kLog2e);
     }
     const float dtb = (cvalid && p.dt_bias) ? __ldg(p.dt_bias + c) : 0.f;
@@ -993,16 +998,18 @@ scan_bwd_ckpt_kernel(const BwdParams p)
         if constexpr (ASYNC) return to_f32(r.act[arr][tl][cl]);
         else return ld1((arr == 0 ? DT : U) + t * p.D + c);
     };
-    auto bquad = [&](int tl, int qq) { return *reinterpret_cast<const float4 *>(sB + tl * kN + 4 * qq); };
+    auto bquad = [&](int tl, int qq) {
+        return *reinterpret_cast<const float4 *>(sB + tl * kN + 8 * sub + 4 * qq);
+    };
 
     f32x2 h[NP];
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
-        const int64_t o = (s * p.D + c) * kN + 2 * j;
+        const int64_t o = (s * p.D + c) * kN + 8 * sub + 2 * j;
         h[j] = (cvalid && p.h0) ? pk2(p.h0[o], p.h0[o + 1]) : 0ull;
     }
     if (ASYNC && nchunks > 0) {
-        w_issue<T>(p, raw[0], start, (int)min((int64_t)kWTS, len), cbase, nch, false);
+        w_issue<T, kCkThreads>(p, raw[0], start, (int)min((int64_t)kWTS, len), cbase, nch, false);
         cp_commit();
     }
     for (int64_t k = 0; k < nchunks; ++k) {
@@ -1022,7 +1029,7 @@ scan_bwd_ckpt_kernel(const BwdParams p)
         __syncthreads();  // chunk k has landed; chunk k - 1 is no longer read
         if (ASYNC && k + 1 < nchunks) {
             const int64_t t1 = t0 + kWTS;
-            w_issue<T>(p, raw[(k + 1) & 1], t1, (int)min((int64_t)kWTS, end - t1),
+            w_issue<T, kCkThreads>(p, raw[(k + 1) & 1], t1, (int)min((int64_t)kWTS, end - t1),
                                    cbase, nch, false);
             cp_commit();
         }
@@ -1132,7 +1139,7 @@ static cudaError_t run_wide(const BwdParams &p, dim3 grid, cudaStream_t stream, 
     cudaError_t e = cudaFuncSetAttribute(scan_bwd_ckpt_kernel<T, ASYNC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ck_smem);
     if (e != cudaSuccess) return e;
-    scan_bwd_ckpt_kernel<T, ASYNC><<<grid, kWCh, ck_smem, stream>>>(p);
+    scan_bwd_ckpt_kernel<T, ASYNC><<<grid, kCkThreads, ck_smem, stream>>>(p);
     ++*launches;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
