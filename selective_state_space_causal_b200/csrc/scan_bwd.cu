@@ -945,17 +945,18 @@ scan_bwd_wide_kernel(const BwdParams p)
 // Two adjacent lanes share a channel, 8 states each, which halves each thread's
 // serial chain: with packed sequences of mixed lengths the pass is bound by
 // its longest sequence.
-constexpr int kCkThreads = 2 * kWCh;
+constexpr int kCkLanes = 2;                   // lanes per channel (4 measured slower)
+constexpr int kCkThreads = kCkLanes * kWCh;
 
 template <typename T, bool ASYNC>
 __global__ void __launch_bounds__(kCkThreads)
 scan_bwd_ckpt_kernel(const BwdParams p)
 {
-    constexpr int NP = 4, NQ = 2;  // this lane's packed state pairs and state quads
+    constexpr int SPL = kN / kCkLanes, NP = SPL / 2, NQ = SPL / 4;  // states, pairs, quads per lane
     extern __shared__ __align__(128) unsigned char c_smem[];
     WRaw<T> *raw = reinterpret_cast<WRaw<T> *>(c_smem);
     float *sB = reinterpret_cast<float *>(c_smem + 2 * sizeof(WRaw<T>));  // [kWTS][kN]
-    const int tid = threadIdx.x, cl = tid >> 1, sub = tid & 1;
+    const int tid = threadIdx.x, cl = tid / kCkLanes, sub = tid % kCkLanes;
     const int64_t cbase = (int64_t)blockIdx.x * kWCh, c = cbase + cl;
     const int nch = (int)min((int64_t)kWCh, p.D - cbase);
     const bool cvalid = c < p.D;
@@ -970,13 +971,13 @@ scan_bwd_ckpt_kernel(const BwdParams p)
     }
     const int64_t len = end - start;
     const int64_t nchunks = (len + kWTS - 1) / kWTS;
-    float *ck = p.ckpt + ((start / kWTS + s) * p.D + c) * kN + 8 * sub;
+    float *ck = p.ckpt + ((start / kWTS + s) * p.D + c) * kN + SPL * sub;
     const int64_t ck_stride = p.D * kN;
     f32x2 A2[NP];
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
-        const float a0 = cvalid ? __ldg(p.A + c * kN + 8 * sub + 2 * j) : 0.f;
-        const float a1 = cvalid ? __ldg(p.A + c * kN + 8 * sub + 2 * j + 1) : 0.f;
+        const float a0 = cvalid ? __ldg(p.A + c * kN + SPL * sub + 2 * j) : 0.f;
+        const float a1 = cvalid ? __ldg(p.A + c * kN + SPL * sub + 2 * j + 1) : 0.f;
         A2[j] = pk2(a0 * kLog2e, a1 * kLog2e);
     }
     const float dtb = (cvalid && p.dt_bias) ? __ldg(p.dt_bias + c) : 0.f;
@@ -999,13 +1000,13 @@ scan_bwd_ckpt_kernel(const BwdParams p)
         else return ld1((arr == 0 ? DT : U) + t * p.D + c);
     };
     auto bquad = [&](int tl, int qq) {
-        return *reinterpret_cast<const float4 *>(sB + tl * kN + 8 * sub + 4 * qq);
+        return *reinterpret_cast<const float4 *>(sB + tl * kN + SPL * sub + 4 * qq);
     };
 
     f32x2 h[NP];
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
-        const int64_t o = (s * p.D + c) * kN + 8 * sub + 2 * j;
+        const int64_t o = (s * p.D + c) * kN + SPL * sub + 2 * j;
         h[j] = (cvalid && p.h0) ? pk2(p.h0[o], p.h0[o + 1]) : 0ull;
     }
     if (ASYNC && nchunks > 0) {
