@@ -64,9 +64,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--replay-windows", type=int, nargs="+", default=[3], metavar="W",
                     help="checkpoint intervals of the replay decode measurement")
-    ap.add_argument("--profile-scan-bwd", action="store_true",
-                    help="instead of the step: run 3 backward scans over 16384 packed tokens of "
-                         "5120 channels (about 1.5 GB), untimed, for ncu captures")
+    ap.add_argument("--profile-scan-bwd", nargs="?", const="packed", default=None,
+                    choices=["packed", "layer"],
+                    help="instead of the step: run 3 backward scans, untimed, for ncu captures: "
+                         "over 16384 packed tokens of 5120 channels (packed, about 2.2 GB) or "
+                         "over the Mamba-130M layer's 8 x 2048 x 1536 (layer)")
     ap.add_argument("--profile-decode", type=int, default=None, metavar="W",
                     help="instead of the step: run 3 windows of replay decode steps (checkpoint "
                          "every W tokens, bf16 copy) and 3 eager decode steps at 256 x 8192 from "
@@ -877,15 +879,20 @@ def scan_sweep(variants, peaks):
     return 0
 
 
-def profile_scan_bwd():
-    """Three backward scans on a quarter of the packed workload, for profiler captures."""
+def profile_scan_bwd(shape="packed"):
+    """Three backward scans, for profiler captures: on a quarter of the packed
+    workload, or on the Mamba-130M layer shape (8 dense rows)."""
     import torch
 
     import selective_state_space_causal_b200 as ssm
     from selective_state_space_causal_b200 import synth
 
-    D, tot = 5120, 16384
-    lens = synth.sample_lengths(0, tot, 128, 8192)
+    if shape == "layer":
+        D, tot = 1536, 8 * 2048
+        lens = [2048] * 8
+    else:
+        D, tot = 5120, 16384
+        lens = synth.sample_lengths(0, tot, 128, 8192)
     cu = torch.from_numpy(synth.cu_from_lengths(lens)).cuda()
     ly = Layer(D)
     a = synth.device_activations(0, tot, D)
@@ -945,7 +952,7 @@ def main():
         profile_decode(args.profile_decode)
         return
     if args.profile_scan_bwd:
-        profile_scan_bwd()
+        profile_scan_bwd(args.profile_scan_bwd)
         return
     if args.impl == "reference":
         return bench_reference(args)
