@@ -69,6 +69,21 @@ struct BwdParams {
     int vec_atomics;  // dB and dC are 16-byte aligned: sums go out as float4 atomics
 };
 
+// The sequence of this CTA row (blockIdx.y; the longest-first order when one
+// is given) and its token range, with the offsets clamped into [0, tok].
+__device__ __forceinline__ void bwd_sequence(const BwdParams &p, int64_t &s, int64_t &start,
+                                             int64_t &end)
+{
+    s = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    if (p.cu) {
+        start = clamp_off(p.cu[s], p.tok);
+        end = max(clamp_off(p.cu[s + 1], p.tok), start);
+    } else {
+        start = s * p.L;
+        end = start + p.L;
+    }
+}
+
 // Shared memory of one CTA.
 struct Smem {
     float d[kTS][kCh];     // delta
@@ -244,15 +259,8 @@ scan_bwd_kernel(const BwdParams p)
     const int64_t cbase = (int64_t)blockIdx.x * kCh, c = cbase + cl;
     const int nch = (int)min((int64_t)kCh, p.D - cbase);
     const bool cvalid = c < p.D;
-    const int64_t s = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
-    int64_t start, end;
-    if (p.cu) {
-        start = clamp_off(p.cu[s], p.tok);
-        end = max(clamp_off(p.cu[s + 1], p.tok), start);
-    } else {
-        start = s * p.L;
-        end = start + p.L;
-    }
+    int64_t s, start, end;
+    bwd_sequence(p, s, start, end);
     const int64_t len = end - start;
     const int64_t nchunks = (len + kTS - 1) / kTS;
     // checkpoint slots of this sequence: floor(start / kTS) + s + k never collide
@@ -641,15 +649,8 @@ scan_bwd_wide_kernel(const BwdParams p)
     const int64_t cbase = (int64_t)blockIdx.x * kWCh, c = cbase + cl;
     const int nch = (int)min((int64_t)kWCh, p.D - cbase);
     const bool cvalid = c < p.D;
-    const int64_t s = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
-    int64_t start, end;
-    if (p.cu) {
-        start = clamp_off(p.cu[s], p.tok);
-        end = max(clamp_off(p.cu[s + 1], p.tok), start);
-    } else {
-        start = s * p.L;
-        end = start + p.L;
-    }
+    int64_t s, start, end;
+    bwd_sequence(p, s, start, end);
     const int64_t len = end - start;
     const int64_t nchunks = (len + kWTS - 1) / kWTS;
     // checkpoint slots of this sequence: floor(start / kWTS) + s + k never collide
@@ -960,15 +961,8 @@ scan_bwd_ckpt_kernel(const BwdParams p)
     const int64_t cbase = (int64_t)blockIdx.x * kWCh, c = cbase + cl;
     const int nch = (int)min((int64_t)kWCh, p.D - cbase);
     const bool cvalid = c < p.D;
-    const int64_t s = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
-    int64_t start, end;
-    if (p.cu) {
-        start = clamp_off(p.cu[s], p.tok);
-        end = max(clamp_off(p.cu[s + 1], p.tok), start);
-    } else {
-        start = s * p.L;
-        end = start + p.L;
-    }
+    int64_t s, start, end;
+    bwd_sequence(p, s, start, end);
     const int64_t len = end - start;
     const int64_t nchunks = (len + kWTS - 1) / kWTS;
     float *ck = p.ckpt + ((start / kWTS + s) * p.D + c) * kN + SPL * sub;
