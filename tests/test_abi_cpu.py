@@ -282,3 +282,25 @@ def conv_scan(**kw):
 def test_conv_scan_rejects(kw, code):
     assert conv_scan(**kw) == code
     assert _err()
+
+
+@pytest.mark.parametrize("chunk", [8, 16])
+def test_bwd_checkpoint_slots_are_distinct_and_fit_the_workspace(chunk):
+    """The backward kernels keep sequence s's checkpoint k (k < ceil(len/chunk))
+    at slot floor(start/chunk) + s + k, 64 bytes per channel, in a workspace of
+    ssm_scan_bwd_workspace_size bytes (the thread-per-channel kernels use
+    8-token chunks, the lane-split one 16): no two checkpoints share a slot, and
+    every slot and the sequence order after them fit."""
+    rng = np.random.default_rng(5)
+    for trial in range(200):
+        S = int(rng.integers(1, 60))
+        lens = rng.integers(0, 300, size=S) * (rng.random(S) > 0.2)  # some empty
+        starts = np.concatenate([[0], np.cumsum(lens)[:-1]])
+        tok = int(lens.sum())
+        slots = [start // chunk + s + k
+                 for s, (start, n) in enumerate(zip(starts, lens)) for k in range(-(-n // chunk))]
+        assert len(slots) == len(set(slots))
+        D = 8
+        ws = ssm.ssm_scan_bwd_workspace_size(max(tok, 0), D, 16, S)
+        top = (max(slots) + 1) if slots else 0
+        assert top * D * 64 + S * 4 <= ws
