@@ -276,11 +276,12 @@ size_t ssm_scan_bwd_workspace_size(int64_t tok, int64_t D, int N, int64_t S);
 /*
  * Tuning knob for ssm_selective_scan_bwd's kernel: 1 splits each channel's
  * 16 states over 4 lanes (16-token chunks, per-token sums over states and
- * channels by shuffles); 2 gives each channel one thread with all 16 states
- * (8-token chunks whose states are summed over channels from shared memory;
- * about half of variant 1's instructions per token and channel, a quarter of
- * its threads); 0 lets the library choose (2 once S * ceil(D / 128) reaches
- * twice the SM count, else 1). Process-wide; not
+ * channels by shuffles); 2 runs a checkpointing forward pass (two lanes per
+ * channel), then a reverse pass that gives each channel one thread with all 16
+ * states (8-token chunks whose states are summed over channels from shared
+ * memory; about half of variant 1's instructions per token and channel, a
+ * quarter of its threads); 0 lets the library choose (2 once
+ * S * ceil(D / 128) reaches twice the SM count, else 1). Process-wide; not
  * thread-safe against concurrent backward calls. Returns SSM_OK or
  * SSM_ERR_INVALID_ARGUMENT. The variants differ only in the order of their
  * floating-point sums.
