@@ -435,13 +435,18 @@ int ssm_replay_flush(float *ckpt, void *ckpt_lo, const float *buf, const float *
  *
  * Arguments, results and errors are those of ssm_selective_scan_fwd. The
  * longest-first schedule of packed sequences lives in a fixed 16 KB array
- * inside the library instead of a workspace, so a call may name at most 4096
- * packed sequences; larger S with cu_seqlens is rejected with
- * SSM_ERR_INVALID_ARGUMENT before anything is launched. The library allocates
- * nothing for this call: every GPU that loads the library holds the array
- * until the process exits. The first call on a device looks the array's
- * address up (with that device current) and caches it; make that first call
- * before any stream capture. All calls on a device share the one array and
+ * inside the library instead of a workspace, so a packed call (cu_seqlens
+ * given) may name at most 4096 sequences; larger S with cu_seqlens is
+ * rejected with SSM_ERR_INVALID_ARGUMENT before anything is launched. Dense
+ * calls (cu_seqlens NULL) and single sequences need no schedule and accept any
+ * S. The library allocates nothing for this call: every GPU that loads the
+ * library holds the array until the process exits. The first packed call on a
+ * device looks the array's address up (with that device current) and caches
+ * it for the life of the process; make that first call before any stream
+ * capture, and do not use this entry point on a device after a
+ * cudaDeviceReset (or any other teardown of its primary context) in the same
+ * process, since the cached address would then be stale. All calls on a
+ * device share the one array and
  * each overwrites it completely before reading it, so nothing needs clearing,
  * but two such calls that run at the same time on one GPU (different streams
  * without ordering between them) race on it and give unspecified results.
@@ -452,6 +457,28 @@ int ssm_selective_scan_fwd_noalloc(const void *u, const void *delta, const float
                                    const float *h0, const int32_t *cu_seqlens, int64_t S,
                                    void *y, float *h_final, int64_t tok, int64_t D, int N,
                                    ssm_dtype act_dtype, ssm_stream_t stream);
+
+/*
+ * Measurement helpers (not part of the method; the pages have no counterpart).
+ * The selective scan's roofline is set by the special-function unit (one ex2
+ * per state and token), so its denominator is measured on the device at hand
+ * instead of derived from unit counts.
+ *
+ * ssm_probe_rate launches one throughput probe over every SM (8 CTAs of 256
+ * threads each, 8 independent dependency chains per thread) and writes the
+ * operations it performs to *ops; time the launch with CUDA events on
+ * `stream` and divide. kind: 0 ex2.approx.ftz.f32 (special-function unit;
+ * ops = ex2 results), 1 packed fp32x2 FMA (ops = fp32 FMAs, two per
+ * instruction), 2 scalar fp32 FMA, 3 the scan recurrence's mix of one ex2 per
+ * two packed FMA-pipe operations (ops = ex2 results). `iters` loop steps per
+ * thread set the run time (each step is 8 operations per thread, 16 FMAs for
+ * kind 1). sink: device fp32 buffer of at least ssm_probe_sink_floats()
+ * entries, overwritten with one value per thread. Returns SSM_OK,
+ * SSM_ERR_INVALID_ARGUMENT, SSM_ERR_MISALIGNED or SSM_ERR_CUDA.
+ */
+int64_t ssm_probe_sink_floats(void);
+int ssm_probe_rate(int kind, int iters, float *sink, int64_t sink_floats, double *ops,
+                   ssm_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -16,6 +16,8 @@ from ._lib import (  # noqa: F401
     ssm_check_cu_seqlens,
     ssm_last_error,
     ssm_launch_count,
+    ssm_probe_rate,
+    ssm_probe_sink_floats,
     ssm_device_status,
     ssm_replay_flush,
     ssm_replay_reset,

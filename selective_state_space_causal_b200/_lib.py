@@ -55,6 +55,8 @@ SIGNATURES = [
     ("ssm_replay_reset", _int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp]),
     ("ssm_replay_flush", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _i64, _i64, _i64,
                                 _int, _vp]),
+    ("ssm_probe_sink_floats", _i64, []),
+    ("ssm_probe_rate", _int, [_int, _int, _vp, _i64, ctypes.POINTER(ctypes.c_double), _vp]),
 ]
 
 
@@ -132,6 +134,20 @@ def ssm_scan_variant_for(S: int, D: int) -> tuple[int, int]:
     npt, sched = _int(0), _int(0)
     _check(lib.ssm_scan_variant_for(int(S), int(D), ctypes.byref(npt), ctypes.byref(sched)))
     return npt.value, sched.value
+
+
+def ssm_probe_sink_floats() -> int:
+    return int(lib.ssm_probe_sink_floats())
+
+
+def ssm_probe_rate(kind: int, iters: int, sink, stream=None) -> float:
+    """Launches throughput probe `kind` (0 ex2, 1 packed fp32x2 FMA, 2 fp32
+    FMA, 3 the recurrence mix) on the current stream; returns its operation
+    count. The caller times the launch."""
+    ops = ctypes.c_double(0.0)
+    _check(lib.ssm_probe_rate(int(kind), int(iters), _ptr(sink), sink.numel(), ctypes.byref(ops),
+                              _stream(stream)))
+    return ops.value
 
 
 def ssm_device_status(clear: bool = False) -> int:

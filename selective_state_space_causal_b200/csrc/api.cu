@@ -23,6 +23,9 @@ int read_decode_status(bool clear);
 cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
 int64_t noalloc_max_sequences();
 int read_replay_status(bool clear);
+int probe_sink_floats();
+cudaError_t launch_probe(int kind, int iters, float *sink, double *ops, cudaStream_t stream,
+                         int *launches);
 
 struct ScanBwdArgs {
     const void *u, *dt, *B, *C, *z, *dy;
@@ -566,15 +569,40 @@ int ssm_selective_scan_fwd_noalloc(const void *u, const void *delta, const float
                     "%s: at most %lld packed sequences per call (got %lld); the fixed scratch "
                     "holds one schedule entry per sequence",
                     fn, (long long)ssm::noalloc_max_sequences(), (long long)S);
+    // Only packed calls of two or more sequences use the schedule; dense rows
+    // and a single sequence run without it, whatever S is.
     void *scratch = nullptr;
     size_t bytes = 0;
-    cudaError_t e = ssm::noalloc_scratch(&scratch, &bytes);
-    if (e != cudaSuccess)
-        return fail(SSM_ERR_CUDA, "%s: looking up the fixed scratch failed: %s", fn,
-                    cudaGetErrorString(e));
+    if (cu_seqlens && S > 1) {
+        cudaError_t e = ssm::noalloc_scratch(&scratch, &bytes);
+        if (e != cudaSuccess)
+            return fail(SSM_ERR_CUDA, "%s: looking up the fixed scratch failed: %s", fn,
+                        cudaGetErrorString(e));
+    }
     return ssm_selective_scan_fwd(u, delta, A, B, C, Dskip, z, dt_bias, delta_softplus, h0,
                                   cu_seqlens, S, y, h_final, tok, D, N, act_dtype, scratch, bytes,
                                   stream);
+}
+
+int64_t ssm_probe_sink_floats(void) { return (int64_t)ssm::probe_sink_floats(); }
+
+int ssm_probe_rate(int kind, int iters, float *sink, int64_t sink_floats, double *ops,
+                   ssm_stream_t stream)
+{
+    const char *fn = "ssm_probe_rate";
+    if (kind < 0 || kind > 3)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: kind must be 0..3 (got %d)", fn, kind);
+    if (iters < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: iters must be >= 1", fn);
+    if (!sink || !ops) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: sink and ops are required", fn);
+    if (!aligned(sink, 4)) return fail(SSM_ERR_MISALIGNED, "%s: sink misaligned", fn);
+    const int64_t need = ssm_probe_sink_floats();
+    if (sink_floats < need)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: sink holds %lld floats, needs %lld", fn,
+                    (long long)sink_floats, (long long)need);
+    int launched = 0;
+    cudaError_t e = ssm::launch_probe(kind, iters, sink, ops,
+                                      reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
 }
 
 }  // extern "C"

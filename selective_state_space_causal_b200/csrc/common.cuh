@@ -121,9 +121,10 @@ __device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b)
 // 2^x for two values on the FMA pipe instead of the special-function unit.
 // x is clamped to [-126, 126] and split as n + f with n = round(x) (adding and
 // subtracting 1.5 * 2^23 rounds to an integer held in the low mantissa bits)
-// and f in [-0.5, 0.5]; 2^f comes from a degree-5 polynomial whose
-// coefficients were fitted here for minimal relative error on [-0.5, 0.5]
-// (2.3e-7 when evaluated in fp32), and 2^n is added into the exponent bits:
+// and f in [-0.5, 0.5]; 2^f comes from a degree-5 polynomial, the minimax
+// fit for relative error on [-0.5, 0.5] with its coefficients rounded to fp32
+// (1.5e-7 in exact arithmetic, 2.3e-7 when evaluated in fp32;
+// tests/test_fastmath_fit.py re-derives the fit), and 2^n is added into the exponent bits:
 // the float bits of x + 1.5 * 2^23 are 0x4B400000 + n, and shifting them left
 // by 23 leaves exactly n << 23 (mod 2^32).
 __device__ __forceinline__ void exp2_fma2(float x0, float x1, float &r0, float &r1)
@@ -182,8 +183,9 @@ __device__ __forceinline__ float silu_f(float v)
 
 // softplus(v) = max(v, 0) + log1p(e) with e = exp(-|v|) in (0, 1], and
 // log1p(e) = 2 atanh(s), s = e / (2 + e) in (0, 1/3]. 2 atanh(s) / s is a
-// polynomial in s^2; the degree-4 coefficients below were fitted here for
-// minimal relative error on [0, 1/9] (max 4e-9, below fp32 resolution). Two
+// polynomial in s^2; the degree-4 coefficients below are the minimax fit for
+// relative error on [0, 1/9] (max 4e-9, below fp32 resolution;
+// tests/test_fastmath_fit.py re-derives it). Two
 // special-function ops (2^x and 1/x) and ten FMA-pipe ops; relative error of
 // the result ~5e-7.
 __device__ __forceinline__ float softplus_fast(float v)

@@ -5,11 +5,12 @@ Tolerances (max-abs error, per output element):
 
 * fp32 activations: |gpu - oracle| <= 1e-4 * rms(oracle).
 * bf16 activations with fp32 state: |gpu - oracle| <= 2e-2 * rms(oracle)
-  + 2^-8 * |oracle| for outputs stored in bf16. The second term is one bf16
-  ulp: rounding the exact result to bf16 alone moves it by up to 2^-9 |y|,
-  and y is heavy-tailed (max |y| is ~60 rms(y) on Mamba-shaped inputs), so no
-  bf16-output implementation could meet the first term alone. fp32 outputs
-  (the SSM state) get the first term only.
+  + 2^-8 * |oracle| for outputs stored in bf16. The second term is the
+  largest error of rounding the exact result to bf16: half a bf16 ulp, which
+  is at most 2^-8 |y| (bf16 keeps 8 significant bits). y is heavy-tailed (max
+  |y| is ~60 rms(y) on Mamba-shaped inputs), so that rounding alone can exceed
+  the first term and no bf16-output implementation could meet it alone. fp32
+  outputs (the SSM state) get the first term only.
 """
 
 from __future__ import annotations
