@@ -125,10 +125,24 @@ int ssm_scan_variant_for(int64_t S, int64_t D, int *states_per_lane, int *schedu
  * every bounded wait for a TMA tile or bulk copy completed; bit 0 set once a
  * scan kernel's wait gave up, bit 1 once a conv kernel's did, bit 2 once a
  * decode kernel's did, bit 3 once a replay decode kernel's did (the results
- * of that call are then unspecified; the kernel still terminates). Synchronises the device.
+ * of that call are then unspecified; the kernel still terminates), bit 4 once
+ * ssm_selftest_wait_timeout's wait gave up. Synchronises the device.
  * clear != 0 resets the flags. Returns SSM_ERR_CUDA if the query itself fails.
  */
 int ssm_device_status(int clear);
+
+/*
+ * Self-test of the bounded device waits (failure detection; the pages have no
+ * counterpart). Every kernel that waits for a TMA tile or bulk copy waits on an
+ * mbarrier with a bounded number of suspending tries (2^17, about half a
+ * second at most) and, when they run out, sets its status bit and returns
+ * instead of hanging. This call launches one small kernel whose barrier
+ * expects 16 bytes that no copy delivers, with the limit lowered to `tries`
+ * (1..131072): its wait runs out, it sets bit 4 of ssm_device_status and
+ * returns with nothing in flight, and the context stays usable. Asynchronous on
+ * `stream`. Returns SSM_OK, SSM_ERR_INVALID_ARGUMENT or SSM_ERR_CUDA.
+ */
+int ssm_selftest_wait_timeout(int tries, ssm_stream_t stream);
 
 /*
  * Checks a HOST copy of cu_seqlens (S+1 entries): cu[0] == 0, non-decreasing,
@@ -464,8 +478,9 @@ int ssm_selective_scan_fwd_noalloc(const void *u, const void *delta, const float
  * per state and token), so its denominator is measured on the device at hand
  * instead of derived from unit counts.
  *
- * ssm_probe_rate launches one throughput probe over every SM (8 CTAs of 256
- * threads each, 8 independent dependency chains per thread) and writes the
+ * ssm_probe_rate launches one throughput probe over every SM (warps_per_sm / 8
+ * CTAs of 256 threads on each SM, 8 independent dependency chains per thread;
+ * warps_per_sm is 8, 16, ..., 64, and 64 gives the peak) and writes the
  * operations it performs to *ops; time the launch with CUDA events on
  * `stream` and divide. kind: 0 ex2.approx.ftz.f32 (special-function unit;
  * ops = ex2 results), 1 packed fp32x2 FMA (ops = fp32 FMAs, two per
@@ -477,8 +492,8 @@ int ssm_selective_scan_fwd_noalloc(const void *u, const void *delta, const float
  * SSM_ERR_INVALID_ARGUMENT, SSM_ERR_MISALIGNED or SSM_ERR_CUDA.
  */
 int64_t ssm_probe_sink_floats(void);
-int ssm_probe_rate(int kind, int iters, float *sink, int64_t sink_floats, double *ops,
-                   ssm_stream_t stream);
+int ssm_probe_rate(int kind, int iters, int warps_per_sm, float *sink, int64_t sink_floats,
+                   double *ops, ssm_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -28,6 +28,7 @@ from ._lib import (  # noqa: F401
     ssm_selective_scan_fwd,
     ssm_selective_scan_fwd_noalloc,
     ssm_selective_state_update,
+    ssm_selftest_wait_timeout,
     ssm_scan_bwd_variant_for,
     ssm_scan_variant_for,
     ssm_set_scan_bwd_variant,

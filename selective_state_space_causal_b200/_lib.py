@@ -55,8 +55,9 @@ SIGNATURES = [
     ("ssm_replay_reset", _int, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _int, _vp]),
     ("ssm_replay_flush", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _i64, _i64, _i64,
                                 _int, _vp]),
+    ("ssm_selftest_wait_timeout", _int, [_int, _vp]),
     ("ssm_probe_sink_floats", _i64, []),
-    ("ssm_probe_rate", _int, [_int, _int, _vp, _i64, ctypes.POINTER(ctypes.c_double), _vp]),
+    ("ssm_probe_rate", _int, [_int, _int, _int, _vp, _i64, ctypes.POINTER(ctypes.c_double), _vp]),
 ]
 
 
@@ -140,14 +141,19 @@ def ssm_probe_sink_floats() -> int:
     return int(lib.ssm_probe_sink_floats())
 
 
-def ssm_probe_rate(kind: int, iters: int, sink, stream=None) -> float:
+def ssm_probe_rate(kind: int, iters: int, sink, warps_per_sm: int = 64, stream=None) -> float:
     """Launches throughput probe `kind` (0 ex2, 1 packed fp32x2 FMA, 2 fp32
-    FMA, 3 the recurrence mix) on the current stream; returns its operation
-    count. The caller times the launch."""
+    FMA, 3 the recurrence mix) with `warps_per_sm` resident warps per SM on the
+    current stream; returns its operation count. The caller times the launch."""
     ops = ctypes.c_double(0.0)
-    _check(lib.ssm_probe_rate(int(kind), int(iters), _ptr(sink), sink.numel(), ctypes.byref(ops),
-                              _stream(stream)))
+    _check(lib.ssm_probe_rate(int(kind), int(iters), int(warps_per_sm), _ptr(sink), sink.numel(),
+                              ctypes.byref(ops), _stream(stream)))
     return ops.value
+
+
+def ssm_selftest_wait_timeout(tries: int = 64, stream=None) -> None:
+    """Launches the bounded-wait self-test (its wait must run out)."""
+    _check(lib.ssm_selftest_wait_timeout(int(tries), _stream(stream)))
 
 
 def ssm_device_status(clear: bool = False) -> int:

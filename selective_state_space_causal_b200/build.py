@@ -105,7 +105,9 @@ def build_library(force: bool = False, verbose: bool = False, extra: list[str] |
             raise RuntimeError(f"nvcc failed compiling {os.path.basename(src)}")
         if verbose:
             sys.stderr.write(res.stderr)
-    cmd = [nvcc, *ARCH, "-shared", "-o", LIBRARY + ".tmp", *[_object(s) for s in srcs]]
+    # --no-undefined: a symbol missing across translation units fails the build, not the import
+    cmd = [nvcc, *ARCH, "-shared", "-Xlinker", "--no-undefined", "-o", LIBRARY + ".tmp",
+           *[_object(s) for s in srcs]]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)

@@ -24,8 +24,10 @@ cudaError_t noalloc_scratch(void **ptr, size_t *bytes);
 int64_t noalloc_max_sequences();
 int read_replay_status(bool clear);
 int probe_sink_floats();
-cudaError_t launch_probe(int kind, int iters, float *sink, double *ops, cudaStream_t stream,
-                         int *launches);
+int read_selftest_status(bool clear);
+cudaError_t launch_wait_selftest(unsigned tries, cudaStream_t stream, int *launches);
+cudaError_t launch_probe(int kind, int iters, int per_sm, float *sink, double *ops,
+                         cudaStream_t stream, int *launches);
 
 struct ScanBwdArgs {
     const void *u, *dt, *B, *C, *z, *dy;
@@ -152,10 +154,10 @@ unsigned long long ssm_launch_count(void) { return g_launches.load(std::memory_o
 int ssm_set_scan_variant(int npt, int sched)
 {
     const bool npt_ok = npt == 0 || npt == 2 || npt == 4 || npt == 8 || npt == 16;
-    const bool sched_ok = sched >= 0 && sched <= 8;
+    const bool sched_ok = sched >= 0 && sched <= 10;
     if (!npt_ok || !sched_ok)
         return fail(SSM_ERR_INVALID_ARGUMENT,
-                    "ssm_set_scan_variant: states per lane 0, 2, 4, 8 or 16; schedule 0..8");
+                    "ssm_set_scan_variant: states per lane 0, 2, 4, 8 or 16; schedule 0..10");
     ssm::set_scan_variant(npt, sched);
     return ok();
 }
@@ -175,10 +177,11 @@ int ssm_device_status(int clear)
     const int b = ssm::read_conv_status(clear != 0);
     const int d = ssm::read_decode_status(clear != 0);
     const int r = ssm::read_replay_status(clear != 0);
-    if (a < 0 || b < 0 || d < 0 || r < 0)
+    const int t = ssm::read_selftest_status(clear != 0);
+    if (a < 0 || b < 0 || d < 0 || r < 0 || t < 0)
         return fail(SSM_ERR_CUDA, "ssm_device_status: CUDA query failed");
     g_error.clear();
-    return (a ? 1 : 0) | (b ? 2 : 0) | (d ? 4 : 0) | (r ? 8 : 0);
+    return (a ? 1 : 0) | (b ? 2 : 0) | (d ? 4 : 0) | (r ? 8 : 0) | (t ? 16 : 0);
 }
 
 int ssm_check_cu_seqlens(const int32_t *cu, int64_t S, int64_t tok)
@@ -584,14 +587,28 @@ int ssm_selective_scan_fwd_noalloc(const void *u, const void *delta, const float
                                   stream);
 }
 
+int ssm_selftest_wait_timeout(int tries, ssm_stream_t stream)
+{
+    const char *fn = "ssm_selftest_wait_timeout";
+    if (tries < 1 || tries > (1 << 17))
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: tries must be 1..131072 (got %d)", fn, tries);
+    int launched = 0;
+    cudaError_t e = ssm::launch_wait_selftest((unsigned)tries,
+                                              reinterpret_cast<cudaStream_t>(stream), &launched);
+    return finish(e, launched, fn);
+}
+
 int64_t ssm_probe_sink_floats(void) { return (int64_t)ssm::probe_sink_floats(); }
 
-int ssm_probe_rate(int kind, int iters, float *sink, int64_t sink_floats, double *ops,
-                   ssm_stream_t stream)
+int ssm_probe_rate(int kind, int iters, int warps_per_sm, float *sink, int64_t sink_floats,
+                   double *ops, ssm_stream_t stream)
 {
     const char *fn = "ssm_probe_rate";
     if (kind < 0 || kind > 3)
         return fail(SSM_ERR_INVALID_ARGUMENT, "%s: kind must be 0..3 (got %d)", fn, kind);
+    if (warps_per_sm < 8 || warps_per_sm > 64 || warps_per_sm % 8 != 0)
+        return fail(SSM_ERR_INVALID_ARGUMENT, "%s: warps_per_sm must be 8, 16, ..., 64 (got %d)",
+                    fn, warps_per_sm);
     if (iters < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: iters must be >= 1", fn);
     if (!sink || !ops) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: sink and ops are required", fn);
     if (!aligned(sink, 4)) return fail(SSM_ERR_MISALIGNED, "%s: sink misaligned", fn);
@@ -600,7 +617,7 @@ int ssm_probe_rate(int kind, int iters, float *sink, int64_t sink_floats, double
         return fail(SSM_ERR_INVALID_ARGUMENT, "%s: sink holds %lld floats, needs %lld", fn,
                     (long long)sink_floats, (long long)need);
     int launched = 0;
-    cudaError_t e = ssm::launch_probe(kind, iters, sink, ops,
+    cudaError_t e = ssm::launch_probe(kind, iters, warps_per_sm / 8, sink, ops,
                                       reinterpret_cast<cudaStream_t>(stream), &launched);
     return finish(e, launched, fn);
 }

@@ -11,8 +11,13 @@
 #include <cuda_runtime.h>
 
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace ssm {
+
+// Set by the wait self-test when its bounded wait gives up (as it must).
+__device__ int g_selftest_status = 0;
+
 namespace {
 
 constexpr int kProbeThreads = 256;
@@ -109,19 +114,51 @@ probe_mix_kernel(float *sink, int iters)
     sink[blockIdx.x * blockDim.x + threadIdx.x] = s;
 }
 
+// Self-test of the bounded mbarrier wait every TMA-staged kernel uses: the
+// barrier expects 16 transaction bytes that no copy ever delivers, so the
+// wait runs out after `tries` suspending tries, sets the status bit and the
+// kernel returns. Nothing is in flight when it exits.
+__global__ void wait_selftest_kernel(unsigned tries)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) mbar_init(&bar);
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_expect_tx(&bar, 16);
+    bool failed = false;
+    mbar_wait(&bar, 0u, failed, &g_selftest_status, 1, tries);
+}
+
 }  // namespace
 
 int device_sm_count();
 
+int read_selftest_status(bool clear)
+{
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_selftest_status, sizeof(int)) != cudaSuccess) return -1;
+    if (clear && v) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_selftest_status, &zero, sizeof(int)) != cudaSuccess) return -1;
+    }
+    return v;
+}
+
+cudaError_t launch_wait_selftest(unsigned tries, cudaStream_t stream, int *launches)
+{
+    wait_selftest_kernel<<<1, 32, 0, stream>>>(tries);
+    ++*launches;
+    return cudaGetLastError();
+}
+
 int probe_sink_floats() { return device_sm_count() * kProbeBlocksPerSM * kProbeThreads; }
 
 // Launches probe `kind` (0 ex2, 1 packed fp32x2 FMA, 2 scalar fp32 FMA, 3 the
-// recurrence mix) and returns the operations it performs (ex2 results for 0
-// and 3, FMAs for 1 and 2) in *ops.
-cudaError_t launch_probe(int kind, int iters, float *sink, double *ops, cudaStream_t stream,
-                         int *launches)
+// recurrence mix) with `per_sm` CTAs of 8 warps per SM (1..8) and returns the
+// operations it performs (ex2 results for 0 and 3, FMAs for 1 and 2) in *ops.
+cudaError_t launch_probe(int kind, int iters, int per_sm, float *sink, double *ops,
+                         cudaStream_t stream, int *launches)
 {
-    const int blocks = device_sm_count() * kProbeBlocksPerSM;
+    const int blocks = device_sm_count() * per_sm;
     const double lanes = (double)blocks * kProbeThreads * iters;
     switch (kind) {
     case 0:

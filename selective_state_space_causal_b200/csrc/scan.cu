@@ -1501,6 +1501,13 @@ cudaError_t run_ts(const Params &p, cudaStream_t stream, int *launches)
     return cudaGetLastError();
 }
 
+}  // namespace
+
+cudaError_t launch_scan_pipe(const Params &p, bool bf16, int npt, int sched, cudaStream_t stream,
+                             int *launches);
+
+namespace {
+
 int g_forced_npt = 0, g_forced_sched = 0;
 
 // Variants: NPT states per lane; schedule 1: register prefetch, 2: TMA
@@ -1513,6 +1520,10 @@ cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n
         (void)npt; (void)sched;
         return run<Cfg<T, 4, 0, 32, 64, 1>, T>(p, s, n);
     } else {
+        if ((sched == 9 || sched == 10) && p.tok > 0) {
+            cudaError_t e = launch_scan_pipe(p, sizeof(T) == 2, npt, sched, s, n);
+            if (e != cudaErrorNotSupported) return e;
+        }
         if (sched == 3 && p.tok > 0) {
             cudaError_t e = npt == 2 ? run_ts<TsCfg<T, 2, 4, 8, 8>, T>(p, s, n)
                                      : run_ts<TsCfg<T, 4, 4, 8, 8>, T>(p, s, n);
@@ -1625,7 +1636,7 @@ void scan_variant_for(int64_t S, int64_t D, int *npt, int *sched) { pick_variant
 void set_scan_variant(int npt, int sched)
 {
     g_forced_npt = (npt == 2 || npt == 4 || npt == 8 || npt == 16) ? npt : 0;
-    g_forced_sched = (sched >= 1 && sched <= 8) ? sched : 0;
+    g_forced_sched = (sched >= 1 && sched <= 10) ? sched : 0;
 }
 
 size_t scan_order_bytes(int64_t S) { return (size_t)((S * 4 + 255) / 256) * 256; }
@@ -1641,6 +1652,8 @@ cudaError_t launch_seq_order(const int32_t *cu, int64_t S, int64_t tok, int32_t 
 
 int device_sm_count() { return sm_count(); }
 
+int read_pipe_status(bool clear);
+
 int read_scan_status(bool clear)
 {
     int v = 0;
@@ -1649,7 +1662,9 @@ int read_scan_status(bool clear)
         const int zero = 0;
         if (cudaMemcpyToSymbol(g_scan_status, &zero, sizeof(int)) != cudaSuccess) return -1;
     }
-    return v;
+    const int w = read_pipe_status(clear);
+    if (w < 0) return -1;
+    return v | w;
 }
 
 cudaError_t launch_scan(const ScanArgs &a, cudaStream_t stream, int *launches)

@@ -12,10 +12,9 @@
 #include "common.cuh"
 
 namespace ssm {
-namespace {
 
-constexpr int kN = 16;
-
+// Launch parameters of every forward scan kernel (external linkage: the
+// schedules live in more than one translation unit).
 struct Params {
     const void *u, *delta, *B, *C, *z;
     const float *A, *Dskip, *dt_bias, *h0;
@@ -26,6 +25,10 @@ struct Params {
     int64_t S, tok, D, L;
     int delta_softplus;
 };
+
+namespace {
+
+constexpr int kN = 16;
 
 constexpr size_t align128(size_t v) { return (v + 127) / 128 * 128; }
 

@@ -101,14 +101,14 @@ __device__ __forceinline__ void fence_proxy_async()
 }
 
 // Waits for phase `parity` of the barrier with a bounded number of
-// suspending tries. On timeout it sets bit `code` of *status and marks
-// `failed`, after which this thread no longer waits at all, so a kernel
-// always terminates.
+// suspending tries (kWaitTries unless a smaller count is given). On timeout it
+// sets bit `code` of *status and marks `failed`, after which this thread no
+// longer waits at all, so a kernel always terminates.
 __device__ __forceinline__ void mbar_wait(uint64_t *bar, uint32_t parity, bool &failed,
-                                          int *status, int code)
+                                          int *status, int code, unsigned tries = kWaitTries)
 {
     if (failed) return;
-    for (unsigned i = 0; i < kWaitTries; ++i) {
+    for (unsigned i = 0; i < tries; ++i) {
         uint32_t done;
         asm volatile(
             "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"

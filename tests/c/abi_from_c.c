@@ -120,11 +120,16 @@ int main(void)
 
     {
         double ops = 0.0;
-        expect("probe kind out of range", ssm_probe_rate(9, 10, wf, 1 << 20, &ops, NULL),
+        expect("probe kind out of range", ssm_probe_rate(9, 10, 64, wf, 1 << 20, &ops, NULL),
                SSM_ERR_INVALID_ARGUMENT);
-        expect("probe without a sink", ssm_probe_rate(0, 10, NULL, 0, &ops, NULL),
+        expect("probe occupancy not a multiple of 8 warps",
+               ssm_probe_rate(0, 10, 12, wf, 1 << 20, &ops, NULL), SSM_ERR_INVALID_ARGUMENT);
+        expect("probe without a sink", ssm_probe_rate(0, 10, 64, NULL, 0, &ops, NULL),
                SSM_ERR_INVALID_ARGUMENT);
     }
+
+    expect("wait self-test limit out of range", ssm_selftest_wait_timeout(0, NULL),
+           SSM_ERR_INVALID_ARGUMENT);
 
     if (failures) return 1;
     printf("ok\n");

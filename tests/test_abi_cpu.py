@@ -132,7 +132,7 @@ def test_check_cu_seqlens_host():
 def test_tuning_knob():
     for n, c in ((0, 0), (2, 1), (4, 1), (4, 2), (4, 3), (8, 2), (16, 1), (16, 2)):
         ssm.ssm_set_scan_variant(n, c)
-    for n, c in ((3, 1), (16, 9), (4, -1)):
+    for n, c in ((3, 1), (16, 11), (4, -1)):
         with pytest.raises(ssm.SsmError):
             ssm.ssm_set_scan_variant(n, c)
     ssm.ssm_set_scan_variant(0, 0)

@@ -89,7 +89,8 @@ def test_conv_no_silu(orc):
 # ---------------------------------------------------------------------------
 
 VARIANTS = [(2, 1), (2, 2), (2, 3), (4, 1), (4, 2), (4, 3), (4, 4), (4, 5), (8, 1), (8, 2), (8, 4),
-            (8, 5), (16, 1), (16, 2), (16, 4), (16, 5), (2, 6), (4, 6), (8, 6), (16, 6), (4, 7), (8, 7), (16, 7), (2, 8), (4, 8), (8, 8), (16, 8)]
+            (8, 5), (16, 1), (16, 2), (16, 4), (16, 5), (2, 6), (4, 6), (8, 6), (16, 6), (4, 7), (8, 7), (16, 7), (2, 8), (4, 8), (8, 8), (16, 8),
+            (2, 9), (4, 9), (8, 9), (4, 10), (8, 10)]
 
 
 def _scan_case(orc, seed, lens, D, bf16, variant=(0, 0), with_z=True, with_h0=True,
@@ -134,10 +135,12 @@ def test_scan_scalar_path(orc, variant):
     _scan_case(orc, 11, [50, 77], 30, True, variant=variant)
 
 
-def test_scan_options(orc):
-    _scan_case(orc, 12, [90, 40], 72, True, with_z=False, with_h0=False)
-    _scan_case(orc, 13, [90, 40], 72, False, softplus=False)
-    _scan_case(orc, 14, [90, 40], 72, True, inplace=True)
+@pytest.mark.parametrize("variant", [(0, 0), (4, 9), (8, 9), (2, 9), (4, 10)])
+def test_scan_options(orc, variant):
+    _scan_case(orc, 12, [90, 40], 72, True, with_z=False, with_h0=False, variant=variant)
+    _scan_case(orc, 13, [90, 40], 72, False, softplus=False, variant=variant)
+    _scan_case(orc, 13, [90, 40], 72, True, softplus=False, with_z=False, variant=variant)
+    _scan_case(orc, 14, [90, 40], 72, True, inplace=True, variant=variant)
 
 
 def test_scan_workspace_schedule_is_bit_identical(orc):
