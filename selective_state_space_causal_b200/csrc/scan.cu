@@ -1616,14 +1616,14 @@ void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
     const int64_t per_sm = chains / sm_count();
     int npt_auto, sched_auto;
     if (per_sm >= 8 * 640) {
-        npt_auto = 8;
-        sched_auto = 2;
-    } else if (per_sm >= 4 * 320) {
-        npt_auto = 4;
-        sched_auto = 1;
+        npt_auto = 8;           // about 20 warps per SM of 8-state lanes
+        sched_auto = 9;
+    } else if (per_sm >= 4 * 128) {
+        npt_auto = 4;           // 32-token chunks keep more loads in flight
+        sched_auto = 10;
     } else {
-        npt_auto = 2;
-        sched_auto = 8;
+        npt_auto = 2;           // too few channels to fill the SMs otherwise
+        sched_auto = 9;
     }
     *npt = g_forced_npt ? g_forced_npt : npt_auto;
     *sched = g_forced_sched ? g_forced_sched : sched_auto;

@@ -23,6 +23,12 @@
 //              state and token; after each group a transposed shuffle butterfly
 //              over the channel's TPC lanes leaves token `sub` of the group in
 //              full in lane `sub`, which applies skip and gate and stores y
+// Within a warp a channel's TPC lanes sit WCH = 32 / TPC lanes apart. Shared
+// memory, not the special-function unit, is the limit to design for: every
+// shared load shares the MIO path with ex2, and a 16-byte load costs two
+// wavefronts when groups of lanes read one address but four when neighbouring
+// lanes differ; with this lane order a token's B and C rows cost two each and
+// its (delta, delta*u) pair (8 bytes) two.
 // The state-free part of a group (shared loads, exponent arguments, ex2,
 // delta*u*B) is issued one group ahead of the state chain, so a warp keeps a
 // group's exponentials in flight while it runs the previous group's chain.
@@ -67,17 +73,20 @@ __device__ __forceinline__ float rcp_approx(float x)
     return r;
 }
 
-// Shared loads straight into packed fp32x2 registers (no register moves to
-// form the pairs): one 16-byte load as two pairs, one 8-byte load as a pair.
+// Shared loads as packed fp32x2 pairs: one 16-byte load as two pairs, one
+// 8-byte load as a pair. Plain loads (not inline assembly), so the compiler
+// addresses them off a register with constant offsets and keeps the pairs in
+// the load's aligned registers.
 __device__ __forceinline__ void lds_2x2(const void *p, f32x2 &a, f32x2 &b)
 {
-    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(saddr(p)));
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    a = pk2(v.x, v.y);
+    b = pk2(v.z, v.w);
 }
 __device__ __forceinline__ f32x2 lds_x2(const void *p)
 {
-    f32x2 a;
-    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(a) : "r"(saddr(p)));
-    return a;
+    const float2 v = *reinterpret_cast<const float2 *>(p);
+    return pk2(v.x, v.y);
 }
 
 // y[...] = v when pred, as one predicated store.
@@ -103,7 +112,11 @@ struct PipeCfg {
     static constexpr size_t RAW_ACT = sizeof(T) * TCH * CH;
     static constexpr size_t RAW_BC = sizeof(T) * TCH * kN;
     static constexpr size_t STAGE = 3 * align128(RAW_ACT) + 2 * align128(RAW_BC);
-    static constexpr size_t DD_BUF = 16 * (size_t)TCH * CH;  // (delta, delta, delta*u, delta*u) [t][c]
+    static constexpr int WCH = 32 / TPC;                     // channels per warp
+    // (delta, delta*u) of (token t, channel c) at t * ROWD + c: 64 bytes of
+    // padding per row put the pre-pass's four-token stores on two bank halves
+    static constexpr int ROWD = CH + 8;
+    static constexpr size_t DD_BUF = 8 * (size_t)TCH * ROWD;
     static constexpr size_t BC_BUF = 4 * (size_t)TCH * kN;
     static constexpr int RS = 4;                             // raw tile stages
     static constexpr size_t OFF_RAW = 0;
@@ -112,13 +125,17 @@ struct PipeCfg {
     static constexpr size_t OFF_C = align128(OFF_B + 2 * BC_BUF);
     static constexpr size_t OFF_BAR = align128(OFF_C + 2 * BC_BUF);
     static constexpr size_t SMEM = OFF_BAR + 8 * RS;
-    static constexpr int PE = 16 / sizeof(T);                // B (or C) elements per 16-byte piece
-    static constexpr int BCP = TCH * kN / PE;                // 16-byte B (or C) pieces per chunk
+    // B and C rows are widened to fp32 in pieces of PE elements, one or more
+    // pieces per thread (at most 16 bytes of raw data a piece)
+    static constexpr int PE = (TCH * kN / THREADS) < (16 / (int)sizeof(T)) ? (TCH * kN / THREADS)
+                                                                           : (16 / (int)sizeof(T));
+    static constexpr int BCP = TCH * kN / PE;                // pieces of B (or C) per chunk
     static constexpr int BPT = BCP / THREADS;                // pieces per thread
+    static constexpr int PW = PE * sizeof(T) / 4;            // 32-bit words of a raw piece
     static_assert(NPT == 2 || NPT == 4 || NPT == 8, "states per lane");
     static_assert(G % 2 == 0, "token pairs per lane");
     static_assert(BCP % THREADS == 0, "whole B and C pieces per thread");
-    static_assert(PE % 4 == 0, "B and C pieces are whole float4 rows");
+    static_assert(PE >= 2 && (PE & (PE - 1)) == 0, "B and C pieces of 2, 4 or 8 elements");
     static_assert(TCH % TPC == 0, "whole token groups per chunk");
     static_assert(RAW_ACT % 128 == 0 && RAW_BC % 128 == 0, "TMA tiles stay 128-byte aligned");
     static_assert((CH * sizeof(T)) % 16 == 0, "TMA box rows are whole 16-byte units");
@@ -213,9 +230,9 @@ struct Pipe {
                          : 3 * align128(K::RAW_ACT) + (size_t)(which - 3) * align128(K::RAW_BC);
         return reinterpret_cast<T *>(smem + off);
     }
-    __device__ __forceinline__ float4 *sDD(int buf) const
+    __device__ __forceinline__ float2 *sDD(int buf) const
     {
-        return reinterpret_cast<float4 *>(smem + K::OFF_DD + buf * K::DD_BUF);
+        return reinterpret_cast<float2 *>(smem + K::OFF_DD + buf * K::DD_BUF);
     }
     __device__ __forceinline__ float *sB(int buf) const
     {
@@ -229,7 +246,7 @@ struct Pipe {
     // ---- pre-pass of one chunk: loads at the top, stores at the bottom -------
     struct Pre {
         float dt[G], u[G], z[G];
-        uint4 rb[K::BPT], rc[K::BPT];  // 16-byte pieces of B and C, raw
+        uint32_t rb[K::BPT][K::PW], rc[K::BPT][K::PW];  // pieces of B and C, raw
     };
 
     __device__ __forceinline__ void pre_load(Pre &q, int stage) const
@@ -244,8 +261,20 @@ struct Pipe {
         }
 #pragma unroll
         for (int i = 0; i < K::BPT; ++i) {
-            q.rb[i] = reinterpret_cast<const uint4 *>(raw(stage, 3))[tid + i * THREADS];
-            q.rc[i] = reinterpret_cast<const uint4 *>(raw(stage, 4))[tid + i * THREADS];
+            const uint32_t *rb = reinterpret_cast<const uint32_t *>(raw(stage, 3)) + (tid + i * THREADS) * K::PW;
+            const uint32_t *rc = reinterpret_cast<const uint32_t *>(raw(stage, 4)) + (tid + i * THREADS) * K::PW;
+            if constexpr (K::PW == 4) {
+                const uint4 b4 = *reinterpret_cast<const uint4 *>(rb), c4 = *reinterpret_cast<const uint4 *>(rc);
+                q.rb[i][0] = b4.x; q.rb[i][1] = b4.y; q.rb[i][2] = b4.z; q.rb[i][3] = b4.w;
+                q.rc[i][0] = c4.x; q.rc[i][1] = c4.y; q.rc[i][2] = c4.z; q.rc[i][3] = c4.w;
+            } else if constexpr (K::PW == 2) {
+                const uint2 b2 = *reinterpret_cast<const uint2 *>(rb), c2 = *reinterpret_cast<const uint2 *>(rc);
+                q.rb[i][0] = b2.x; q.rb[i][1] = b2.y;
+                q.rc[i][0] = c2.x; q.rc[i][1] = c2.y;
+            } else {
+                q.rb[i][0] = *rb;
+                q.rc[i][0] = *rc;
+            }
         }
     }
 
@@ -254,7 +283,7 @@ struct Pipe {
     template <int BUF, bool MASK>
     __device__ __forceinline__ void pre_pair(const Pre &q, int g, int nt)
     {
-        float4 *dd = sDD(BUF);
+        float2 *dd = sDD(BUF);
         const f32x2 v = add2(pk2(q.dt[g], q.dt[g + 1]), pk2(dtb, dtb));
         const f32x2 u = pk2(q.u[g], q.u[g + 1]);
         f32x2 d, gt = pk2(1.0f, 1.0f);
@@ -278,8 +307,8 @@ struct Pipe {
             d1 = l1 ? d1 : 0.f;
             x1 = l1 ? x1 : 0.f;
         }
-        dd[(sub + TPC * g) * CH + cl] = make_float4(d0, d0, x0, x0);
-        dd[(sub + TPC * (g + 1)) * CH + cl] = make_float4(d1, d1, x1, x1);
+        dd[(sub + TPC * g) * K::ROWD + cl] = make_float2(d0, x0);
+        dd[(sub + TPC * (g + 1)) * K::ROWD + cl] = make_float2(d1, x1);
     }
 
     // B and C rows to fp32 for chunk buffer BUF (tokens past the sequence end
@@ -289,21 +318,25 @@ struct Pipe {
     {
 #pragma unroll
         for (int i = 0; i < K::BPT; ++i) {
-            float4 *b4 = reinterpret_cast<float4 *>(sB(BUF)) + (tid + i * THREADS) * (K::PE / 4);
-            float4 *c4 = reinterpret_cast<float4 *>(sC(BUF)) + (tid + i * THREADS) * (K::PE / 4);
-            if constexpr (sizeof(T) == 2) {
-                const uint4 rb = q.rb[i], rc = q.rc[i];
-                b4[0] = make_float4(__uint_as_float(rb.x << 16), __uint_as_float(rb.x & 0xffff0000u),
-                                    __uint_as_float(rb.y << 16), __uint_as_float(rb.y & 0xffff0000u));
-                b4[1] = make_float4(__uint_as_float(rb.z << 16), __uint_as_float(rb.z & 0xffff0000u),
-                                    __uint_as_float(rb.w << 16), __uint_as_float(rb.w & 0xffff0000u));
-                c4[0] = make_float4(__uint_as_float(rc.x << 16), __uint_as_float(rc.x & 0xffff0000u),
-                                    __uint_as_float(rc.y << 16), __uint_as_float(rc.y & 0xffff0000u));
-                c4[1] = make_float4(__uint_as_float(rc.z << 16), __uint_as_float(rc.z & 0xffff0000u),
-                                    __uint_as_float(rc.w << 16), __uint_as_float(rc.w & 0xffff0000u));
-            } else {
-                b4[0] = *reinterpret_cast<const float4 *>(&q.rb[i]);
-                c4[0] = *reinterpret_cast<const float4 *>(&q.rc[i]);
+            float fb[K::PE], fc[K::PE];
+#pragma unroll
+            for (int w = 0; w < K::PW; ++w) {
+                if constexpr (sizeof(T) == 2) {
+                    fb[2 * w] = __uint_as_float(q.rb[i][w] << 16);
+                    fb[2 * w + 1] = __uint_as_float(q.rb[i][w] & 0xffff0000u);
+                    fc[2 * w] = __uint_as_float(q.rc[i][w] << 16);
+                    fc[2 * w + 1] = __uint_as_float(q.rc[i][w] & 0xffff0000u);
+                } else {
+                    fb[w] = __uint_as_float(q.rb[i][w]);
+                    fc[w] = __uint_as_float(q.rc[i][w]);
+                }
+            }
+            float *b = sB(BUF) + (tid + i * THREADS) * K::PE;
+            float *c = sC(BUF) + (tid + i * THREADS) * K::PE;
+#pragma unroll
+            for (int e = 0; e < K::PE; e += 2) {
+                *reinterpret_cast<float2 *>(b + e) = make_float2(fb[e], fb[e + 1]);
+                *reinterpret_cast<float2 *>(c + e) = make_float2(fc[e], fc[e + 1]);
             }
         }
     }
@@ -331,10 +364,11 @@ struct Pipe {
 
     __device__ __forceinline__ void front_tok(Tok &E, int buf, int t) const
     {
-        const float4 *dd = sDD(buf);
+        const float2 *dd = sDD(buf);
         const float *b = sB(buf);
-        f32x2 dv, xv, bb[NP];
-        lds_2x2(dd + t * CH + cl, dv, xv);
+        f32x2 bb[NP];
+        const float2 v = dd[t * K::ROWD + cl];
+        const f32x2 dv = pk2(v.x, v.x), xv = pk2(v.y, v.y);
 #pragma unroll
         for (int j = 0; j < NP; j += 2) {
             if (j + 1 < NP) lds_2x2(b + t * kN + sub * NPT + 2 * j, bb[j], bb[j + 1]);
@@ -375,7 +409,7 @@ struct Pipe {
 
     // The butterfly over the channel's lanes for a group's partials, then
     // skip, gate and store of token g * TPC + sub.
-    template <int BUF>
+    template <int BUF, bool FULL>
     __device__ __forceinline__ void group_out(float (&P)[TPC], int g, int64_t t0, int nt) const
     {
         // transposed butterfly: after log2(TPC) steps P[0] of lane `sub` is
@@ -387,18 +421,23 @@ struct Pipe {
             for (int i = 0; i < w; ++i) {
                 const float send = upper ? P[i] : P[i + w];
                 const float keep = upper ? P[i + w] : P[i];
-                P[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                P[i] = keep + __shfl_xor_sync(0xffffffffu, send, w * K::WCH);
             }
         }
         const int t = g * TPC + sub;
-        stg_if(static_cast<T *>(p.y) + (t0 + t) * p.D + c0,
-               from_f32<T>((P[0] + gdu[BUF][g]) * gg[BUF][g]), t < nt && cvalid);
+        const T yv = from_f32<T>((P[0] + gdu[BUF][g]) * gg[BUF][g]);
+        T *dst = static_cast<T *>(p.y) + (t0 + t) * p.D + c0;
+        if (FULL) {
+            if (cvalid) *dst = yv;
+        } else {
+            if (cvalid && t < nt) *dst = yv;
+        }
     }
 
     // Iteration: the recurrence of the chunk in buffer BUF (nt valid tokens
     // from t0) and, if PRE, the pre-pass of the next chunk (raw stage `stage`,
     // buffer BUF ^ 1, ntn valid tokens).
-    template <int BUF, bool PRE, bool MASK>
+    template <int BUF, bool PRE, bool MASK, bool FULL>
     __device__ __forceinline__ void iteration(int64_t t0, int nt, int ntn, int stage)
     {
         Pre q;
@@ -414,7 +453,7 @@ struct Pipe {
             if (t + LA < TCH) front_tok(E[(t + LA) % (2 * LA)], BUF, t + LA);
             if (t + 1 < TCH) load_c(C[(t + 1) & 1], BUF, t + 1);
             P[t % TPC] = chain_tok(E[t % (2 * LA)], C[t & 1]);
-            if (t % TPC == TPC - 1) group_out<BUF>(P, t / TPC, t0, nt);
+            if (t % TPC == TPC - 1) group_out<BUF, FULL>(P, t / TPC, t0, nt);
             // the next chunk's pre-pass arithmetic, spread over the chunk
             if (PRE && t % (TCH / (G / 2)) == TCH / (G / 2) - 1)
                 pre_pair<BUF ^ 1, MASK>(q, 2 * (t / (TCH / (G / 2))), ntn);
@@ -433,10 +472,10 @@ __device__ __forceinline__ void cta_sync()
     else __syncthreads();
 }
 
-// At least 11 resident one-warp CTAs per SM (up to 186 registers a thread):
-// enough for every (sequence, channel) warp of the Mamba-130M layer at once.
+// At least three 4-warp CTAs per SM (up to 168 registers a thread): every
+// (sequence, channel) warp of the Mamba-130M layer resident at once.
 template <class K, typename T, bool SP, bool GZ>
-__global__ void __launch_bounds__(K::THREADS, K::THREADS == 32 ? 11 : 5)
+__global__ void __launch_bounds__(K::THREADS, 3)
 scan_pipe_kernel(const Params p, const __grid_constant__ Maps m)
 {
     constexpr int TCH = K::TCH, CH = K::CH, NPT = K::NPT, TPC = K::TPC;
@@ -445,9 +484,12 @@ scan_pipe_kernel(const Params p, const __grid_constant__ Maps m)
     uint64_t *const bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
 
     P.tid = threadIdx.x;
+    // lane = sub * WCH + channel-in-warp: a channel's TPC lanes sit WCH apart,
+    // so shared loads of B and C rows (one address per `sub`) serve groups of
+    // WCH neighbouring lanes in two wavefronts
     P.lane = P.tid & 31;
-    P.cl = P.tid / TPC;
-    P.sub = P.tid % TPC;
+    P.cl = (P.tid >> 5) * K::WCH + P.lane % K::WCH;
+    P.sub = P.lane / K::WCH;
     P.cbase = (int64_t)blockIdx.x * CH;
     P.c0 = P.cbase + P.cl;
     P.cvalid = P.c0 < p.D;
@@ -520,10 +562,10 @@ scan_pipe_kernel(const Params p, const __grid_constant__ Maps m)
         }
         if (k + 1 < nch) {
             wait_raw(k + 1);
-            if (k + 2 < nch) P.template iteration<BUF, true, false>(t0, TCH, TCH, (k + 1) % K::RS);
-            else P.template iteration<BUF, true, true>(t0, TCH, ntok(k + 1), (k + 1) % K::RS);
+            if (k + 2 < nch) P.template iteration<BUF, true, false, true>(t0, TCH, TCH, (k + 1) % K::RS);
+            else P.template iteration<BUF, true, true, true>(t0, TCH, ntok(k + 1), (k + 1) % K::RS);
         } else {
-            P.template iteration<BUF, false, false>(t0, ntok(k), 0, 0);
+            P.template iteration<BUF, false, false, false>(t0, ntok(k), 0, 0);
         }
         cta_sync<K::THREADS>();
     };
@@ -595,23 +637,22 @@ int read_pipe_status(bool clear)
 
 // Schedules 9 and 10 (16- and 32-token chunks) for 16-byte aligned rows (D a
 // multiple of 8 for bf16, of 4 for fp32); cudaErrorNotSupported when the
-// tensor maps cannot be encoded. A CTA is one warp (4 or 8 states per lane)
-// or two (2 states per lane, whose one-warp tile would be 8 bytes wide).
+// tensor maps cannot be encoded. CTAs of four warps.
 cudaError_t launch_scan_pipe(const Params &p, bool bf16, int npt, int sched, cudaStream_t stream,
                              int *launches)
 {
     const bool lng = sched == 10;
     if (bf16) {
         using T = __nv_bfloat16;
-        if (npt == 8) return lng ? run_pipe<PipeCfg<T, 8, 16, 32>, T>(p, stream, launches)
-                                 : run_pipe<PipeCfg<T, 8, 16, 16>, T>(p, stream, launches);
-        if (npt == 2) return run_pipe<PipeCfg<T, 2, 8, 32>, T>(p, stream, launches);
-        return lng ? run_pipe<PipeCfg<T, 4, 8, 32>, T>(p, stream, launches)
-                   : run_pipe<PipeCfg<T, 4, 8, 16>, T>(p, stream, launches);
+        if (npt == 8) return lng ? run_pipe<PipeCfg<T, 8, 64, 32>, T>(p, stream, launches)
+                                 : run_pipe<PipeCfg<T, 8, 64, 16>, T>(p, stream, launches);
+        if (npt == 2) return run_pipe<PipeCfg<T, 2, 16, 32>, T>(p, stream, launches);
+        return lng ? run_pipe<PipeCfg<T, 4, 32, 32>, T>(p, stream, launches)
+                   : run_pipe<PipeCfg<T, 4, 32, 16>, T>(p, stream, launches);
     }
-    if (npt == 8) return run_pipe<PipeCfg<float, 8, 16, 16>, float>(p, stream, launches);
-    if (npt == 2) return run_pipe<PipeCfg<float, 2, 8, 32>, float>(p, stream, launches);
-    return run_pipe<PipeCfg<float, 4, 8, 16>, float>(p, stream, launches);
+    if (npt == 8) return run_pipe<PipeCfg<float, 8, 64, 16>, float>(p, stream, launches);
+    if (npt == 2) return run_pipe<PipeCfg<float, 2, 16, 32>, float>(p, stream, launches);
+    return run_pipe<PipeCfg<float, 4, 32, 16>, float>(p, stream, launches);
 }
 
 }  // namespace ssm

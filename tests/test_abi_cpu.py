@@ -162,17 +162,18 @@ def test_bwd_variant_knob_and_choice():
 
 def test_variant_choice():
     """The automatic choice follows (sequence, channel, state) recurrences per
-    SM (148 SMs when no device is visible): 8 states per lane with TMA staging
-    when the GPU holds about 20 warps per SM of them, else 4 states per lane
-    with register prefetch while that gives about 10 warps per SM, else 2 states
-    per lane in the single-stage TMA layout. A forced variant is reported as
+    SM (148 SMs when no device is visible): 8 states per lane in the pipelined
+    kernel with 16-token chunks when the GPU holds about 20 warps per SM of
+    them, else 4 states per lane with 32-token chunks while that still gives
+    every SM a block, else 2 states per lane. A forced variant is reported as
     forced."""
     ssm.ssm_set_scan_variant(0, 0)
-    assert ssm.ssm_scan_variant_for(8, 1536) == (4, 1)      # 8 x 2048 x 1536 layer
-    assert ssm.ssm_scan_variant_for(43, 5120) == (8, 2)     # packed 65536 x 5120
-    assert ssm.ssm_scan_variant_for(1, 8192) == (2, 8)      # one 8192-channel sequence
-    assert ssm.ssm_scan_variant_for(4, 8192) == (4, 1)
-    assert ssm.ssm_scan_variant_for(1, 32) == (2, 8)
+    assert ssm.ssm_scan_variant_for(8, 1536) == (4, 10)     # 8 x 2048 x 1536 layer
+    assert ssm.ssm_scan_variant_for(43, 5120) == (8, 9)     # packed 65536 x 5120
+    assert ssm.ssm_scan_variant_for(1, 8192) == (4, 10)     # one 8192-channel sequence
+    assert ssm.ssm_scan_variant_for(4, 8192) == (4, 10)
+    assert ssm.ssm_scan_variant_for(1, 2048) == (2, 9)
+    assert ssm.ssm_scan_variant_for(1, 32) == (2, 9)
     ssm.ssm_set_scan_variant(16, 7)
     assert ssm.ssm_scan_variant_for(1, 32) == (16, 7)
     ssm.ssm_set_scan_variant(0, 0)

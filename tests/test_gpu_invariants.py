@@ -50,7 +50,8 @@ def _acts(seed, tok, D):
     return {k: dev(v, BF) for k, v in a.items()}
 
 
-@pytest.mark.parametrize("variant", [(4, 1), (4, 2), (4, 3), (2, 3), (8, 2), (16, 2), (4, 6), (8, 6), (4, 7), (8, 7), (2, 8), (4, 8)])
+@pytest.mark.parametrize("variant", [(4, 1), (4, 2), (4, 3), (2, 3), (8, 2), (16, 2), (4, 6), (8, 6), (4, 7), (8, 7), (2, 8), (4, 8),
+                                     (2, 9), (4, 9), (8, 9), (4, 10), (8, 10)])
 def test_pack_equals_separate(variant):
     ssm.ssm_set_scan_variant(*variant)
     lens = [100, 0, 3, 1, 257, 64]
