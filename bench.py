@@ -294,6 +294,26 @@ def scan_roofline(kernel, variant, exps, bytes_, kernel_ms, mufu, peaks, workloa
             "hbm_peak_gbs": peaks["hbm_gbs"], "hbm_peak_source": peaks["source"]}
 
 
+def conv_bytes(tok, D, S, state_in):
+    """Algorithmic bytes of one bf16 conv call: x in and xc out (2 B each per
+    token and channel), the conv state out (and in), 3 bf16 per sequence and
+    channel, and the fp32 weights and bias."""
+    return tok * D * 4 + S * D * 6 * (2 if state_in else 1) + D * 20
+
+
+def conv_roofline(bytes_, kernel_ms, peaks, workload, two_launches=False):
+    """The roofline block of a conv call: bound by HBM. With the state updated
+    in place the state output is a second, small launch, timed with it."""
+    achieved = bytes_ / (kernel_ms * 1e-3) / 1e9
+    kernel = "conv1d_tma_kernel" + (" + conv_state_out_kernel" if two_launches else "")
+    return {"kernel": kernel, "bound": "hbm", "unit": "GB/s", "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"], "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "peak_source": peaks["source"],
+            "traffic": recorded_traffic("conv1d_tma_kernel", workload,
+                                        source_sha("conv1d.cu", "common.cuh", "tma.cuh")),
+            "kernel_ms": round(kernel_ms, 5), "algorithmic_bytes_per_launch": int(bytes_)}
+
+
 def scan_bytes(tok, D, S):
     """Algorithmic bytes of one bf16 scan call: u, dt, z in and y out (2 B each
     per token and channel), B and C (64 B per token), the final state (64 B
@@ -335,15 +355,17 @@ class LongCtxStep:
         self.h.zero_()
         for j in range(self.nch):
             sl = slice(j * self.chunk, (j + 1) * self.chunk)
+            if ev is not None:
+                ev[j][0].record()
             ssm.ssm_causal_conv1d(a["x"][sl], self.xc, ly.w, bias=ly.b, conv_state_in=self.cs,
                                   conv_state_out=self.cs)
             if ev is not None:
-                ev[j][0].record()
+                ev[j][1].record()
             ssm.ssm_selective_scan_fwd(self.xc, a["dt"][sl], ly.A, a["B"][sl], a["C"][sl],
                                        self.y[sl], Dskip=ly.Dskip, z=a["z"][sl],
                                        dt_bias=ly.dt_bias, h0=self.h, h_final=self.h)
             if ev is not None:
-                ev[j][1].record()
+                ev[j][2].record()
         d = self.dec
         ssm.ssm_selective_state_update(self.cs, self.h, d["x"], d["dt"], d["B"], d["C"], self.yd,
                                        ly.w, ly.A, z=d["z"], conv_b=ly.b, Dskip=ly.Dskip,
@@ -357,7 +379,7 @@ def bench_headline(args, world, peaks, rank_dev, mufu):
     for _ in range(args.warmup):
         st.run()
     K = args.steps
-    evs = [[_events(2) for _ in range(st.nch)] for _ in range(K)]
+    evs = [[_events(3) for _ in range(st.nch)] for _ in range(K)]
     start, stop = _events(2)
     launches0 = st.ssm.ssm_launch_count()
     clocks = ClockSampler(rank_dev)
@@ -374,7 +396,8 @@ def bench_headline(args, world, peaks, rank_dev, mufu):
     if st.ssm.ssm_device_status() != 0:
         raise RuntimeError("a bounded device wait timed out during the timed region")
     ms = start.elapsed_time(stop) / K
-    scan_ms = sum(e[0].elapsed_time(e[1]) for row in evs for e in row) / (K * st.nch)
+    conv_ms = sum(e[0].elapsed_time(e[1]) for row in evs for e in row) / (K * st.nch)
+    scan_ms = sum(e[1].elapsed_time(e[2]) for row in evs for e in row) / (K * st.nch)
     ms_max = _max_over_ranks(ms, world)
     value = whole_job_rate(st.units(), world, ms_max)
     sha = source_sha(*SCAN_SOURCES)
@@ -386,6 +409,8 @@ def bench_headline(args, world, peaks, rank_dev, mufu):
     res = {"value": value, "ms_per_step": ms_max, "step_ms_this_rank": ms, "roofline": roofline,
            "clocks": clk, "gpu_launches": int(launches),
            "scan_ms_per_step": round(scan_ms * st.nch, 4),
+           "conv_roofline": conv_roofline(conv_bytes(st.chunk, st.D, 1, True), conv_ms, peaks,
+                                          "longctx_call_8192x8192", two_launches=True),
            "launches_per_step": launches / K}
     if not args.no_e2e:
         res["e2e"] = e2e_longctx(st, world, max(3, K // 4))
@@ -532,14 +557,16 @@ class LayerStep:
         d = dec_inputs if dec_inputs is not None else self.dec[i % self.SETS]
         y = self.y if y is None else y
         yd = self.yd if yd is None else yd
+        if ev is not None:
+            ev[0].record()
         ssm.ssm_causal_conv1d(a["x"], self.xc, ly.w, bias=ly.b, S=self.Bn,
                               conv_state_out=self.cs)
         if ev is not None:
-            ev[0].record()
+            ev[1].record()
         ssm.ssm_selective_scan_fwd(self.xc, a["dt"], ly.A, a["B"], a["C"], y, Dskip=ly.Dskip,
                                    z=a["z"], dt_bias=ly.dt_bias, h_final=self.h, S=self.Bn)
         if ev is not None:
-            ev[1].record()
+            ev[2].record()
         ssm.ssm_selective_state_update(self.cs, self.h, d["x"], d["dt"], d["B"], d["C"], yd,
                                        ly.w, ly.A, z=d["z"], conv_b=ly.b, Dskip=ly.Dskip,
                                        dt_bias=ly.dt_bias)
@@ -600,7 +627,7 @@ def bench_layer(args, world, peaks, mufu):
     for i in range(args.warmup):
         st.run(i)
     K = max(args.steps, 50)
-    evs = [_events(2) for _ in range(K)]
+    evs = [_events(3) for _ in range(K)]
     s0, s1 = _events(2)
     l0 = st.ssm.ssm_launch_count()
     _barrier_sync(world)
@@ -611,13 +638,16 @@ def bench_layer(args, world, peaks, mufu):
     _barrier_sync(world)
     launches = st.ssm.ssm_launch_count() - l0
     ms = _max_over_ranks(s0.elapsed_time(s1) / K, world)
-    scan_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    conv_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    scan_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
     variant = st.ssm.ssm_scan_variant_for(st.Bn, st.D)
     res = {"value": whole_job_rate(st.units(), world, ms), "unit": UNIT, "ms_per_step": ms,
            "gpu_launches_per_step": launches / K,
            "roofline": scan_roofline(SCAN_KERNELS.get(variant[1], "scan_kernel"), variant,
                                      st.tok * st.D * N_STATE, scan_bytes(st.tok, st.D, st.Bn),
                                      scan_ms, mufu, peaks, LAYER, source_sha(*SCAN_SOURCES)),
+           "conv_roofline": conv_roofline(conv_bytes(st.tok, st.D, st.Bn, False), conv_ms, peaks,
+                                          LAYER),
            "step": "causal_conv1d+silu -> selective_scan (h_final) -> 1 decode step; "
                    "4 rotating input sets (~600 MB) larger than L2"}
 
@@ -695,14 +725,16 @@ def bench_packed(args, world, peaks, mufu):
                      device="cuda")
 
     def step(ev=None, src=a, yy=y):
-        ssm.ssm_causal_conv1d(src["x"], xc, ly.w, bias=ly.b, cu_seqlens=cu, conv_state_out=cs)
         if ev:
             ev[0].record()
+        ssm.ssm_causal_conv1d(src["x"], xc, ly.w, bias=ly.b, cu_seqlens=cu, conv_state_out=cs)
+        if ev:
+            ev[1].record()
         ssm.ssm_selective_scan_fwd(xc, src["dt"], ly.A, src["B"], src["C"], yy, Dskip=ly.Dskip,
                                    z=src["z"], dt_bias=ly.dt_bias, h_final=h, cu_seqlens=cu,
                                    workspace=ws)
         if ev:
-            ev[1].record()
+            ev[2].record()
 
     def fused(ev=None):
         if ev:
@@ -713,10 +745,11 @@ def bench_packed(args, world, peaks, mufu):
         if ev:
             ev[1].record()
 
-    def timed(fn, n):
+    def timed(fn, n, marks):
+        """Step time and the mean time between consecutive marks."""
         for _ in range(3):
             fn()
-        evs = [_events(2) for _ in range(n)]
+        evs = [_events(marks) for _ in range(n)]
         s0, s1 = _events(2)
         _barrier_sync(world)
         s0.record()
@@ -725,17 +758,18 @@ def bench_packed(args, world, peaks, mufu):
         s1.record()
         _barrier_sync(world)
         return (_max_over_ranks(s0.elapsed_time(s1) / n, world),
-                sum(e[0].elapsed_time(e[1]) for e in evs) / n)
+                [sum(e[m].elapsed_time(e[m + 1]) for e in evs) / n for m in range(marks - 1)])
 
     n = max(5, args.steps)
-    ms, scan_ms = timed(step, n)
-    fms, fk = timed(fused, n)
+    ms, (conv_ms, scan_ms) = timed(step, n, 3)
+    fms, (fk,) = timed(fused, n, 2)
     variant = ssm.ssm_scan_variant_for(S, D)
     res = {"value": whole_job_rate(tot * D, world, ms), "unit": UNIT, "ms_per_step": ms,
            "sequences": S,
            "roofline": scan_roofline(SCAN_KERNELS.get(variant[1], "scan_kernel"), variant,
                                      tot * D * N_STATE, scan_bytes(tot, D, S), scan_ms, mufu,
                                      peaks, PACKED, source_sha(*SCAN_SOURCES)),
+           "conv_roofline": conv_roofline(conv_bytes(tot, D, S, False), conv_ms, peaks, PACKED),
            "fused_step": {"value": whole_job_rate(tot * D, world, fms), "ms_per_step": fms,
                           "conv_scan_kernel_ms": round(fk, 5)},
            "step": "conv1d+silu -> selective_scan over 43 packed sequences (longest first)"}
@@ -793,20 +827,27 @@ def bench_decode(args, world, peaks, mufu):
     yd = torch.empty((Bt, D), dtype=bf, device="cuda")
     s0, s1 = _events(2)
     total_ms, done, kernel_ms = 0.0, 0, []
+    def one(s):
+        ssm.ssm_selective_state_update(cs, h, s["x"], s["dt"], s["B"], s["C"], yd, ly.w, ly.A,
+                                       z=s["z"], conv_b=ly.b, Dskip=ly.Dskip, dt_bias=ly.dt_bias)
+
     for b0 in range(0, steps, block):
         blk = [synth.device_activations(5000 + b0 + i, Bt, D) for i in range(block)]
-        evs = [_events(2) for _ in range(block)]
+        # the steps/s value: the block back to back, no events between steps
         _barrier_sync(world)
         s0.record()
-        for s, ev in zip(blk, evs):
-            ev[0].record()
-            ssm.ssm_selective_state_update(cs, h, s["x"], s["dt"], s["B"], s["C"], yd, ly.w, ly.A,
-                                           z=s["z"], conv_b=ly.b, Dskip=ly.Dskip,
-                                           dt_bias=ly.dt_bias)
-            ev[1].record()
+        for s in blk:
+            one(s)
         s1.record()
         _barrier_sync(world)
         total_ms += _max_over_ranks(s0.elapsed_time(s1), world)
+        # the kernel time: the same block again, an event pair around each step
+        evs = [_events(2) for _ in range(block)]
+        for s, ev in zip(blk, evs):
+            ev[0].record()
+            one(s)
+            ev[1].record()
+        torch.cuda.synchronize()
         kernel_ms += [e[0].elapsed_time(e[1]) for e in evs]
         done += block
         del blk
@@ -1172,9 +1213,13 @@ def profile_scan(kind):
         tok, D, cu, S = 16384, 1536, None, 8
     elif kind in ("long", "conv_long"):
         tok, D, cu, S = 8192, 8192, None, 1
-    else:  # a 16384-token slice of the packed workload's length mix
+    else:  # a 16384-token slice of the packed workload's length mix, in the
+        # variant the library picks for the whole packed workload
         lens = synth.sample_lengths(0, 16384)
         tok, D, cu, S = 16384, 5120, synth.cu_from_lengths(lens), len(lens)
+        w = synth.WORKLOADS[PACKED]
+        full = len(synth.sample_lengths(0, w["total"], w["len_lo"], w["len_hi"]))
+        ssm.ssm_set_scan_variant(*ssm.ssm_scan_variant_for(full, D))
     ly = Layer(D)
     cu_d = torch.from_numpy(cu).cuda() if cu is not None else None
     a = synth.device_activations(0, tok, D)
@@ -1321,7 +1366,8 @@ def main():
                        "parallelism": f"replicas x{world}"},
             "roofline": res["roofline"], "mufu_peak": mufu, "clocks": res["clocks"],
             "e2e": res.get("e2e"), "gpu_launches": res["gpu_launches"],
-            "launches_per_step": res["launches_per_step"],
+            "launches_per_step": res["launches_per_step"], "conv_roofline": res["conv_roofline"],
+            "scan_ms_per_step": res["scan_ms_per_step"],
             "cpu_baseline": cpu, "workloads": workloads,
         }
         print(json.dumps(line), flush=True)
