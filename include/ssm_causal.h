@@ -99,7 +99,8 @@ unsigned long long ssm_launch_count(void);
  * 4, 8 or 16 states per lane; 8: the layout of schedule 1 with TMA staging;
  * 9 and 10: the chunk-pipelined kernel, TMA staging four stages deep, the next
  * chunk's per-token work interleaved with this chunk's recurrence, 16- and
- * 32-token chunks, 2, 4 or 8 states per lane; the library's choice).
+ * 32-token chunks, 2, 4 or 8 states per lane; 11: schedule 10 at 4 states
+ * per lane with the register budget of two CTAs per SM; the library's choice).
  * 0 lets the library choose. Applies to the
  * 16-byte vector path; the scalar path always uses 4 states per lane and
  * register prefetch. A variant whose alignment needs the inputs do not meet

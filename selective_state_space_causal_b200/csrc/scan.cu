@@ -1520,7 +1520,7 @@ cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n
         (void)npt; (void)sched;
         return run<Cfg<T, 4, 0, 32, 64, 1>, T>(p, s, n);
     } else {
-        if ((sched == 9 || sched == 10) && p.tok > 0) {
+        if (sched >= 9 && sched <= 11 && p.tok > 0) {
             cudaError_t e = launch_scan_pipe(p, sizeof(T) == 2, npt, sched, s, n);
             if (e != cudaErrorNotSupported) return e;
         }
@@ -1620,7 +1620,8 @@ void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
         sched_auto = 9;
     } else if (per_sm >= 4 * 128) {
         npt_auto = 4;           // 32-token chunks keep more loads in flight
-        sched_auto = 10;
+        // at most two CTAs per SM: the register budget of two
+        sched_auto = S * ((D + 31) / 32) <= 2 * (int64_t)sm_count() ? 11 : 10;
     } else {
         npt_auto = 2;           // too few channels to fill the SMs otherwise
         sched_auto = 9;
@@ -1636,7 +1637,7 @@ void scan_variant_for(int64_t S, int64_t D, int *npt, int *sched) { pick_variant
 void set_scan_variant(int npt, int sched)
 {
     g_forced_npt = (npt == 2 || npt == 4 || npt == 8 || npt == 16) ? npt : 0;
-    g_forced_sched = (sched >= 1 && sched <= 10) ? sched : 0;
+    g_forced_sched = (sched >= 1 && sched <= 11) ? sched : 0;
 }
 
 size_t scan_order_bytes(int64_t S) { return (size_t)((S * 4 + 255) / 256) * 256; }

@@ -102,9 +102,13 @@ __device__ __forceinline__ void stg_if(float *dst, float v, bool pred)
                  :: "l"(dst), "f"(v), "r"((unsigned)pred) : "memory");
 }
 
-template <typename T, int NPT_, int CH_, int TCH_>
+template <typename T, int NPT_, int CH_, int TCH_, int MINB_ = 3>
 struct PipeCfg {
     static constexpr int NPT = NPT_, CH = CH_, TCH = TCH_;
+    // resident CTAs per SM the register budget must allow: 3 (up to 168
+    // registers a thread) or, for grids of at most two CTAs per SM, 2 (up to
+    // 255), which gives the compiler room to keep more of the look-ahead live
+    static constexpr int MINB = MINB_;
     static constexpr int NP = NPT / 2;                       // packed state pairs per lane
     static constexpr int TPC = kN / NPT;                     // lanes per channel = tokens per group
     static constexpr int THREADS = CH * TPC;
@@ -472,10 +476,10 @@ __device__ __forceinline__ void cta_sync()
     else __syncthreads();
 }
 
-// At least three 4-warp CTAs per SM (up to 168 registers a thread): every
-// (sequence, channel) warp of the Mamba-130M layer resident at once.
+// At least MINB 4-warp CTAs per SM: with three (up to 168 registers a thread)
+// every (sequence, channel) warp of the Mamba-130M layer is resident at once.
 template <class K, typename T, bool SP, bool GZ>
-__global__ void __launch_bounds__(K::THREADS, 3)
+__global__ void __launch_bounds__(K::THREADS, K::MINB)
 scan_pipe_kernel(const Params p, const __grid_constant__ Maps m)
 {
     constexpr int TCH = K::TCH, CH = K::CH, NPT = K::NPT, TPC = K::TPC;
@@ -635,15 +639,18 @@ int read_pipe_status(bool clear)
     return v;
 }
 
-// Schedules 9 and 10 (16- and 32-token chunks) for 16-byte aligned rows (D a
-// multiple of 8 for bf16, of 4 for fp32); cudaErrorNotSupported when the
-// tensor maps cannot be encoded. CTAs of four warps.
+// Schedules 9 and 10 (16- and 32-token chunks) and 11 (schedule 10 at 4 states
+// per lane with up to 255 registers, two CTAs per SM; for bf16) for 16-byte
+// aligned rows (D a multiple of 8 for bf16, of 4 for fp32);
+// cudaErrorNotSupported when the tensor maps cannot be encoded. CTAs of four
+// warps.
 cudaError_t launch_scan_pipe(const Params &p, bool bf16, int npt, int sched, cudaStream_t stream,
                              int *launches)
 {
     const bool lng = sched == 10;
     if (bf16) {
         using T = __nv_bfloat16;
+        if (sched == 11) return run_pipe<PipeCfg<T, 4, 32, 32, 2>, T>(p, stream, launches);
         if (npt == 8) return lng ? run_pipe<PipeCfg<T, 8, 64, 32>, T>(p, stream, launches)
                                  : run_pipe<PipeCfg<T, 8, 64, 16>, T>(p, stream, launches);
         if (npt == 2) return run_pipe<PipeCfg<T, 2, 16, 32>, T>(p, stream, launches);

@@ -90,7 +90,7 @@ def test_conv_no_silu(orc):
 
 VARIANTS = [(2, 1), (2, 2), (2, 3), (4, 1), (4, 2), (4, 3), (4, 4), (4, 5), (8, 1), (8, 2), (8, 4),
             (8, 5), (16, 1), (16, 2), (16, 4), (16, 5), (2, 6), (4, 6), (8, 6), (16, 6), (4, 7), (8, 7), (16, 7), (2, 8), (4, 8), (8, 8), (16, 8),
-            (2, 9), (4, 9), (8, 9), (4, 10), (8, 10)]
+            (2, 9), (4, 9), (8, 9), (4, 10), (8, 10), (4, 11)]
 
 
 def _scan_case(orc, seed, lens, D, bf16, variant=(0, 0), with_z=True, with_h0=True,
