@@ -62,7 +62,7 @@ SCAN_KERNELS = {1: "scan_kernel", 2: "scan_tma_kernel", 3: "scan_ts_kernel", 4: 
                 5: "scan_tma_kernel", 6: "scan_ws_kernel", 7: "scan_warp_kernel",
                 8: "scan_staged_kernel", 9: "scan_pipe_kernel", 10: "scan_pipe_kernel",
                 11: "scan_pipe_kernel"}
-SCAN_SOURCES = ("scan.cu", "scan_pipe.cu", "scan_parts.cuh", "common.cuh", "tma.cuh")
+SCAN_SOURCES = ("scan.cu", "scan_pipe.cu", "scan_pipe.cuh", "scan_parts.cuh", "common.cuh", "tma.cuh")
 
 
 # ---------------------------------------------------------------------------
@@ -652,6 +652,9 @@ def bench_layer(args, world, peaks, mufu):
            "step": "causal_conv1d+silu -> selective_scan (h_final) -> 1 decode step; "
                    "4 rotating input sets (~600 MB) larger than L2"}
 
+    res["scan_bwd"] = bench_scan_bwd(world, st.layer, st.sets[0], None, st.Bn, mufu, peaks,
+                                     label="Mamba-130M layer 8 x 2048 x 1536", n=10)
+
     # the same step with the fused conv -> scan kernel
     def fused(i, ev=None):
         ly, a, d = st.layer, st.sets[i % st.SETS], st.dec[i % st.SETS]
@@ -938,7 +941,51 @@ def bench_scan_bwd(world, ly, a, cu, S, mufu, peaks, label="packed 65536 x 5120"
            "hbm_frac": round(units * 14 / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
            "variant": ssm.ssm_scan_bwd_variant_for(S, D), "sequences": S,
            "step": f"ssm_selective_scan_bwd over the {label} prefill, all gradients"}
-    del g, ws, dy
+
+    # the training pair: the forward leaves its checkpoints in the workspace,
+    # the backward reads them instead of running its own forward pass
+    y = torch.empty_like(a["x"])
+    fws = torch.empty(max(1, ssm.ssm_scan_workspace_size(tok, D, N_STATE, S)),
+                      dtype=torch.uint8, device="cuda")
+    fkw = dict(Dskip=ly.Dskip, z=a["z"], dt_bias=ly.dt_bias, cu_seqlens=cu, S=S, workspace=fws)
+
+    def fwd():
+        ssm.ssm_selective_scan_fwd(a["x"], a["dt"], ly.A, a["B"], a["C"], y, **fkw)
+
+    def fwd_ck():
+        ssm.ssm_selective_scan_fwd_ckpt(a["x"], a["dt"], ly.A, a["B"], a["C"], y, ws, **fkw)
+
+    def bwd_ck():
+        ssm.ssm_selective_scan_bwd(a["x"], a["dt"], ly.A, a["B"], a["C"], dy, g, Dskip=ly.Dskip,
+                                   z=a["z"], dt_bias=ly.dt_bias, cu_seqlens=cu, S=S,
+                                   workspace=ws, from_fwd_ckpt=True)
+
+    def timed(fns):
+        for _ in range(2):
+            for f in fns:
+                f()
+        evs = [_events(len(fns) + 1) for _ in range(n)]
+        _barrier_sync(world)
+        for i in range(n):
+            evs[i][0].record()
+            for j, f in enumerate(fns):
+                f()
+                evs[i][j + 1].record()
+        _barrier_sync(world)
+        return [_max_over_ranks(sum(e[j].elapsed_time(e[j + 1]) for e in evs) / n, world)
+                for j in range(len(fns))]
+
+    f_ms, fck_ms, bck_ms = timed([fwd, fwd_ck, bwd_ck])
+    res["from_forward_checkpoints"] = {
+        "bwd_ms": round(bck_ms, 4), "fwd_ckpt_ms": round(fck_ms, 4), "fwd_ms": round(f_ms, 4),
+        "value": units * world / (bck_ms * 1e-3) / 1e9, "unit": UNIT,
+        "mufu_frac": round(units * N_STATE / (bck_ms * 1e-3) / 1e9 / mufu["gexp_per_s"], 4),
+        "train_pair_ms": round(fck_ms + bck_ms, 4), "separate_pair_ms": round(f_ms + ms, 4),
+        "step": "ssm_selective_scan_fwd_ckpt (the forward writes the state before every 8th "
+                "token) then ssm_selective_scan_bwd_ckpt (no checkpointing pass); mufu_frac "
+                "counts the 16 exponentials per (token, channel) the backward needs once the "
+                "forward states are given"}
+    del g, ws, dy, y, fws
     return res
 
 

@@ -358,6 +358,51 @@ int ssm_selective_scan_bwd(const void *u, const void *delta, const float *A, con
                            size_t workspace_bytes, ssm_stream_t stream);
 
 /*
+ * Training pair: a forward scan that leaves the backward pass its state
+ * checkpoints, and the backward pass that reads them instead of running its
+ * own checkpointing forward pass (for a training step's forward, whose inputs
+ * the backward sees again).
+ *
+ * ssm_selective_scan_fwd_ckpt computes exactly what ssm_selective_scan_fwd
+ * computes (y and h_final bit for bit, same arguments) and also writes, into
+ * bwd_workspace, the fp32 state of every sequence and channel before each
+ * 8th token of the sequence (before tokens 0, 8, 16, ...; about 8 bytes per
+ * token and channel). The pipelined kernels (schedules 9 to 11) write them as
+ * they go; with any other kernel the library adds a checkpointing pass after
+ * the scan.
+ *   bwd_workspace  >= ssm_scan_bwd_workspace_size(tok, D, N, S) bytes,
+ *                  256-byte aligned, required, owned by the caller; must not
+ *                  overlap `workspace`
+ * Errors: those of ssm_selective_scan_fwd; SSM_ERR_WORKSPACE when
+ * bwd_workspace is NULL or too small; SSM_ERR_MISALIGNED when it is not
+ * 256-byte aligned; SSM_ERR_INVALID_ARGUMENT when the workspaces overlap.
+ *
+ * ssm_selective_scan_bwd_ckpt takes ssm_selective_scan_bwd's arguments, with
+ * `workspace` the bwd_workspace that ssm_selective_scan_fwd_ckpt filled for
+ * the same u, delta, A, B, dt_bias, delta_softplus, h0, cu_seqlens and sizes
+ * (on the same stream, or ordered after it), unchanged since. Gradients as
+ * ssm_selective_scan_bwd's, except that the states come from the forward's
+ * own arithmetic, so results differ from it in the last bits. Checkpoints that
+ * do not match the inputs give wrong gradients; nothing checks them.
+ */
+int ssm_selective_scan_fwd_ckpt(const void *u, const void *delta, const float *A, const void *B,
+                                const void *C, const float *Dskip, const void *z,
+                                const float *dt_bias, int delta_softplus, const float *h0,
+                                const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
+                                int64_t tok, int64_t D, int N, ssm_dtype act_dtype,
+                                void *workspace, size_t workspace_bytes, void *bwd_workspace,
+                                size_t bwd_workspace_bytes, ssm_stream_t stream);
+
+int ssm_selective_scan_bwd_ckpt(const void *u, const void *delta, const float *A, const void *B,
+                                const void *C, const float *Dskip, const void *z,
+                                const float *dt_bias, int delta_softplus, const float *h0,
+                                const int32_t *cu_seqlens, int64_t S, const void *dy,
+                                const float *dh_final, void *du, void *ddelta, void *dz,
+                                float *dB, float *dC, float *dA, float *dDskip, float *ddt_bias,
+                                float *dh0, int64_t tok, int64_t D, int N, ssm_dtype act_dtype,
+                                void *workspace, size_t workspace_bytes, ssm_stream_t stream);
+
+/*
  * Replay decode: one token per row, with each slot's SSM state kept as a
  * checkpoint plus the SSM inputs of the tokens since it.
  * Follows "ReplaySSM: Cache SSM Inputs, Not State" (abstract): the recurrence

@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     ssm_scan_workspace_size,
     ssm_selective_scan_bwd,
     ssm_selective_scan_fwd,
+    ssm_selective_scan_fwd_ckpt,
     ssm_selective_scan_fwd_noalloc,
     ssm_selective_state_update,
     ssm_selftest_wait_timeout,

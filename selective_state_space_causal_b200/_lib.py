@@ -35,6 +35,9 @@ SIGNATURES = [
     ("ssm_scan_workspace_size", _sz, [_i64, _i64, _int, _i64]),
     ("ssm_selective_scan_fwd", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64,
                                       _vp, _vp, _i64, _i64, _int, _int, _vp, _sz, _vp]),
+    ("ssm_selective_scan_fwd_ckpt", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp,
+                                           _i64, _vp, _vp, _i64, _i64, _int, _int, _vp, _sz, _vp,
+                                           _sz, _vp]),
     ("ssm_selective_scan_fwd_noalloc", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp,
                                               _vp, _i64, _vp, _vp, _i64, _i64, _int, _int, _vp]),
     ("ssm_selective_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -49,6 +52,9 @@ SIGNATURES = [
     ("ssm_selective_scan_bwd", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _i64,
                                       _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64,
                                       _i64, _int, _int, _vp, _sz, _vp]),
+    ("ssm_selective_scan_bwd_ckpt", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp,
+                                           _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                           _vp, _i64, _i64, _int, _int, _vp, _sz, _vp]),
     ("ssm_replay_state_update", _int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _vp, _vp, _vp,
                                        _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp, _i64, _vp, _i64,
                                        _i64, _int, _int, _int, _int, _vp]),
@@ -202,6 +208,24 @@ def ssm_selective_scan_fwd(u, delta, A, B, C, y, Dskip=None, z=None, dt_bias=Non
                                       N, _dtype(u), _ptr(workspace), ws_bytes, _stream(stream)))
 
 
+def ssm_selective_scan_fwd_ckpt(u, delta, A, B, C, y, bwd_workspace, Dskip=None, z=None,
+                                dt_bias=None, delta_softplus=True, h0=None, h_final=None,
+                                cu_seqlens=None, S=None, workspace=None, stream=None):
+    """ssm_selective_scan_fwd that also writes, into `bwd_workspace` (a device
+    byte tensor of ssm_scan_bwd_workspace_size() bytes), the state checkpoints
+    that ssm_selective_scan_bwd_ckpt reads instead of recomputing them."""
+    tok, D = u.shape
+    N = A.shape[1]
+    if S is None:
+        S = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    bws_bytes = 0 if bwd_workspace is None else bwd_workspace.numel() * bwd_workspace.element_size()
+    _check(lib.ssm_selective_scan_fwd_ckpt(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(z), _ptr(dt_bias),
+        int(bool(delta_softplus)), _ptr(h0), _ptr(cu_seqlens), S, _ptr(y), _ptr(h_final), tok, D,
+        N, _dtype(u), _ptr(workspace), ws_bytes, _ptr(bwd_workspace), bws_bytes, _stream(stream)))
+
+
 def ssm_selective_scan_fwd_noalloc(u, delta, A, B, C, y, Dskip=None, z=None, dt_bias=None,
                                    delta_softplus=True, h0=None, h_final=None, cu_seqlens=None,
                                    S=None, stream=None):
@@ -310,18 +334,22 @@ def ssm_scan_bwd_variant_for(S: int, D: int) -> int:
 
 def ssm_selective_scan_bwd(u, delta, A, B, C, dy, grads, Dskip=None, z=None, dt_bias=None,
                            delta_softplus=True, h0=None, dh_final=None, cu_seqlens=None, S=None,
-                           workspace=None, stream=None):
+                           workspace=None, stream=None, from_fwd_ckpt=False):
     """Backward of ssm_selective_scan_fwd. `grads` holds the output tensors:
     du, ddelta (like u), dz (like u, or None), dB, dC (tok, N) fp32, dA (D, N)
     fp32, dDskip, ddt_bias (D) fp32 or None, dh0 (S, D, N) fp32 or None.
-    `workspace` is a device byte tensor of ssm_scan_bwd_workspace_size() bytes."""
+    `workspace` is a device byte tensor of ssm_scan_bwd_workspace_size() bytes.
+    from_fwd_ckpt: the workspace holds the checkpoints that
+    ssm_selective_scan_fwd_ckpt wrote for the same inputs
+    (ssm_selective_scan_bwd_ckpt)."""
     tok, D = u.shape
     N = A.shape[1]
     if S is None:
         S = (cu_seqlens.numel() - 1) if cu_seqlens is not None else 1
     g = grads
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.ssm_selective_scan_bwd(
+    fn = lib.ssm_selective_scan_bwd_ckpt if from_fwd_ckpt else lib.ssm_selective_scan_bwd
+    _check(fn(
         _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(Dskip), _ptr(z), _ptr(dt_bias),
         int(bool(delta_softplus)), _ptr(h0), _ptr(cu_seqlens), S, _ptr(dy), _ptr(dh_final),
         _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g.get("dz")), _ptr(g["dB"]), _ptr(g["dC"]),

@@ -40,8 +40,10 @@ struct ScanBwdArgs {
     int64_t tok, D;
     int softplus;
     bool bf16;
+    bool have_ckpt = false;  // ckpt already holds the forward's 8-token checkpoints
 };
 size_t scan_bwd_workspace_bytes(int64_t tok, int64_t D, int64_t S);
+cudaError_t launch_scan_bwd_ckpt_pass(const ScanBwdArgs &a, cudaStream_t stream, int *launches);
 void set_scan_bwd_variant(int v);
 int scan_bwd_variant_for(int64_t S, int64_t D);
 
@@ -238,14 +240,16 @@ size_t ssm_scan_workspace_size(int64_t tok, int64_t D, int N, int64_t S)
     return S > 1 ? ssm::scan_order_bytes(S) : 0;
 }
 
-int ssm_selective_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
-                           const void *C, const float *Dskip, const void *z,
-                           const float *dt_bias, int delta_softplus, const float *h0,
-                           const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
-                           int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
-                           size_t workspace_bytes, ssm_stream_t stream)
+// The forward scan's checks and launch; with bwd_ws (already checked), the
+// state before every 8th token of each sequence also goes there for the
+// backward pass.
+static int scan_fwd_impl(const char *fn, const void *u, const void *delta, const float *A,
+                         const void *B, const void *C, const float *Dskip, const void *z,
+                         const float *dt_bias, int delta_softplus, const float *h0,
+                         const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
+                         int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
+                         size_t workspace_bytes, void *bwd_ws, ssm_stream_t stream)
 {
-    const char *fn = "ssm_selective_scan_fwd";
     if (!valid_dtype(act_dtype)) return fail(SSM_ERR_UNSUPPORTED_DTYPE, "%s: unknown dtype", fn);
     if (N != 16) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: N must be 16 (got %d)", fn, N);
     if (D < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: D must be >= 1", fn);
@@ -278,12 +282,63 @@ int ssm_selective_scan_fwd(const void *u, const void *delta, const float *A, con
     }
     const bool vec = aligned(u, 16) && aligned(delta, 16) && aligned(y, 16) &&
                      (!z || aligned(z, 16));
+    bool written = false;
     ssm::ScanArgs a{u, delta, A, B, C, Dskip, z, dt_bias, delta_softplus, h0, cu_seqlens, S,
                     y, h_final, tok, D, N, dt(act_dtype),
-                    workspace ? static_cast<int32_t *>(workspace) : nullptr, vec};
+                    workspace ? static_cast<int32_t *>(workspace) : nullptr, vec,
+                    static_cast<float *>(bwd_ws), &written};
     int launched = 0;
-    cudaError_t e = ssm::launch_scan(a, reinterpret_cast<cudaStream_t>(stream), &launched);
+    const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = ssm::launch_scan(a, st, &launched);
+    if (e == cudaSuccess && bwd_ws && !written) {
+        // the kernel that ran does not write checkpoints: a pass of its own
+        ssm::ScanBwdArgs b{u, delta, B, C, z, nullptr, A, Dskip, dt_bias, h0, nullptr,
+                           cu_seqlens, S, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                           nullptr, nullptr, nullptr, static_cast<float *>(bwd_ws), tok, D,
+                           delta_softplus, act_dtype == SSM_BF16};
+        e = ssm::launch_scan_bwd_ckpt_pass(b, st, &launched);
+    }
     return finish(e, launched, fn);
+}
+
+int ssm_selective_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                           const void *C, const float *Dskip, const void *z,
+                           const float *dt_bias, int delta_softplus, const float *h0,
+                           const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
+                           int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
+                           size_t workspace_bytes, ssm_stream_t stream)
+{
+    return scan_fwd_impl("ssm_selective_scan_fwd", u, delta, A, B, C, Dskip, z, dt_bias,
+                         delta_softplus, h0, cu_seqlens, S, y, h_final, tok, D, N, act_dtype,
+                         workspace, workspace_bytes, nullptr, stream);
+}
+
+int ssm_selective_scan_fwd_ckpt(const void *u, const void *delta, const float *A, const void *B,
+                                const void *C, const float *Dskip, const void *z,
+                                const float *dt_bias, int delta_softplus, const float *h0,
+                                const int32_t *cu_seqlens, int64_t S, void *y, float *h_final,
+                                int64_t tok, int64_t D, int N, ssm_dtype act_dtype,
+                                void *workspace, size_t workspace_bytes, void *bwd_workspace,
+                                size_t bwd_workspace_bytes, ssm_stream_t stream)
+{
+    const char *fn = "ssm_selective_scan_fwd_ckpt";
+    if (N == 16 && D >= 1 && S >= 0 && tok >= 0) {
+        const size_t need = ssm_scan_bwd_workspace_size(tok, D, N, S);
+        if (!bwd_workspace || bwd_workspace_bytes < need)
+            return fail(SSM_ERR_WORKSPACE, "%s: bwd_workspace has %zu bytes, needs %zu", fn,
+                        bwd_workspace ? bwd_workspace_bytes : (size_t)0, need);
+        if (!aligned(bwd_workspace, 256))
+            return fail(SSM_ERR_MISALIGNED, "%s: bwd_workspace must be 256-byte aligned", fn);
+        if (workspace && bwd_workspace) {
+            const char *a = static_cast<const char *>(workspace);
+            const char *b = static_cast<const char *>(bwd_workspace);
+            if (a < b + need && b < a + workspace_bytes)
+                return fail(SSM_ERR_INVALID_ARGUMENT, "%s: the two workspaces overlap", fn);
+        }
+    }
+    return scan_fwd_impl(fn, u, delta, A, B, C, Dskip, z, dt_bias, delta_softplus, h0,
+                         cu_seqlens, S, y, h_final, tok, D, N, act_dtype, workspace,
+                         workspace_bytes, bwd_workspace, stream);
 }
 
 int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x,
@@ -404,16 +459,17 @@ int ssm_scan_bwd_variant_for(int64_t S, int64_t D, int *variant)
     return ok();
 }
 
-int ssm_selective_scan_bwd(const void *u, const void *delta, const float *A, const void *B,
-                           const void *C, const float *Dskip, const void *z,
-                           const float *dt_bias, int delta_softplus, const float *h0,
-                           const int32_t *cu_seqlens, int64_t S, const void *dy,
-                           const float *dh_final, void *du, void *ddelta, void *dz, float *dB,
-                           float *dC, float *dA, float *dDskip, float *ddt_bias, float *dh0,
-                           int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
-                           size_t workspace_bytes, ssm_stream_t stream)
+// The backward scan's checks and launch; have_ckpt: the workspace holds the
+// forward's checkpoints (ssm_selective_scan_fwd_ckpt).
+static int scan_bwd_impl(const char *fn, bool have_ckpt, const void *u, const void *delta,
+                         const float *A, const void *B, const void *C, const float *Dskip,
+                         const void *z, const float *dt_bias, int delta_softplus,
+                         const float *h0, const int32_t *cu_seqlens, int64_t S, const void *dy,
+                         const float *dh_final, void *du, void *ddelta, void *dz, float *dB,
+                         float *dC, float *dA, float *dDskip, float *ddt_bias, float *dh0,
+                         int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
+                         size_t workspace_bytes, ssm_stream_t stream)
 {
-    const char *fn = "ssm_selective_scan_bwd";
     if (!valid_dtype(act_dtype)) return fail(SSM_ERR_UNSUPPORTED_DTYPE, "%s: unknown dtype", fn);
     if (N != 16) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: N must be 16 (got %d)", fn, N);
     if (D < 1) return fail(SSM_ERR_INVALID_ARGUMENT, "%s: D must be >= 1", fn);
@@ -452,10 +508,40 @@ int ssm_selective_scan_bwd(const void *u, const void *delta, const float *A, con
     ssm::ScanBwdArgs a{u, delta, B, C, z, dy, A, Dskip, dt_bias, h0, dh_final, cu_seqlens, S,
                        du, ddelta, dz, dB, dC, dA, dDskip, ddt_bias, dh0,
                        static_cast<float *>(workspace), tok, D, delta_softplus,
-                       act_dtype == SSM_BF16};
+                       act_dtype == SSM_BF16, have_ckpt};
     int launched = 0;
     cudaError_t e = ssm::launch_scan_bwd(a, reinterpret_cast<cudaStream_t>(stream), &launched);
     return finish(e, launched, fn);
+}
+
+int ssm_selective_scan_bwd(const void *u, const void *delta, const float *A, const void *B,
+                           const void *C, const float *Dskip, const void *z,
+                           const float *dt_bias, int delta_softplus, const float *h0,
+                           const int32_t *cu_seqlens, int64_t S, const void *dy,
+                           const float *dh_final, void *du, void *ddelta, void *dz, float *dB,
+                           float *dC, float *dA, float *dDskip, float *ddt_bias, float *dh0,
+                           int64_t tok, int64_t D, int N, ssm_dtype act_dtype, void *workspace,
+                           size_t workspace_bytes, ssm_stream_t stream)
+{
+    return scan_bwd_impl("ssm_selective_scan_bwd", false, u, delta, A, B, C, Dskip, z, dt_bias,
+                         delta_softplus, h0, cu_seqlens, S, dy, dh_final, du, ddelta, dz, dB, dC,
+                         dA, dDskip, ddt_bias, dh0, tok, D, N, act_dtype, workspace,
+                         workspace_bytes, stream);
+}
+
+int ssm_selective_scan_bwd_ckpt(const void *u, const void *delta, const float *A, const void *B,
+                                const void *C, const float *Dskip, const void *z,
+                                const float *dt_bias, int delta_softplus, const float *h0,
+                                const int32_t *cu_seqlens, int64_t S, const void *dy,
+                                const float *dh_final, void *du, void *ddelta, void *dz,
+                                float *dB, float *dC, float *dA, float *dDskip, float *ddt_bias,
+                                float *dh0, int64_t tok, int64_t D, int N, ssm_dtype act_dtype,
+                                void *workspace, size_t workspace_bytes, ssm_stream_t stream)
+{
+    return scan_bwd_impl("ssm_selective_scan_bwd_ckpt", true, u, delta, A, B, C, Dskip, z,
+                         dt_bias, delta_softplus, h0, cu_seqlens, S, dy, dh_final, du, ddelta,
+                         dz, dB, dC, dA, dDskip, ddt_bias, dh0, tok, D, N, act_dtype, workspace,
+                         workspace_bytes, stream);
 }
 
 // Shared checks of a replay slot list (NULL = slots 0..n-1).

@@ -43,6 +43,11 @@ struct ScanArgs {
     DType dtype;
     int32_t *order;  // nullptr: sequences in index order; else S entries of scratch
     bool vec;
+    // the state before every 8th token of each sequence, for the backward
+    // pass, or nullptr; *ckpt_written reports whether the kernel that ran wrote
+    // them (the pipelined kernel does, the other schedules do not)
+    float *ckpt = nullptr;
+    bool *ckpt_written = nullptr;
 };
 
 struct DecodeArgs {

@@ -1512,17 +1512,21 @@ int g_forced_npt = 0, g_forced_sched = 0;
 
 // Variants: NPT states per lane; schedule 1: register prefetch, 2: TMA
 // staging, 3: TMA staging with time-split chunks; CH channels per CTA, TCH
-// tokens per chunk.
+// tokens per chunk. *piped: set when the pipelined kernel (schedules 9-11)
+// ran; it alone writes p.ckpt.
 template <typename T, int VEC>
-cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n)
+cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n, bool *piped)
 {
     if constexpr (VEC == 1) {
-        (void)npt; (void)sched;
+        (void)npt; (void)sched; (void)piped;
         return run<Cfg<T, 4, 0, 32, 64, 1>, T>(p, s, n);
     } else {
         if (sched >= 9 && sched <= 11 && p.tok > 0) {
             cudaError_t e = launch_scan_pipe(p, sizeof(T) == 2, npt, sched, s, n);
-            if (e != cudaErrorNotSupported) return e;
+            if (e != cudaErrorNotSupported) {
+                *piped = e == cudaSuccess;
+                return e;
+            }
         }
         if (sched == 3 && p.tok > 0) {
             cudaError_t e = npt == 2 ? run_ts<TsCfg<T, 2, 4, 8, 8>, T>(p, s, n)
@@ -1676,6 +1680,9 @@ cudaError_t launch_scan(const ScanArgs &a, cudaStream_t stream, int *launches)
     p.cu = a.cu; p.order = nullptr; p.y = a.y; p.h_final = a.h_final;
     p.S = a.S; p.tok = a.tok; p.D = a.D; p.L = a.cu ? 0 : a.tok / a.S;
     p.delta_softplus = a.delta_softplus;
+    p.ckpt = a.ckpt;
+    bool piped = false;
+    if (a.ckpt_written) *a.ckpt_written = false;
     if (a.cu && a.order && a.S > 1) {
         order_kernel<<<1, 1024, 0, stream>>>(a.cu, a.S, a.tok, a.order);
         ++*launches;
@@ -1685,12 +1692,17 @@ cudaError_t launch_scan(const ScanArgs &a, cudaStream_t stream, int *launches)
     }
     int npt, sched;
     pick_variant(a.S, a.D, &npt, &sched);
+    cudaError_t e;
     if (a.dtype == DType::BF16) {
-        if (a.vec && a.D % 8 == 0) return dispatch<__nv_bfloat16, 8>(p, npt, sched, stream, launches);
-        return dispatch<__nv_bfloat16, 1>(p, npt, sched, stream, launches);
+        if (a.vec && a.D % 8 == 0) e = dispatch<__nv_bfloat16, 8>(p, npt, sched, stream, launches, &piped);
+        else e = dispatch<__nv_bfloat16, 1>(p, npt, sched, stream, launches, &piped);
+    } else if (a.vec && a.D % 4 == 0) {
+        e = dispatch<float, 4>(p, npt, sched, stream, launches, &piped);
+    } else {
+        e = dispatch<float, 1>(p, npt, sched, stream, launches, &piped);
     }
-    if (a.vec && a.D % 4 == 0) return dispatch<float, 4>(p, npt, sched, stream, launches);
-    return dispatch<float, 1>(p, npt, sched, stream, launches);
+    if (a.ckpt_written) *a.ckpt_written = piped;
+    return e;
 }
 
 }  // namespace ssm

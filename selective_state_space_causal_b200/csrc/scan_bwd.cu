@@ -55,6 +55,7 @@ constexpr int kCh = 32;               // channels per CTA
 constexpr int kThreads = kCh * kTPC;  // 128
 constexpr int kWarps = kThreads / 32;
 constexpr int kTS = 16;               // tokens per chunk (one checkpoint each)
+constexpr int kFwdCk = 8;             // tokens per checkpoint when the forward wrote them
 
 struct BwdParams {
     const void *u, *dt, *B, *C, *z, *dy;
@@ -67,6 +68,9 @@ struct BwdParams {
     int64_t S, tok, D, L;
     int softplus;
     int vec_atomics;  // dB and dC are 16-byte aligned: sums go out as float4 atomics
+    // the workspace already holds the state before every 8th token of each
+    // sequence (written by the forward pass): no checkpointing pass here
+    int have_ckpt;
 };
 
 // The sequence of this CTA row (blockIdx.y; the longest-first order when one
@@ -263,8 +267,11 @@ scan_bwd_kernel(const BwdParams p)
     bwd_sequence(p, s, start, end);
     const int64_t len = end - start;
     const int64_t nchunks = (len + kTS - 1) / kTS;
-    // checkpoint slots of this sequence: floor(start / kTS) + s + k never collide
-    float *ck = p.ckpt + ((start / kTS + s) * p.D + c) * kN + sub * kNPT;
+    // checkpoint slots of this sequence: floor(start / kTS) + s + k never
+    // collide; the forward's 8-token checkpoints sit at floor(start / 8) + s
+    // + 2k
+    float *ck = p.ckpt + ((start / (p.have_ckpt ? kFwdCk : kTS) + s) * p.D + c) * kN + sub * kNPT;
+    const int64_t ck_step = (p.have_ckpt ? kTS / kFwdCk : 1) * p.D * kN;
 
     f32x2 A2[2], Aln[2];
 #pragma unroll
@@ -278,47 +285,49 @@ scan_bwd_kernel(const BwdParams p)
     const float dsk = (cvalid && p.Dskip) ? __ldg(p.Dskip + c) : 0.f;
 
     // ---- phase A: forward, checkpoint at every chunk start ----------------
-    f32x2 h[2];
+    if (!p.have_ckpt) {
+        f32x2 h[2];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int64_t o = (s * p.D + c) * kN + sub * kNPT + 2 * j;
-        h[j] = (cvalid && p.h0) ? pk2(p.h0[o], p.h0[o + 1]) : 0ull;
-    }
-    if (ASYNC && nchunks > 0) {
-        issue_chunk<T>(p, raw[0], start, (int)min((int64_t)kTS, len), cbase, nch, false);
-        cp_commit();
-    }
-    for (int64_t k = 0; k < nchunks; ++k) {
-        const int64_t t0 = start + k * kTS;
-        const int nt = (int)min((int64_t)kTS, end - t0);
-        if (cvalid) {
-            float4 v;
-            upk2(h[0], v.x, v.y);
-            upk2(h[1], v.z, v.w);
-            *reinterpret_cast<float4 *>(ck + k * p.D * kN) = v;
+        for (int j = 0; j < 2; ++j) {
+            const int64_t o = (s * p.D + c) * kN + sub * kNPT + 2 * j;
+            h[j] = (cvalid && p.h0) ? pk2(p.h0[o], p.h0[o + 1]) : 0ull;
         }
-        if constexpr (ASYNC) {
-            // the next chunk's copies go out before this one is staged; the
-            // buffer they fill was last read before the previous barrier
-            if (k + 1 < nchunks) {
-                const int64_t t1 = t0 + kTS;
-                issue_chunk<T>(p, raw[(k + 1) & 1], t1, (int)min((int64_t)kTS, end - t1), cbase,
-                               nch, false);
-                cp_commit();
-                cp_wait<1>();
-            } else {
-                cp_wait<0>();
+        if (ASYNC && nchunks > 0) {
+            issue_chunk<T>(p, raw[0], start, (int)min((int64_t)kTS, len), cbase, nch, false);
+            cp_commit();
+        }
+        for (int64_t k = 0; k < nchunks; ++k) {
+            const int64_t t0 = start + k * kTS;
+            const int nt = (int)min((int64_t)kTS, end - t0);
+            if (cvalid) {
+                float4 v;
+                upk2(h[0], v.x, v.y);
+                upk2(h[1], v.z, v.w);
+                *reinterpret_cast<float4 *>(ck + k * ck_step) = v;
             }
-            __syncthreads();  // every thread's copies have landed; the previous chunk is done
-            stage_from_raw<T>(p, sm, raw[k & 1], nt, cbase, false);
-        } else {
-            __syncthreads();  // the previous chunk's values are no longer read
-            stage_chunk<T>(p, sm, t0, nt, cbase, false);
-        }
-        __syncthreads();
-        for (int tl = 0; tl < nt; ++tl) {
-            f32x2 a[2];
-            fwd_token(h, A2, sm.d[tl][cl], sm.u[tl][cl], &sm.B[tl][sub * kNPT], a);
+            if constexpr (ASYNC) {
+                // the next chunk's copies go out before this one is staged; the
+                // buffer they fill was last read before the previous barrier
+                if (k + 1 < nchunks) {
+                    const int64_t t1 = t0 + kTS;
+                    issue_chunk<T>(p, raw[(k + 1) & 1], t1, (int)min((int64_t)kTS, end - t1), cbase,
+                                   nch, false);
+                    cp_commit();
+                    cp_wait<1>();
+                } else {
+                    cp_wait<0>();
+                }
+                __syncthreads();  // every thread's copies have landed; the previous chunk is done
+                stage_from_raw<T>(p, sm, raw[k & 1], nt, cbase, false);
+            } else {
+                __syncthreads();  // the previous chunk's values are no longer read
+                stage_chunk<T>(p, sm, t0, nt, cbase, false);
+            }
+            __syncthreads();
+            for (int tl = 0; tl < nt; ++tl) {
+                f32x2 a[2];
+                fwd_token(h, A2, sm.d[tl][cl], sm.u[tl][cl], &sm.B[tl][sub * kNPT], a);
+            }
         }
     }
 
@@ -359,7 +368,7 @@ scan_bwd_kernel(const BwdParams p)
         // recompute this lane's states over the chunk from its checkpoint
         f32x2 hc[2], hist[kTS][2];
         if (cvalid) {
-            const float4 v = *reinterpret_cast<const float4 *>(ck + k * p.D * kN);
+            const float4 v = *reinterpret_cast<const float4 *>(ck + k * ck_step);
             hc[0] = pk2(v.x, v.y);
             hc[1] = pk2(v.z, v.w);
         } else {
@@ -1086,6 +1095,7 @@ struct ScanBwdArgs {
     int64_t tok, D;
     int softplus;
     bool bf16;
+    bool have_ckpt = false;  // ckpt already holds the forward's 8-token checkpoints
 };
 
 cudaError_t launch_seq_order(const int32_t *cu, int64_t S, int64_t tok, int32_t *order,
@@ -1127,17 +1137,27 @@ int scan_bwd_variant_for(int64_t S, int64_t D)
 }
 
 template <typename T, bool ASYNC>
-static cudaError_t run_wide(const BwdParams &p, dim3 grid, cudaStream_t stream, int *launches)
+static cudaError_t run_ckpt(const BwdParams &p, dim3 grid, cudaStream_t stream, int *launches)
 {
-    // the forward pass that writes the checkpoints, then the reverse pass
     const size_t ck_smem = 2 * sizeof(WRaw<T>) + sizeof(float) * kWTS * kN;
     cudaError_t e = cudaFuncSetAttribute(scan_bwd_ckpt_kernel<T, ASYNC>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ck_smem);
     if (e != cudaSuccess) return e;
     scan_bwd_ckpt_kernel<T, ASYNC><<<grid, kCkThreads, ck_smem, stream>>>(p);
     ++*launches;
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+template <typename T, bool ASYNC>
+static cudaError_t run_wide(const BwdParams &p, dim3 grid, cudaStream_t stream, int *launches)
+{
+    // the forward pass that writes the checkpoints (unless the forward scan
+    // wrote them), then the reverse pass
+    cudaError_t e;
+    if (!p.have_ckpt) {
+        e = run_ckpt<T, ASYNC>(p, grid, stream, launches);
+        if (e != cudaSuccess) return e;
+    }
     const size_t smem = w_smem_bytes(sizeof(WRaw<T>), ASYNC && sizeof(T) == 2);
     e = cudaFuncSetAttribute(scan_bwd_wide_kernel<T, ASYNC>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -1174,7 +1194,7 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *laun
     p.A = a.A; p.Dskip = a.Dskip; p.dt_bias = a.dt_bias; p.h0 = a.h0; p.dh_final = a.dh_final;
     p.cu = a.cu; p.du = a.du; p.ddt = a.ddt; p.dz = a.dz;
     p.dB = a.dB; p.dC = a.dC; p.dA = a.dA; p.dDskip = a.dDskip; p.ddt_bias = a.ddt_bias;
-    p.dh0 = a.dh0; p.ckpt = a.ckpt; p.order = nullptr;
+    p.dh0 = a.dh0; p.ckpt = a.ckpt; p.order = nullptr; p.have_ckpt = a.have_ckpt ? 1 : 0;
     p.S = a.S; p.tok = a.tok; p.D = a.D; p.L = a.cu ? 0 : a.tok / a.S; p.softplus = a.softplus;
     p.vec_atomics = ((uintptr_t)a.dB % 16 == 0) && ((uintptr_t)a.dC % 16 == 0);
     if (a.cu && a.S > 1) {
@@ -1212,6 +1232,27 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *laun
     }
     ++*launches;
     return e;
+}
+
+// The checkpointing forward pass alone (the state before every 8th token of
+// each sequence into a.ckpt), for a forward scan whose kernel did not write
+// them. Reads u, dt, B, A, dt_bias and h0; sequences in index order.
+cudaError_t launch_scan_bwd_ckpt_pass(const ScanBwdArgs &a, cudaStream_t stream, int *launches)
+{
+    if (a.S == 0 || a.tok == 0) return cudaSuccess;
+    BwdParams p{};
+    p.u = a.u; p.dt = a.dt; p.B = a.B; p.A = a.A; p.dt_bias = a.dt_bias; p.h0 = a.h0;
+    p.cu = a.cu; p.ckpt = a.ckpt; p.order = nullptr;
+    p.S = a.S; p.tok = a.tok; p.D = a.D; p.L = a.cu ? 0 : a.tok / a.S; p.softplus = a.softplus;
+    const size_t es = a.bf16 ? 2 : 4;
+    const uintptr_t mis = (uintptr_t)a.u | (uintptr_t)a.dt | (uintptr_t)a.B;
+    const bool async_ok = (mis % 16 == 0) && ((size_t)a.D * es) % 16 == 0;
+    const dim3 grid((unsigned)((a.D + kWCh - 1) / kWCh), (unsigned)a.S);
+    if (a.bf16)
+        return async_ok ? run_ckpt<__nv_bfloat16, true>(p, grid, stream, launches)
+                        : run_ckpt<__nv_bfloat16, false>(p, grid, stream, launches);
+    return async_ok ? run_ckpt<float, true>(p, grid, stream, launches)
+                    : run_ckpt<float, false>(p, grid, stream, launches);
 }
 
 }  // namespace ssm

@@ -24,6 +24,9 @@ struct Params {
     float *h_final;
     int64_t S, tok, D, L;
     int delta_softplus;
+    // the state before every 8th token of each sequence, for the backward
+    // pass (written by the pipelined kernel only), or null
+    float *ckpt = nullptr;
 };
 
 namespace {

@@ -258,6 +258,57 @@ def test_scan_bwd_rejects(kw, code):
     assert _err()
 
 
+def bwd_ckpt(**kw):
+    a = dict(u=A16, dt=A16 + 0x200000, A=A16, B=A16, C=A16, Dsk=None, z=None, dtb=None, sp=1,
+             h0=None, cu=None, S=1, dy=A16 + 0x400000, dhf=None, du=A16 + 0x600000,
+             ddt=A16 + 0x800000, dz=None, dB=A16, dC=A16, dA=A16, dDsk=None, ddtb=None,
+             dh0=None, tok=64, D=32, N=16, adt=1, ws=A16, wsb=1 << 30)
+    a.update(kw)
+    return L.ssm_selective_scan_bwd_ckpt(a["u"], a["dt"], a["A"], a["B"], a["C"], a["Dsk"],
+                                         a["z"], a["dtb"], a["sp"], a["h0"], a["cu"], a["S"],
+                                         a["dy"], a["dhf"], a["du"], a["ddt"], a["dz"], a["dB"],
+                                         a["dC"], a["dA"], a["dDsk"], a["ddtb"], a["dh0"],
+                                         a["tok"], a["D"], a["N"], a["adt"], a["ws"], a["wsb"],
+                                         None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(N=8), -1), (dict(dA=None), -1), (dict(ws=None), -5), (dict(wsb=64), -5),
+    (dict(ws=A16 + 16), -3), (dict(u=A16 + 1), -3), (dict(adt=5), -2),
+    (dict(du=A16 + 0x200000), -1),
+])
+def test_scan_bwd_ckpt_rejects(kw, code):
+    """The backward that reads the forward's checkpoints checks its arguments
+    as ssm_selective_scan_bwd does."""
+    assert bwd_ckpt(**kw) == code
+    assert "ssm_selective_scan_bwd_ckpt" in _err()
+
+
+def fwd_ckpt(**kw):
+    need = ssm.ssm_scan_bwd_workspace_size(64, 32, 16, 1)
+    a = dict(u=A16, dt=A16 + 0x200000, A=A16, B=A16, C=A16, Dsk=None, z=None, dtb=None, sp=1,
+             h0=None, cu=None, S=1, y=A16 + 0x400000, hf=None, tok=64, D=32, N=16, adt=1,
+             ws=None, wsb=0, bws=A16 + 0x600000, bwsb=need)
+    a.update(kw)
+    return L.ssm_selective_scan_fwd_ckpt(a["u"], a["dt"], a["A"], a["B"], a["C"], a["Dsk"],
+                                         a["z"], a["dtb"], a["sp"], a["h0"], a["cu"], a["S"],
+                                         a["y"], a["hf"], a["tok"], a["D"], a["N"], a["adt"],
+                                         a["ws"], a["wsb"], a["bws"], a["bwsb"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(bws=None), -5), (dict(bwsb=64), -5), (dict(bws=A16 + 0x600000 + 16), -3),
+    (dict(ws=A16 + 0x600000, wsb=256), -1), (dict(N=8), -1), (dict(A=None), -1),
+    (dict(u=A16 + 1), -3), (dict(adt=5), -2), (dict(y=A16 + 0x200000), -1),
+])
+def test_scan_fwd_ckpt_rejects(kw, code):
+    """The forward that writes checkpoints for the backward needs a 256-byte
+    aligned backward workspace of ssm_scan_bwd_workspace_size() bytes apart
+    from its own workspace, and checks the rest as ssm_selective_scan_fwd."""
+    assert fwd_ckpt(**kw) == code
+    assert _err()
+
+
 def test_scan_bwd_workspace_size():
     n = ssm.ssm_scan_bwd_workspace_size(16384, 1536, 16, 8)
     # a 64-byte state per 8 tokens, sequence and channel, plus the sequence order

@@ -28,7 +28,11 @@ def variant(request):
     ssm.ssm_set_scan_bwd_variant(0)
 
 
-def _run_bwd(u, dt, A, B, C, dy, Dskip, z, dt_bias, h0, dh_final, cu, S, softplus=True):
+def _run_bwd(u, dt, A, B, C, dy, Dskip, z, dt_bias, h0, dh_final, cu, S, softplus=True,
+             from_fwd=False):
+    """from_fwd: the workspace is filled by ssm_selective_scan_fwd_ckpt first,
+    whose y and h_final must be those of ssm_selective_scan_fwd bit for bit,
+    and the backward reads its checkpoints (ssm_selective_scan_bwd_ckpt)."""
     tok, D = u.shape
     N = A.shape[1]
     f32 = dict(device="cuda", dtype=torch.float32)
@@ -39,14 +43,28 @@ def _run_bwd(u, dt, A, B, C, dy, Dskip, z, dt_bias, h0, dh_final, cu, S, softplu
          "ddt_bias": torch.full((D,), 7.0, **f32), "dh0": torch.full((S, D, N), 7.0, **f32)}
     ws = torch.empty(max(1, ssm.ssm_scan_bwd_workspace_size(tok, D, N, S)), dtype=torch.uint8,
                      device="cuda")
+    if from_fwd:
+        fws = torch.empty(max(1, ssm.ssm_scan_workspace_size(tok, D, N, S)), dtype=torch.uint8,
+                          device="cuda")
+        ys = [torch.full_like(u, 3.0) for _ in range(2)]
+        hs = [torch.full((S, D, N), 3.0, device="cuda") for _ in range(2)]
+        kw = dict(Dskip=Dskip, z=z, dt_bias=dt_bias, delta_softplus=softplus, h0=h0,
+                  cu_seqlens=cu, S=S, workspace=fws)
+        ws.fill_(0xFF)  # NaN everywhere a checkpoint is not written
+        ssm.ssm_selective_scan_fwd_ckpt(u, dt, A, B, C, ys[0], ws, h_final=hs[0], **kw)
+        ssm.ssm_selective_scan_fwd(u, dt, A, B, C, ys[1], h_final=hs[1], **kw)
+        torch.cuda.synchronize()
+        assert torch.equal(ys[0], ys[1]), "y of the checkpointing forward"
+        assert torch.equal(hs[0], hs[1]), "h_final of the checkpointing forward"
     ssm.ssm_selective_scan_bwd(u, dt, A, B, C, dy, g, Dskip=Dskip, z=z, dt_bias=dt_bias,
                                delta_softplus=softplus, h0=h0, dh_final=dh_final, cu_seqlens=cu,
-                               S=S, workspace=ws)
+                               S=S, workspace=ws, from_fwd_ckpt=from_fwd)
     torch.cuda.synchronize()
     return g
 
 
-def _check(orc, bf16, lens, D, gate=True, softplus=True, dense_rows=None, seed=0):
+def _check(orc, bf16, lens, D, gate=True, softplus=True, dense_rows=None, seed=0,
+           from_fwd=False):
     dt_ = act_dtype(bf16)
     if dense_rows:
         tok = dense_rows[0] * dense_rows[1]
@@ -71,7 +89,7 @@ def _check(orc, bf16, lens, D, gate=True, softplus=True, dense_rows=None, seed=0
         dtb = None
     g = _run_bwd(dev(act["x"], dt_), dev(delta, dt_), dev(prm.A), dev(act["B"], dt_),
                  dev(act["C"], dt_), dev(dy, dt_), dev(prm.Dskip), dev(z, dt_) if gate else None,
-                 dev(dtb), dev(st["h0"]), dev(dhf), cu_d, S, softplus)
+                 dev(dtb), dev(st["h0"]), dev(dhf), cu_d, S, softplus, from_fwd)
     r = orc.selective_scan_bwd(act["x"], delta, prm.A, act["B"], act["C"], dy,
                                Dskip=prm.Dskip, z=z, dt_bias=dtb, delta_softplus=softplus,
                                h0=st["h0"], cu_seqlens=None if dense_rows else cu_h,
@@ -234,3 +252,37 @@ def test_bwd_many_short_sequences_past_the_sort_limit(orc, variant):
     handles (the order stays as given), with h0 and dh_final for each."""
     lens = list(np.random.default_rng(23).integers(0, 7, size=5000))
     _check(orc, True, lens, 128, seed=23)
+
+
+@pytest.fixture(params=[(0, 0), (2, 9), (4, 10), (8, 9), (4, 11), (4, 1)],
+                ids=["fwd_pick", "pipe2", "pipe4", "pipe8", "pipe4_255reg", "fwd_sched1"])
+def fwd_sched(request):
+    """The forward that writes the checkpoints: the library's pick, the
+    pipelined kernel at 2, 4 and 8 states per lane (it writes them as it goes),
+    and schedule 1 (no checkpoint output: the library adds its checkpointing
+    pass)."""
+    ssm.ssm_set_scan_variant(*request.param)
+    yield request.param
+    ssm.ssm_set_scan_variant(0, 0)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_bwd_from_forward_checkpoints(orc, bf16, variant, fwd_sched):
+    """ssm_selective_scan_fwd_ckpt then ssm_selective_scan_bwd_ckpt: the same
+    y and h_final as the plain forward, gradients against the oracle; chunk
+    and checkpoint edges (8, 16, 32 tokens) below, at and across, an empty and
+    a one-token sequence, a partial channel block. The workspace starts as
+    NaN, so a checkpoint the forward fails to write shows up."""
+    _check(orc, bf16, [37, 0, 1, 130, 16, 17, 5, 64, 33], 40, from_fwd=True)
+
+
+def test_bwd_from_forward_checkpoints_dense_wide(orc, variant, fwd_sched):
+    """Dense rows over several channel blocks with a ragged channel tail."""
+    _check(orc, True, None, 200, dense_rows=(2, 96), seed=4, from_fwd=True)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_bwd_from_forward_checkpoints_unaligned(orc, bf16, variant):
+    """D = 36: no pipelined forward for bf16 rows of 72 bytes; the
+    checkpointing pass writes them."""
+    _check(orc, bf16, [19, 40, 2], 36, seed=11, from_fwd=True)
