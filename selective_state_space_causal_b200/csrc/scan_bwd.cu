@@ -97,8 +97,9 @@ struct Smem {
     float dzf[kTS][kCh];   // dy * silu'(z)
     float B[kTS][kN];
     float C[kTS][kN];
-    float red[kWarps][kTS][32];  // dB / dC partial sums of each warp's 8 channels
+    float red[kWarps][kTS][32];  // dB (states 0..15) then dC (16..31) sums of each warp's 8 channels
     float out[3][kTS][kCh];      // du, ddt, dz of the chunk
+    float wbuf[kWarps][2][8][32];  // a token pair's dB / dC terms of each warp's 8 channels
 };
 
 // Raw chunk inputs as they sit in global memory, copied in one chunk ahead.
@@ -256,8 +257,10 @@ template <typename T, bool ASYNC>
 __global__ void __launch_bounds__(kThreads)
 scan_bwd_kernel(const BwdParams p)
 {
-    __shared__ Smem sm;
-    __shared__ __align__(16) RawChunk<T> raw[ASYNC ? 2 : 1];
+    // dynamic: with fp32 inputs and copies in flight it is above 48 KB
+    extern __shared__ __align__(16) unsigned char l_smem[];
+    Smem &sm = *reinterpret_cast<Smem *>(l_smem);
+    RawChunk<T> *raw = reinterpret_cast<RawChunk<T> *>(l_smem + sizeof(Smem));
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sub = tid % kTPC, cl = tid / kTPC;
     const int64_t cbase = (int64_t)blockIdx.x * kCh, c = cbase + cl;
@@ -386,10 +389,17 @@ scan_bwd_kernel(const BwdParams p)
                 hist[tl][1] = hr[1];
             }
         }
-        // walk the chunk backwards
+        // walk the chunk backwards. Sums over a channel's 4 lanes wait for a
+        // group of kTPC tokens and then take a transposed butterfly that leaves
+        // token tl + sub's sums in lane `sub`, which writes that token's
+        // outputs; dB / dC terms go through the warp's buffer a token pair at a
+        // time and are summed over the warp's 8 channels from there.
+        float Pq[kTPC], Pu[kTPC], Px[kTPC];  // C.h, G.B, G.(u B + A a h_{t-1}) of my states
+        const int cw = lane >> 2;            // channel within the warp
 #pragma unroll
         for (int tl = kTS - 1; tl >= 0; --tl) {
             float pb[2 * kNPT];  // this lane's dB then dC terms of token tl
+            float q = 0.f, us = 0.f, xs = 0.f;
             if (tl < nt) {
                 const float d = sm.d[tl][cl], u = sm.u[tl][cl], dq = sm.dq[tl][cl];
                 const float *Bn = &sm.B[tl][sub * kNPT], *Cn = &sm.C[tl][sub * kNPT];
@@ -418,26 +428,13 @@ scan_bwd_kernel(const BwdParams p)
                     pb[kNPT + 2 * j + 1] = h1_;
                     G[j] = mul2(a, G[j]);                             // towards h_{t-1}
                 }
-                // sums over the channel's 4 lanes
                 float q0, q1, u0, u1, x0, x1;
                 upk2(qp, q0, q1);
                 upk2(dup, u0, u1);
                 upk2(ddp, x0, x1);
-                float qs = q0 + q1, us = u0 + u1, xs = x0 + x1;
-#pragma unroll
-                for (int w = 1; w < kTPC; w <<= 1) {
-                    qs += __shfl_xor_sync(0xffffffffu, qs, w);
-                    us += __shfl_xor_sync(0xffffffffu, us, w);
-                    xs += __shfl_xor_sync(0xffffffffu, xs, w);
-                }
-                if (sub == 0) {
-                    const float ddt = xs * sm.dsp[tl][cl];
-                    sm.out[0][tl][cl] = dq * dsk + d * us;
-                    sm.out[1][tl][cl] = ddt;
-                    sm.out[2][tl][cl] = sm.dzf[tl][cl] * (qs + dsk * u);
-                    dDsk += dq * u;
-                    ddtb += ddt;
-                }
+                q = q0 + q1;
+                us = u0 + u1;
+                xs = x0 + x1;
             } else {
 #pragma unroll
                 for (int i = 0; i < 2 * kNPT; ++i) pb[i] = 0.f;
@@ -446,35 +443,66 @@ scan_bwd_kernel(const BwdParams p)
 #pragma unroll
                 for (int i = 0; i < 2 * kNPT; ++i) pb[i] = 0.f;
             }
-            // dB / dC: transposed sum over the warp's 8 channels (lane bits 2..4);
-            // afterwards lane (chl, sub) holds the sum of term chl of its sub
+            Pq[tl % kTPC] = q;
+            Pu[tl % kTPC] = us;
+            Px[tl % kTPC] = xs;
+            float *wb = &sm.wbuf[warp][tl & 1][cw][0];
+            *reinterpret_cast<float4 *>(wb + sub * kNPT) = make_float4(pb[0], pb[1], pb[2], pb[3]);
+            *reinterpret_cast<float4 *>(wb + kN + sub * kNPT) = make_float4(pb[4], pb[5], pb[6], pb[7]);
+            if ((tl & 1) == 0) {
+                // tokens tl and tl + 1: lane L sums values 2 (L % 16), +1 of token
+                // tl + L / 16 over the warp's 8 channels
+                __syncwarp();
+                const int sl = lane >> 4, vv = 2 * (lane & 15);
+                f32x2 acc = 0ull;
 #pragma unroll
-            for (int w = 16, half = kNPT; w >= 4; w >>= 1, half >>= 1) {
-                const bool upper = (lane & w) != 0;
+                for (int ch = 0; ch < 8; ++ch) {
+                    const float2 v = *reinterpret_cast<const float2 *>(&sm.wbuf[warp][sl][ch][vv]);
+                    acc = add2(acc, pk2(v.x, v.y));
+                }
+                float r0, r1;
+                upk2(acc, r0, r1);
+                *reinterpret_cast<float2 *>(&sm.red[warp][tl + sl][vv]) = make_float2(r0, r1);
+                __syncwarp();
+            }
+            if (tl % kTPC == 0) {
+                // the group tl .. tl + 3 is complete: transposed butterfly over
+                // the channel's lanes (xor 2, then 1)
 #pragma unroll
-                for (int i = 0; i < half; ++i) {
-                    const float send = upper ? pb[i] : pb[i + half];
-                    const float keep = upper ? pb[i + half] : pb[i];
-                    pb[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                for (int w = kTPC / 2; w >= 1; w >>= 1) {
+                    const bool upper = (sub & w) != 0;
+#pragma unroll
+                    for (int i = 0; i < w; ++i) {
+                        const float sq = upper ? Pq[i] : Pq[i + w], kq = upper ? Pq[i + w] : Pq[i];
+                        const float su = upper ? Pu[i] : Pu[i + w], ku = upper ? Pu[i + w] : Pu[i];
+                        const float sx = upper ? Px[i] : Px[i + w], kx = upper ? Px[i + w] : Px[i];
+                        Pq[i] = kq + __shfl_xor_sync(0xffffffffu, sq, w);
+                        Pu[i] = ku + __shfl_xor_sync(0xffffffffu, su, w);
+                        Px[i] = kx + __shfl_xor_sync(0xffffffffu, sx, w);
+                    }
+                }
+                const int tg = tl + sub;  // the token whose sums this lane now holds
+                if (tg < nt) {
+                    const float d = sm.d[tg][cl], u = sm.u[tg][cl], dq = sm.dq[tg][cl];
+                    const float ddt = Px[0] * sm.dsp[tg][cl];
+                    sm.out[0][tg][cl] = dq * dsk + d * Pu[0];
+                    sm.out[1][tg][cl] = ddt;
+                    sm.out[2][tg][cl] = sm.dzf[tg][cl] * (Pq[0] + dsk * u);
+                    dDsk += dq * u;
+                    ddtb += ddt;
                 }
             }
-            // term index held by this lane: bits (16, 8, 4) of the lane pick
-            // halves (4, 2, 1) of the 8 terms
-            const int term = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
-            sm.red[warp][tl][term * kTPC + sub] = pb[0];
         }
         __syncthreads();
         // dB / dC of the chunk: sum over warps, one atomic per (token, state)
         for (int e = tid; e < kTS * 2 * kN; e += kThreads) {
-            const int tl = e / (2 * kN), r = e % (2 * kN);  // r = term * 4 + sub
+            const int tl = e / (2 * kN), r = e % (2 * kN);  // r < 16: dB state r, else dC state r - 16
             if (tl >= nt) continue;
-            const int term = r / kTPC, sb = r % kTPC;
             float v = 0.f;
 #pragma unroll
             for (int w = 0; w < kWarps; ++w) v += sm.red[w][tl][r];
-            const int n = sb * kNPT + (term % kNPT);
-            float *dst = term < kNPT ? p.dB : p.dC;
-            atomicAdd(dst + (t0 + tl) * kN + n, v);
+            float *dst = r < kN ? p.dB : p.dC;
+            atomicAdd(dst + (t0 + tl) * kN + (r % kN), v);
         }
         // du, ddt, dz of the chunk, channels contiguous
         for (int e = tid; e < kTS * kCh; e += kThreads) {
@@ -502,10 +530,16 @@ scan_bwd_kernel(const BwdParams p)
             atomicAdd(p.dA + c * kN + n, a0);
             atomicAdd(p.dA + c * kN + n + 1, a1);
         }
-        if (sub == 0) {
-            if (p.dDskip) atomicAdd(p.dDskip + c, dDsk);
-            if (p.ddt_bias) atomicAdd(p.ddt_bias + c, ddtb);
-        }
+    }
+    // each lane summed its own tokens' dDskip and ddt_bias terms
+#pragma unroll
+    for (int w = 1; w < kTPC; w <<= 1) {
+        dDsk += __shfl_xor_sync(0xffffffffu, dDsk, w);
+        ddtb += __shfl_xor_sync(0xffffffffu, ddtb, w);
+    }
+    if (cvalid && sub == 0) {
+        if (p.dDskip) atomicAdd(p.dDskip + c, dDsk);
+        if (p.ddt_bias) atomicAdd(p.ddt_bias + c, ddtb);
     }
 }
 
@@ -1137,6 +1171,17 @@ int scan_bwd_variant_for(int64_t S, int64_t D)
 }
 
 template <typename T, bool ASYNC>
+static cudaError_t run_lanes(const BwdParams &p, dim3 grid, cudaStream_t stream)
+{
+    const size_t smem = sizeof(Smem) + (ASYNC ? 2 : 1) * sizeof(RawChunk<T>);
+    cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T, ASYNC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    scan_bwd_kernel<T, ASYNC><<<grid, kThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, bool ASYNC>
 static cudaError_t run_ckpt(const BwdParams &p, dim3 grid, cudaStream_t stream, int *launches)
 {
     const size_t ck_smem = 2 * sizeof(WRaw<T>) + sizeof(float) * kWTS * kN;
@@ -1221,14 +1266,12 @@ cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *laun
                          : run_wide<float, false>(p, grid, stream, launches);
     } else {
         const dim3 grid((unsigned)((a.D + kCh - 1) / kCh), (unsigned)a.S);
-        if (a.bf16) {
-            if (async_ok) scan_bwd_kernel<__nv_bfloat16, true><<<grid, kThreads, 0, stream>>>(p);
-            else scan_bwd_kernel<__nv_bfloat16, false><<<grid, kThreads, 0, stream>>>(p);
-        } else {
-            if (async_ok) scan_bwd_kernel<float, true><<<grid, kThreads, 0, stream>>>(p);
-            else scan_bwd_kernel<float, false><<<grid, kThreads, 0, stream>>>(p);
-        }
-        e = cudaGetLastError();
+        if (a.bf16)
+            e = async_ok ? run_lanes<__nv_bfloat16, true>(p, grid, stream)
+                         : run_lanes<__nv_bfloat16, false>(p, grid, stream);
+        else
+            e = async_ok ? run_lanes<float, true>(p, grid, stream)
+                         : run_lanes<float, false>(p, grid, stream);
     }
     ++*launches;
     return e;
