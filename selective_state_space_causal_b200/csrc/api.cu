@@ -492,15 +492,17 @@ static int scan_bwd_impl(const char *fn, bool have_ckpt, const void *u, const vo
     if (!aligned(workspace, 256))
         return fail(SSM_ERR_MISALIGNED, "%s: workspace must be 256-byte aligned", fn);
     if (tok > 0) {
-        const size_t bytes = (size_t)tok * D * es;
+        // (tok, D) activations against (tok, D) inputs and the (tok, N) B, C rows
+        const size_t bytes = (size_t)tok * D * es, bc_bytes = (size_t)tok * N * es;
         const void *outs[] = {du, ddelta, dz};
         const void *ins[] = {u, delta, z, dy, B, C};
+        const size_t in_bytes[] = {bytes, bytes, bytes, bytes, bc_bytes, bc_bytes};
         for (const void *o : outs) {
             if (!o) continue;
-            for (const void *in : ins) {
-                if (!in) continue;
-                const char *a = static_cast<const char *>(o), *b = static_cast<const char *>(in);
-                if (a < b + bytes && b < a + bytes)
+            for (int i = 0; i < 6; ++i) {
+                if (!ins[i]) continue;
+                const char *a = static_cast<const char *>(o), *b = static_cast<const char *>(ins[i]);
+                if (a < b + in_bytes[i] && b < a + bytes)
                     return fail(SSM_ERR_INVALID_ARGUMENT, "%s: a gradient overlaps an input", fn);
             }
         }

@@ -258,6 +258,16 @@ def test_scan_bwd_rejects(kw, code):
     assert _err()
 
 
+def test_scan_bwd_overlap_uses_bc_extent():
+    """B and C are (tok, N): a gradient right after B's tok x N elements does not
+    overlap it, one that starts inside does."""
+    B = A16 + 0x1000000
+    assert bwd(B=B, C=B, du=B + 64 * 16 * 2 - 2) == -1  # inside B (bf16)
+    assert "overlaps" in _err()
+    bwd(B=B, C=B, du=B + 64 * 16 * 2)  # just past B: no overlap (fails later without a GPU)
+    assert "overlaps" not in _err()
+
+
 def bwd_ckpt(**kw):
     a = dict(u=A16, dt=A16 + 0x200000, A=A16, B=A16, C=A16, Dsk=None, z=None, dtb=None, sp=1,
              h0=None, cu=None, S=1, dy=A16 + 0x400000, dhf=None, du=A16 + 0x600000,

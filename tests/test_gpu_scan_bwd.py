@@ -143,10 +143,12 @@ def test_bwd_deterministic_outputs(variant):
         assert torch.allclose(x, y, rtol=1e-5, atol=1e-5 * float(y.abs().max())), k
 
 
-def test_bwd_packmamba_workload_sampled(orc, variant):
+@pytest.mark.parametrize("from_fwd", [False, True], ids=["own_ckpt", "fwd_ckpt"])
+def test_bwd_packmamba_workload_sampled(orc, variant, from_fwd):
     """The packed 65536-token, 5120-channel training shape: per-token gradients,
     dA, dDskip, ddt_bias and dh0 of sampled channels against the oracle run on
-    those channels alone (channels are independent for these)."""
+    those channels alone (channels are independent for these); also with the
+    checkpoints written by the forward (2.7 GB of them at this shape)."""
     w = synth.WORKLOADS["packmamba_2p8b_varlen_65536"]
     D, tot = w["D"], w["total"]
     lens = synth.sample_lengths(0, tot, w["len_lo"], w["len_hi"])
@@ -157,7 +159,7 @@ def test_bwd_packmamba_workload_sampled(orc, variant):
     a = synth.device_activations(0, tot, D)
     dy = synth.device_activations(1, tot, D)["x"]
     g = _run_bwd(a["x"], a["dt"], p["A"], a["B"], a["C"], dy, p["Dskip"], a["z"], p["dt_bias"],
-                 None, None, cu_d, S)
+                 None, None, cu_d, S, from_fwd=from_fwd)
     rng = np.random.default_rng(0)
     ch = np.sort(rng.choice(D, size=6, replace=False))
     chd = torch.from_numpy(ch).cuda()
