@@ -79,6 +79,8 @@ def parse_args(argv=None):
                     help="skip the Mamba-130M layer, packed, decode and backward workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the headline step as plain launches instead of a CUDA graph")
     ap.add_argument("--replay-windows", type=int, nargs="+", default=[3], metavar="W",
                     help="checkpoint intervals of the replay decode measurement")
     ap.add_argument("--profile-scan-bwd", nargs="?", const="packed", default=None,
@@ -343,7 +345,10 @@ class LongCtxStep:
         bf = torch.bfloat16
         self.xc = torch.empty((self.chunk, self.D), dtype=bf, device="cuda")
         self.y = torch.empty((self.L, self.D), dtype=bf, device="cuda")
-        self.cs = torch.zeros((1, self.D, self.K - 1), dtype=bf, device="cuda")
+        # the conv state alternates between two buffers (chunk j reads cs[j % 2]
+        # and writes cs[(j + 1) % 2]), so the state output rides along with the
+        # conv kernel instead of a second launch after it
+        self.cs = [torch.zeros((1, self.D, self.K - 1), dtype=bf, device="cuda") for _ in range(2)]
         self.h = torch.zeros((1, self.D, N_STATE), device="cuda")
         self.yd = torch.empty((1, self.D), dtype=bf, device="cuda")
 
@@ -352,14 +357,15 @@ class LongCtxStep:
 
     def run(self, ev=None):
         ssm, ly, a = self.ssm, self.layer, self.a
-        self.cs.zero_()
+        self.cs[0].zero_()
         self.h.zero_()
         for j in range(self.nch):
             sl = slice(j * self.chunk, (j + 1) * self.chunk)
             if ev is not None:
                 ev[j][0].record()
-            ssm.ssm_causal_conv1d(a["x"][sl], self.xc, ly.w, bias=ly.b, conv_state_in=self.cs,
-                                  conv_state_out=self.cs)
+            ssm.ssm_causal_conv1d(a["x"][sl], self.xc, ly.w, bias=ly.b,
+                                  conv_state_in=self.cs[j % 2],
+                                  conv_state_out=self.cs[(j + 1) % 2])
             if ev is not None:
                 ev[j][1].record()
             ssm.ssm_selective_scan_fwd(self.xc, a["dt"][sl], ly.A, a["B"][sl], a["C"][sl],
@@ -368,9 +374,9 @@ class LongCtxStep:
             if ev is not None:
                 ev[j][2].record()
         d = self.dec
-        ssm.ssm_selective_state_update(self.cs, self.h, d["x"], d["dt"], d["B"], d["C"], self.yd,
-                                       ly.w, ly.A, z=d["z"], conv_b=ly.b, Dskip=ly.Dskip,
-                                       dt_bias=ly.dt_bias)
+        ssm.ssm_selective_state_update(self.cs[self.nch % 2], self.h, d["x"], d["dt"], d["B"],
+                                       d["C"], self.yd, ly.w, ly.A, z=d["z"], conv_b=ly.b,
+                                       Dskip=ly.Dskip, dt_bias=ly.dt_bias)
 
 
 def bench_headline(args, world, peaks, rank_dev, mufu):
@@ -380,25 +386,54 @@ def bench_headline(args, world, peaks, rank_dev, mufu):
     for _ in range(args.warmup):
         st.run()
     K = args.steps
+    # kernel times: the step with an event pair around every conv and scan call
     evs = [[_events(3) for _ in range(st.nch)] for _ in range(K)]
-    start, stop = _events(2)
     launches0 = st.ssm.ssm_launch_count()
+    p0, p1 = _events(2)
+    _barrier_sync(world)
+    p0.record()
+    for i in range(K):
+        st.run(ev=evs[i])
+    p1.record()
+    _barrier_sync(world)
+    launches_per_step = (st.ssm.ssm_launch_count() - launches0) / K
+    plain_ms = p0.elapsed_time(p1) / K
+    conv_ms = sum(e[0].elapsed_time(e[1]) for row in evs for e in row) / (K * st.nch)
+    scan_ms = sum(e[1].elapsed_time(e[2]) for row in evs for e in row) / (K * st.nch)
+    # the timed steps: the step captured once as a CUDA graph (its 33 library
+    # launches and 2 fills) and replayed, which removes the host's launch gaps
+    graph = None
+    if not args.no_graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            st.run()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            st.run()
+        for _ in range(2):
+            graph.replay()
+    step = graph.replay if graph is not None else st.run
+    launches0 = st.ssm.ssm_launch_count()
+    start, stop = _events(2)
     clocks = ClockSampler(rank_dev)
     clocks.start()
     time.sleep(0.05)
     _barrier_sync(world)
     start.record()
-    for i in range(K):
-        st.run(ev=evs[i])
+    for _ in range(K):
+        step()
     stop.record()
     _barrier_sync(world)
     clk = clocks.stop()
-    launches = st.ssm.ssm_launch_count() - launches0
+    # a replayed graph launches the captured kernels without calling the library
+    launches = launches_per_step * K if graph is not None else (st.ssm.ssm_launch_count()
+                                                                 - launches0)
     if st.ssm.ssm_device_status() != 0:
         raise RuntimeError("a bounded device wait timed out during the timed region")
     ms = start.elapsed_time(stop) / K
-    conv_ms = sum(e[0].elapsed_time(e[1]) for row in evs for e in row) / (K * st.nch)
-    scan_ms = sum(e[1].elapsed_time(e[2]) for row in evs for e in row) / (K * st.nch)
     ms_max = _max_over_ranks(ms, world)
     value = whole_job_rate(st.units(), world, ms_max)
     sha = source_sha(*SCAN_SOURCES)
@@ -408,11 +443,13 @@ def bench_headline(args, world, peaks, rank_dev, mufu):
                              scan_bytes(st.chunk, st.D, 2), scan_ms, mufu, peaks,
                              "longctx_call_8192x8192", sha)
     res = {"value": value, "ms_per_step": ms_max, "step_ms_this_rank": ms, "roofline": roofline,
-           "clocks": clk, "gpu_launches": int(launches),
+           "clocks": clk, "gpu_launches": int(launches), "cuda_graph": graph is not None,
+           "step_ms_without_graph": round(plain_ms, 4),
            "scan_ms_per_step": round(scan_ms * st.nch, 4),
            "conv_roofline": conv_roofline(conv_bytes(st.chunk, st.D, 1, True), conv_ms, peaks,
-                                          "longctx_call_8192x8192", two_launches=True),
-           "launches_per_step": launches / K}
+                                          "longctx_call_8192x8192"),
+           "launches_per_step": launches_per_step}
+    del graph
     if not args.no_e2e:
         res["e2e"] = e2e_longctx(st, world, max(3, K // 4))
     del st
@@ -459,7 +496,7 @@ def e2e_longctx(st, world, steps):
                 dec_dev[k].copy_(host_dec[k], non_blocking=True)
             ev_dec.record(s_in)
         with torch.cuda.stream(s_cmp):
-            st.cs.zero_()
+            st.cs[0].zero_()
             st.h.zero_()
         for j in range(st.nch):
             b, n = g[0] % 2, g[0]
@@ -475,8 +512,8 @@ def e2e_longctx(st, world, steps):
                 if n >= 2:
                     s_cmp.wait_event(ev_out[b])  # its output has been copied out
                 a = stage[b]
-                ssm.ssm_causal_conv1d(a["x"], st.xc, ly.w, bias=ly.b, conv_state_in=st.cs,
-                                      conv_state_out=st.cs)
+                ssm.ssm_causal_conv1d(a["x"], st.xc, ly.w, bias=ly.b, conv_state_in=st.cs[j % 2],
+                                      conv_state_out=st.cs[(j + 1) % 2])
                 ssm.ssm_selective_scan_fwd(st.xc, a["dt"], ly.A, a["B"], a["C"], ystage[b],
                                            Dskip=ly.Dskip, z=a["z"], dt_bias=ly.dt_bias,
                                            h0=st.h, h_final=st.h)
@@ -488,9 +525,9 @@ def e2e_longctx(st, world, steps):
         with torch.cuda.stream(s_cmp):
             s_cmp.wait_event(ev_dec)
             d = dec_dev
-            ssm.ssm_selective_state_update(st.cs, st.h, d["x"], d["dt"], d["B"], d["C"], st.yd,
-                                           ly.w, ly.A, z=d["z"], conv_b=ly.b, Dskip=ly.Dskip,
-                                           dt_bias=ly.dt_bias)
+            ssm.ssm_selective_state_update(st.cs[st.nch % 2], st.h, d["x"], d["dt"], d["B"],
+                                           d["C"], st.yd, ly.w, ly.A, z=d["z"], conv_b=ly.b,
+                                           Dskip=ly.Dskip, dt_bias=ly.dt_bias)
             ev_decdone.record(s_cmp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev_decdone)
@@ -1409,13 +1446,15 @@ def main():
             "config": {"workload": HEADLINE, "batch": 1, "seq_len": 131072, "chunk": 8192,
                        "d_inner": 8192, "d_state": 16, "d_conv": 4,
                        "step": "16 x (causal_conv1d+silu -> selective_scan) over 8192-token "
-                               "chunks, conv state and h carried in place, then 1 decode step",
+                               "chunks, h carried in place and the conv state between two "
+                               "buffers, then 1 decode step; replayed as one CUDA graph",
                        "l2": "inputs (6.4 GB) far larger than L2; no rotation needed",
                        "parallelism": f"replicas x{world}"},
             "roofline": res["roofline"], "mufu_peak": mufu, "clocks": res["clocks"],
             "e2e": res.get("e2e"), "gpu_launches": res["gpu_launches"],
             "launches_per_step": res["launches_per_step"], "conv_roofline": res["conv_roofline"],
-            "scan_ms_per_step": res["scan_ms_per_step"],
+            "scan_ms_per_step": res["scan_ms_per_step"], "cuda_graph": res["cuda_graph"],
+            "step_ms_without_graph": res["step_ms_without_graph"],
             "cpu_baseline": cpu, "workloads": workloads,
         }
         print(json.dumps(line), flush=True)

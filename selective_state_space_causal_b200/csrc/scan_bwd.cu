@@ -28,8 +28,10 @@
 //     dy silu'(z)) and fp32 B and C rows in shared memory; each lane recomputes
 //     its states for the chunk into registers from the checkpoint, then walks
 //     the chunk backwards carrying G in registers.
-// Sums over a channel's 4 lanes use butterflies; dB and dC, summed over
-// channels, go through a transposed shuffle over the warp's 8 channels, a
+// Sums over a channel's 4 lanes wait for a group of 4 tokens and take a
+// transposed butterfly that leaves one token's sums in each lane; dB and dC,
+// summed over channels, go through a per-warp shared buffer a token pair at a
+// time (each lane sums one pair of values over the warp's 8 channels), a
 // shared-memory sum over the CTA's warps, and one fp32 atomic per (token,
 // state) and CTA. dA, dDskip and ddt_bias (summed over sequences) take one
 // atomic per CTA and channel. The atomics make the last bits of those sums
