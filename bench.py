@@ -343,7 +343,14 @@ class LongCtxStep:
         self.a = synth.device_activations(seed + 1, self.L, self.D)
         self.dec = synth.device_activations(seed + 101, 1, self.D)
         bf = torch.bfloat16
-        self.xc = torch.empty((self.chunk, self.D), dtype=bf, device="cuda")
+        # chunk j's conv output goes to xcs[j % 2]: the conv of chunk j + 1 runs
+        # on a second stream while the scan of chunk j runs (it needs only the
+        # conv state, not h), on the SMs the scan's grid leaves half empty
+        self.xcs = [torch.empty((self.chunk, self.D), dtype=bf, device="cuda") for _ in range(2)]
+        self.xc = self.xcs[0]
+        self.s_conv = torch.cuda.Stream()
+        self.ev_conv = [torch.cuda.Event() for _ in range(self.nch)]
+        self.ev_scan = [torch.cuda.Event() for _ in range(self.nch)]
         self.y = torch.empty((self.L, self.D), dtype=bf, device="cuda")
         # the conv state alternates between two buffers (chunk j reads cs[j % 2]
         # and writes cs[(j + 1) % 2]), so the state output rides along with the
@@ -355,24 +362,48 @@ class LongCtxStep:
     def units(self):
         return self.L * self.D
 
-    def run(self, ev=None):
+    def conv_only(self):
+        """The step's 16 conv calls alone, one after another."""
         ssm, ly, a = self.ssm, self.layer, self.a
-        self.cs[0].zero_()
-        self.h.zero_()
         for j in range(self.nch):
             sl = slice(j * self.chunk, (j + 1) * self.chunk)
-            if ev is not None:
-                ev[j][0].record()
-            ssm.ssm_causal_conv1d(a["x"][sl], self.xc, ly.w, bias=ly.b,
+            ssm.ssm_causal_conv1d(a["x"][sl], self.xcs[j % 2], ly.w, bias=ly.b,
                                   conv_state_in=self.cs[j % 2],
                                   conv_state_out=self.cs[(j + 1) % 2])
+
+    def run(self, ev=None):
+        """One step; ev[j] (4 events per chunk) brackets chunk j's conv (on the
+        conv stream) and scan (on the current stream)."""
+        import torch
+
+        ssm, ly, a = self.ssm, self.layer, self.a
+        main, sc = torch.cuda.current_stream(), self.s_conv
+        self.cs[0].zero_()
+        self.h.zero_()
+        sc.wait_stream(main)
+        for j in range(self.nch):
+            sl = slice(j * self.chunk, (j + 1) * self.chunk)
+            with torch.cuda.stream(sc):
+                if j >= 2:
+                    sc.wait_event(self.ev_scan[j - 2])  # the scan two back has read xcs[j % 2]
+                if ev is not None:
+                    ev[j][0].record(sc)
+                ssm.ssm_causal_conv1d(a["x"][sl], self.xcs[j % 2], ly.w, bias=ly.b,
+                                      conv_state_in=self.cs[j % 2],
+                                      conv_state_out=self.cs[(j + 1) % 2])
+                if ev is not None:
+                    ev[j][1].record(sc)
+                self.ev_conv[j].record(sc)
+            main.wait_event(self.ev_conv[j])
             if ev is not None:
-                ev[j][1].record()
-            ssm.ssm_selective_scan_fwd(self.xc, a["dt"][sl], ly.A, a["B"][sl], a["C"][sl],
+                ev[j][2].record(main)
+            ssm.ssm_selective_scan_fwd(self.xcs[j % 2], a["dt"][sl], ly.A, a["B"][sl], a["C"][sl],
                                        self.y[sl], Dskip=ly.Dskip, z=a["z"][sl],
                                        dt_bias=ly.dt_bias, h0=self.h, h_final=self.h)
             if ev is not None:
-                ev[j][2].record()
+                ev[j][3].record(main)
+            self.ev_scan[j].record(main)
+        main.wait_stream(sc)
         d = self.dec
         ssm.ssm_selective_state_update(self.cs[self.nch % 2], self.h, d["x"], d["dt"], d["B"],
                                        d["C"], self.yd, ly.w, ly.A, z=d["z"], conv_b=ly.b,
@@ -387,7 +418,7 @@ def bench_headline(args, world, peaks, rank_dev, mufu):
         st.run()
     K = args.steps
     # kernel times: the step with an event pair around every conv and scan call
-    evs = [[_events(3) for _ in range(st.nch)] for _ in range(K)]
+    evs = [[_events(4) for _ in range(st.nch)] for _ in range(K)]
     launches0 = st.ssm.ssm_launch_count()
     p0, p1 = _events(2)
     _barrier_sync(world)
@@ -398,8 +429,17 @@ def bench_headline(args, world, peaks, rank_dev, mufu):
     _barrier_sync(world)
     launches_per_step = (st.ssm.ssm_launch_count() - launches0) / K
     plain_ms = p0.elapsed_time(p1) / K
-    conv_ms = sum(e[0].elapsed_time(e[1]) for row in evs for e in row) / (K * st.nch)
-    scan_ms = sum(e[1].elapsed_time(e[2]) for row in evs for e in row) / (K * st.nch)
+    conv_in_step_ms = sum(e[0].elapsed_time(e[1]) for row in evs for e in row) / (K * st.nch)
+    scan_ms = sum(e[2].elapsed_time(e[3]) for row in evs for e in row) / (K * st.nch)
+    # the conv calls alone (in the step they run beside the scans, so their
+    # event times there measure waiting for room, not the kernel)
+    cevs = [_events(2) for _ in range(K)]
+    for i in range(K):
+        cevs[i][0].record()
+        st.conv_only()
+        cevs[i][1].record()
+    torch.cuda.synchronize()
+    conv_ms = sum(e[0].elapsed_time(e[1]) for e in cevs) / (K * st.nch)
     # the timed steps: the step captured once as a CUDA graph (its 33 library
     # launches and 2 fills) and replayed, which removes the host's launch gaps
     graph = None
@@ -446,8 +486,11 @@ def bench_headline(args, world, peaks, rank_dev, mufu):
            "clocks": clk, "gpu_launches": int(launches), "cuda_graph": graph is not None,
            "step_ms_without_graph": round(plain_ms, 4),
            "scan_ms_per_step": round(scan_ms * st.nch, 4),
-           "conv_roofline": conv_roofline(conv_bytes(st.chunk, st.D, 1, True), conv_ms, peaks,
-                                          "longctx_call_8192x8192"),
+           "conv_roofline": dict(conv_roofline(conv_bytes(st.chunk, st.D, 1, True), conv_ms,
+                                               peaks, "longctx_call_8192x8192"),
+                                 measured="the 16 conv calls alone; in the step each runs "
+                                          "beside a scan",
+                                 in_step_event_ms=round(conv_in_step_ms, 5)),
            "launches_per_step": launches_per_step}
     del graph
     if not args.no_e2e:
@@ -1447,7 +1490,8 @@ def main():
                        "d_inner": 8192, "d_state": 16, "d_conv": 4,
                        "step": "16 x (causal_conv1d+silu -> selective_scan) over 8192-token "
                                "chunks, h carried in place and the conv state between two "
-                               "buffers, then 1 decode step; replayed as one CUDA graph",
+                               "buffers, chunk j+1's conv on a second stream beside chunk j's "
+                               "scan, then 1 decode step; replayed as one CUDA graph",
                        "l2": "inputs (6.4 GB) far larger than L2; no rotation needed",
                        "parallelism": f"replicas x{world}"},
             "roofline": res["roofline"], "mufu_peak": mufu, "clocks": res["clocks"],
