@@ -708,29 +708,53 @@ def bench_layer(args, world, peaks, mufu):
     for i in range(args.warmup):
         st.run(i)
     K = max(args.steps, 50)
+    # kernel times: event pairs around the conv and the scan of every step
     evs = [_events(3) for _ in range(K)]
-    s0, s1 = _events(2)
     l0 = st.ssm.ssm_launch_count()
+    for i in range(K):
+        st.run(i, ev=evs[i])
+    torch.cuda.synchronize()
+    launches_per_step = (st.ssm.ssm_launch_count() - l0) / K
+    conv_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
+    scan_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    # the timed steps: each input set's step captured once as a CUDA graph
+    graphs = []
+    if not args.no_graph:
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for i in range(st.SETS):
+                st.run(i)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        for i in range(st.SETS):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                st.run(i)
+            graphs.append(g)
+        for g in graphs:
+            g.replay()
+    step = (lambda i: graphs[i % st.SETS].replay()) if graphs else st.run
+    s0, s1 = _events(2)
     _barrier_sync(world)
     s0.record()
     for i in range(K):
-        st.run(i, ev=evs[i])
+        step(i)
     s1.record()
     _barrier_sync(world)
-    launches = st.ssm.ssm_launch_count() - l0
     ms = _max_over_ranks(s0.elapsed_time(s1) / K, world)
-    conv_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / K
-    scan_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / K
+    del graphs
     variant = st.ssm.ssm_scan_variant_for(st.Bn, st.D)
     res = {"value": whole_job_rate(st.units(), world, ms), "unit": UNIT, "ms_per_step": ms,
-           "gpu_launches_per_step": launches / K,
+           "gpu_launches_per_step": launches_per_step, "cuda_graph": not args.no_graph,
            "roofline": scan_roofline(SCAN_KERNELS.get(variant[1], "scan_kernel"), variant,
                                      st.tok * st.D * N_STATE, scan_bytes(st.tok, st.D, st.Bn),
                                      scan_ms, mufu, peaks, LAYER, source_sha(*SCAN_SOURCES)),
            "conv_roofline": conv_roofline(conv_bytes(st.tok, st.D, st.Bn, False), conv_ms, peaks,
                                           LAYER),
            "step": "causal_conv1d+silu -> selective_scan (h_final) -> 1 decode step; "
-                   "4 rotating input sets (~600 MB) larger than L2"}
+                   "4 rotating input sets (~600 MB) larger than L2; each set's step "
+                   "replayed as a CUDA graph"}
 
     res["scan_bwd"] = bench_scan_bwd(world, st.layer, st.sets[0], None, st.Bn, mufu, peaks,
                                      label="Mamba-130M layer 8 x 2048 x 1536", n=10)
