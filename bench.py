@@ -910,6 +910,34 @@ def decode_bytes_per_step(Bt, D):
             + Bt * N_STATE * 2 * 2 + D * (4 * 4 + 3 * 4 + N_STATE * 4))
 
 
+def _time_block(world, steps, use_graph):
+    """Device time (ms, max over ranks) of a block of step callables run back
+    to back: captured as one CUDA graph outside the timed region and replayed
+    inside it, or as plain launches."""
+    import torch
+
+    g = None
+    if use_graph:
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):  # recorded, not run
+            for f in steps:
+                f()
+    s0, s1 = _events(2)
+    _barrier_sync(world)
+    s0.record()
+    if g is not None:
+        g.replay()
+    else:
+        for f in steps:
+            f()
+    s1.record()
+    _barrier_sync(world)
+    ms = _max_over_ranks(s0.elapsed_time(s1), world)
+    del g
+    return ms
+
+
 def bench_decode(args, world, peaks, mufu):
     import torch
 
@@ -933,22 +961,17 @@ def bench_decode(args, world, peaks, mufu):
     cs0, h0 = cs.clone(), h.clone()
     block = 100
     yd = torch.empty((Bt, D), dtype=bf, device="cuda")
-    s0, s1 = _events(2)
     total_ms, done, kernel_ms = 0.0, 0, []
+
     def one(s):
         ssm.ssm_selective_state_update(cs, h, s["x"], s["dt"], s["B"], s["C"], yd, ly.w, ly.A,
                                        z=s["z"], conv_b=ly.b, Dskip=ly.Dskip, dt_bias=ly.dt_bias)
 
     for b0 in range(0, steps, block):
         blk = [synth.device_activations(5000 + b0 + i, Bt, D) for i in range(block)]
-        # the steps/s value: the block back to back, no events between steps
-        _barrier_sync(world)
-        s0.record()
-        for s in blk:
-            one(s)
-        s1.record()
-        _barrier_sync(world)
-        total_ms += _max_over_ranks(s0.elapsed_time(s1), world)
+        # the steps/s value: the block back to back (one CUDA graph), no events
+        # between steps
+        total_ms += _time_block(world, [lambda s=s: one(s) for s in blk], not args.no_graph)
         # the kernel time: the same block again, an event pair around each step
         evs = [_events(2) for _ in range(block)]
         for s, ev in zip(blk, evs):
@@ -971,7 +994,8 @@ def bench_decode(args, world, peaks, mufu):
                         "traffic": recorded_traffic("decode_bulk_kernel", DECODE,
                                                     source_sha("decode.cu", "common.cuh",
                                                                "tma.cuh"))},
-           "step": "ssm_selective_state_update, 256 rows x 8192 channels, fresh inputs per step"}
+           "step": "ssm_selective_state_update, 256 rows x 8192 channels, fresh inputs per "
+                   "step; blocks of 100 steps replayed as CUDA graphs"}
     if not args.no_e2e:
         one = synth.device_activations(6000, Bt, D)
         host_in = {k: v.cpu().pin_memory() for k, v in one.items()}
@@ -993,7 +1017,8 @@ def bench_decode(args, world, peaks, mufu):
                              "copied out; states stay on the device; pipelined"}
         del csx, hx
     for W in args.replay_windows:
-        res[f"replay_w{W}"] = bench_replay(peaks, world, ly, cs0, h0, W, steps, mufu)
+        res[f"replay_w{W}"] = bench_replay(peaks, world, ly, cs0, h0, W, steps, mufu,
+                                           not args.no_graph)
     del cs, h, cs0, h0
     torch.cuda.empty_cache()
     return res
@@ -1119,7 +1144,7 @@ def replay_bytes_per_step(Bt, D, W, keep_lo=True):
     return total / W
 
 
-def bench_replay(peaks, world, ly, cs, h, W, steps, mufu):
+def bench_replay(peaks, world, ly, cs, h, W, steps, mufu, use_graph=True):
     """Batch-256 decode through the replay kernels (checkpoint + input buffer,
     bf16 checkpoint copy), on the same prefill states and the same kind of
     fresh per-step inputs as the eager decode measurement."""
@@ -1134,22 +1159,18 @@ def bench_replay(peaks, world, ly, cs, h, W, steps, mufu):
     csr = cs.clone()
     ssm.ssm_replay_reset(rep)
     yd = torch.empty((Bt, D), dtype=torch.bfloat16, device="cuda")
-    s0, s1 = _events(2)
     block = 100
     total_ms = 0.0
     done = 0
     l0 = ssm.ssm_launch_count()
+
+    def one(s):
+        ssm.ssm_replay_state_update(csr, rep, s["x"], s["dt"], s["B"], s["C"], yd, ly.w, ly.A,
+                                    z=s["z"], conv_b=ly.b, Dskip=ly.Dskip, dt_bias=ly.dt_bias)
+
     for b0 in range(0, steps, block):
         blk = [synth.device_activations(5000 + b0 + i, Bt, D) for i in range(block)]
-        _barrier_sync(world)
-        s0.record()
-        for s in blk:
-            ssm.ssm_replay_state_update(csr, rep, s["x"], s["dt"], s["B"], s["C"], yd, ly.w, ly.A,
-                                        z=s["z"], conv_b=ly.b, Dskip=ly.Dskip,
-                                        dt_bias=ly.dt_bias)
-        s1.record()
-        _barrier_sync(world)
-        total_ms += _max_over_ranks(s0.elapsed_time(s1), world)
+        total_ms += _time_block(world, [lambda s=s: one(s) for s in blk], use_graph)
         done += block
         del blk
     launches = ssm.ssm_launch_count() - l0
@@ -1163,7 +1184,8 @@ def bench_replay(peaks, world, ly, cs, h, W, steps, mufu):
         "mufu_frac": round(exps_step / (per * 1e-3) / 1e9 / mufu["gexp_per_s"], 4),
         "gpu_launches_per_step": launches / done,
         "step": f"ssm_replay_state_update (checkpoint every {W} tokens, bf16 copy for outputs), "
-                "256 rows x 8192 channels, fresh inputs per step"}
+                "256 rows x 8192 channels, fresh inputs per step; blocks of 100 steps "
+                "replayed as CUDA graphs"}
     del rep, csr
     return res
 
