@@ -4,11 +4,14 @@
 Headline step: one long-context prefill at the Falcon-Mamba-7B layer shape,
 then one decode token. The 131072-token sequence (d_inner 8192, N 16, conv
 width 4, bf16 activations, fp32 state) is processed in 16 calls of 8192
-tokens, each a causal conv1d + SiLU and a selective scan, with the conv state
-and the SSM state carried in place between calls; the row then takes one
-decode step from the final states. The headline value is tokens x channels per
-second of the whole step (Gtoken*ch/s), with the inputs resident in HBM (6.4 GB
-of inputs, far larger than the 126 MB L2, so no step finds them in L2).
+tokens, each a causal conv1d + SiLU and a selective scan, with the SSM state
+carried in place and the conv state between two buffers; the conv of chunk
+j+1 runs on a second stream beside the scan of chunk j (it needs only the conv
+state); the row then takes one decode step from the final states. The step is
+captured once as a CUDA graph and replayed (--no-graph: plain launches). The
+headline value is tokens x channels per second of the whole step
+(Gtoken*ch/s), with the inputs resident in HBM (6.4 GB of inputs, far larger
+than the 126 MB L2, so no step finds them in L2).
 
 The scan, which dominates the step, is bound by the special-function unit (16
 ex2 per token and channel); its roofline is exps per second against the
