@@ -64,7 +64,7 @@ ORACLE_CHANNELS = 256     # channel sample of the CPU baseline on the large work
 SCAN_KERNELS = {1: "scan_kernel", 2: "scan_tma_kernel", 3: "scan_ts_kernel", 4: "scan_tma_kernel",
                 5: "scan_tma_kernel", 6: "scan_ws_kernel", 7: "scan_warp_kernel",
                 8: "scan_staged_kernel", 9: "scan_pipe_kernel", 10: "scan_pipe_kernel",
-                11: "scan_pipe_kernel"}
+                11: "scan_pipe_kernel", 12: "scan_wide_kernel"}
 SCAN_SOURCES = ("scan.cu", "scan_pipe.cu", "scan_pipe.cuh", "scan_parts.cuh", "common.cuh", "tma.cuh")
 
 
@@ -1302,7 +1302,7 @@ def bench_reference(args):
 # sweeps and profiler cases
 # ---------------------------------------------------------------------------
 
-SWEEP_VARIANTS = [(0, 0), (4, 10), (4, 11), (4, 9), (8, 9), (2, 9), (2, 8), (4, 1), (8, 2)]
+SWEEP_VARIANTS = [(0, 0), (4, 10), (4, 11), (4, 9), (8, 9), (16, 12), (2, 9), (2, 8), (4, 1), (8, 2)]
 
 
 def scan_sweep(variants, peaks):

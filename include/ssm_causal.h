@@ -100,7 +100,10 @@ unsigned long long ssm_launch_count(void);
  * 9 and 10: the chunk-pipelined kernel, TMA staging four stages deep, the next
  * chunk's per-token work interleaved with this chunk's recurrence, 16- and
  * 32-token chunks, 2, 4 or 8 states per lane; 11: schedule 10 at 4 states
- * per lane with the register budget of two CTAs per SM; the library's choice).
+ * per lane with the register budget of two CTAs per SM; 12: one lane per
+ * channel with all 16 states, 128-lane CTAs, TMA staging, no shuffles, for
+ * shapes with many (sequence, channel) pairs; it takes any states_per_lane
+ * value and reports 16; the library's choice).
  * 0 lets the library choose. Applies to the
  * 16-byte vector path; the scalar path always uses 4 states per lane and
  * register prefetch. A variant whose alignment needs the inputs do not meet

@@ -156,10 +156,10 @@ unsigned long long ssm_launch_count(void) { return g_launches.load(std::memory_o
 int ssm_set_scan_variant(int npt, int sched)
 {
     const bool npt_ok = npt == 0 || npt == 2 || npt == 4 || npt == 8 || npt == 16;
-    const bool sched_ok = sched >= 0 && sched <= 11;
+    const bool sched_ok = sched >= 0 && sched <= 12;
     if (!npt_ok || !sched_ok)
         return fail(SSM_ERR_INVALID_ARGUMENT,
-                    "ssm_set_scan_variant: states per lane 0, 2, 4, 8 or 16; schedule 0..11");
+                    "ssm_set_scan_variant: states per lane 0, 2, 4, 8 or 16; schedule 0..12");
     ssm::set_scan_variant(npt, sched);
     return ok();
 }

@@ -1512,8 +1512,8 @@ int g_forced_npt = 0, g_forced_sched = 0;
 
 // Variants: NPT states per lane; schedule 1: register prefetch, 2: TMA
 // staging, 3: TMA staging with time-split chunks; CH channels per CTA, TCH
-// tokens per chunk. *piped: set when the pipelined kernel (schedules 9-11)
-// ran; it alone writes p.ckpt.
+// tokens per chunk. *piped: set when the pipelined kernels (schedules 9-12)
+// ran; they alone write p.ckpt.
 template <typename T, int VEC>
 cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n, bool *piped)
 {
@@ -1521,7 +1521,7 @@ cudaError_t dispatch(const Params &p, int npt, int sched, cudaStream_t s, int *n
         (void)npt; (void)sched; (void)piped;
         return run<Cfg<T, 4, 0, 32, 64, 1>, T>(p, s, n);
     } else {
-        if (sched >= 9 && sched <= 11 && p.tok > 0) {
+        if (sched >= 9 && sched <= 12 && p.tok > 0) {
             cudaError_t e = launch_scan_pipe(p, sizeof(T) == 2, npt, sched, s, n);
             if (e != cudaErrorNotSupported) {
                 *piped = e == cudaSuccess;
@@ -1606,6 +1606,10 @@ int sm_count()
 }
 
 // Measured on B200 (exponential rate against the special-function peak):
+// with at least two waves of its 128-lane CTAs (three per SM), one lane per
+// channel (schedule 12) beats 8 states per lane in the pipelined kernel on
+// the packed 65536 x 5120 workload (0.684 against 0.668) and on 32 x 2048 x
+// 5120 (0.657 against 0.643). Earlier measurements of the other schedules:
 // 8 states per lane with double-buffered TMA staging has the fewest
 // instructions per exponential and wins once the GPU holds about 20 warps per
 // SM of it (packed 65536 x 5120: 0.60 against 0.52 for the next best); below
@@ -1619,7 +1623,10 @@ void pick_variant(int64_t S, int64_t D, int *npt, int *sched)
     const int64_t chains = S * D * kN;            // (sequence, channel, state) recurrences
     const int64_t per_sm = chains / sm_count();
     int npt_auto, sched_auto;
-    if (per_sm >= 8 * 640) {
+    if (per_sm >= 2 * 3 * 128 * kN) {
+        npt_auto = 16;          // one lane per channel: two full waves of 3 CTAs per SM
+        sched_auto = 12;
+    } else if (per_sm >= 8 * 640) {
         npt_auto = 8;           // about 20 warps per SM of 8-state lanes
         sched_auto = 9;
     } else if (per_sm >= 4 * 128) {
@@ -1641,7 +1648,8 @@ void scan_variant_for(int64_t S, int64_t D, int *npt, int *sched) { pick_variant
 void set_scan_variant(int npt, int sched)
 {
     g_forced_npt = (npt == 2 || npt == 4 || npt == 8 || npt == 16) ? npt : 0;
-    g_forced_sched = (sched >= 1 && sched <= 11) ? sched : 0;
+    g_forced_sched = (sched >= 1 && sched <= 12) ? sched : 0;
+    if (g_forced_sched == 12) g_forced_npt = 16;  // one lane per channel, whatever was asked
 }
 
 size_t scan_order_bytes(int64_t S) { return (size_t)((S * 4 + 255) / 256) * 256; }

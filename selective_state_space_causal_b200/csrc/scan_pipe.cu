@@ -14,8 +14,9 @@ int read_pipe_status(bool clear)
     return (a < 0 || b < 0) ? -1 : (a | b);
 }
 
-// Schedules 9 and 10 (16- and 32-token chunks) and 11 (schedule 10 at 4 states
-// per lane with up to 255 registers, two CTAs per SM; for bf16) for 16-byte
+// Schedules 9 and 10 (16- and 32-token chunks), 11 (schedule 10 at 4 states
+// per lane with up to 255 registers, two CTAs per SM; for bf16) and 12 (one
+// lane per channel with all 16 states, 128-lane CTAs) for 16-byte
 // aligned rows (D a multiple of 8 for bf16, of 4 for fp32);
 // cudaErrorNotSupported when the tensor maps cannot be encoded. CTAs of four
 // warps. With p.ckpt the kernels that also write the backward pass's

@@ -1,4 +1,4 @@
-// scan_pipe.cuh -- the chunk-pipelined selective scan (schedules 9 to 11,
+// scan_pipe.cuh -- the chunk-pipelined selective scan (schedules 9 to 12,
 // sm_100a). Included by scan_pipe.cu (the kernels as the forward uses them)
 // and scan_pipe_ckpt.cu (the same kernels, also writing the state before every
 // 8th token of each sequence for the backward pass); the two compile apart.
@@ -675,9 +675,13 @@ cudaError_t run_pipe(const Params &p, cudaStream_t stream, int *launches)
 }
 
 template <bool CK>
+cudaError_t launch_wide_cfg(const Params &p, bool bf16, cudaStream_t stream, int *launches);
+
+template <bool CK>
 cudaError_t launch_pipe_cfg(const Params &p, bool bf16, int npt, int sched, cudaStream_t stream,
                             int *launches)
 {
+    if (sched == 12) return launch_wide_cfg<CK>(p, bf16, stream, launches);
     const bool lng = sched == 10;
     if (bf16) {
         using T = __nv_bfloat16;
@@ -691,6 +695,382 @@ cudaError_t launch_pipe_cfg(const Params &p, bool bf16, int npt, int sched, cuda
     if (npt == 8) return run_pipe<PipeCfg<float, 8, 64, 16>, float, CK>(p, stream, launches);
     if (npt == 2) return run_pipe<PipeCfg<float, 2, 16, 32>, float, CK>(p, stream, launches);
     return run_pipe<PipeCfg<float, 4, 32, 16>, float, CK>(p, stream, launches);
+}
+
+// ---------------------------------------------------------------------------
+// Schedule 12: one lane per channel, all 16 states of the channel in the lane.
+//
+// For shapes with many (sequence, channel) pairs per SM. With a channel's
+// states in one lane the readout needs no shuffles, every lane of a warp reads
+// a token's B and C rows at one address (one shared-memory wavefront per
+// 16-byte load, where the split-lane kernels pay two), and the per-token
+// pre-pass (softplus, silu, delta*u) stays in the lane's registers instead of
+// going through shared memory. Per token and warp that is 8 broadcast loads
+// and 3 two-byte column loads against 16 warp-wide ex2, about half the
+// shared-memory wavefronts per exponential of the 8-state kernel. The price is
+// a longer chain: a lane walks all 16 exponentials of each token, so one
+// sequence takes twice as long as with 8 states per lane, and the kernel needs
+// enough (sequence, channel) pairs to fill the SMs (the packed workload has
+// 43 x 5120).
+//
+// A CTA of 128 lanes owns one sequence and 128 channels. Raw u, dt, z tiles
+// (TCH x 128) and B, C rows (TCH x 16) arrive by TMA (plain per-CTA copies of
+// this GPU's memory, no multicast) into one of RS stages; chunk j is issued
+// after the barrier that ends iteration j - RS, so RS - 1 chunks are in
+// flight. Iteration k runs chunk k's tokens straight from its raw stage and
+// its fp32 B and C rows, then widens chunk k+1's B and C rows to fp32 (bf16
+// inputs; fp32 rows are read from the raw stage), then one CTA barrier.
+// Tokens past the sequence end get delta = 0 and delta*u = 0 (the state is
+// unchanged) and are not stored.
+template <typename T, int TCH_, int RS_, int MINB_>
+struct WideCfg {
+    static constexpr int CH = 128, THREADS = 128, TCH = TCH_, RS = RS_, MINB = MINB_;
+    static constexpr size_t RAW_ACT = sizeof(T) * TCH * CH;
+    static constexpr size_t RAW_BC = sizeof(T) * TCH * kN;
+    static constexpr size_t STAGE = 3 * align128(RAW_ACT) + 2 * align128(RAW_BC);
+    static constexpr size_t BCF = 4 * (size_t)TCH * kN;   // one chunk's B (or C) rows in fp32
+    static constexpr size_t OFF_B = RS * STAGE;
+    static constexpr size_t OFF_C = OFF_B + 2 * BCF;
+    static constexpr size_t OFF_BAR = align128(OFF_C + 2 * BCF);
+    static constexpr size_t SMEM = OFF_BAR + 8 * RS;
+    // B or C elements one thread widens per chunk (threads 0-63: B, 64-127: C)
+    static constexpr int EPT = TCH * kN / (THREADS / 2);
+    static_assert(TCH % 2 == 0, "token pairs");
+    static_assert(sizeof(T) == 4 || EPT == 4 || EPT == 8, "8- or 16-byte raw B and C pieces");
+    static_assert(RAW_ACT % 128 == 0 && RAW_BC % 128 == 0, "TMA tiles stay 128-byte aligned");
+    static_assert(RS >= 2, "at least one chunk in flight");
+};
+
+template <class K, typename T, bool SP, bool GZ, bool CK>
+struct Wide {
+    static constexpr int TCH = K::TCH, CH = K::CH;
+    static_assert(TCH % kCkTok == 0, "checkpoints fall on chunk boundaries");
+    unsigned char *smem;
+    const Params &p;
+    int tid;
+    int64_t c0, end;
+    bool cvalid;
+    float dtb, dsk;
+    f32x2 A2p[8], hp[8];  // A * log2(e) and the state, two states per register
+    float *ckb;  // this lane's state checkpoints for the backward pass, or null
+
+    // The lane's 16 states as checkpoint j of its sequence (the state before
+    // the sequence's token 8j).
+    __device__ __forceinline__ void store_ckpt(int64_t j) const
+    {
+        float4 *dst = reinterpret_cast<float4 *>(ckb + j * p.D * kN);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float4 v;
+            upk2(hp[2 * q], v.x, v.y);
+            upk2(hp[2 * q + 1], v.z, v.w);
+            dst[q] = v;
+        }
+    }
+
+    __device__ __forceinline__ Wide(unsigned char *s, const Params &p_) : smem(s), p(p_) {}
+
+    __device__ __forceinline__ T *raw(int stage, int which) const
+    {
+        size_t off = (size_t)stage * K::STAGE;
+        off += which < 3 ? (size_t)which * align128(K::RAW_ACT)
+                         : 3 * align128(K::RAW_ACT) + (size_t)(which - 3) * align128(K::RAW_BC);
+        return reinterpret_cast<T *>(smem + off);
+    }
+    // fp32 B (which 0) or C (which 1) rows of the chunk in `stage` / buffer `buf`
+    __device__ __forceinline__ const float *bc(int which, int buf, int stage) const
+    {
+        if constexpr (sizeof(T) == 4) {
+            (void)buf;
+            return reinterpret_cast<const float *>(raw(stage, 3 + which));
+        } else {
+            (void)stage;
+            return reinterpret_cast<const float *>(smem + (which ? K::OFF_C : K::OFF_B) + buf * K::BCF);
+        }
+    }
+
+    // B and C rows of the chunk in `stage` to fp32 buffer BUF (bf16 only).
+    template <int BUF>
+    __device__ __forceinline__ void widen(int stage) const
+    {
+        if constexpr (sizeof(T) == 2) {
+            const int which = tid >= K::THREADS / 2, i = tid & (K::THREADS / 2 - 1);
+            const uint32_t *src = reinterpret_cast<const uint32_t *>(raw(stage, 3 + which)) + i * (K::EPT / 2);
+            float *dst = reinterpret_cast<float *>(smem + (which ? K::OFF_C : K::OFF_B) + BUF * K::BCF) +
+                         i * K::EPT;
+            if constexpr (K::EPT == 4) {
+                const uint2 v = *reinterpret_cast<const uint2 *>(src);
+                *reinterpret_cast<float4 *>(dst) = make_float4(
+                    __uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                    __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+            } else {
+                const uint4 v = *reinterpret_cast<const uint4 *>(src);
+                *reinterpret_cast<float4 *>(dst) = make_float4(
+                    __uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                    __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+                *reinterpret_cast<float4 *>(dst + 4) = make_float4(
+                    __uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u),
+                    __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
+            }
+        } else {
+            (void)stage;
+        }
+    }
+
+    // One token: 16 exponentials, the state update, the readout, skip, gate.
+    __device__ __forceinline__ float token(float d, float du, const float *b, const float *c)
+    {
+        const f32x2 dv = pk2(d, d), xv = pk2(du, du);
+        f32x2 bb[8], cc[8];
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) lds_2x2(b + 2 * j, bb[j], bb[j + 1]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float a0, a1;
+            upk2(mul2(dv, A2p[j]), a0, a1);
+            hp[j] = fma2(pk2(ex2_approx(a0), ex2_approx(a1)), hp[j], mul2(xv, bb[j]));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) lds_2x2(c + 2 * j, cc[j], cc[j + 1]);
+        f32x2 acc0 = mul2(cc[0], hp[0]), acc1 = mul2(cc[1], hp[1]);
+#pragma unroll
+        for (int j = 2; j < 8; j += 2) {
+            acc0 = fma2(cc[j], hp[j], acc0);
+            acc1 = fma2(cc[j + 1], hp[j + 1], acc1);
+        }
+        float s0, s1;
+        upk2(add2(acc0, acc1), s0, s1);
+        return s0 + s1;
+    }
+
+    // The tokens of chunk k (nt valid, starting at t0) from raw stage `stage`
+    // and B/C buffer BUF; kc: the checkpoint index of the chunk's first token.
+    template <int BUF, bool MASK>
+    __device__ __forceinline__ void chunk(int stage, int64_t t0, int nt, int64_t kc)
+    {
+        const T *rU = raw(stage, 0), *rDT = raw(stage, 1), *rZ = raw(stage, 2);
+        const float *b = bc(0, BUF, stage), *c = bc(1, BUF, stage);
+        T *dst = static_cast<T *>(p.y) + t0 * p.D + c0;
+        // one token pair per trip: unrolled further, the compiler hoists the
+        // B and C rows of later tokens (174 registers at two pairs per trip,
+        // 255 and spills at a full chunk), which leaves two CTAs per SM
+        // instead of three, and ran slower (packed workload 0.62 against
+        // 0.68 of the ex2 peak)
+#pragma unroll 1
+        for (int t = 0; t < TCH; t += 2) {
+            const f32x2 v = add2(pk2(raw_f32(rDT + t * CH + tid), raw_f32(rDT + (t + 1) * CH + tid)),
+                                 pk2(dtb, dtb));
+            const f32x2 u = pk2(raw_f32(rU + t * CH + tid), raw_f32(rU + (t + 1) * CH + tid));
+            f32x2 d, gt = pk2(1.0f, 1.0f);
+            if (SP && GZ) {
+                softplus_silu2(v, pk2(raw_f32(rZ + t * CH + tid), raw_f32(rZ + (t + 1) * CH + tid)), d, gt);
+            } else if (SP) {
+                d = softplus2p(v);
+            } else {
+                d = v;
+                if (GZ) gt = silu2p(pk2(raw_f32(rZ + t * CH + tid), raw_f32(rZ + (t + 1) * CH + tid)));
+            }
+            float d0, d1, x0, x1, s0, s1, g0, g1;
+            upk2(d, d0, d1);
+            upk2(mul2(d, u), x0, x1);
+            upk2(mul2(pk2(dsk, dsk), u), s0, s1);
+            upk2(gt, g0, g1);
+            if (MASK) {
+                d0 = t < nt ? d0 : 0.f;
+                x0 = t < nt ? x0 : 0.f;
+                d1 = t + 1 < nt ? d1 : 0.f;
+                x1 = t + 1 < nt ? x1 : 0.f;
+            }
+            const float r0 = token(d0, x0, b + t * kN, c + t * kN);
+            const float r1 = token(d1, x1, b + (t + 1) * kN, c + (t + 1) * kN);
+            const T y0 = from_f32<T>((r0 + s0) * g0), y1 = from_f32<T>((r1 + s1) * g1);
+            if (MASK) {
+                if (cvalid && t < nt) dst[(int64_t)t * p.D] = y0;
+                if (cvalid && t + 1 < nt) dst[(int64_t)(t + 1) * p.D] = y1;
+            } else if (cvalid) {
+                dst[(int64_t)t * p.D] = y0;
+                dst[(int64_t)(t + 1) * p.D] = y1;
+            }
+            // after every 8th token of the sequence, unless it was the last
+            if constexpr (CK) {
+                if ((t + 2) % kCkTok == 0 && ckb && t0 + t + 2 < end) store_ckpt(kc + (t + 2) / kCkTok);
+            }
+        }
+    }
+};
+
+template <class K, typename T, bool SP, bool GZ, bool CK>
+__global__ void __launch_bounds__(K::THREADS, K::MINB)
+scan_wide_kernel(const Params p, const __grid_constant__ Maps m)
+{
+    constexpr int TCH = K::TCH;
+    extern __shared__ __align__(128) unsigned char smem[];
+    Wide<K, T, SP, GZ, CK> W(smem, p);
+    uint64_t *const bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+    W.tid = threadIdx.x;
+    const int64_t cbase = (int64_t)blockIdx.x * K::CH;
+    W.c0 = cbase + W.tid;
+    W.cvalid = W.c0 < p.D;
+    int64_t seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
+    int64_t start, end;
+    if (p.cu) {
+        start = clamp_off(p.cu[seq], p.tok);
+        end = max(clamp_off(p.cu[seq + 1], p.tok), start);
+    } else {
+        start = seq * p.L;
+        end = start + p.L;
+    }
+    W.end = end;
+    const int nch = (int)((end - start + TCH - 1) / TCH);
+    constexpr uint32_t tx_bytes = (uint32_t)((GZ ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
+
+    if (W.tid == 0) {
+#pragma unroll
+        for (int st = 0; st < K::RS; ++st) mbar_init(&bar[st]);
+    }
+    __syncthreads();
+    auto issue = [&](int j) {  // TMA of chunk j into stage j % RS
+        const int stage = j % K::RS;
+        mbar_expect_tx(&bar[stage], tx_bytes);
+        const int x = (int)cbase, y = (int)(start + (int64_t)j * TCH);
+        tma_2d(W.raw(stage, 0), &m.u, &bar[stage], x, y);
+        tma_2d(W.raw(stage, 1), &m.dt, &bar[stage], x, y);
+        if (GZ) tma_2d(W.raw(stage, 2), &m.z, &bar[stage], x, y);
+        tma_2d(W.raw(stage, 3), &m.b, &bar[stage], 0, y);
+        tma_2d(W.raw(stage, 4), &m.c, &bar[stage], 0, y);
+    };
+    if (W.tid == 0) {
+        for (int j = 0; j < K::RS && j < nch; ++j) issue(j);
+    }
+
+    if (W.cvalid) {
+        const float4 *a4 = reinterpret_cast<const float4 *>(p.A + W.c0 * kN);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 a = __ldg(a4 + q);
+            W.A2p[2 * q] = pk2(a.x * kLog2e, a.y * kLog2e);
+            W.A2p[2 * q + 1] = pk2(a.z * kLog2e, a.w * kLog2e);
+        }
+        if (p.h0) {
+            const float4 *h4 = reinterpret_cast<const float4 *>(p.h0 + (seq * p.D + W.c0) * kN);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 h = h4[q];
+                W.hp[2 * q] = pk2(h.x, h.y);
+                W.hp[2 * q + 1] = pk2(h.z, h.w);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) W.hp[j] = 0ull;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            W.A2p[j] = 0ull;
+            W.hp[j] = 0ull;
+        }
+    }
+    W.dtb = (W.cvalid && p.dt_bias) ? __ldg(p.dt_bias + W.c0) : 0.f;
+    W.dsk = (W.cvalid && p.Dskip) ? __ldg(p.Dskip + W.c0) : 0.f;
+    // checkpoint j of sequence `seq` (the state before its token 8j) lives in
+    // row floor(start / 8) + seq + j of D x 16 floats: sequences never collide
+    W.ckb = (CK && W.cvalid) ? p.ckpt + ((start / kCkTok + seq) * p.D + W.c0) * kN : nullptr;
+    if (CK && W.ckb && end > start) W.store_ckpt(0);
+
+    bool failed = false;
+    auto wait_raw = [&](int j) {
+        mbar_wait(&bar[j % K::RS], (uint32_t)((j / K::RS) & 1), failed, &g_pipe_status, 1);
+    };
+    if (nch > 0) {
+        wait_raw(0);
+        W.template widen<0>(0);
+    }
+    __syncthreads();
+
+    // iteration k: chunk k from stage k % RS and B/C buffer k & 1; then chunk
+    // k+1's B and C rows widened into buffer (k+1) & 1
+    auto step = [&](auto tag, int k) {
+        constexpr int BUF = decltype(tag)::value;
+        // stage (k-1) % RS was last read in iteration k-1, before the last barrier
+        if (W.tid == 0 && k >= 1 && k - 1 + K::RS < nch) {
+            fence_proxy_async();
+            issue(k - 1 + K::RS);
+        }
+        const int64_t t0 = start + (int64_t)k * TCH;
+        const int64_t kc = (int64_t)k * (TCH / kCkTok);
+        const int nt = (int)min((int64_t)TCH, end - t0);
+        if (nt == TCH) W.template chunk<BUF, false>(k % K::RS, t0, TCH, kc);
+        else W.template chunk<BUF, true>(k % K::RS, t0, nt, kc);
+        if (k + 1 < nch) {
+            wait_raw(k + 1);
+            W.template widen<BUF ^ 1>((k + 1) % K::RS);
+        }
+        __syncthreads();
+    };
+    int k = 0;
+    for (; k + 1 < nch; k += 2) {
+        step(BufTag<0>{}, k);
+        step(BufTag<1>{}, k + 1);
+    }
+    if (k < nch) step(BufTag<0>{}, k);
+
+    if (p.h_final && W.cvalid) {
+        float4 *o4 = reinterpret_cast<float4 *>(p.h_final + (seq * p.D + W.c0) * kN);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float4 v;
+            upk2(W.hp[2 * q], v.x, v.y);
+            upk2(W.hp[2 * q + 1], v.z, v.w);
+            o4[q] = v;
+        }
+    }
+}
+
+template <class K, typename T, bool SP, bool GZ, bool CK>
+cudaError_t run_wide_t(const Params &p, const Maps &m, cudaStream_t stream, int *launches)
+{
+    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
+    cudaError_t e = cudaFuncSetAttribute(scan_wide_kernel<K, T, SP, GZ, CK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
+    if (e != cudaSuccess) return e;
+    scan_wide_kernel<K, T, SP, GZ, CK><<<grid, K::THREADS, K::SMEM, stream>>>(p, m);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+template <class K, typename T, bool CK>
+cudaError_t run_wide(const Params &p, cudaStream_t stream, int *launches)
+{
+    Maps m;
+    const bool bf = sizeof(T) == 2;
+    bool ok = p.tok > 0 && encode_2d(&m.u, p.u, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+              encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+    if (ok) {
+        if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+        else m.z = m.u;  // never loaded
+    }
+    if (!ok) return cudaErrorNotSupported;
+    if (p.delta_softplus)
+        return p.z ? run_wide_t<K, T, true, true, CK>(p, m, stream, launches)
+                   : run_wide_t<K, T, true, false, CK>(p, m, stream, launches);
+    return p.z ? run_wide_t<K, T, false, true, CK>(p, m, stream, launches)
+               : run_wide_t<K, T, false, false, CK>(p, m, stream, launches);
+}
+
+// Schedule 12 (one lane per channel); cudaErrorNotSupported when the tensor
+// maps cannot be encoded. bf16: 32-token chunks in two stages (60 KB of
+// shared memory), 142 registers, three CTAs (12 warps) per SM. Measured on
+// the packed and uniform workloads against 16-token chunks in three or four
+// stages (0.661-0.669 / 0.628-0.634 of the ex2 peak) and four CTAs per SM
+// capped at 128 registers (0.623 / 0.647): 0.684 / 0.657.
+template <bool CK>
+cudaError_t launch_wide_cfg(const Params &p, bool bf16, cudaStream_t stream, int *launches)
+{
+    if (bf16) return run_wide<WideCfg<__nv_bfloat16, 32, 2, 3>, __nv_bfloat16, CK>(p, stream, launches);
+    return run_wide<WideCfg<float, 16, 3, 2>, float, CK>(p, stream, launches);
 }
 
 // This translation unit's status word (-1 when it cannot be read).

@@ -130,9 +130,9 @@ def test_check_cu_seqlens_host():
 
 
 def test_tuning_knob():
-    for n, c in ((0, 0), (2, 1), (4, 1), (4, 2), (4, 3), (8, 2), (16, 1), (16, 2)):
+    for n, c in ((0, 0), (2, 1), (4, 1), (4, 2), (4, 3), (8, 2), (16, 1), (16, 2), (16, 12)):
         ssm.ssm_set_scan_variant(n, c)
-    for n, c in ((3, 1), (16, 12), (4, -1)):
+    for n, c in ((3, 1), (16, 13), (4, -1)):
         with pytest.raises(ssm.SsmError):
             ssm.ssm_set_scan_variant(n, c)
     ssm.ssm_set_scan_variant(0, 0)
@@ -162,15 +162,18 @@ def test_bwd_variant_knob_and_choice():
 
 def test_variant_choice():
     """The automatic choice follows (sequence, channel, state) recurrences per
-    SM (148 SMs when no device is visible): 8 states per lane in the pipelined
-    kernel with 16-token chunks when the GPU holds about 20 warps per SM of
-    them, else 4 states per lane with 32-token chunks while that still gives
+    SM (148 SMs when no device is visible): one lane per channel (schedule 12)
+    with at least two waves of its three 128-lane CTAs per SM, else 8 states
+    per lane in the pipelined kernel with 16-token chunks when the GPU holds
+    about 20 warps per SM of them, else 4 states per lane with 32-token chunks while that still gives
     every SM a block (with the two-CTAs-per-SM register budget when the grid
     has at most two CTAs per SM), else 2 states per lane. A forced variant is
     reported as forced."""
     ssm.ssm_set_scan_variant(0, 0)
     assert ssm.ssm_scan_variant_for(8, 1536) == (4, 10)     # 8 x 2048 x 1536 layer
-    assert ssm.ssm_scan_variant_for(43, 5120) == (8, 9)     # packed 65536 x 5120
+    assert ssm.ssm_scan_variant_for(43, 5120) == (16, 12)   # packed 65536 x 5120
+    assert ssm.ssm_scan_variant_for(32, 5120) == (16, 12)   # 32 x 2048 x 5120
+    assert ssm.ssm_scan_variant_for(16, 5120) == (8, 9)     # below two waves of schedule 12
     assert ssm.ssm_scan_variant_for(1, 8192) == (4, 11)     # one 8192-channel sequence
     assert ssm.ssm_scan_variant_for(4, 8192) == (4, 10)
     assert ssm.ssm_scan_variant_for(1, 2048) == (2, 9)

@@ -51,7 +51,8 @@ def _acts(seed, tok, D):
 
 
 @pytest.mark.parametrize("variant", [(4, 1), (4, 2), (4, 3), (2, 3), (8, 2), (16, 2), (4, 6), (8, 6), (4, 7), (8, 7), (2, 8), (4, 8),
-                                     (2, 9), (4, 9), (8, 9), (4, 10), (8, 10), (4, 11)])
+                                     (2, 9), (4, 9), (8, 9), (4, 10), (8, 10), (4, 11), (16, 12)],
+                         ids=lambda v: f"{v[0]}x{v[1]}")
 def test_pack_equals_separate(variant):
     ssm.ssm_set_scan_variant(*variant)
     lens = [100, 0, 3, 1, 257, 64]

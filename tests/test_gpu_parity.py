@@ -90,7 +90,7 @@ def test_conv_no_silu(orc):
 
 VARIANTS = [(2, 1), (2, 2), (2, 3), (4, 1), (4, 2), (4, 3), (4, 4), (4, 5), (8, 1), (8, 2), (8, 4),
             (8, 5), (16, 1), (16, 2), (16, 4), (16, 5), (2, 6), (4, 6), (8, 6), (16, 6), (4, 7), (8, 7), (16, 7), (2, 8), (4, 8), (8, 8), (16, 8),
-            (2, 9), (4, 9), (8, 9), (4, 10), (8, 10), (4, 11)]
+            (2, 9), (4, 9), (8, 9), (4, 10), (8, 10), (4, 11), (16, 12)]
 
 
 def _scan_case(orc, seed, lens, D, bf16, variant=(0, 0), with_z=True, with_h0=True,
@@ -124,18 +124,19 @@ def _scan_case(orc, seed, lens, D, bf16, variant=(0, 0), with_z=True, with_h0=Tr
     return host(y), host(hf)
 
 
-@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("variant", VARIANTS, ids=lambda v: f"{v[0]}x{v[1]}")
 @pytest.mark.parametrize("bf16", [False, True])
 def test_scan_variants_packed(orc, variant, bf16):
     _scan_case(orc, 10, [130, 0, 1, 7, 64, 65, 200], 200, bf16, variant=variant)
 
 
-@pytest.mark.parametrize("variant", VARIANTS)
+@pytest.mark.parametrize("variant", VARIANTS, ids=lambda v: f"{v[0]}x{v[1]}")
 def test_scan_scalar_path(orc, variant):
     _scan_case(orc, 11, [50, 77], 30, True, variant=variant)
 
 
-@pytest.mark.parametrize("variant", [(0, 0), (4, 9), (8, 9), (2, 9), (4, 10)])
+@pytest.mark.parametrize("variant", [(0, 0), (4, 9), (8, 9), (2, 9), (4, 10), (16, 12)],
+                         ids=lambda v: f"{v[0]}x{v[1]}")
 def test_scan_options(orc, variant):
     _scan_case(orc, 12, [90, 40], 72, True, with_z=False, with_h0=False, variant=variant)
     _scan_case(orc, 13, [90, 40], 72, False, softplus=False, variant=variant)

@@ -256,13 +256,14 @@ def test_bwd_many_short_sequences_past_the_sort_limit(orc, variant):
     _check(orc, True, lens, 128, seed=23)
 
 
-@pytest.fixture(params=[(0, 0), (2, 9), (4, 10), (8, 9), (4, 11), (4, 1)],
-                ids=["fwd_pick", "pipe2", "pipe4", "pipe8", "pipe4_255reg", "fwd_sched1"])
+@pytest.fixture(params=[(0, 0), (2, 9), (4, 10), (8, 9), (4, 11), (4, 1), (16, 12)],
+                ids=["fwd_pick", "pipe2", "pipe4", "pipe8", "pipe4_255reg", "fwd_sched1", "wide16"])
 def fwd_sched(request):
     """The forward that writes the checkpoints: the library's pick, the
     pipelined kernel at 2, 4 and 8 states per lane (it writes them as it goes),
-    and schedule 1 (no checkpoint output: the library adds its checkpointing
-    pass)."""
+    schedule 1 (no checkpoint output: the library adds its checkpointing
+    pass) and schedule 12 (one lane per channel, also writing them as it
+    goes)."""
     ssm.ssm_set_scan_variant(*request.param)
     yield request.param
     ssm.ssm_set_scan_variant(0, 0)
