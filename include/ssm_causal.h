@@ -370,7 +370,7 @@ int ssm_selective_scan_bwd(const void *u, const void *delta, const float *A, con
  * computes (y and h_final bit for bit, same arguments) and also writes, into
  * bwd_workspace, the fp32 state of every sequence and channel before each
  * 8th token of the sequence (before tokens 0, 8, 16, ...; about 8 bytes per
- * token and channel). The pipelined kernels (schedules 9 to 11) write them as
+ * token and channel). The pipelined kernels (schedules 9 to 12) write them as
  * they go; with any other kernel the library adds a checkpointing pass after
  * the scan.
  *   bwd_workspace  >= ssm_scan_bwd_workspace_size(tok, D, N, S) bytes,
