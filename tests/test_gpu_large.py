@@ -9,13 +9,24 @@ import numpy as np
 import pytest
 import torch
 
+import selective_state_space_causal_b200 as ssm
 from selective_state_space_causal_b200 import synth
 from gpu_helpers import TOL_BF16, assert_close, dev, host, run_conv, run_scan
 
 pytestmark = pytest.mark.gpu
 
 
-def test_conv_and_scan_past_2_31_elements(orc):
+@pytest.fixture(params=[(0, 0), (16, 12)], ids=["pick", "one_lane_per_channel"])
+def scan_variant(request):
+    """The library's pick for one 8192-channel sequence (4 states per lane),
+    and schedule 12 forced (one lane per channel), whose offsets are computed
+    apart from the other schedules'."""
+    ssm.ssm_set_scan_variant(*request.param)
+    yield request.param
+    ssm.ssm_set_scan_variant(0, 0)
+
+
+def test_conv_and_scan_past_2_31_elements(orc, scan_variant):
     D, L = 8192, 270336
     assert L * D > 2 ** 31
     prm = synth.make_params(7, D)
