@@ -273,10 +273,16 @@ int ssm_selective_state_update(void *conv_state, float *ssm_state, const void *x
  *   delta, A, B, C, Dskip, z, dt_bias, delta_softplus, h0, cu_seqlens, S, y,
  *   h_final, tok, D, N, act_dtype: as ssm_selective_scan_fwd (u is the conv
  *                  output); y must not overlap x, delta or z
- * Always one kernel: the scan's register-prefetch layout (4 or 8 states per
- * lane as ssm_scan_variant_for reports it, 4 when rows are not 16-byte
- * aligned), sequences in index order. Where the scan alone would pick a TMA
- * schedule (many sequence-channel pairs) the two-call path can be faster.
+ * Always one kernel. Where ssm_scan_variant_for reports schedule 12 (many
+ * sequence-channel pairs) and every row is 16-byte aligned: one lane per
+ * channel with the conv window in the lane's registers, sequences longest
+ * first when S <= 128 (each CTA ranks the lengths itself; no workspace),
+ * else in index order. Otherwise the scan's register-prefetch layout (4 or 8
+ * states per lane as ssm_scan_variant_for reports it, 4 when rows are not
+ * 16-byte aligned), sequences in index order. The conv output takes the conv
+ * kernel's operations in its order, so an xc copy equals ssm_causal_conv1d's
+ * output bit for bit. Where the scan alone would pick a TMA schedule the
+ * two-call path can be as fast or faster.
  */
 int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
                       const void *conv_state_in, void *conv_state_out, void *xc, int K,

@@ -57,7 +57,9 @@ struct ConvScanArgs {
     DType state_dtype;
     ScanArgs scan;
 };
-cudaError_t launch_conv_scan(const ConvScanArgs &a, int npt, cudaStream_t stream, int *launches);
+cudaError_t launch_conv_scan(const ConvScanArgs &a, int npt, int sched, cudaStream_t stream,
+                             int *launches);
+int read_conv_scan_status(bool clear);
 cudaError_t launch_scan_bwd(const ScanBwdArgs &a, cudaStream_t stream, int *launches);
 
 struct ReplayStepArgs {
@@ -175,7 +177,9 @@ int ssm_scan_variant_for(int64_t S, int64_t D, int *states_per_lane, int *schedu
 
 int ssm_device_status(int clear)
 {
-    const int a = ssm::read_scan_status(clear != 0);
+    const int a0 = ssm::read_scan_status(clear != 0);
+    const int a1 = ssm::read_conv_scan_status(clear != 0);
+    const int a = (a0 < 0 || a1 < 0) ? -1 : (a0 | a1);
     const int b = ssm::read_conv_status(clear != 0);
     const int d = ssm::read_decode_status(clear != 0);
     const int r = ssm::read_replay_status(clear != 0);
@@ -431,7 +435,7 @@ int ssm_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
     ssm::ConvScanArgs a{x, conv_w, conv_b, conv_state_in, conv_state_out, xc, K,
                         dt(conv_state_dtype), sa};
     int launched = 0;
-    cudaError_t e = ssm::launch_conv_scan(a, npt == 8 ? 8 : 4,
+    cudaError_t e = ssm::launch_conv_scan(a, npt == 8 ? 8 : 4, sched,
                                           reinterpret_cast<cudaStream_t>(stream), &launched);
     return finish(e, launched, fn);
 }

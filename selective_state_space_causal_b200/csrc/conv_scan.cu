@@ -20,9 +20,12 @@
 // chunk and no extra barrier is needed. The conv takes the same operations in
 // the same order as the conv kernel (taps oldest first, bias first, SiLU as
 // x * 1/(1 + 2^(-x log2 e))), and xc stays in fp32.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 #include "scan_parts.cuh"
+#include "scan_pipe.cuh"
 
 namespace ssm {
 
@@ -313,6 +316,362 @@ cudaError_t by_kw(const Params &p, const ConvParams &cp, int K, int npt, bool ve
     }
 }
 
+
+// ---------------------------------------------------------------------------
+// One lane per channel (the scan's schedule 12) with the conv in the lane.
+//
+// A lane walks its channel's tokens in order, so the conv window is the
+// lane's last KW-1 inputs, kept in registers across chunks (the sequence's
+// carried conv state at its start): no halo rows and no shared-memory tile.
+// Each token's conv output is formed with the conv kernel's operations in its
+// order (bias first, taps oldest first, SiLU as x / (1 + 2^(-x log2 e))),
+// stays in fp32 as the scan's u and is optionally stored as xc. The rest is
+// scan_wide_kernel: raw x, dt, z tiles and B, C rows by TMA in two stages of 32
+// tokens, B and C widened to fp32 once per CTA, one lane per channel with all
+// 16 states, no shuffles. Packed sequences run longest first: with at most
+// kRankMax sequences each CTA ranks the lengths itself (the entry point takes
+// no workspace for an order); above that, in index order.
+constexpr int kRankMax = 128;
+
+template <class K, typename T, typename TS, int KW>
+struct FusedWide {
+    static constexpr int TCH = K::TCH, CH = K::CH;
+    unsigned char *smem;
+    const Params &p;
+    const ConvParams &cp;
+    int tid;
+    int64_t c0;
+    bool cvalid, sp, gz;
+    float dtb, dsk, cb;
+    float cw[KW], win[KW - 1];  // conv taps; the channel's last KW-1 inputs, oldest first
+    f32x2 A2p[8], hp[8];        // A * log2(e) and the state, two states per register
+
+    __device__ __forceinline__ FusedWide(unsigned char *s, const Params &p_, const ConvParams &cp_)
+        : smem(s), p(p_), cp(cp_) {}
+
+    __device__ __forceinline__ T *raw(int stage, int which) const
+    {
+        size_t off = (size_t)stage * K::STAGE;
+        off += which < 3 ? (size_t)which * align128(K::RAW_ACT)
+                         : 3 * align128(K::RAW_ACT) + (size_t)(which - 3) * align128(K::RAW_BC);
+        return reinterpret_cast<T *>(smem + off);
+    }
+    __device__ __forceinline__ const float *bc(int which, int buf, int stage) const
+    {
+        if constexpr (sizeof(T) == 4) {
+            (void)buf;
+            return reinterpret_cast<const float *>(raw(stage, 3 + which));
+        } else {
+            (void)stage;
+            return reinterpret_cast<const float *>(smem + (which ? K::OFF_C : K::OFF_B) + buf * K::BCF);
+        }
+    }
+    template <int BUF>
+    __device__ __forceinline__ void widen(int stage) const
+    {
+        if constexpr (sizeof(T) == 2) {
+            const int which = tid >= K::THREADS / 2, i = tid & (K::THREADS / 2 - 1);
+            const uint32_t *src = reinterpret_cast<const uint32_t *>(raw(stage, 3 + which)) + i * (K::EPT / 2);
+            float *dst = reinterpret_cast<float *>(smem + (which ? K::OFF_C : K::OFF_B) + BUF * K::BCF) +
+                         i * K::EPT;
+#pragma unroll
+            for (int e = 0; e < K::EPT / 2; e += 2)
+                *reinterpret_cast<float4 *>(dst + 2 * e) = make_float4(
+                    __uint_as_float(src[e] << 16), __uint_as_float(src[e] & 0xffff0000u),
+                    __uint_as_float(src[e + 1] << 16), __uint_as_float(src[e + 1] & 0xffff0000u));
+        } else {
+            (void)stage;
+        }
+    }
+
+    // One token of the recurrence and its readout (as scan_wide_kernel).
+    __device__ __forceinline__ float token(float d, float du, const float *b, const float *c)
+    {
+        const f32x2 dv = pk2(d, d), xv = pk2(du, du);
+        f32x2 bb[8], cc[8];
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) lds_2x2(b + 2 * j, bb[j], bb[j + 1]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float a0, a1;
+            upk2(mul2(dv, A2p[j]), a0, a1);
+            hp[j] = fma2(pk2(ex2_approx(a0), ex2_approx(a1)), hp[j], mul2(xv, bb[j]));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) lds_2x2(c + 2 * j, cc[j], cc[j + 1]);
+        f32x2 acc0 = mul2(cc[0], hp[0]), acc1 = mul2(cc[1], hp[1]);
+#pragma unroll
+        for (int j = 2; j < 8; j += 2) {
+            acc0 = fma2(cc[j], hp[j], acc0);
+            acc1 = fma2(cc[j + 1], hp[j + 1], acc1);
+        }
+        float s0, s1;
+        upk2(add2(acc0, acc1), s0, s1);
+        return s0 + s1;
+    }
+
+    template <int BUF, bool MASK>
+    __device__ __forceinline__ void chunk(int stage, int64_t t0, int nt)
+    {
+        const T *rX = raw(stage, 0), *rDT = raw(stage, 1), *rZ = raw(stage, 2);
+        const float *b = bc(0, BUF, stage), *c = bc(1, BUF, stage);
+        T *dst = static_cast<T *>(p.y) + t0 * p.D + c0;
+        T *xcd = cp.xc ? static_cast<T *>(cp.xc) + t0 * p.D + c0 : nullptr;
+#pragma unroll 1
+        for (int t = 0; t < TCH; t += 2) {
+            // the conv of tokens t and t + 1 over [window, x_t, x_t+1]
+            float ext[KW + 1];
+#pragma unroll
+            for (int k = 0; k < KW - 1; ++k) ext[k] = win[k];
+            ext[KW - 1] = raw_f32(rX + t * CH + tid);
+            ext[KW] = raw_f32(rX + (t + 1) * CH + tid);
+            float a0 = cb, a1 = cb;
+#pragma unroll
+            for (int k = 0; k < KW; ++k) {
+                a0 = fmaf(cw[k], ext[k], a0);
+                a1 = fmaf(cw[k], ext[k + 1], a1);
+            }
+            const float u0 = conv_silu_f(a0), u1 = conv_silu_f(a1);
+            const bool l0 = !MASK || t < nt, l1 = !MASK || t + 1 < nt;
+#pragma unroll
+            for (int k = 0; k < KW - 1; ++k) win[k] = l1 ? ext[k + 2] : (l0 ? ext[k + 1] : ext[k]);
+
+            const f32x2 v = add2(pk2(raw_f32(rDT + t * CH + tid), raw_f32(rDT + (t + 1) * CH + tid)),
+                                 pk2(dtb, dtb));
+            const f32x2 u = pk2(u0, u1);
+            f32x2 d, gt = pk2(1.0f, 1.0f);
+            if (sp && gz) {
+                softplus_silu2(v, pk2(raw_f32(rZ + t * CH + tid), raw_f32(rZ + (t + 1) * CH + tid)), d, gt);
+            } else if (sp) {
+                d = softplus2p(v);
+            } else {
+                d = v;
+                if (gz) gt = silu2p(pk2(raw_f32(rZ + t * CH + tid), raw_f32(rZ + (t + 1) * CH + tid)));
+            }
+            float d0, d1, x0, x1, s0, s1, g0, g1;
+            upk2(d, d0, d1);
+            upk2(mul2(d, u), x0, x1);
+            upk2(mul2(pk2(dsk, dsk), u), s0, s1);
+            upk2(gt, g0, g1);
+            if (MASK) {
+                d0 = l0 ? d0 : 0.f;
+                x0 = l0 ? x0 : 0.f;
+                d1 = l1 ? d1 : 0.f;
+                x1 = l1 ? x1 : 0.f;
+            }
+            const float r0 = token(d0, x0, b + t * kN, c + t * kN);
+            const float r1 = token(d1, x1, b + (t + 1) * kN, c + (t + 1) * kN);
+            if (cvalid) {
+                if (l0) dst[(int64_t)t * p.D] = from_f32<T>((r0 + s0) * g0);
+                if (l1) dst[(int64_t)(t + 1) * p.D] = from_f32<T>((r1 + s1) * g1);
+                if (xcd) {
+                    if (l0) xcd[(int64_t)t * p.D] = from_f32<T>(u0);
+                    if (l1) xcd[(int64_t)(t + 1) * p.D] = from_f32<T>(u1);
+                }
+            }
+        }
+    }
+};
+
+template <class K, typename T, typename TS, int KW>
+__global__ void __launch_bounds__(K::THREADS, K::MINB)
+conv_scan_wide_kernel(const Params p, const ConvParams cp, const __grid_constant__ Maps m)
+{
+    constexpr int TCH = K::TCH;
+    extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ int cu_s[kRankMax + 1];
+    __shared__ int seq_s;
+    FusedWide<K, T, TS, KW> W(smem, p, cp);
+    uint64_t *const bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
+    W.tid = threadIdx.x;
+    const int64_t cbase = (int64_t)blockIdx.x * K::CH;
+    W.c0 = cbase + W.tid;
+    W.cvalid = W.c0 < p.D;
+    W.sp = p.delta_softplus != 0;
+    W.gz = p.z != nullptr;
+
+    // the sequence: blockIdx.y-th longest (ties by index) when the CTA can
+    // rank the lengths itself, else sequence blockIdx.y
+    int64_t seq = blockIdx.y;
+    if (p.cu && p.S > 1 && p.S <= kRankMax) {
+        const int S = (int)p.S;
+        for (int i = W.tid; i <= S; i += K::THREADS) cu_s[i] = (int)clamp_off(p.cu[i], p.tok);
+        if (W.tid == 0) seq_s = (int)blockIdx.y;
+        __syncthreads();
+        for (int i = W.tid; i < S; i += K::THREADS) {
+            const int li = max(cu_s[i + 1] - cu_s[i], 0);
+            int rank = 0;
+            for (int j = 0; j < S; ++j) {
+                const int lj = max(cu_s[j + 1] - cu_s[j], 0);
+                rank += (lj > li) || (lj == li && j < i);
+            }
+            if (rank == (int)blockIdx.y) seq_s = i;
+        }
+        __syncthreads();
+        seq = seq_s;
+    }
+    seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
+    int64_t start, end;
+    if (p.cu) {
+        start = clamp_off(p.cu[seq], p.tok);
+        end = max(clamp_off(p.cu[seq + 1], p.tok), start);
+    } else {
+        start = seq * p.L;
+        end = start + p.L;
+    }
+    const int nch = (int)((end - start + TCH - 1) / TCH);
+    const uint32_t tx_bytes = (uint32_t)((W.gz ? 3 : 2) * K::RAW_ACT + 2 * K::RAW_BC);
+
+    if (W.tid == 0) {
+#pragma unroll
+        for (int st = 0; st < K::RS; ++st) mbar_init(&bar[st]);
+    }
+    __syncthreads();
+    auto issue = [&](int j) {  // TMA of chunk j into stage j % RS
+        const int stage = j % K::RS;
+        mbar_expect_tx(&bar[stage], tx_bytes);
+        const int x = (int)cbase, y = (int)(start + (int64_t)j * TCH);
+        tma_2d(W.raw(stage, 0), &m.u, &bar[stage], x, y);
+        tma_2d(W.raw(stage, 1), &m.dt, &bar[stage], x, y);
+        if (W.gz) tma_2d(W.raw(stage, 2), &m.z, &bar[stage], x, y);
+        tma_2d(W.raw(stage, 3), &m.b, &bar[stage], 0, y);
+        tma_2d(W.raw(stage, 4), &m.c, &bar[stage], 0, y);
+    };
+    if (W.tid == 0) {
+        for (int j = 0; j < K::RS && j < nch; ++j) issue(j);
+    }
+
+    const TS *SIN = static_cast<const TS *>(cp.state_in);
+    TS *SOUT = static_cast<TS *>(cp.state_out);
+    if (W.cvalid) {
+        const float4 *a4 = reinterpret_cast<const float4 *>(p.A + W.c0 * kN);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float4 a = __ldg(a4 + q);
+            W.A2p[2 * q] = pk2(a.x * kLog2e, a.y * kLog2e);
+            W.A2p[2 * q + 1] = pk2(a.z * kLog2e, a.w * kLog2e);
+        }
+        if (p.h0) {
+            const float4 *h4 = reinterpret_cast<const float4 *>(p.h0 + (seq * p.D + W.c0) * kN);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float4 h = h4[q];
+                W.hp[2 * q] = pk2(h.x, h.y);
+                W.hp[2 * q + 1] = pk2(h.z, h.w);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) W.hp[j] = 0ull;
+        }
+#pragma unroll
+        for (int k = 0; k < KW; ++k) W.cw[k] = __ldg(cp.w + W.c0 * KW + k);
+#pragma unroll
+        for (int k = 0; k < KW - 1; ++k)
+            W.win[k] = SIN ? to_f32(SIN[(seq * p.D + W.c0) * (KW - 1) + k]) : 0.f;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            W.A2p[j] = 0ull;
+            W.hp[j] = 0ull;
+        }
+#pragma unroll
+        for (int k = 0; k < KW; ++k) W.cw[k] = 0.f;
+#pragma unroll
+        for (int k = 0; k < KW - 1; ++k) W.win[k] = 0.f;
+    }
+    W.cb = (W.cvalid && cp.bias) ? __ldg(cp.bias + W.c0) : 0.f;
+    W.dtb = (W.cvalid && p.dt_bias) ? __ldg(p.dt_bias + W.c0) : 0.f;
+    W.dsk = (W.cvalid && p.Dskip) ? __ldg(p.Dskip + W.c0) : 0.f;
+
+    bool failed = false;
+    auto wait_raw = [&](int j) {
+        mbar_wait(&bar[j % K::RS], (uint32_t)((j / K::RS) & 1), failed, &g_pipe_status, 1);
+    };
+    if (nch > 0) {
+        wait_raw(0);
+        W.template widen<0>(0);
+    }
+    __syncthreads();
+
+    auto step = [&](auto tag, int k) {
+        constexpr int BUF = decltype(tag)::value;
+        // stage (k-1) % RS was last read in iteration k-1, before the last barrier
+        if (W.tid == 0 && k >= 1 && k - 1 + K::RS < nch) {
+            fence_proxy_async();
+            issue(k - 1 + K::RS);
+        }
+        const int64_t t0 = start + (int64_t)k * TCH;
+        const int nt = (int)min((int64_t)TCH, end - t0);
+        if (nt == TCH) W.template chunk<BUF, false>(k % K::RS, t0, TCH);
+        else W.template chunk<BUF, true>(k % K::RS, t0, nt);
+        if (k + 1 < nch) {
+            wait_raw(k + 1);
+            W.template widen<BUF ^ 1>((k + 1) % K::RS);
+        }
+        __syncthreads();
+    };
+    int k = 0;
+    for (; k + 1 < nch; k += 2) {
+        step(BufTag<0>{}, k);
+        step(BufTag<1>{}, k + 1);
+    }
+    if (k < nch) step(BufTag<0>{}, k);
+
+    if (W.cvalid) {
+        if (p.h_final) {
+            float4 *o4 = reinterpret_cast<float4 *>(p.h_final + (seq * p.D + W.c0) * kN);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float4 v;
+                upk2(W.hp[2 * q], v.x, v.y);
+                upk2(W.hp[2 * q + 1], v.z, v.w);
+                o4[q] = v;
+            }
+        }
+        // the sequence's last KW-1 inputs (the carried state where it is
+        // shorter); the lane read its own entries of the input state above
+        if (SOUT) {
+#pragma unroll
+            for (int k2 = 0; k2 < KW - 1; ++k2)
+                SOUT[(seq * p.D + W.c0) * (KW - 1) + k2] = from_f32<TS>(W.win[k2]);
+        }
+    }
+}
+
+template <class K, typename T, typename TS, int KW>
+cudaError_t run_fused_wide(const Params &p, const ConvParams &cp, cudaStream_t stream, int *launches)
+{
+    Maps m;
+    const bool bf = sizeof(T) == 2;
+    bool ok = p.tok > 0 && encode_2d(&m.u, cp.x, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.dt, p.delta, bf, p.D, p.tok, K::CH, K::TCH) &&
+              encode_2d(&m.b, p.B, bf, kN, p.tok, kN, K::TCH) &&
+              encode_2d(&m.c, p.C, bf, kN, p.tok, kN, K::TCH);
+    if (ok) {
+        if (p.z) ok = encode_2d(&m.z, p.z, bf, p.D, p.tok, K::CH, K::TCH);
+        else m.z = m.u;  // never loaded
+    }
+    if (!ok) return cudaErrorNotSupported;
+    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
+    cudaError_t e = cudaFuncSetAttribute(conv_scan_wide_kernel<K, T, TS, KW>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
+    if (e != cudaSuccess) return e;
+    conv_scan_wide_kernel<K, T, TS, KW><<<grid, K::THREADS, K::SMEM, stream>>>(p, cp, m);
+    ++*launches;
+    return cudaGetLastError();
+}
+
+template <typename T, typename TS>
+cudaError_t wide_by_kw(const Params &p, const ConvParams &cp, int KW, cudaStream_t s, int *n)
+{
+    using K = std::conditional_t<sizeof(T) == 2, WideCfg<__nv_bfloat16, 32, 2, 3>, WideCfg<float, 16, 3, 2>>;
+    switch (KW) {
+    case 2: return run_fused_wide<K, T, TS, 2>(p, cp, s, n);
+    case 3: return run_fused_wide<K, T, TS, 3>(p, cp, s, n);
+    default: return run_fused_wide<K, T, TS, 4>(p, cp, s, n);
+    }
+}
+
 }  // namespace
 
 struct ConvScanArgs {
@@ -326,10 +685,16 @@ struct ConvScanArgs {
     ScanArgs scan;
 };
 
-// The fused kernel: 16-byte channel vectors (4 or 8 states per lane, as the
-// scan's variant choice says) where every row is 16-byte aligned, else scalar
-// channels with 4 states per lane.
-cudaError_t launch_conv_scan(const ConvScanArgs &a, int npt, cudaStream_t stream, int *launches)
+// This translation unit's status word of bounded TMA waits (-1 when it
+// cannot be read).
+int read_conv_scan_status(bool clear) { return read_tu_pipe_status(clear); }
+
+// The fused kernel: one lane per channel where the scan would take schedule
+// 12 and every row is 16-byte aligned; else 16-byte channel vectors (4 or 8
+// states per lane, as the scan's variant choice says) where every row is
+// 16-byte aligned, else scalar channels with 4 states per lane.
+cudaError_t launch_conv_scan(const ConvScanArgs &a, int npt, int sched, cudaStream_t stream,
+                             int *launches)
 {
     const ScanArgs &s = a.scan;
     if (s.S == 0) return cudaSuccess;
@@ -345,6 +710,14 @@ cudaError_t launch_conv_scan(const ConvScanArgs &a, int npt, cudaStream_t stream
     p.delta_softplus = s.delta_softplus;
     ConvParams cp{a.x, a.w, a.bias, a.state_in, a.state_out, a.xc};
     const bool xb = s.dtype == DType::BF16, sb = a.state_dtype == DType::BF16;
+    if (sched == 12 && vec && s.tok > 0) {
+        cudaError_t e;
+        if (xb && sb) e = wide_by_kw<__nv_bfloat16, __nv_bfloat16>(p, cp, a.K, stream, launches);
+        else if (xb) e = wide_by_kw<__nv_bfloat16, float>(p, cp, a.K, stream, launches);
+        else if (sb) e = wide_by_kw<float, __nv_bfloat16>(p, cp, a.K, stream, launches);
+        else e = wide_by_kw<float, float>(p, cp, a.K, stream, launches);
+        if (e != cudaErrorNotSupported) return e;
+    }
     if (xb && sb) return by_kw<__nv_bfloat16, __nv_bfloat16>(p, cp, a.K, npt, vec, stream, launches);
     if (xb) return by_kw<__nv_bfloat16, float>(p, cp, a.K, npt, vec, stream, launches);
     if (sb) return by_kw<float, __nv_bfloat16>(p, cp, a.K, npt, vec, stream, launches);

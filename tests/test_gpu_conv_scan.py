@@ -65,17 +65,33 @@ def _case(orc, bf16, K, lens, D, seed, inplace=False, want_xc=True, dense=None):
     return y
 
 
+@pytest.fixture(params=[(0, 0), (16, 12)], ids=["pick", "one_lane_per_channel"])
+def fused_variant(request):
+    """The kernel the library picks for the shape, and the one-lane-per-channel
+    fused kernel (taken where the scan would run schedule 12), forced."""
+    ssm.ssm_set_scan_variant(*request.param)
+    yield request.param
+    ssm.ssm_set_scan_variant(0, 0)
+
+
 @pytest.mark.parametrize("bf16", [False, True])
 @pytest.mark.parametrize("K", [2, 3, 4])
-def test_fused_packed(orc, bf16, K):
+def test_fused_packed(orc, bf16, K, fused_variant):
     # empty and shorter-than-K-1 sequences, chunk edges at 64 tokens, a
     # partial channel block
     _case(orc, bf16, K, [70, 0, 1, 2, 64, 129, 5], 96, 3 + K)
 
 
-def test_fused_in_place_conv_state_and_dense(orc):
+def test_fused_in_place_conv_state_and_dense(orc, fused_variant):
     _case(orc, True, 4, [33, 65, 1], 64, 21, inplace=True, want_xc=False)
     _case(orc, True, 4, None, 128, 22, dense=(3, 100))
+
+
+def test_fused_many_sequences(orc, fused_variant):
+    """More sequences than a CTA ranks by itself (index order then), with a
+    ragged channel tail over two channel blocks."""
+    lens = list(np.random.default_rng(41).integers(0, 40, size=150))
+    _case(orc, True, 4, lens, 200, 41)
 
 
 @pytest.mark.parametrize("bf16", [False, True])
@@ -84,7 +100,7 @@ def test_fused_unaligned_rows(orc, bf16):
     _case(orc, bf16, 4, [40, 7, 90], 36, 31)
 
 
-def test_fused_mamba130m_layer(orc):
+def test_fused_mamba130m_layer(orc, fused_variant):
     """The Mamba-130M layer shape: y and h_final of sampled channels against the
     oracle's conv then scan, and the conv state output and the optional xc copy
     bit for bit equal to the two-call path's (the fused kernel computes the
@@ -111,6 +127,38 @@ def test_fused_mamba130m_layer(orc):
     ry, rh = orc.selective_scan(rxc, sel(a["dt"]), prm.A[ch], host(a["B"]), host(a["C"]),
                                 Dskip=prm.Dskip[ch], z=sel(a["z"]), dt_bias=prm.dt_bias[ch], S=Bn,
                                 want_state=True)
+    assert_close(sel(y1), ry, True, TOL_BF16, "y")
+    assert_close(host(h1)[:, ch], rh, False, TOL_BF16, "h_final")
+    assert ssm.ssm_device_status() == 0
+
+
+def test_fused_packed_workload(orc):
+    """The packed 65536 x 5120 workload (43 sequences) in the kernel the library
+    picks for it (one lane per channel): the conv state output and the xc copy
+    bit for bit equal to the conv kernel's, y and h_final of sampled channels
+    (the first and last among them) against the oracle's conv then scan."""
+    w = synth.WORKLOADS["packmamba_2p8b_varlen_65536"]
+    D = w["D"]
+    lens = synth.sample_lengths(0, w["total"], w["len_lo"], w["len_hi"])
+    cu_d, cu_h = cu_tensor(lens)
+    tok, S = int(cu_h[-1]), len(lens)
+    prm = synth.make_params(0, D)
+    p = {k: dev(getattr(prm, k)) for k in ("conv_w", "conv_b", "A", "Dskip", "dt_bias")}
+    a = synth.device_activations(0, tok, D)
+    xc, cs2 = run_conv(a["x"], p["conv_w"], p["conv_b"], cu=cu_d, S=S, want_state=True)
+    y1, h1, cs1, xc1 = _fused(a["x"], p["conv_w"], p["conv_b"], a["dt"], p["A"], a["B"], a["C"],
+                              p["Dskip"], a["z"], p["dt_bias"], None, None, cu_d, S,
+                              want_xc=True)
+    assert torch.equal(cs1, cs2)
+    assert torch.equal(xc1, xc), "the fused kernel's xc rounds to the conv kernel's bits"
+    rng = np.random.default_rng(1)
+    ch = np.unique(np.concatenate([[0, D - 1], rng.choice(D, size=10, replace=False)]))
+    chd = torch.from_numpy(ch).cuda()
+    sel = lambda t: host(t.index_select(1, chd))  # noqa: E731
+    rxc = orc.causal_conv1d(sel(a["x"]), prm.conv_w[ch], prm.conv_b[ch], cu_seqlens=cu_h)
+    ry, rh = orc.selective_scan(rxc, sel(a["dt"]), prm.A[ch], host(a["B"]), host(a["C"]),
+                                Dskip=prm.Dskip[ch], z=sel(a["z"]), dt_bias=prm.dt_bias[ch],
+                                cu_seqlens=cu_h, want_state=True)
     assert_close(sel(y1), ry, True, TOL_BF16, "y")
     assert_close(host(h1)[:, ch], rh, False, TOL_BF16, "h_final")
     assert ssm.ssm_device_status() == 0
