@@ -84,8 +84,11 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time the headline step as plain launches instead of a CUDA graph")
-    ap.add_argument("--replay-windows", type=int, nargs="+", default=[3], metavar="W",
+    ap.add_argument("--replay-windows", type=int, nargs="+", default=[2, 3], metavar="W",
                     help="checkpoint intervals of the replay decode measurement")
+    ap.add_argument("--replay-copy", choices=["both", "bf16", "none"], default="both",
+                    help="replay decode with the bf16 checkpoint copy for outputs (bf16), "
+                         "with outputs from the fp32 checkpoint (none), or both")
     ap.add_argument("--profile-scan-bwd", nargs="?", const="packed", default=None,
                     choices=["packed", "layer"],
                     help="instead of the step: run 3 backward scans, untimed, for ncu captures: "
@@ -1020,8 +1023,12 @@ def bench_decode(args, world, peaks, mufu):
                              "copied out; states stay on the device; pipelined"}
         del csx, hx
     for W in args.replay_windows:
-        res[f"replay_w{W}"] = bench_replay(peaks, world, ly, cs0, h0, W, steps, mufu,
-                                           not args.no_graph)
+        if args.replay_copy != "none":
+            res[f"replay_w{W}"] = bench_replay(peaks, world, ly, cs0, h0, W, steps, mufu,
+                                               not args.no_graph)
+        if args.replay_copy != "bf16":
+            res[f"replay_w{W}_fp32_ckpt"] = bench_replay(peaks, world, ly, cs0, h0, W, steps, mufu,
+                                                         not args.no_graph, keep_lo=False)
     del cs, h, cs0, h0
     torch.cuda.empty_cache()
     return res
@@ -1147,17 +1154,17 @@ def replay_bytes_per_step(Bt, D, W, keep_lo=True):
     return total / W
 
 
-def bench_replay(peaks, world, ly, cs, h, W, steps, mufu, use_graph=True):
+def bench_replay(peaks, world, ly, cs, h, W, steps, mufu, use_graph=True, keep_lo=True):
     """Batch-256 decode through the replay kernels (checkpoint + input buffer,
-    bf16 checkpoint copy), on the same prefill states and the same kind of
-    fresh per-step inputs as the eager decode measurement."""
+    with or without the bf16 checkpoint copy), on the same prefill states and
+    the same kind of fresh per-step inputs as the eager decode measurement."""
     import torch
 
     import selective_state_space_causal_b200 as ssm
 
     synth = load_synth()
     Bt, D = h.shape[0], h.shape[1]
-    rep = ssm.replay_buffers(Bt, D, W, "cuda", keep_lo=True)
+    rep = ssm.replay_buffers(Bt, D, W, "cuda", keep_lo=keep_lo)
     rep["ckpt"].copy_(h)
     csr = cs.clone()
     ssm.ssm_replay_reset(rep)
@@ -1178,7 +1185,7 @@ def bench_replay(peaks, world, ly, cs, h, W, steps, mufu, use_graph=True):
         del blk
     launches = ssm.ssm_launch_count() - l0
     per = total_ms / done
-    bytes_step = replay_bytes_per_step(Bt, D, W)
+    bytes_step = replay_bytes_per_step(Bt, D, W, keep_lo)
     exps_step = Bt * D * N_STATE * (W + 1) / 2
     res = {
         "value": 1e3 / per * world, "unit": "steps/s", "ms_per_step": per, "steps": done,
@@ -1186,7 +1193,8 @@ def bench_replay(peaks, world, ly, cs, h, W, steps, mufu, use_graph=True):
         "hbm_frac": round(bytes_step / (per * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "mufu_frac": round(exps_step / (per * 1e-3) / 1e9 / mufu["gexp_per_s"], 4),
         "gpu_launches_per_step": launches / done,
-        "step": f"ssm_replay_state_update (checkpoint every {W} tokens, bf16 copy for outputs), "
+        "step": f"ssm_replay_state_update (checkpoint every {W} tokens, "
+                f"{'bf16 copy' if keep_lo else 'the fp32 checkpoint'} for outputs), "
                 "256 rows x 8192 channels, fresh inputs per step; blocks of 100 steps "
                 "replayed as CUDA graphs"}
     del rep, csr

@@ -50,7 +50,7 @@ def _step(cs, rep, s, y, p, dt_, idx=None):
 
 @pytest.mark.parametrize("bf16", [False, True])
 @pytest.mark.parametrize("K", [2, 4])
-@pytest.mark.parametrize("W,keep_lo", [(1, True), (3, False), (4, True), (8, True)])
+@pytest.mark.parametrize("W,keep_lo", [(1, True), (2, False), (3, False), (4, True), (8, True)])
 def test_replay_matches_oracle(orc, bf16, K, W, keep_lo):
     n_slots, Bt, D, steps = 9, 6, 200, 10
     prm = _params(30 + K, D, K)
