@@ -186,7 +186,9 @@ int ssm_causal_conv1d(const void *x, void *xc, const float *weight, const float 
 /*
  * Bytes of optional scratch for ssm_selective_scan_fwd with S packed
  * sequences (a longest-first schedule of the sequences). Passing a NULL
- * workspace is always allowed: sequences are then scheduled in index order.
+ * workspace is always allowed: sequences are then scheduled in index order,
+ * except by schedule 12, whose CTAs rank up to 128 sequences by length
+ * themselves.
  */
 size_t ssm_scan_workspace_size(int64_t tok, int64_t D, int N, int64_t S);
 

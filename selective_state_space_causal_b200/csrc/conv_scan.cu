@@ -331,7 +331,6 @@ cudaError_t by_kw(const Params &p, const ConvParams &cp, int K, int npt, bool ve
 // 16 states, no shuffles. Packed sequences run longest first: with at most
 // kRankMax sequences each CTA ranks the lengths itself (the entry point takes
 // no workspace for an order); above that, in index order.
-constexpr int kRankMax = 128;
 
 template <class K, typename T, typename TS, int KW>
 struct FusedWide {
@@ -479,8 +478,6 @@ conv_scan_wide_kernel(const Params p, const ConvParams cp, const __grid_constant
 {
     constexpr int TCH = K::TCH;
     extern __shared__ __align__(128) unsigned char smem[];
-    __shared__ int cu_s[kRankMax + 1];
-    __shared__ int seq_s;
     FusedWide<K, T, TS, KW> W(smem, p, cp);
     uint64_t *const bar = reinterpret_cast<uint64_t *>(smem + K::OFF_BAR);
     W.tid = threadIdx.x;
@@ -490,26 +487,9 @@ conv_scan_wide_kernel(const Params p, const ConvParams cp, const __grid_constant
     W.sp = p.delta_softplus != 0;
     W.gz = p.z != nullptr;
 
-    // the sequence: blockIdx.y-th longest (ties by index) when the CTA can
-    // rank the lengths itself, else sequence blockIdx.y
-    int64_t seq = blockIdx.y;
-    if (p.cu && p.S > 1 && p.S <= kRankMax) {
-        const int S = (int)p.S;
-        for (int i = W.tid; i <= S; i += K::THREADS) cu_s[i] = (int)clamp_off(p.cu[i], p.tok);
-        if (W.tid == 0) seq_s = (int)blockIdx.y;
-        __syncthreads();
-        for (int i = W.tid; i < S; i += K::THREADS) {
-            const int li = max(cu_s[i + 1] - cu_s[i], 0);
-            int rank = 0;
-            for (int j = 0; j < S; ++j) {
-                const int lj = max(cu_s[j + 1] - cu_s[j], 0);
-                rank += (lj > li) || (lj == li && j < i);
-            }
-            if (rank == (int)blockIdx.y) seq_s = i;
-        }
-        __syncthreads();
-        seq = seq_s;
-    }
+    // longest first (ranked by the CTA when there is no order and at most
+    // kRankMax sequences)
+    int64_t seq = ranked_seq(p);
     seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
     int64_t start, end;
     if (p.cu) {

@@ -114,6 +114,38 @@ __device__ __forceinline__ void stg_if(float *dst, float v, bool pred)
 // Tokens per checkpoint of the state written for the backward pass.
 constexpr int kCkTok = 8;
 
+// Packed sequences run longest first. In the one-lane-per-channel kernels,
+// without a precomputed order (no workspace) and with at most kRankMax
+// sequences, each CTA ranks the lengths itself (their longest chains are twice
+// as long as the split-lane kernels', so the order matters more there): cu_seqlens into shared memory, one rank per thread (ties by index),
+// and the CTA takes the blockIdx.y-th longest. Otherwise sequence blockIdx.y.
+// The branch is the same for the whole CTA, and every thread must call this
+// (it holds two CTA barriers).
+constexpr int kRankMax = 128;
+
+__device__ __forceinline__ int64_t ranked_seq(const Params &p)
+{
+    __shared__ int cu_s[kRankMax + 1];
+    __shared__ int seq_s;
+    if (p.order) return (int64_t)p.order[blockIdx.y];
+    if (!p.cu || p.S <= 1 || p.S > kRankMax) return (int64_t)blockIdx.y;
+    const int S = (int)p.S;
+    for (int i = threadIdx.x; i <= S; i += blockDim.x) cu_s[i] = (int)clamp_off(p.cu[i], p.tok);
+    if (threadIdx.x == 0) seq_s = (int)blockIdx.y;
+    __syncthreads();
+    for (int i = threadIdx.x; i < S; i += blockDim.x) {
+        const int li = max(cu_s[i + 1] - cu_s[i], 0);
+        int rank = 0;
+        for (int j = 0; j < S; ++j) {
+            const int lj = max(cu_s[j + 1] - cu_s[j], 0);
+            rank += (lj > li) || (lj == li && j < i);
+        }
+        if (rank == (int)blockIdx.y) seq_s = i;
+    }
+    __syncthreads();
+    return (int64_t)seq_s;
+}
+
 template <typename T, int NPT_, int CH_, int TCH_, int MINB_ = 3>
 struct PipeCfg {
     static constexpr int NPT = NPT_, CH = CH_, TCH = TCH_;
@@ -911,7 +943,7 @@ scan_wide_kernel(const Params p, const __grid_constant__ Maps m)
     const int64_t cbase = (int64_t)blockIdx.x * K::CH;
     W.c0 = cbase + W.tid;
     W.cvalid = W.c0 < p.D;
-    int64_t seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
+    int64_t seq = ranked_seq(p);
     seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
     int64_t start, end;
     if (p.cu) {

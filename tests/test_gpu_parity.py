@@ -135,6 +135,33 @@ def test_scan_scalar_path(orc, variant):
     _scan_case(orc, 11, [50, 77], 30, True, variant=variant)
 
 
+@pytest.mark.parametrize("nseq", [43, 150])
+def test_scan_order_keeps_results(nseq):
+    """One lane per channel (schedule 12) over packed sequences run in three
+    orders: longest first from the workspace, longest first as each CTA ranks
+    the lengths itself (no workspace, at most 128 sequences), and in index
+    order (no workspace, more than 128). Each sequence's arithmetic does not
+    depend on the order, so y and h_final agree bit for bit."""
+    lens = list(np.random.default_rng(nseq).integers(0, 200, size=nseq))
+    D = 256
+    tok = int(sum(lens))
+    prm, act = _layer_inputs(nseq, tok, D, True)
+    cu_d, _ = cu_tensor(lens)
+    args = (dev(act["x"], torch.bfloat16), dev(act["dt"], torch.bfloat16), dev(prm.A),
+            dev(act["B"], torch.bfloat16), dev(act["C"], torch.bfloat16))
+    kw = dict(Dskip=dev(prm.Dskip), z=dev(act["z"], torch.bfloat16), dt_bias=dev(prm.dt_bias),
+              cu=cu_d)
+    ssm.ssm_set_scan_variant(16, 12)
+    try:
+        y0, h0 = run_scan(*args, workspace=True, **kw)
+        y1, h1 = run_scan(*args, workspace=False, **kw)
+    finally:
+        ssm.ssm_set_scan_variant(0, 0)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, y1) and torch.equal(h0, h1)
+    assert ssm.ssm_device_status() == 0
+
+
 @pytest.mark.parametrize("variant", [(0, 0), (4, 9), (8, 9), (2, 9), (4, 10), (16, 12)],
                          ids=lambda v: f"{v[0]}x{v[1]}")
 def test_scan_options(orc, variant):
