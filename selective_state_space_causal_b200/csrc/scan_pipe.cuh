@@ -931,7 +931,10 @@ struct Wide {
     }
 };
 
-template <class K, typename T, bool SP, bool GZ, bool CK>
+// RK: the CTAs rank the sequences themselves (no order given, at most
+// kRankMax packed sequences); a separate instantiation, so that the kernel
+// with an order (or without packing) keeps its own register allocation.
+template <class K, typename T, bool SP, bool GZ, bool CK, bool RK>
 __global__ void __launch_bounds__(K::THREADS, K::MINB)
 scan_wide_kernel(const Params p, const __grid_constant__ Maps m)
 {
@@ -943,7 +946,9 @@ scan_wide_kernel(const Params p, const __grid_constant__ Maps m)
     const int64_t cbase = (int64_t)blockIdx.x * K::CH;
     W.c0 = cbase + W.tid;
     W.cvalid = W.c0 < p.D;
-    int64_t seq = ranked_seq(p);
+    int64_t seq;
+    if constexpr (RK) seq = ranked_seq(p);
+    else seq = p.order ? (int64_t)p.order[blockIdx.y] : (int64_t)blockIdx.y;
     seq = seq < 0 ? 0 : (seq >= p.S ? p.S - 1 : seq);
     int64_t start, end;
     if (p.cu) {
@@ -1059,16 +1064,24 @@ scan_wide_kernel(const Params p, const __grid_constant__ Maps m)
     }
 }
 
+template <class K, typename T, bool SP, bool GZ, bool CK, bool RK>
+cudaError_t run_wide_k(const Params &p, const Maps &m, cudaStream_t stream, int *launches)
+{
+    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
+    cudaError_t e = cudaFuncSetAttribute(scan_wide_kernel<K, T, SP, GZ, CK, RK>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
+    if (e != cudaSuccess) return e;
+    scan_wide_kernel<K, T, SP, GZ, CK, RK><<<grid, K::THREADS, K::SMEM, stream>>>(p, m);
+    ++*launches;
+    return cudaGetLastError();
+}
+
 template <class K, typename T, bool SP, bool GZ, bool CK>
 cudaError_t run_wide_t(const Params &p, const Maps &m, cudaStream_t stream, int *launches)
 {
-    const dim3 grid((unsigned)((p.D + K::CH - 1) / K::CH), (unsigned)p.S);
-    cudaError_t e = cudaFuncSetAttribute(scan_wide_kernel<K, T, SP, GZ, CK>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)K::SMEM);
-    if (e != cudaSuccess) return e;
-    scan_wide_kernel<K, T, SP, GZ, CK><<<grid, K::THREADS, K::SMEM, stream>>>(p, m);
-    ++*launches;
-    return cudaGetLastError();
+    if (!p.order && p.cu && p.S > 1 && p.S <= kRankMax)
+        return run_wide_k<K, T, SP, GZ, CK, true>(p, m, stream, launches);
+    return run_wide_k<K, T, SP, GZ, CK, false>(p, m, stream, launches);
 }
 
 template <class K, typename T, bool CK>
