@@ -99,11 +99,13 @@ def parse_args(argv=None):
                          "every W tokens, bf16 copy) and 3 eager decode steps at 256 x 8192 from "
                          "random states, untimed, as a small case for ncu captures")
     ap.add_argument("--profile-scan", default=None,
-                    choices=["layer", "long", "packed", "conv_long", "decode_fresh"],
+                    choices=["layer", "long", "packed", "packed_fused", "conv_long",
+                             "decode_fresh"],
                     help="instead of the step: 3 untimed calls of one kernel's workload for ncu "
                          "captures (the Mamba-130M layer scan, one 8192 x 8192 long-context scan "
-                         "call, a 16384-token slice of the packed scan, one 8192 x 8192 conv "
-                         "call, or 3 eager decode steps at 256 x 8192 on fresh inputs)")
+                         "call, a 16384-token slice of the packed scan, the same slice through "
+                         "the fused conv -> scan, one 8192 x 8192 conv call, or 3 eager decode "
+                         "steps at 256 x 8192 on fresh inputs)")
     ap.add_argument("--scan-sweep", nargs="*", metavar="NPT,SCHED", default=None,
                     help="instead of the step: time the scan alone for each variant "
                          "(states per lane, schedule; default: a standard list) on the "
@@ -1417,6 +1419,10 @@ def profile_scan(kind):
         if kind == "conv_long":
             ssm.ssm_causal_conv1d(a["x"], y, ly.w, bias=ly.b, conv_state_in=cs,
                                   conv_state_out=cs)
+        elif kind == "packed_fused":
+            ssm.ssm_conv_scan_fwd(a["x"], ly.w, a["dt"], ly.A, a["B"], a["C"], y, conv_b=ly.b,
+                                  conv_state_in=cs, conv_state_out=cs, Dskip=ly.Dskip, z=a["z"],
+                                  dt_bias=ly.dt_bias, h0=h, h_final=h, cu_seqlens=cu_d, S=S)
         else:
             ssm.ssm_selective_scan_fwd(a["x"], a["dt"], ly.A, a["B"], a["C"], y, Dskip=ly.Dskip,
                                        z=a["z"], dt_bias=ly.dt_bias, h0=h, h_final=h,
